@@ -1,0 +1,443 @@
+"""Benchmark of the paged decode path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl pkv|reference]
+
+One step = one decode step of the whole path for a batch: the block manager's
+append (slot mapping), the KV append kernel for the batch's new tokens, and
+paged decode attention (plus its partition merge) over the updated cache.
+Default workload: the Llama-2-7B-shaped decode batch (B=64, 32/32 heads,
+D=128, bf16, block size 16, context lengths U[512,2048], random placement in
+a 16384-block pool).
+
+Printed metric (one JSON line on rank 0): achieved HBM GB/s of the step
+(algorithmic bytes: every K/V byte of every context read once, Q, the output,
+block tables and lengths, and the appended tokens read and written) with its
+fraction of the measured HBM peak, plus decode tokens/s. `value` is timed with
+per-step inputs already in HBM; `e2e` times the same steps through the public
+API from host buffers (host block manager, pinned H2D copies of the step's
+queries / new K,V / metadata, the kernels, D2H of the output).
+
+Multi-GPU (torchrun): every rank runs its own replica of the batch (decode
+batches are independent; there is no data exchange), times are the max over
+ranks, and `value` is the sum of all ranks' bytes over that time.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_322_b200 import workloads as wl  # noqa: E402
+
+L2_BYTES = 126 * 2 ** 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="pkv", choices=["pkv", "reference"])
+    ap.add_argument("--workload", default="llama2_7b", choices=list(wl.WORKLOADS))
+    ap.add_argument("--partition-tokens", type=int, default=-1, help="-1: the workload's, 0: library default")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_init(args):
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def all_max(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def all_sum(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.samples, self._stop = index, [], threading.Event()
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                r = subprocess.run(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                    "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
+                if r.returncode == 0 and r.stdout.strip():
+                    self.samples.append([x.strip() for x in r.stdout.strip().split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._t.join(timeout=10)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4)
+                          if len(s) > 3 + i and s[3 + i].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def traffic_record():
+    """ncu DRAM traffic of the attention kernel, if taken on the current source."""
+    path = os.path.join(ROOT, "profiles", "attention_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("source_sha1") != kernel_source_sha1():
+        return None
+    return rec
+
+
+def kernel_source_sha1() -> str:
+    h = hashlib.sha1()
+    for name in ("paged_attention.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "paged_kv_cache_322_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+# ---------------------------------------------------------------------------
+# byte accounting (algorithmic: each byte the method must move, once)
+# ---------------------------------------------------------------------------
+def attention_bytes(w: wl.Workload, lens_after: np.ndarray, out_elt: int) -> int:
+    eb = w.elt_bytes
+    kv = int(lens_after.sum()) * w.num_kv_heads * w.head_dim * eb * 2
+    q = w.num_seqs * w.num_q_heads * w.head_dim * eb
+    out = w.num_seqs * w.num_q_heads * w.head_dim * out_elt
+    tables = int(sum(-(-int(n) // w.block_size) for n in lens_after)) * 4
+    return kv + q + out + tables + 4 * w.num_seqs
+
+
+def append_bytes(w: wl.Workload) -> int:
+    row = w.num_kv_heads * w.head_dim * w.elt_bytes
+    return w.num_seqs * (2 * row * 2 + 8)          # K and V rows read and written, slot ids
+
+
+# ---------------------------------------------------------------------------
+# the library arm
+# ---------------------------------------------------------------------------
+def run_pkv(args, ws, rank, local):
+    import torch
+    from paged_kv_cache_322_b200 import binding
+    from paged_kv_cache_322_b200.engine import PagedKVCache
+
+    dev = torch.device("cuda", local)
+    w = wl.WORKLOADS[args.workload]
+    if rank:
+        w = dataclasses.replace(w, seed=w.seed + 7919 * rank)     # each replica its own batch
+    part = w.partition_tokens if args.partition_tokens < 0 else args.partition_tokens
+    K, W = args.steps, args.warmup
+    total_steps = 2 * (K + W) + 2
+    lens0 = wl.context_lens(w)
+    dt = torch.float32 if w.kv_dtype == "f32" else torch.bfloat16
+    mb = -(-int(lens0.max() + total_steps) // w.block_size)
+
+    # ---- set-up (untimed): prompts into the cache through the library ----
+    cache = PagedKVCache(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, dt, dev,
+                         free_order=wl.free_order(w), max_blocks_per_seq=mb)
+    kvs = wl.prompt_kv_all(w, lens0)
+    for s in range(w.num_seqs):
+        k, v = kvs[s]
+        cache.add_sequence(s, torch.from_numpy(k).to(dev, dt), torch.from_numpy(v).to(dev, dt))
+    del kvs
+    ids = np.arange(w.num_seqs, dtype=np.int64)
+    if w.ctx == "shared_prefix":
+        raise SystemExit("the shared-prefix workload is a parity case; bench the decode workloads")
+    torch.cuda.synchronize()
+
+    # ---- per-step inputs, resident in HBM before timing ----
+    steps = []
+    for i in range(K + W):
+        slots, src, dst = cache.bm.append_slots(ids)
+        assert src.size == 0
+        tables, lens = cache.block_tables(ids)
+        q = wl.decode_q(w, i)
+        kn, vn = wl.decode_kv(w, i)
+        steps.append(dict(
+            q=torch.from_numpy(q).to(dev, dt), kn=torch.from_numpy(kn).to(dev, dt),
+            vn=torch.from_numpy(vn).to(dev, dt), slots=torch.from_numpy(slots).to(dev),
+            tables=torch.from_numpy(tables).to(dev), lens=torch.from_numpy(lens).to(dev),
+            maxlen=int(lens.max()), bytes_attn=attention_bytes(w, lens, 2)))
+    out = torch.empty((w.num_seqs, w.num_q_heads, w.head_dim), dtype=torch.bfloat16, device=dev)
+    ws_bytes = binding.workspace_bytes(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, mb,
+                                       max(s["maxlen"] for s in steps), part if part > 0 else 0)
+    workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    part_used = binding.partition_tokens(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, mb,
+                                         max(s["maxlen"] for s in steps), part if part > 0 else 0)
+    stream = torch.cuda.current_stream(dev)
+    maxctx = max(s["maxlen"] for s in steps)
+
+    def step_device(st, ev0=None, ev1=None):
+        binding.reshape_and_cache(st["kn"], st["vn"], cache.k_cache, cache.v_cache, st["slots"])
+        if ev0 is not None:
+            ev0.record(stream)
+        binding.paged_attention_decode(out, st["q"], cache.k_cache, cache.v_cache, st["tables"], st["lens"],
+                                       w.scale, max_context_len=maxctx, partition_tokens=part if part > 0 else 0,
+                                       workspace=workspace)
+        if ev1 is not None:
+            ev1.record(stream)
+
+    for i in range(W):
+        step_device(steps[i])
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t0.record(stream)
+        for i in range(K):
+            step_device(steps[W + i], *ev[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    ms = t0.elapsed_time(t1)
+    attn_ms = [a.elapsed_time(b) for a, b in ev]
+    assert binding.get_device_error() == 0
+    timed = steps[W:]
+    bytes_step = [s["bytes_attn"] + append_bytes(w) for s in timed]
+    local_bytes = float(sum(bytes_step))
+    ms_max = all_max(ms, ws)
+    total_bytes = all_sum(local_bytes, ws)
+    gbs = total_bytes / (ms_max * 1e-3) / 1e9
+    tokens_s = ws * w.num_seqs * K / (ms_max * 1e-3)
+    peak, peak_kind = measured_peaks()
+    attn_avg_ms = statistics.mean(attn_ms)
+    attn_bytes_avg = statistics.mean(s["bytes_attn"] for s in timed)
+    achieved = attn_bytes_avg / (attn_avg_ms * 1e-3) / 1e9
+    launches_per_step = 2 + (1 if (part_used and maxctx > part_used) else 0)
+    del steps
+
+    # ---- end to end through the public API from host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        host = []
+        for i in range(K + W):
+            q = wl.decode_q(w, 1000 + i)
+            kn, vn = wl.decode_kv(w, 1000 + i)
+            host.append(tuple(torch.from_numpy(x).to(dt).pin_memory() for x in (q, kn, vn)))
+        out_host = torch.empty(out.shape, dtype=torch.bfloat16, pin_memory=True)
+        q_d = torch.empty(host[0][0].shape, dtype=dt, device=dev)
+        k_d = torch.empty(host[0][1].shape, dtype=dt, device=dev)
+        v_d = torch.empty(host[0][2].shape, dtype=dt, device=dev)
+        e2e_bytes = []
+
+        def step_host(hq, hk, hv):
+            q_d.copy_(hq, non_blocking=True)
+            k_d.copy_(hk, non_blocking=True)
+            v_d.copy_(hv, non_blocking=True)
+            o = cache.decode_step(ids, q_d, k_d, v_d, w.scale, out=out, partition_tokens=part if part > 0 else 0)
+            out_host.copy_(o, non_blocking=True)
+            stream.synchronize()
+
+        lens_now = np.array([cache.bm.seq_len(int(s)) for s in ids])
+        for i in range(K):
+            e2e_bytes.append(attention_bytes(w, lens_now + W + i + 1, 2) + append_bytes(w))
+
+        for i in range(W):
+            step_host(*host[i])
+        barrier(ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(K):
+            step_host(*host[W + i])
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(ws)
+        e_ms = all_max(e0.elapsed_time(e1), ws)
+        e_total = all_sum(float(sum(e2e_bytes)), ws)
+        eb = w.elt_bytes
+        h2d = (w.num_seqs * w.num_q_heads * w.head_dim * eb + 2 * w.num_seqs * w.num_kv_heads * w.head_dim * eb +
+               w.num_seqs * 8 + w.num_seqs * mb * 4 + w.num_seqs * 4)
+        d2h = w.num_seqs * w.num_q_heads * w.head_dim * 2
+        e2e = {"value": round(e_total / (e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+               "decode_tokens_per_s": round(ws * w.num_seqs * K / (e_ms * 1e-3), 1),
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e_ms / K, 4)}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_seconds)
+
+    tr = traffic_record()
+    result = {
+        "metric": "paged decode attention achieved HBM GB/s (% of B200 peak); decode tokens/s",
+        "value": round(gbs, 1), "unit": "GB/s", "n_gpus": ws, "steps": K, "warmup": W,
+        "ms_per_step": round(ms_max / K, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.kv_dtype, "data": "synthetic",
+        "pct_of_peak": round(100 * gbs / ws / peak, 1),
+        "decode_tokens_per_s": round(tokens_s, 1),
+        "attention_layer_tokens_per_s_per_32_layers": round(tokens_s / 32, 1),
+        "config": {"workload": w.description, "global_batch": w.num_seqs * ws, "seq_len": f"U[{w.lo},{w.hi}]",
+                   "block_size": w.block_size, "partition_tokens": part_used,
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                   "l2": f"inputs larger than L2 ({int(lens0.sum()) * w.num_kv_heads * w.head_dim * w.elt_bytes * 2 / 1e9:.2f} GB KV per step vs 126 MB L2); no flush",
+                   "seed": w.seed},
+        "roofline": {"bound": "hbm", "kernel": "paged_decode_kernel + merge_partitions_kernel (one attention call)",
+                     "achieved": round(achieved, 1), "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "avg_launch_ms": round(attn_avg_ms, 5),
+                     "algorithmic_bytes_per_launch": int(attn_bytes_avg),
+                     "traffic": (tr["traffic_bytes_per_launch"] if tr else None)},
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * K,
+        "clocks": clocks.summary(),
+        "cpu_baseline": cpu,
+    }
+    return result
+
+
+def cpu_baseline(w: wl.Workload, target_s: float):
+    """The oracle, as it stands, on a bounded sample of the same workload: whole
+    sequences (their logical K/V regenerated from the seeded generator, written
+    into an oracle pool, attention in fp64), until ~target_s seconds of CPU."""
+    from oracle import cache_ops as ocache
+    from oracle import paged_attention as oattn
+    from oracle.block_manager import BlockManager as OracleBM
+    lens = wl.context_lens(w)
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    q = wl.decode_q(w, 0)
+    done, nbytes, t_total = 0, 0, 0.0
+    for s in range(w.num_seqs):
+        n = int(lens[s])
+        k, v = wl.prompt_kv(w, s, n)
+        nblk = -(-n // w.block_size)
+        bm = OracleBM(nblk, w.block_size)
+        kc = np.zeros((nblk, w.block_size, w.num_kv_heads, w.head_dim), np.float32)
+        vc = np.zeros_like(kc)
+        t0 = time.perf_counter()
+        ocache.reshape_and_cache(k, v, kc, vc, np.asarray(bm.allocate(0, n)))
+        oattn.paged_attention_decode(q[s:s + 1], kc, vc, [bm.block_table(0)], [n], w.scale, w.block_size)
+        t_total += time.perf_counter() - t0
+        done += 1
+        nbytes += n * w.num_kv_heads * w.head_dim * w.elt_bytes * 2 + 2 * w.num_q_heads * w.head_dim * w.elt_bytes
+        if t_total >= target_s:
+            break
+    return {"value": round(nbytes / t_total / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} of {w.num_seqs} sequences of the bench workload (KV append + fp64 attention), "
+                      f"{t_total:.1f} s", "decode_tokens_per_s": round(done / t_total, 2)}
+
+
+def run_reference(args, ws, rank):
+    """The reference arm: the CPU oracle, timed per step on a bounded sample."""
+    w = wl.WORKLOADS[args.workload]
+    if rank != 0:
+        return None
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    per_step_s = max(0.5, min(10.0, 90.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(w, per_step_s)
+        if i >= args.warmup:
+            vals.append(r)
+    v = statistics.mean(x["value"] for x in vals)
+    return {"impl": "reference", "metric": "paged decode attention achieved HBM GB/s (% of B200 peak); decode tokens/s",
+            "value": round(v, 4), "unit": "GB/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.description},
+            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": f"per step: {vals[0]['sample']}"},
+            "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        ws = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        r = run_reference(args, ws, rank)
+        if r is not None:
+            print(json.dumps(r), flush=True)
+        return
+    ws, rank, local = dist_init(args)
+    try:
+        r = run_pkv(args, ws, rank, local)
+        if rank == 0:
+            print(json.dumps(r), flush=True)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,241 @@
+/*
+ * pkv.h -- C ABI of the paged KV-cache decode library (libpkv.so, sm_100a).
+ *
+ * The library implements the data-parallel decode path of PagedAttention:
+ *   - pkv_paged_attention_decode : decode attention of one query token per
+ *     sequence over a KV cache split into fixed-size physical blocks and
+ *     reached through per-sequence block tables (MHA and grouped-query).
+ *   - pkv_reshape_and_cache      : the per-token KV append into the cache.
+ *   - pkv_copy_blocks            : physical block copies for copy-on-write forks.
+ *   - pkv_bm_*                   : a host-side block manager (free list, block
+ *     tables, slot mapping, reference counts, copy-on-write) that produces the
+ *     block tables, slot mappings and copy lists the kernels consume.
+ *
+ * Sources of the definitions (web pages on vLLM's PagedAttention):
+ *   [BT]  "为什么PagedAttention能让大模型推理吞吐量提升数倍：从KV Cache内存碎片到分页管理的
+ *         系统级优化", section "Block Table：GPU上的页表" (block tables, the 7-token
+ *         walkthrough) and section "Memory Sharing" (shared blocks, copy-on-write).
+ *   [ENG] "LLM 推理引擎内部原理：PagedAttention、Continuous Batching 与现代推理架构剖析",
+ *         §2.3 (Block 分配器: free list, allocate, append_slot, free) and §2.4
+ *         (CUDA kernel: cache layout [num_blocks, block_size, num_heads, head_dim],
+ *         two-level addressing block table -> physical block -> in-block offset).
+ *   [VP]  "vLLM PagedAttention 深度解析" (cyqw.cn), §3.3 (single-request prefill and
+ *         decode flow), §4.1 (parallel sampling, reference counts, copy-on-write),
+ *         §4.2 (beam search, blocks freed when their count reaches 0).
+ *
+ * Conventions shared by every call:
+ *   - Every data pointer passed to a kernel entry point is a DEVICE pointer
+ *     on the current CUDA device. The caller allocates and owns all memory;
+ *     no kernel entry point allocates, frees or synchronises (pkv_get_device_error
+ *     excepted). Calls are asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream).
+ *   - Tensors are dense, row-major and 16-byte aligned:
+ *       q, out          [num_seqs, num_q_heads, head_dim]
+ *       k, v (new)      [num_tokens, num_kv_heads, head_dim]
+ *       k_cache,v_cache [num_blocks, block_size, num_kv_heads, head_dim]   ([ENG] §2.4)
+ *       block_tables    int32 [num_seqs, max_blocks_per_seq]; entry j of row s is the
+ *                       physical block holding tokens [j*block_size, (j+1)*block_size)
+ *       context_lens    int32 [num_seqs]
+ *       slot_mapping    int64 [num_tokens]; slot = physical_block*block_size + offset
+ *   - Supported: head_dim 64 or 128; block_size 16; num_q_heads a multiple of
+ *     num_kv_heads with group size num_q_heads/num_kv_heads in {1, 2, 4, 8};
+ *     kv dtype f32 or bf16 (q has the kv dtype). Query head h reads KV head
+ *     h / group (a reading: the pages do not discuss grouped-query attention).
+ *   - Errors detected on the host (bad sizes, null pointers, unsupported shapes,
+ *     a launch failure) are returned at once and nothing is launched.
+ *     Errors that need device data (a block id or slot outside the pool, a context
+ *     longer than the block table) cannot be seen by the host without a
+ *     synchronisation: the kernel skips the bad access, records the error in a
+ *     device error word and carries on; read it with pkv_get_device_error.
+ *     No kernel traps or asserts.
+ */
+#ifndef PKV_H
+#define PKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pkv_status {
+    PKV_OK = 0,
+    PKV_ERR_INVALID_ARG = 1,     /* a size, pointer or alignment is invalid */
+    PKV_ERR_UNSUPPORTED = 2,     /* valid but not built (head_dim, block_size, group) */
+    PKV_ERR_CUDA = 3,            /* a CUDA runtime call or launch failed */
+    PKV_ERR_DEVICE_BOUNDS = 4,   /* (device word) a block id / slot / length was out of range */
+    PKV_ERR_OUT_OF_BLOCKS = 5,   /* (block manager) the free list is empty */
+    PKV_ERR_DEVICE_TIMEOUT = 6   /* (device word) a bounded wait inside a kernel gave up */
+} pkv_status;
+
+typedef enum pkv_dtype { PKV_F32 = 0, PKV_BF16 = 1 } pkv_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* pkv_status_string(int status);
+
+/* ------------------------------------------------------------------------- */
+/* Decode attention                                                          */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * Decode attention over the paged cache ([ENG] §2.4; [BT] "Block Table"):
+ * for every sequence s and query head h (KV head g = h / group),
+ *     out[s,h,:] = sum_j softmax_j(scale * q[s,h,:] . K_s[j,g,:]) * V_s[j,g,:]
+ * over the first context_lens[s] logical tokens j of sequence s, where token j
+ * is read from physical block block_tables[s][j / block_size], offset
+ * j % block_size. A sequence with context length 0 gets a zero output.
+ *
+ * Long contexts are cut into partitions of `partition_tokens` tokens (a
+ * multiple of block_size; 0 picks one from the shapes) that are processed in
+ * parallel and merged exactly with a log-sum-exp reduction. Partial results
+ * live in `workspace` (device memory, at least
+ * pkv_paged_attention_workspace_bytes(...) bytes, 256-byte aligned; it may be
+ * NULL when that size is 0). Its contents need no initialisation and are
+ * scratch between calls; two calls in flight at once need two workspaces.
+ *
+ *   out            device, [num_seqs, num_q_heads, head_dim], out_dtype (f32 or bf16)
+ *   q              device, [num_seqs, num_q_heads, head_dim], kv_dtype
+ *   k_cache,v_cache device, [num_blocks, block_size, num_kv_heads, head_dim], kv_dtype
+ *   block_tables   device int32 [num_seqs, max_blocks_per_seq]
+ *   context_lens   device int32 [num_seqs], each in [0, max_blocks_per_seq*block_size]
+ *   max_context_len host upper bound of context_lens (sizes the partition grid);
+ *                  0 means max_blocks_per_seq*block_size. A length above it or
+ *                  above the table's capacity is clamped and flagged
+ *                  PKV_ERR_DEVICE_BOUNDS in the device error word.
+ *   Block ids outside [0, num_blocks) are flagged the same way and read as zeros.
+ */
+pkv_status pkv_paged_attention_decode(
+    void* out, pkv_dtype out_dtype,
+    const void* q, const void* k_cache, const void* v_cache, pkv_dtype kv_dtype,
+    const int32_t* block_tables, const int32_t* context_lens, float scale,
+    int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+    int block_size, int max_blocks_per_seq, int num_blocks,
+    int max_context_len, int partition_tokens,
+    void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace pkv_paged_attention_decode needs for these sizes (0 when
+ * no sequence can span more than one partition). Same partition rule as the
+ * decode call; pass the same max_context_len and partition_tokens. Returns
+ * (size_t)-1 for invalid sizes. */
+size_t pkv_paged_attention_workspace_bytes(
+    int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+    int max_blocks_per_seq, int max_context_len, int partition_tokens);
+
+/* The partition length (tokens) the decode call uses for these sizes. */
+int pkv_paged_attention_partition_tokens(
+    int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+    int max_blocks_per_seq, int max_context_len, int partition_tokens);
+
+/* ------------------------------------------------------------------------- */
+/* Cache-side kernels                                                        */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * KV append ([VP] §3.3, prefill step 3 and decode step 2: each new token's K
+ * and V are written to the physical slot its block table maps it to):
+ *     k_cache[slot / block_size, slot % block_size, :, :] = k[t, :, :]   (same for v)
+ * for every token t with slot = slot_mapping[t] >= 0; negative slots are
+ * skipped (padding). Slots >= num_blocks*block_size are skipped and flagged
+ * PKV_ERR_DEVICE_BOUNDS. Two tokens with the same slot in one call race.
+ *
+ *   k, v           device, [num_tokens, num_kv_heads, head_dim], dtype
+ *   k_cache,v_cache device, [num_blocks, block_size, num_kv_heads, head_dim], dtype
+ *   slot_mapping   device int64 [num_tokens]
+ * num_tokens may be 0 (nothing is launched).
+ */
+pkv_status pkv_reshape_and_cache(
+    const void* k, const void* v, void* k_cache, void* v_cache, pkv_dtype dtype,
+    const int64_t* slot_mapping, int num_tokens,
+    int num_kv_heads, int head_dim, int block_size, int num_blocks, void* stream);
+
+/*
+ * Block copy for copy-on-write ([VP] §4.1: the shared physical block is copied
+ * to a fresh block for the sample that writes next):
+ *     k_cache[dst[i]] = k_cache[src[i]],  v_cache[dst[i]] = v_cache[src[i]]
+ * for i < num_pairs, every slot of the block. Destination ids must be distinct
+ * and must not appear among the sources of the same call (the copies run in
+ * parallel). Ids outside [0, num_blocks) are skipped and flagged
+ * PKV_ERR_DEVICE_BOUNDS.
+ *
+ *   src_block_ids, dst_block_ids  device int64 [num_pairs]
+ * num_pairs may be 0 (nothing is launched).
+ */
+pkv_status pkv_copy_blocks(
+    void* k_cache, void* v_cache, pkv_dtype dtype,
+    const int64_t* src_block_ids, const int64_t* dst_block_ids, int num_pairs,
+    int block_size, int num_kv_heads, int head_dim, int num_blocks, void* stream);
+
+/*
+ * Reads and clears the current device's error word (0 or a pkv_status code set
+ * by a kernel). Synchronises `stream` first. `code` is a host pointer.
+ */
+pkv_status pkv_get_device_error(int* code, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Host block manager ([ENG] §2.3; [VP] §3.3, §4.1, §4.2; [BT])              */
+/* ------------------------------------------------------------------------- */
+/*
+ * Plain host memory, not thread-safe (one manager per scheduler thread).
+ * Sequences are named by caller-chosen int64 ids. All array arguments here are
+ * HOST pointers.
+ *
+ * Free list: FIFO of block ids, taken from the front, returned to the back
+ * ([ENG] §2.3). Reference counts: a block shared by k sequences has count k;
+ * a block whose count falls to 0 goes back to the free list ([VP] §4.2).
+ */
+typedef struct pkv_block_manager pkv_block_manager;
+
+/* free_order: the initial free-list order (a permutation of 0..num_blocks-1),
+ * or NULL for 0,1,2,... The manager copies it. */
+pkv_status pkv_bm_create(int num_blocks, int block_size, const int32_t* free_order,
+                         pkv_block_manager** out);
+void pkv_bm_destroy(pkv_block_manager* bm);
+
+/* New sequence of num_tokens prompt tokens: takes ceil(num_tokens/block_size)
+ * blocks and writes the slot of every prompt token to slots_out (may be NULL).
+ * PKV_ERR_OUT_OF_BLOCKS (nothing taken) if the free list is too short;
+ * PKV_ERR_INVALID_ARG if seq_id already exists. */
+pkv_status pkv_bm_allocate(pkv_block_manager* bm, int64_t seq_id, int num_tokens,
+                           int64_t* slots_out);
+
+/* One decode step: appends one token to each listed sequence, in order, and
+ * writes its slot to slot_mapping_out[i]. A sequence whose last block still has
+ * room writes into it, after a copy-on-write if that block is shared (the
+ * (src, dst) pair is appended to copy_src_out/copy_dst_out, capacity n); a full
+ * last block gets a new block. *num_copies_out receives the number of pairs.
+ * On PKV_ERR_OUT_OF_BLOCKS, *num_done_out sequences were appended and the rest
+ * untouched. num_done_out may be NULL. */
+pkv_status pkv_bm_append_slots(pkv_block_manager* bm, const int64_t* seq_ids, int n,
+                               int64_t* slot_mapping_out, int64_t* copy_src_out,
+                               int64_t* copy_dst_out, int* num_copies_out, int* num_done_out);
+
+/* Copy-on-write of one logical block of a sequence: if its physical block is
+ * shared, the sequence gets a fresh block and (*src, *dst) is the copy to run;
+ * otherwise *src = *dst = -1. */
+pkv_status pkv_bm_make_writable(pkv_block_manager* bm, int64_t seq_id, int logical_block,
+                                int64_t* src, int64_t* dst);
+
+/* child shares all of parent's blocks (each count + 1) and its length. */
+pkv_status pkv_bm_fork(pkv_block_manager* bm, int64_t parent, int64_t child);
+
+/* Drops a sequence: each of its blocks' counts falls by one, blocks at 0 return
+ * to the back of the free list in table order. */
+pkv_status pkv_bm_free(pkv_block_manager* bm, int64_t seq_id);
+
+/* Block tables and lengths of the listed sequences, rows of max_blocks int32
+ * entries padded with 0, ready to copy to the device. PKV_ERR_INVALID_ARG if a
+ * sequence has more than max_blocks blocks. context_lens_out may be NULL. */
+pkv_status pkv_bm_block_tables(const pkv_block_manager* bm, const int64_t* seq_ids, int n,
+                               int max_blocks, int32_t* tables_out, int32_t* context_lens_out);
+
+int pkv_bm_num_free(const pkv_block_manager* bm);
+int pkv_bm_ref_count(const pkv_block_manager* bm, int block);
+/* Number of tokens of a sequence, or -1 if unknown. */
+int pkv_bm_seq_len(const pkv_block_manager* bm, int64_t seq_id);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H */

@@ -1,0 +1,275 @@
+"""Thin Python binding of libpkv.so (ctypes).
+
+Argument marshalling only: shapes, dtypes and pointers are read from torch
+tensors and passed to the C ABI declared in include/pkv.h; every step of the
+path runs in the library's CUDA kernels (or, for the block manager, its C++
+host code). There is no fallback: if libpkv.so is missing, every call raises.
+Build it with `python -m paged_kv_cache_322_b200.build`.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpkv.so")
+
+PKV_F32, PKV_BF16 = 0, 1
+STATUS = {0: "PKV_OK", 1: "PKV_ERR_INVALID_ARG", 2: "PKV_ERR_UNSUPPORTED", 3: "PKV_ERR_CUDA",
+          4: "PKV_ERR_DEVICE_BOUNDS", 5: "PKV_ERR_OUT_OF_BLOCKS", 6: "PKV_ERR_DEVICE_TIMEOUT"}
+
+
+class PkvError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        name = STATUS.get(status, str(status))
+        super().__init__(f"{what}: {name} ({_lib().pkv_status_string(status).decode()})")
+
+
+_L = None
+_c = ctypes
+_vp, _i32, _i64, _f32, _sz = _c.c_void_p, _c.c_int, _c.c_int64, _c.c_float, _c.c_size_t
+_pi32, _pi64 = _c.POINTER(_c.c_int32), _c.POINTER(_c.c_int64)
+
+_SIGS = {
+    "pkv_status_string": (_c.c_char_p, [_i32]),
+    "pkv_paged_attention_decode": (_i32, [_vp, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _f32, _i32, _i32, _i32, _i32,
+                                          _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp]),
+    "pkv_paged_attention_workspace_bytes": (_sz, [_i32] * 8),
+    "pkv_paged_attention_partition_tokens": (_i32, [_i32] * 8),
+    "pkv_reshape_and_cache": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
+    "pkv_copy_blocks": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
+    "pkv_get_device_error": (_i32, [_c.POINTER(_c.c_int), _vp]),
+    "pkv_bm_create": (_i32, [_i32, _i32, _pi32, _c.POINTER(_vp)]),
+    "pkv_bm_destroy": (None, [_vp]),
+    "pkv_bm_allocate": (_i32, [_vp, _i64, _i32, _pi64]),
+    "pkv_bm_append_slots": (_i32, [_vp, _pi64, _i32, _pi64, _pi64, _pi64, _c.POINTER(_c.c_int),
+                                   _c.POINTER(_c.c_int)]),
+    "pkv_bm_make_writable": (_i32, [_vp, _i64, _i32, _pi64, _pi64]),
+    "pkv_bm_fork": (_i32, [_vp, _i64, _i64]),
+    "pkv_bm_free": (_i32, [_vp, _i64]),
+    "pkv_bm_block_tables": (_i32, [_vp, _pi64, _i32, _i32, _pi32, _pi32]),
+    "pkv_bm_num_free": (_i32, [_vp]),
+    "pkv_bm_ref_count": (_i32, [_vp, _i32]),
+    "pkv_bm_seq_len": (_i32, [_vp, _i64]),
+}
+
+
+def _lib():
+    global _L
+    if _L is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built; run `python -m paged_kv_cache_322_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(lib, name)
+            f.restype = res
+            f.argtypes = args
+        _L = lib
+    return _L
+
+
+def library():
+    """The loaded ctypes library (loads it on first use)."""
+    return _lib()
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise PkvError(status, what)
+
+
+def _ptr(a: np.ndarray, ctype):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+# ---------------------------------------------------------------------------
+# torch-facing kernel calls
+# ---------------------------------------------------------------------------
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return PKV_F32
+    if t.dtype == torch.bfloat16:
+        return PKV_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _stream(t, stream) -> int:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream(t.device)
+    return s.cuda_stream
+
+
+def _cuda_contig(*ts):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must be CUDA tensors")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                    max_context_len=0, partition_tokens=0) -> int:
+    n = _lib().pkv_paged_attention_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                                   max_blocks_per_seq, max_context_len, partition_tokens)
+    if n == ctypes.c_size_t(-1).value:
+        raise PkvError(1, "pkv_paged_attention_workspace_bytes")
+    return n
+
+
+def partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                     max_context_len=0, partition_tokens=0) -> int:
+    return _lib().pkv_paged_attention_partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                                       max_blocks_per_seq, max_context_len, partition_tokens)
+
+
+def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                           max_context_len: int = 0, partition_tokens: int = 0, workspace=None, stream=None):
+    """out[s,h] = softmax(scale q[s,h] K_s^T) V_s over the block-table-addressed cache.
+
+    out, q [B, Hq, D]; caches [NB, bs, Hkv, D]; block_tables int32 [B, MB];
+    context_lens int32 [B]. `workspace` (uint8 CUDA tensor) is allocated from
+    torch's allocator when not given."""
+    torch = _torch()
+    _cuda_contig(out, q, k_cache, v_cache, block_tables, context_lens)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    B, hq, d = q.shape
+    nb, bs, hkv, d2 = k_cache.shape
+    if d2 != d or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != (B, hq, d):
+        raise ValueError("shape mismatch")
+    if q.dtype != k_cache.dtype or v_cache.dtype != k_cache.dtype:
+        raise TypeError("q, k_cache and v_cache must share a dtype")
+    mb = block_tables.shape[1]
+    need = workspace_bytes(B, hq, hkv, d, bs, mb, max_context_len, partition_tokens)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_n = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = _lib().pkv_paged_attention_decode(
+        out.data_ptr(), _dtype_code(out), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+        _dtype_code(k_cache), block_tables.data_ptr(), context_lens.data_ptr(), float(scale), B, hq, hkv, d, bs,
+        mb, nb, int(max_context_len), int(partition_tokens), ws_ptr, ws_n, _stream(q, stream))
+    _check(st, "pkv_paged_attention_decode")
+    return out
+
+
+def reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, stream=None):
+    """Writes k[t], v[t] ([T, Hkv, D]) into cache slot slot_mapping[t] (int64; < 0 skipped)."""
+    torch = _torch()
+    _cuda_contig(k, v, k_cache, v_cache, slot_mapping)
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    nb, bs, hkv, d = k_cache.shape
+    T = k.shape[0]
+    if tuple(k.shape) != (T, hkv, d) or tuple(v.shape) != (T, hkv, d) or slot_mapping.numel() != T:
+        raise ValueError("shape mismatch")
+    if not (k.dtype == v.dtype == k_cache.dtype == v_cache.dtype):
+        raise TypeError("k, v and the caches must share a dtype")
+    st = _lib().pkv_reshape_and_cache(k.data_ptr(), v.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                      _dtype_code(k_cache), slot_mapping.data_ptr(), T, hkv, d, bs, nb,
+                                      _stream(k_cache, stream))
+    _check(st, "pkv_reshape_and_cache")
+
+
+def copy_blocks(k_cache, v_cache, src, dst, stream=None):
+    """cache[dst[i]] = cache[src[i]] for K and V (src, dst int64 CUDA tensors)."""
+    torch = _torch()
+    _cuda_contig(k_cache, v_cache, src, dst)
+    if src.dtype != torch.int64 or dst.dtype != torch.int64 or src.numel() != dst.numel():
+        raise TypeError("src and dst must be int64 tensors of equal length")
+    nb, bs, hkv, d = k_cache.shape
+    st = _lib().pkv_copy_blocks(k_cache.data_ptr(), v_cache.data_ptr(), _dtype_code(k_cache), src.data_ptr(),
+                                dst.data_ptr(), src.numel(), bs, hkv, d, nb, _stream(k_cache, stream))
+    _check(st, "pkv_copy_blocks")
+
+
+def get_device_error(stream=None) -> int:
+    """Reads and clears the current device's error word (synchronises the stream)."""
+    torch = _torch()
+    code = ctypes.c_int(0)
+    s = stream if stream is not None else torch.cuda.current_stream()
+    _check(_lib().pkv_get_device_error(ctypes.byref(code), s.cuda_stream), "pkv_get_device_error")
+    return code.value
+
+
+# ---------------------------------------------------------------------------
+# host block manager
+# ---------------------------------------------------------------------------
+class BlockManager:
+    """The library's C++ block manager (free list, tables, slots, refcounts, CoW)."""
+
+    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+        self._h = ctypes.c_void_p()
+        order = None
+        if free_order is not None:
+            order = np.ascontiguousarray(free_order, dtype=np.int32)
+            if order.size != num_blocks:
+                raise ValueError("free_order must list every block")
+        _check(_lib().pkv_bm_create(num_blocks, block_size, _ptr(order, ctypes.c_int32) if order is not None else None,
+                                    ctypes.byref(self._h)), "pkv_bm_create")
+        self.num_blocks, self.block_size = num_blocks, block_size
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value and _L is not None:
+            _L.pkv_bm_destroy(h)
+            self._h = None
+
+    def allocate(self, seq_id: int, num_tokens: int) -> np.ndarray:
+        slots = np.empty(max(num_tokens, 1), dtype=np.int64)
+        _check(_lib().pkv_bm_allocate(self._h, seq_id, num_tokens, _ptr(slots, ctypes.c_int64)), "pkv_bm_allocate")
+        return slots[:num_tokens]
+
+    def append_slots(self, seq_ids):
+        """One decode step for the listed sequences -> (slot_mapping, copy_src, copy_dst)."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = ids.size
+        slots = np.empty(max(n, 1), np.int64)
+        src = np.empty(max(n, 1), np.int64)
+        dst = np.empty(max(n, 1), np.int64)
+        nc, nd = ctypes.c_int(0), ctypes.c_int(0)
+        st = _lib().pkv_bm_append_slots(self._h, _ptr(ids, ctypes.c_int64), n, _ptr(slots, ctypes.c_int64),
+                                        _ptr(src, ctypes.c_int64), _ptr(dst, ctypes.c_int64), ctypes.byref(nc),
+                                        ctypes.byref(nd))
+        _check(st, "pkv_bm_append_slots")
+        return slots[:n], src[:nc.value], dst[:nc.value]
+
+    def make_writable(self, seq_id: int, logical_block: int):
+        s, d = ctypes.c_int64(-1), ctypes.c_int64(-1)
+        _check(_lib().pkv_bm_make_writable(self._h, seq_id, logical_block, ctypes.byref(s), ctypes.byref(d)),
+               "pkv_bm_make_writable")
+        return None if s.value < 0 else (s.value, d.value)
+
+    def fork(self, parent: int, child: int):
+        _check(_lib().pkv_bm_fork(self._h, parent, child), "pkv_bm_fork")
+
+    def free(self, seq_id: int):
+        _check(_lib().pkv_bm_free(self._h, seq_id), "pkv_bm_free")
+
+    def block_tables(self, seq_ids, max_blocks: int):
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        tables = np.zeros((ids.size, max_blocks), np.int32)
+        lens = np.zeros(ids.size, np.int32)
+        _check(_lib().pkv_bm_block_tables(self._h, _ptr(ids, ctypes.c_int64), ids.size, max_blocks,
+                                          _ptr(tables, ctypes.c_int32), _ptr(lens, ctypes.c_int32)),
+               "pkv_bm_block_tables")
+        return tables, lens
+
+    def num_free(self) -> int:
+        return _lib().pkv_bm_num_free(self._h)
+
+    def ref_count(self, block: int) -> int:
+        return _lib().pkv_bm_ref_count(self._h, block)
+
+    def seq_len(self, seq_id: int) -> int:
+        return _lib().pkv_bm_seq_len(self._h, seq_id)

@@ -1,0 +1,212 @@
+// Host block manager: FIFO free list, per-sequence block tables, slot mapping,
+// reference counts and copy-on-write.
+//
+// Follows "LLM 推理引擎内部原理" §2.3 (Block 分配器): the free pool is a FIFO of
+// block ids; a new request takes ceil(n / block_size) blocks; appending a token
+// writes into the last block while it has room, else takes one block from the
+// front of the free list; freed blocks go to the back. "vLLM PagedAttention 深度
+// 解析" §4.1 adds sharing: forked samples point at the same physical blocks with
+// a reference count, and the first write into a shared block copies it for the
+// writer (old count - 1, new count 1); §4.2: a block returns to the pool when its
+// count reaches 0.
+//
+// The free list is a ring buffer of capacity num_blocks (each id is either in
+// the ring or referenced, never both), so every call is O(1) per block.
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <unordered_map>
+#include <vector>
+
+#include "../../include/pkv.h"
+
+namespace {
+
+struct Seq {
+    std::vector<int32_t> table;
+    int64_t len = 0;
+};
+
+}  // namespace
+
+struct pkv_block_manager {
+    int num_blocks = 0;
+    int block_size = 0;
+    std::vector<int32_t> ring;      // free list, FIFO
+    size_t head = 0, count = 0;
+    std::vector<int32_t> ref;
+    std::unordered_map<int64_t, Seq> seqs;
+
+    bool take(int32_t* b) {
+        if (count == 0) return false;
+        *b = ring[head];
+        head = (head + 1) % ring.size();
+        --count;
+        ref[*b] = 1;
+        return true;
+    }
+    void give_back(int32_t b) {
+        ring[(head + count) % ring.size()] = b;
+        ++count;
+    }
+    void release(int32_t b) {
+        if (--ref[b] == 0) give_back(b);
+    }
+    int64_t slot(const Seq& s, int64_t pos) const {
+        return (int64_t)s.table[pos / block_size] * block_size + pos % block_size;
+    }
+};
+
+extern "C" {
+
+pkv_status pkv_bm_create(int num_blocks, int block_size, const int32_t* free_order,
+                         pkv_block_manager** out) {
+    if (!out || num_blocks <= 0 || block_size <= 0) return PKV_ERR_INVALID_ARG;
+    *out = nullptr;
+    pkv_block_manager* bm = new (std::nothrow) pkv_block_manager();
+    if (!bm) return PKV_ERR_INVALID_ARG;
+    bm->num_blocks = num_blocks;
+    bm->block_size = block_size;
+    bm->ring.resize(num_blocks);
+    bm->ref.assign(num_blocks, 0);
+    if (free_order) {
+        std::vector<char> seen(num_blocks, 0);
+        for (int i = 0; i < num_blocks; ++i) {
+            int32_t b = free_order[i];
+            if (b < 0 || b >= num_blocks || seen[b]) { delete bm; return PKV_ERR_INVALID_ARG; }
+            seen[b] = 1;
+            bm->ring[i] = b;
+        }
+    } else {
+        for (int i = 0; i < num_blocks; ++i) bm->ring[i] = i;
+    }
+    bm->head = 0;
+    bm->count = num_blocks;
+    *out = bm;
+    return PKV_OK;
+}
+
+void pkv_bm_destroy(pkv_block_manager* bm) { delete bm; }
+
+pkv_status pkv_bm_allocate(pkv_block_manager* bm, int64_t seq_id, int num_tokens, int64_t* slots_out) {
+    if (!bm || num_tokens < 0) return PKV_ERR_INVALID_ARG;
+    if (bm->seqs.count(seq_id)) return PKV_ERR_INVALID_ARG;
+    const int64_t nblk = ((int64_t)num_tokens + bm->block_size - 1) / bm->block_size;
+    if ((size_t)nblk > bm->count) return PKV_ERR_OUT_OF_BLOCKS;
+    Seq s;
+    s.table.resize(nblk);
+    for (int64_t i = 0; i < nblk; ++i) bm->take(&s.table[i]);
+    s.len = num_tokens;
+    if (slots_out)
+        for (int64_t p = 0; p < num_tokens; ++p) slots_out[p] = bm->slot(s, p);
+    bm->seqs.emplace(seq_id, std::move(s));
+    return PKV_OK;
+}
+
+pkv_status pkv_bm_append_slots(pkv_block_manager* bm, const int64_t* seq_ids, int n,
+                               int64_t* slot_mapping_out, int64_t* copy_src_out,
+                               int64_t* copy_dst_out, int* num_copies_out, int* num_done_out) {
+    if (num_done_out) *num_done_out = 0;
+    if (num_copies_out) *num_copies_out = 0;
+    if (!bm || n < 0 || (n > 0 && (!seq_ids || !slot_mapping_out || !copy_src_out ||
+                                   !copy_dst_out || !num_copies_out)))
+        return PKV_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i)
+        if (!bm->seqs.count(seq_ids[i])) return PKV_ERR_INVALID_ARG;
+    int ncopy = 0;
+    for (int i = 0; i < n; ++i) {
+        Seq& s = bm->seqs[seq_ids[i]];
+        const int64_t len = s.len;
+        if (len % bm->block_size != 0) {
+            int32_t last = s.table.back();
+            if (bm->ref[last] > 1) {             // shared partially filled block: copy-on-write
+                int32_t fresh;
+                if (!bm->take(&fresh)) { *num_copies_out = ncopy; return PKV_ERR_OUT_OF_BLOCKS; }
+                bm->ref[last] -= 1;
+                s.table.back() = fresh;
+                copy_src_out[ncopy] = last;
+                copy_dst_out[ncopy] = fresh;
+                ++ncopy;
+            }
+        } else {
+            int32_t fresh;
+            if (!bm->take(&fresh)) { *num_copies_out = ncopy; return PKV_ERR_OUT_OF_BLOCKS; }
+            s.table.push_back(fresh);
+        }
+        slot_mapping_out[i] = bm->slot(s, len);
+        s.len = len + 1;
+        if (num_done_out) *num_done_out = i + 1;
+    }
+    *num_copies_out = ncopy;
+    return PKV_OK;
+}
+
+pkv_status pkv_bm_make_writable(pkv_block_manager* bm, int64_t seq_id, int logical_block,
+                                int64_t* src, int64_t* dst) {
+    if (!bm || !src || !dst) return PKV_ERR_INVALID_ARG;
+    *src = *dst = -1;
+    auto it = bm->seqs.find(seq_id);
+    if (it == bm->seqs.end()) return PKV_ERR_INVALID_ARG;
+    Seq& s = it->second;
+    if (logical_block < 0 || (size_t)logical_block >= s.table.size()) return PKV_ERR_INVALID_ARG;
+    int32_t old = s.table[logical_block];
+    if (bm->ref[old] <= 1) return PKV_OK;
+    int32_t fresh;
+    if (!bm->take(&fresh)) return PKV_ERR_OUT_OF_BLOCKS;
+    bm->ref[old] -= 1;
+    s.table[logical_block] = fresh;
+    *src = old;
+    *dst = fresh;
+    return PKV_OK;
+}
+
+pkv_status pkv_bm_fork(pkv_block_manager* bm, int64_t parent, int64_t child) {
+    if (!bm) return PKV_ERR_INVALID_ARG;
+    auto it = bm->seqs.find(parent);
+    if (it == bm->seqs.end() || bm->seqs.count(child)) return PKV_ERR_INVALID_ARG;
+    Seq c = it->second;
+    for (int32_t b : c.table) bm->ref[b] += 1;
+    bm->seqs.emplace(child, std::move(c));
+    return PKV_OK;
+}
+
+pkv_status pkv_bm_free(pkv_block_manager* bm, int64_t seq_id) {
+    if (!bm) return PKV_ERR_INVALID_ARG;
+    auto it = bm->seqs.find(seq_id);
+    if (it == bm->seqs.end()) return PKV_ERR_INVALID_ARG;
+    for (int32_t b : it->second.table) bm->release(b);
+    bm->seqs.erase(it);
+    return PKV_OK;
+}
+
+pkv_status pkv_bm_block_tables(const pkv_block_manager* bm, const int64_t* seq_ids, int n,
+                               int max_blocks, int32_t* tables_out, int32_t* context_lens_out) {
+    if (!bm || n < 0 || max_blocks <= 0 || (n > 0 && (!seq_ids || !tables_out)))
+        return PKV_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) {
+        auto it = bm->seqs.find(seq_ids[i]);
+        if (it == bm->seqs.end()) return PKV_ERR_INVALID_ARG;
+        const Seq& s = it->second;
+        if (s.table.size() > (size_t)max_blocks || s.len > INT32_MAX) return PKV_ERR_INVALID_ARG;
+        int32_t* row = tables_out + (size_t)i * max_blocks;
+        std::memcpy(row, s.table.data(), s.table.size() * sizeof(int32_t));
+        std::memset(row + s.table.size(), 0, (max_blocks - s.table.size()) * sizeof(int32_t));
+        if (context_lens_out) context_lens_out[i] = (int32_t)s.len;
+    }
+    return PKV_OK;
+}
+
+int pkv_bm_num_free(const pkv_block_manager* bm) { return bm ? (int)bm->count : -1; }
+
+int pkv_bm_ref_count(const pkv_block_manager* bm, int block) {
+    if (!bm || block < 0 || block >= bm->num_blocks) return -1;
+    return bm->ref[block];
+}
+
+int pkv_bm_seq_len(const pkv_block_manager* bm, int64_t seq_id) {
+    if (!bm) return -1;
+    auto it = bm->seqs.find(seq_id);
+    return it == bm->seqs.end() ? -1 : (int)it->second.len;
+}
+
+}  // extern "C"

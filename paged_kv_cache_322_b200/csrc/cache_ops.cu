@@ -1,0 +1,139 @@
+// Cache-side kernels: KV append (reshape_and_cache) and block copy (copy_blocks).
+//
+// Layout ("LLM 推理引擎内部原理" §2.4): cache[num_blocks, block_size, Hkv, D].
+// One token's K (or V) for all heads is one contiguous row of Hkv*D elements
+// at (slot / block_size, slot % block_size), so the append is a row copy, and a
+// physical block is one contiguous span of block_size*Hkv*D elements, so the
+// block copy is a span copy. Both move 16-byte vectors, several in flight per
+// thread, with non-allocating loads of the read-once source.
+#include "common.cuh"
+
+namespace pkv {
+namespace {
+
+__device__ __forceinline__ int4 ld_stream(const int4* p) {
+    int4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.s32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+// grid.x = token, grid.y = 0 (K) / 1 (V). Each CTA copies one row of
+// row_vecs 16-byte vectors.
+__global__ void __launch_bounds__(256) reshape_and_cache_kernel(
+    const int4* __restrict__ k, const int4* __restrict__ v, int4* __restrict__ k_cache,
+    int4* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, int row_vecs,
+    int64_t num_slots, int* err) {
+    const int t = blockIdx.x;
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) return;
+    if (slot >= num_slots) {
+        if (threadIdx.x == 0) flag_error(err, PKV_ERR_DEVICE_BOUNDS);
+        return;
+    }
+    const int4* src = (blockIdx.y == 0 ? k : v) + (int64_t)t * row_vecs;
+    int4* dst = (blockIdx.y == 0 ? k_cache : v_cache) + slot * row_vecs;
+    int i = threadIdx.x;
+    for (; i + 3 * 256 < row_vecs; i += 4 * 256) {
+        int4 a = ld_stream(src + i), b = ld_stream(src + i + 256);
+        int4 c = ld_stream(src + i + 512), d = ld_stream(src + i + 768);
+        dst[i] = a;
+        dst[i + 256] = b;
+        dst[i + 512] = c;
+        dst[i + 768] = d;
+    }
+    for (; i < row_vecs; i += 256) dst[i] = ld_stream(src + i);
+}
+
+// grid.x = chunk of the block span (kChunkVecs vectors), grid.y = pair,
+// grid.z = 0 (K) / 1 (V).
+constexpr int kCopyThreads = 256;
+constexpr int kCopyUnroll = 4;
+constexpr int kChunkVecs = kCopyThreads * kCopyUnroll;
+
+__global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
+    int4* __restrict__ k_cache, int4* __restrict__ v_cache, const int64_t* __restrict__ src_ids,
+    const int64_t* __restrict__ dst_ids, int64_t block_vecs, int64_t num_blocks, int* err) {
+    const int64_t s = src_ids[blockIdx.y], d = dst_ids[blockIdx.y];
+    if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks) {
+        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0) flag_error(err, PKV_ERR_DEVICE_BOUNDS);
+        return;
+    }
+    int4* cache = blockIdx.z == 0 ? k_cache : v_cache;
+    const int4* src = cache + s * block_vecs;
+    int4* dst = cache + d * block_vecs;
+    const int64_t base = (int64_t)blockIdx.x * kChunkVecs + threadIdx.x;
+    int4 r[kCopyUnroll];
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+        const int64_t i = base + u * kCopyThreads;
+        if (i < block_vecs) r[u] = ld_stream(src + i);
+    }
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+        const int64_t i = base + u * kCopyThreads;
+        if (i < block_vecs) dst[i] = r[u];
+    }
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elt_bytes(pkv_dtype t) { return t == PKV_F32 ? 4 : (t == PKV_BF16 ? 2 : 0); }
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" {
+
+pkv_status pkv_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,
+                                 pkv_dtype dtype, const int64_t* slot_mapping, int num_tokens,
+                                 int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                 void* stream) {
+    using namespace pkv;
+    const int eb = elt_bytes(dtype);
+    if (eb == 0 || num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        num_blocks <= 0)
+        return PKV_ERR_INVALID_ARG;
+    const int64_t row_bytes = (int64_t)num_kv_heads * head_dim * eb;
+    if (row_bytes % 16 != 0 || row_bytes / 16 > INT32_MAX) return PKV_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PKV_OK;
+    if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+        return PKV_ERR_INVALID_ARG;
+    int* err = device_error_word();
+    if (!err) return PKV_ERR_CUDA;
+    dim3 grid(num_tokens, 2);
+    reshape_and_cache_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const int4*>(k), static_cast<const int4*>(v), static_cast<int4*>(k_cache),
+        static_cast<int4*>(v_cache), slot_mapping, (int)(row_bytes / 16),
+        (int64_t)num_blocks * block_size, err);
+    return cuda_status(cudaGetLastError());
+}
+
+pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, pkv_dtype dtype,
+                           const int64_t* src_block_ids, const int64_t* dst_block_ids, int num_pairs,
+                           int block_size, int num_kv_heads, int head_dim, int num_blocks,
+                           void* stream) {
+    using namespace pkv;
+    const int eb = elt_bytes(dtype);
+    if (eb == 0 || num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        num_blocks <= 0 || num_pairs > 65535)
+        return PKV_ERR_INVALID_ARG;
+    const int64_t block_bytes = (int64_t)block_size * num_kv_heads * head_dim * eb;
+    if (block_bytes % 16 != 0) return PKV_ERR_UNSUPPORTED;
+    if (num_pairs == 0) return PKV_OK;
+    if (!k_cache || !v_cache || !src_block_ids || !dst_block_ids) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(k_cache) || !aligned16(v_cache)) return PKV_ERR_INVALID_ARG;
+    int* err = device_error_word();
+    if (!err) return PKV_ERR_CUDA;
+    const int64_t block_vecs = block_bytes / 16;
+    const int64_t chunks = (block_vecs + kChunkVecs - 1) / kChunkVecs;
+    if (chunks > INT32_MAX) return PKV_ERR_UNSUPPORTED;
+    dim3 grid((unsigned)chunks, num_pairs, 2);
+    copy_blocks_kernel<<<grid, kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<int4*>(k_cache), static_cast<int4*>(v_cache), src_block_ids, dst_block_ids,
+        block_vecs, num_blocks, err);
+    return cuda_status(cudaGetLastError());
+}
+
+}  // extern "C"

@@ -1,0 +1,113 @@
+"""One layer's paged KV cache on the device plus the host block manager, and
+the decode step that runs the whole path in order:
+
+    block manager append (slot mapping, copy-on-write pairs)      [host, C++]
+    -> copy_blocks for the copy-on-write pairs                      [CUDA]
+    -> reshape_and_cache of the new tokens' K/V into their slots    [CUDA]
+    -> paged decode attention over the updated cache                [CUDA]
+
+("vLLM PagedAttention 深度解析" §3.3 decode step: write the new token's KV into
+its logical block through the block table, allocate a new block when the last
+one is full; §4.1: copy a shared block before writing into it.)
+
+Host metadata (slot mapping, copy lists, block tables, lengths) goes to the
+device through pinned staging buffers on the caller's stream. This module only
+sequences calls of the C ABI; it computes nothing itself.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import binding
+
+
+class PagedKVCache:
+    def __init__(self, num_blocks: int, block_size: int, num_kv_heads: int, head_dim: int,
+                 dtype: torch.dtype, device, free_order=None, max_blocks_per_seq: int = 0,
+                 fill_value: float | None = None):
+        self.num_blocks, self.block_size = num_blocks, block_size
+        self.num_kv_heads, self.head_dim, self.dtype = num_kv_heads, head_dim, dtype
+        self.device = torch.device(device)
+        shape = (num_blocks, block_size, num_kv_heads, head_dim)
+        if fill_value is None:
+            self.k_cache = torch.empty(shape, dtype=dtype, device=self.device)
+            self.v_cache = torch.empty(shape, dtype=dtype, device=self.device)
+        else:
+            self.k_cache = torch.full(shape, fill_value, dtype=dtype, device=self.device)
+            self.v_cache = torch.full(shape, fill_value, dtype=dtype, device=self.device)
+        self.bm = binding.BlockManager(num_blocks, block_size, free_order)
+        self.max_blocks_per_seq = max_blocks_per_seq or num_blocks
+        self._pinned = {}
+
+    # -- staging ---------------------------------------------------------
+    def _to_device(self, name: str, arr: np.ndarray, stream=None) -> torch.Tensor:
+        """Copies a host array to the device through a reusable pinned buffer."""
+        t = torch.from_numpy(np.ascontiguousarray(arr))
+        buf = self._pinned.get(name)
+        if buf is None or buf.numel() < t.numel() or buf.dtype != t.dtype:
+            buf = torch.empty(max(t.numel(), 1), dtype=t.dtype, pin_memory=True)
+            self._pinned[name] = buf
+        # the previous async copy out of this buffer must be done before reuse
+        ev = self._pinned.get(name + "/ev")
+        if ev is not None:
+            ev.synchronize()
+        view = buf[:t.numel()].view(t.shape)
+        view.copy_(t)
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        with torch.cuda.stream(s):
+            dev = view.to(self.device, non_blocking=True)
+            e = torch.cuda.Event()
+            e.record(s)
+        self._pinned[name + "/ev"] = e
+        return dev
+
+    # -- sequences ---------------------------------------------------------
+    def add_sequence(self, seq_id: int, k: torch.Tensor, v: torch.Tensor, stream=None):
+        """New sequence with prompt K/V [n, Hkv, D] (device tensors): allocates
+        its blocks and writes the prompt into them."""
+        slots = self.bm.allocate(seq_id, k.shape[0])
+        if k.shape[0]:
+            binding.reshape_and_cache(k, v, self.k_cache, self.v_cache, self._to_device("slots", slots, stream),
+                                      stream=stream)
+        return slots
+
+    def fork(self, parent: int, child: int):
+        self.bm.fork(parent, child)
+
+    def make_writable(self, seq_ids, logical_block: int, stream=None):
+        """Copy-on-write of one logical block for each listed sequence; runs the
+        copies. Returns the (src, dst) pairs."""
+        pairs = [p for p in (self.bm.make_writable(s, logical_block) for s in seq_ids) if p is not None]
+        if pairs:
+            arr = np.asarray(pairs, dtype=np.int64)
+            binding.copy_blocks(self.k_cache, self.v_cache, self._to_device("cow_src", arr[:, 0], stream),
+                                self._to_device("cow_dst", arr[:, 1], stream), stream=stream)
+        return pairs
+
+    def free(self, seq_id: int):
+        self.bm.free(seq_id)
+
+    def block_tables(self, seq_ids):
+        return self.bm.block_tables(seq_ids, self.max_blocks_per_seq)
+
+    # -- the decode step -----------------------------------------------------
+    def decode_step(self, seq_ids, q, k_new, v_new, scale: float, out=None, out_dtype=torch.float32,
+                    partition_tokens: int = 0, stream=None):
+        """Appends one token per sequence (k_new, v_new [B, Hkv, D]) and returns
+        attention of q [B, Hq, D] over each sequence's updated context."""
+        seq_ids = np.asarray(seq_ids, dtype=np.int64)
+        slots, src, dst = self.bm.append_slots(seq_ids)
+        if src.size:
+            binding.copy_blocks(self.k_cache, self.v_cache, self._to_device("src", src, stream),
+                                self._to_device("dst", dst, stream), stream=stream)
+        binding.reshape_and_cache(k_new, v_new, self.k_cache, self.v_cache, self._to_device("slots", slots, stream),
+                                  stream=stream)
+        tables, lens = self.block_tables(seq_ids)
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=self.device)
+        binding.paged_attention_decode(out, q, self.k_cache, self.v_cache, self._to_device("tables", tables, stream),
+                                       self._to_device("lens", lens, stream), scale,
+                                       max_context_len=int(lens.max()) if lens.size else 0,
+                                       partition_tokens=partition_tokens, stream=stream)
+        return out

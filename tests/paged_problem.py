@@ -1,0 +1,174 @@
+"""Test harness: builds the same decode problem twice from the seeded inputs,
+once with the oracle (CPU, fp64) and once through the library (GPU), each side
+with its own block manager. Nothing here computes attention or addresses."""
+from __future__ import annotations
+
+import numpy as np
+
+from oracle import cache_ops as ocache
+from oracle import paged_attention as oattn
+from oracle.block_manager import BlockManager as OracleBM
+from paged_kv_cache_322_b200 import workloads as wl
+
+
+class SparsePool:
+    """A cache [num_blocks, bs, Hkv, D] that stores only written blocks; unwritten
+    blocks read as NaN (like the sentinel-filled device pool)."""
+
+    def __init__(self, num_blocks, bs, hkv, d):
+        self.shape = (num_blocks, bs, hkv, d)
+        self.blocks = {}
+
+    def _blk(self, b):
+        b = int(b)
+        if b not in self.blocks:
+            self.blocks[b] = np.full(self.shape[1:], np.nan, dtype=np.float32)
+        return self.blocks[b]
+
+    def __getitem__(self, key):
+        if isinstance(key, tuple):
+            return self._blk(key[0])[key[1]]
+        if isinstance(key, (int, np.integer)):
+            return self._blk(key)
+        return np.stack([self._blk(b) for b in np.asarray(key).tolist()]) if len(key) else \
+            np.zeros((0,) + self.shape[1:], np.float32)
+
+    def __setitem__(self, key, val):
+        if isinstance(key, tuple):
+            self._blk(key[0])[key[1]] = val
+        else:
+            self._blk(key)[...] = val
+
+
+class OracleProblem:
+    """Oracle side of a workload: block tables from the oracle block manager,
+    cache contents for the listed sequences only (`keep`, default all)."""
+
+    def __init__(self, w: wl.Workload, keep=None, dense=False):
+        self.w = w
+        self.lens = wl.context_lens(w)
+        self.bm = OracleBM(w.num_blocks, w.block_size, wl.free_order(w))
+        shape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
+        if dense:
+            self.kc = np.full(shape, np.nan, np.float32)
+            self.vc = np.full(shape, np.nan, np.float32)
+        else:
+            self.kc = SparsePool(*shape)
+            self.vc = SparsePool(*shape)
+        self.keep = set(range(w.num_seqs)) if keep is None else set(int(s) for s in keep)
+        if w.ctx == "shared_prefix":
+            self._build_shared()
+        else:
+            for s in range(w.num_seqs):
+                slots = self.bm.allocate(s, int(self.lens[s]))
+                if s in self.keep:
+                    k, v = wl.prompt_kv(w, s, int(self.lens[s]))
+                    ocache.reshape_and_cache(k, v, self.kc, self.vc, np.asarray(slots))
+        self.cow_pairs = []
+
+    def _build_shared(self):
+        w = self.w
+        p = w.shared_prefix
+        slots = self.bm.allocate(-1, p)
+        k0, v0 = wl.prompt_kv(w, 0, int(self.lens[0]))
+        ocache.reshape_and_cache(k0[:p], v0[:p], self.kc, self.vc, np.asarray(slots))
+        for s in range(w.num_seqs):
+            self.bm.fork(-1, s)
+        self.bm.free_seq(-1)
+        for s in range(w.num_seqs):
+            n = int(self.lens[s])
+            tail = [self.bm.append_slot(s)[0] for _ in range(n - p)]
+            if s in self.keep:
+                k, v = wl.prompt_kv(w, s, n)
+                ocache.reshape_and_cache(k[p:], v[p:], self.kc, self.vc, np.asarray(tail))
+
+    def fork_last_shared_block(self):
+        """Copy-on-write of the last shared prefix block for every sequence
+        (all but the last one copy; the last keeps the original)."""
+        last = self.w.shared_prefix // self.w.block_size - 1
+        pairs = [self.bm.make_writable(s, last) for s in range(self.w.num_seqs)]
+        pairs = [x for x in pairs if x is not None]
+        if pairs:
+            ocache.copy_blocks(self.kc, self.vc, [a for a, _ in pairs], [b for _, b in pairs])
+        self.cow_pairs = pairs
+        return pairs
+
+    def decode_step(self, step: int, seqs=None):
+        """Appends step `step`'s token to every sequence; returns the fp64
+        attention output of the listed sequences (default: kept ones)."""
+        w = self.w
+        q = wl.decode_q(w, step)
+        kn, vn = wl.decode_kv(w, step)
+        slots = []
+        for s in range(w.num_seqs):
+            slot, copy = self.bm.append_slot(s)
+            assert copy is None
+            slots.append(slot if s in self.keep else -1)
+        ocache.reshape_and_cache(kn, vn, self.kc, self.vc, np.asarray(slots))
+        return self.attend(q, seqs)
+
+    def attend(self, q, seqs=None):
+        seqs = sorted(self.keep) if seqs is None else list(seqs)
+        tables = {s: self.bm.block_table(s) for s in seqs}
+        lens = {s: self.bm.lens[s] for s in seqs}
+        out = oattn.paged_attention_decode(q, self.kc, self.vc, _TableView(tables), _TableView(lens),
+                                           self.w.scale, self.w.block_size, seqs=seqs)
+        return out
+
+
+class _TableView:
+    def __init__(self, d):
+        self.d = d
+
+    def __getitem__(self, s):
+        return self.d[int(s)]
+
+
+def gpu_problem(w: wl.Workload, device="cuda", fill_nan=True, max_new_tokens=4):
+    """Library side: a PagedKVCache with the workload's prompts written by
+    reshape_and_cache through the library's block manager."""
+    import torch
+    from paged_kv_cache_322_b200.engine import PagedKVCache
+    lens = wl.context_lens(w)
+    dt = torch.float32 if w.kv_dtype == "f32" else torch.bfloat16
+    mb = -(-int(lens.max() + max_new_tokens) // w.block_size)
+    cache = PagedKVCache(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, dt, device,
+                         free_order=wl.free_order(w), max_blocks_per_seq=mb,
+                         fill_value=float("nan") if fill_nan else None)
+    def dev(x):
+        return torch.from_numpy(x).to(device=device, dtype=dt)
+    if w.ctx == "shared_prefix":
+        p = w.shared_prefix
+        k0, v0 = wl.prompt_kv(w, 0, int(lens[0]))
+        cache.add_sequence(-1, dev(k0[:p]), dev(v0[:p]))
+        for s in range(w.num_seqs):
+            cache.fork(-1, s)
+        cache.free(-1)
+        for s in range(w.num_seqs):
+            n = int(lens[s])
+            k, v = wl.prompt_kv(w, s, n)
+            kt, vt = dev(k[p:]), dev(v[p:])
+            slots = np.concatenate([cache.bm.append_slots([s])[0] for _ in range(n - p)])
+            from paged_kv_cache_322_b200 import binding
+            binding.reshape_and_cache(kt, vt, cache.k_cache, cache.v_cache,
+                                      torch.from_numpy(slots).to(device))
+    else:
+        kvs = wl.prompt_kv_all(w, lens)
+        for s in range(w.num_seqs):
+            k, v = kvs[s]
+            cache.add_sequence(s, dev(k), dev(v))
+    return cache, lens
+
+
+def step_inputs(w: wl.Workload, step: int, device="cuda"):
+    import torch
+    dt = torch.float32 if w.kv_dtype == "f32" else torch.bfloat16
+    q = torch.from_numpy(wl.decode_q(w, step)).to(device=device, dtype=dt)
+    kn, vn = wl.decode_kv(w, step)
+    return q, torch.from_numpy(kn).to(device=device, dtype=dt), torch.from_numpy(vn).to(device=device, dtype=dt)
+
+
+def tolerance(w: wl.Workload) -> float:
+    """Max abs error allowed against the fp64 oracle: 1e-5 for fp32 inputs,
+    2e-3 for bf16-rounded inputs (fp32 accumulation, fp32 output)."""
+    return 1e-5 if w.kv_dtype == "f32" else 2e-3

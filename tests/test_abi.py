@@ -1,0 +1,273 @@
+"""The C-ABI library on the CPU: it loads, exports every declared symbol, its
+host block manager matches the oracle's bit for bit, and host-side argument
+checks reject bad calls before anything reaches a GPU."""
+import ctypes
+import os
+import random
+import re
+
+import numpy as np
+import pytest
+
+from oracle.block_manager import BlockManager as OracleBM
+from paged_kv_cache_322_b200 import binding, workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(binding.LIB_PATH):
+        from paged_kv_cache_322_b200 import build
+        build.build()
+    return binding.library()
+
+
+def _declared():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(pkv_\w+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert len(names) >= 17
+    for n in sorted(names):
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert lib.pkv_status_string(code)
+    assert lib.pkv_status_string(99) == b"unknown status"
+
+
+def test_walkthrough_and_cow_match_the_pages(lib, golden_dir):
+    import json
+    g = json.load(open(os.path.join(golden_dir, "block_table_walkthrough.json")))
+    bm = binding.BlockManager(g["num_blocks"], g["block_size"], g["free_order"])
+    assert bm.allocate(7, g["prompt_tokens"]).tolist() == g["after_prefill"]["slots"]
+    t, n = bm.block_tables([7], 4)
+    assert t[0, :2].tolist() == g["after_prefill"]["table"] and n[0] == 7
+    for step in g["decode"]:
+        slots, src, dst = bm.append_slots([7])
+        assert slots.tolist() == [step["slot"]] and src.size == 0
+        t, _ = bm.block_tables([7], 4)
+        assert t[0, :len(step["table"])].tolist() == step["table"]
+        assert bm.num_free() == step["num_free"]
+    c = json.load(open(os.path.join(golden_dir, "cow_fork.json")))
+    bm = binding.BlockManager(c["num_blocks"], c["block_size"], c["free_order"])
+    bm.allocate(1, c["prompt_tokens"])
+    bm.fork(1, 2)
+    slots, src, dst = bm.append_slots([1, 2])
+    assert slots.tolist() == [c["A1_append"]["slot"], c["A2_append"]["slot"]]
+    assert list(zip(src.tolist(), dst.tolist())) == [tuple(c["A1_append"]["copy"])]
+    for b, r in c["ref_after"].items():
+        assert bm.ref_count(int(b)) == r
+
+
+def _run_both(ops, nb, bs, order):
+    """Runs one op list on the oracle and on the library's block manager."""
+    o = OracleBM(nb, bs, order)
+    p = binding.BlockManager(nb, bs, order)
+    for op in ops:
+        kind = op[0]
+        if kind == "alloc":
+            r_o = o.allocate(op[1], op[2])
+            try:
+                r_p = p.allocate(op[1], op[2]).tolist()
+            except binding.PkvError as e:
+                assert e.status == 5
+                r_p = None
+            assert r_o == r_p
+        elif kind == "fork":
+            o.fork(op[1], op[2])
+            p.fork(op[1], op[2])
+        elif kind == "append":
+            exp_slots, exp_pairs = [], []
+            oom = False
+            for s in op[1]:
+                r = o.append_slot(s)
+                if r is None:
+                    oom = True
+                    break
+                exp_slots.append(r[0])
+                if r[1] is not None:
+                    exp_pairs.append(r[1])
+            if oom:
+                with pytest.raises(binding.PkvError):
+                    p.append_slots(op[1])
+                return o, p, False
+            slots, src, dst = p.append_slots(op[1])
+            assert slots.tolist() == exp_slots
+            assert list(zip(src.tolist(), dst.tolist())) == exp_pairs
+        elif kind == "cow":
+            r_o = o.make_writable(op[1], op[2])
+            assert p.make_writable(op[1], op[2]) == r_o
+        elif kind == "free":
+            o.free_seq(op[1])
+            p.free(op[1])
+        assert o.num_free() == p.num_free()
+    return o, p, True
+
+
+@pytest.mark.parametrize("seed", range(25))
+def test_random_ops_bit_exact_vs_oracle(lib, seed):
+    rng = random.Random(seed)
+    bs = rng.choice([1, 4, 16])
+    nb = 96
+    order = rng.sample(range(nb), nb)
+    ops, live, nxt = [], [], 0
+    for _ in range(150):
+        x = rng.random()
+        if x < 0.2 or not live:
+            ops.append(("alloc", nxt, rng.randint(0, 3 * bs)))
+            live.append(nxt)
+            nxt += 1
+        elif x < 0.3:
+            ops.append(("fork", rng.choice(live), nxt))
+            live.append(nxt)
+            nxt += 1
+        elif x < 0.8:
+            ops.append(("append", rng.sample(live, rng.randint(1, len(live)))))
+        elif x < 0.9:
+            ops.append(("free", live.pop(rng.randrange(len(live)))))
+        else:
+            ops.append(("cow", rng.choice(live), 0))
+    # an allocation can fail (then the id does not exist): replay with the oracle first
+    o = OracleBM(nb, bs, order)
+    valid, alive = [], set()
+    for op in ops:
+        if op[0] == "alloc":
+            if o.allocate(op[1], op[2]) is not None:
+                alive.add(op[1])
+            valid.append(op)
+        elif op[0] == "fork":
+            if op[1] in alive:
+                o.fork(op[1], op[2])
+                alive.add(op[2])
+                valid.append(op)
+        elif op[0] == "append":
+            ids = [s for s in op[1] if s in alive]
+            if ids:
+                if any(o.append_slot(s) is None for s in ids):
+                    valid.append(("append", ids))
+                    break
+                valid.append(("append", ids))
+        elif op[0] == "free":
+            if op[1] in alive:
+                o.free_seq(op[1])
+                alive.discard(op[1])
+                valid.append(op)
+        else:
+            if op[1] in alive and o.tables[op[1]]:
+                try:
+                    o.make_writable(op[1], 0)
+                except Exception:
+                    break
+                valid.append(op)
+    _run_both(valid, nb, bs, order)
+
+
+@pytest.mark.parametrize("name", list(wl.WORKLOADS))
+def test_workload_prefill_and_steps_bit_exact(lib, name):
+    w = wl.WORKLOADS[name]
+    lens = wl.context_lens(w)
+    order = wl.free_order(w)
+    o = OracleBM(w.num_blocks, w.block_size, order)
+    p = binding.BlockManager(w.num_blocks, w.block_size, order)
+    if w.ctx == "shared_prefix":
+        assert o.allocate(-1, w.shared_prefix) == p.allocate(-1, w.shared_prefix).tolist()
+        for s in range(w.num_seqs):
+            o.fork(-1, s)
+            p.fork(-1, s)
+        o.free_seq(-1)
+        p.free(-1)
+        for s in range(w.num_seqs):
+            exp = [o.append_slot(s)[0] for _ in range(int(lens[s]) - w.shared_prefix)]
+            got = []
+            for _ in range(int(lens[s]) - w.shared_prefix):
+                got.append(int(p.append_slots([s])[0][0]))
+            assert exp == got
+        last = w.shared_prefix // w.block_size - 1
+        pairs_o = [o.make_writable(s, last) for s in range(w.num_seqs)]
+        pairs_p = [p.make_writable(s, last) for s in range(w.num_seqs)]
+        assert pairs_o == pairs_p and sum(x is not None for x in pairs_p) == w.num_seqs - 1
+    else:
+        for s in range(w.num_seqs):
+            assert o.allocate(s, int(lens[s])) == p.allocate(s, int(lens[s])).tolist()
+    ids = list(range(w.num_seqs))
+    mb = -(-int(lens.max() + 3) // w.block_size)
+    for _ in range(3):
+        exp = [o.append_slot(s)[0] for s in ids]
+        slots, src, dst = p.append_slots(ids)
+        assert slots.tolist() == exp and src.size == 0
+        tables, plens = p.block_tables(ids, mb)
+        for s in ids:
+            t = o.block_table(s)
+            assert tables[s, :len(t)].tolist() == t and plens[s] == o.lens[s]
+
+
+def test_block_manager_errors(lib):
+    with pytest.raises(binding.PkvError):
+        binding.BlockManager(4, 2, [0, 1, 1, 3])           # not a permutation
+    bm = binding.BlockManager(2, 4)
+    bm.allocate(0, 8)
+    with pytest.raises(binding.PkvError) as e:
+        bm.append_slots([0])
+    assert e.value.status == 5
+    with pytest.raises(binding.PkvError) as e:
+        bm.allocate(0, 1)                                   # id exists
+    assert e.value.status == 1
+    with pytest.raises(binding.PkvError):
+        bm.block_tables([0], 1)                             # table longer than the row
+    with pytest.raises(binding.PkvError):
+        bm.fork(5, 6)
+
+
+def test_kernel_entry_points_reject_bad_arguments_on_host(lib):
+    fake = ctypes.c_void_p(1 << 20)
+    # head_dim 96 is not built; group 3 is not built; block size 8 not built
+    assert lib.pkv_paged_attention_decode(fake, 0, fake, fake, fake, 1, fake, fake, 1.0, 2, 8, 8, 96, 16, 4, 64,
+                                          0, 0, None, 0, None) == 2
+    assert lib.pkv_paged_attention_decode(fake, 0, fake, fake, fake, 1, fake, fake, 1.0, 2, 12, 4, 128, 16, 4, 64,
+                                          0, 0, None, 0, None) == 2
+    assert lib.pkv_paged_attention_decode(fake, 0, fake, fake, fake, 1, fake, fake, 1.0, 2, 8, 8, 128, 8, 4, 64,
+                                          0, 0, None, 0, None) == 2
+    # Hq not a multiple of Hkv, negative sizes, bad dtype, NaN scale, misalignment
+    assert lib.pkv_paged_attention_decode(fake, 0, fake, fake, fake, 1, fake, fake, 1.0, 2, 6, 4, 128, 16, 4, 64,
+                                          0, 0, None, 0, None) == 1
+    assert lib.pkv_paged_attention_decode(fake, 0, fake, fake, fake, 1, fake, fake, 1.0, -1, 8, 8, 128, 16, 4, 64,
+                                          0, 0, None, 0, None) == 1
+    assert lib.pkv_paged_attention_decode(fake, 7, fake, fake, fake, 1, fake, fake, 1.0, 2, 8, 8, 128, 16, 4, 64,
+                                          0, 0, None, 0, None) == 1
+    assert lib.pkv_paged_attention_decode(fake, 0, fake, fake, fake, 1, fake, fake, float("nan"), 2, 8, 8, 128, 16,
+                                          4, 64, 0, 0, None, 0, None) == 1
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    assert lib.pkv_paged_attention_decode(odd, 0, fake, fake, fake, 1, fake, fake, 1.0, 2, 8, 8, 128, 16, 4, 64,
+                                          0, 0, None, 0, None) == 1
+    # split-K needs a workspace: none given
+    assert lib.pkv_paged_attention_decode(fake, 0, fake, fake, fake, 1, fake, fake, 1.0, 2, 8, 8, 128, 16, 128, 64,
+                                          0, 512, None, 0, None) == 1
+    # zero sequences / tokens / pairs: nothing to launch
+    assert lib.pkv_paged_attention_decode(None, 0, None, None, None, 1, None, None, 1.0, 0, 8, 8, 128, 16, 4, 64,
+                                          0, 0, None, 0, None) == 0
+    assert lib.pkv_reshape_and_cache(None, None, None, None, 1, None, 0, 8, 128, 16, 64, None) == 0
+    assert lib.pkv_copy_blocks(None, None, 1, None, None, 0, 16, 8, 128, 64, None) == 0
+    assert lib.pkv_reshape_and_cache(fake, fake, fake, fake, 5, fake, 4, 8, 128, 16, 64, None) == 1
+    assert lib.pkv_reshape_and_cache(fake, fake, fake, fake, 1, fake, 4, 1, 4, 16, 64, None) == 2  # 8-byte rows
+    assert lib.pkv_copy_blocks(fake, fake, 1, fake, fake, -1, 16, 8, 128, 64, None) == 1
+
+
+def test_workspace_and_partition_rule(lib):
+    # 512-token partitions over a 32768-token cap: 64 partitions of (D + 2) floats per row
+    n = binding.workspace_bytes(16, 32, 8, 128, 16, 2048, 32768, 512)
+    rows = 16 * 32 * 64
+    assert n >= rows * 128 * 4 + rows * 2 * 4
+    assert binding.workspace_bytes(4, 8, 8, 64, 16, 16, 256, 512) == 0      # one partition
+    assert binding.partition_tokens(16, 32, 8, 128, 16, 2048, 32768, 500) == 512
+    assert binding.partition_tokens(64, 32, 32, 128, 16, 128, 2048, 0) in (256, 512)
