@@ -48,14 +48,16 @@ L2_BYTES = 126 * 2 ** 20
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="pkv", choices=["pkv", "reference"])
     ap.add_argument("--workload", default="llama2_7b", choices=list(wl.WORKLOADS))
     ap.add_argument("--partition-tokens", type=int, default=-1, help="-1: the workload's, 0: library default")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--num-seqs", type=int, default=0, help="override the batch size (profiling a small case)")
+    ap.add_argument("--num-blocks", type=int, default=0, help="override the pool size (profiling a small case)")
     return ap.parse_args()
 
 
@@ -108,27 +110,56 @@ def all_sum(x: float, ws: int) -> float:
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    """Samples SM clock, max clock and throttle reasons through NVML every few
+    milliseconds while the timed region runs (nvidia-smi as a fallback)."""
 
-    def __init__(self, index: int):
-        self.index, self.samples, self._stop = index, [], threading.Event()
+    def __init__(self, index: int, interval_s: float = 0.005):
+        self.index, self.interval, self.samples, self._stop = index, interval_s, [], threading.Event()
         self._t = threading.Thread(target=self._run, daemon=True)
+        self.source = "nvml"
 
     def _run(self):
-        while not self._stop.is_set():
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+            while True:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+                r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((sm, mx, sorted(k for k, b in bits.items() if r & b)))
+                if self._stop.wait(self.interval):
+                    break
+            pynvml.nvmlShutdown()
+        except Exception:
+            self.source = "nvidia-smi"
+            self._run_smi()
+
+    def _run_smi(self):
+        fields = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_power_cap")
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        while True:
             try:
-                r = subprocess.run(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                r = subprocess.run(["nvidia-smi", f"--id={self.index}", f"--query-gpu={fields}",
                                     "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
-                if r.returncode == 0 and r.stdout.strip():
-                    self.samples.append([x.strip() for x in r.stdout.strip().split(",")])
+                v = [x.strip() for x in r.stdout.strip().split(",")]
+                if r.returncode == 0 and len(v) == 6:
+                    self.samples.append((float(v[0]), float(v[1]),
+                                         [names[i] for i in range(4) if v[2 + i].lower() == "active"]))
             except Exception:
                 pass
-            self._stop.wait(0.2)
+            if self._stop.wait(0.2):
+                break
 
     def __enter__(self):
         self._t.start()
+        time.sleep(0.02)                       # first sample lands before the timed region starts
         return self
 
     def __exit__(self, *a):
@@ -137,14 +168,11 @@ class ClockSampler:
 
     def summary(self):
         if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
-        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for s in self.samples for i in range(4)
-                          if len(s) > 3 + i and s[3 + i].strip().lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.samples)}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples),
+                "sm_max_mhz": max(s[1] for s in self.samples),
+                "reasons": sorted({r for s in self.samples for r in s[2]}),
+                "samples": len(self.samples), "source": self.source}
 
 
 def measured_peaks():
@@ -203,6 +231,10 @@ def run_pkv(args, ws, rank, local):
 
     dev = torch.device("cuda", local)
     w = wl.WORKLOADS[args.workload]
+    if args.num_seqs or args.num_blocks:
+        w = dataclasses.replace(w, num_seqs=args.num_seqs or w.num_seqs, num_blocks=args.num_blocks or w.num_blocks,
+                                description=w.description + f" [override: B={args.num_seqs or w.num_seqs}, "
+                                                            f"pool={args.num_blocks or w.num_blocks}]")
     if rank:
         w = dataclasses.replace(w, seed=w.seed + 7919 * rank)     # each replica its own batch
     part = w.partition_tokens if args.partition_tokens < 0 else args.partition_tokens
@@ -357,7 +389,8 @@ def run_pkv(args, ws, rank, local):
                      "achieved": round(achieved, 1), "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "avg_launch_ms": round(attn_avg_ms, 5),
                      "algorithmic_bytes_per_launch": int(attn_bytes_avg),
-                     "traffic": (tr["traffic_bytes_per_launch"] if tr else None)},
+                     "traffic": (int(tr["traffic_per_algorithmic_byte"] * attn_bytes_avg) if tr else None),
+                     "traffic_source": (tr["captured_on"] if tr else None)},
         "e2e": e2e,
         "gpu_launches": launches_per_step * K,
         "clocks": clocks.summary(),
@@ -369,32 +402,36 @@ def run_pkv(args, ws, rank, local):
 def cpu_baseline(w: wl.Workload, target_s: float):
     """The oracle, as it stands, on a bounded sample of the same workload: whole
     sequences (their logical K/V regenerated from the seeded generator, written
-    into an oracle pool, attention in fp64), until ~target_s seconds of CPU."""
+    into an oracle pool, attention in fp64), sequence after sequence and step
+    after step, until ~target_s seconds of CPU time."""
     from oracle import cache_ops as ocache
     from oracle import paged_attention as oattn
     from oracle.block_manager import BlockManager as OracleBM
     lens = wl.context_lens(w)
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
-    q = wl.decode_q(w, 0)
-    done, nbytes, t_total = 0, 0, 0.0
-    for s in range(w.num_seqs):
-        n = int(lens[s])
-        k, v = wl.prompt_kv(w, s, n)
-        nblk = -(-n // w.block_size)
-        bm = OracleBM(nblk, w.block_size)
-        kc = np.zeros((nblk, w.block_size, w.num_kv_heads, w.head_dim), np.float32)
-        vc = np.zeros_like(kc)
-        t0 = time.perf_counter()
-        ocache.reshape_and_cache(k, v, kc, vc, np.asarray(bm.allocate(0, n)))
-        oattn.paged_attention_decode(q[s:s + 1], kc, vc, [bm.block_table(0)], [n], w.scale, w.block_size)
-        t_total += time.perf_counter() - t0
-        done += 1
-        nbytes += n * w.num_kv_heads * w.head_dim * w.elt_bytes * 2 + 2 * w.num_q_heads * w.head_dim * w.elt_bytes
-        if t_total >= target_s:
-            break
+    done, nbytes, t_total, step = 0, 0, 0.0, 0
+    while t_total < target_s:
+        q = wl.decode_q(w, step)
+        for s in range(w.num_seqs):
+            n = int(lens[s])
+            k, v = wl.prompt_kv(w, s, n)
+            nblk = -(-n // w.block_size)
+            bm = OracleBM(nblk, w.block_size)
+            kc = np.zeros((nblk, w.block_size, w.num_kv_heads, w.head_dim), np.float32)
+            vc = np.zeros_like(kc)
+            t0 = time.perf_counter()
+            ocache.reshape_and_cache(k, v, kc, vc, np.asarray(bm.allocate(0, n)))
+            oattn.paged_attention_decode(q[s:s + 1], kc, vc, [bm.block_table(0)], [n], w.scale, w.block_size)
+            t_total += time.perf_counter() - t0
+            done += 1
+            nbytes += n * w.num_kv_heads * w.head_dim * w.elt_bytes * 2 + 2 * w.num_q_heads * w.head_dim * w.elt_bytes
+            if t_total >= target_s:
+                break
+        step += 1
     return {"value": round(nbytes / t_total / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{done} of {w.num_seqs} sequences of the bench workload (KV append + fp64 attention), "
-                      f"{t_total:.1f} s", "decode_tokens_per_s": round(done / t_total, 2)}
+            "sample": f"{done} sequence-steps of the bench workload ({w.num_seqs} sequences per step; KV append "
+                      f"into an oracle pool + fp64 attention), {t_total:.1f} s of CPU time",
+            "decode_tokens_per_s": round(done / t_total, 2)}
 
 
 def run_reference(args, ws, rank):
