@@ -127,6 +127,46 @@ int pkv_paged_attention_partition_tokens(
     int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
     int max_blocks_per_seq, int max_context_len, int partition_tokens);
 
+/* Size of the fixed scratch array behind pkv_paged_attention_decode_noalloc. */
+#define PKV_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/*
+ * pkv_paged_attention_decode for callers that cannot allocate device memory.
+ * (The pages have no counterpart to this call; it is a property of this
+ * library's interface, not of the method.)
+ *
+ * Who needs it: a caller whose device memory is already fully reserved by
+ * someone else (a serving engine that hands nearly all of the GPU to its KV
+ * pool and weights up front), or code that runs inside a plugin or enqueue
+ * hook where cudaMalloc / cudaFree are off limits because they can synchronise
+ * the whole device. Such a caller still owns and passes every input and
+ * output; only the split-K scratch moves into a fixed array of
+ * PKV_NOALLOC_SCRATCH_BYTES that the library keeps in each GPU's memory from
+ * the moment the GPU loads the library until the process exits. The call
+ * allocates nothing.
+ *
+ * Arguments and results are exactly those of pkv_paged_attention_decode,
+ * without workspace / workspace_bytes. The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress, with that device current);
+ * make that first call before any stream capture on that device.
+ *
+ * Limit: when pkv_paged_attention_workspace_bytes(...) for these sizes exceeds
+ * PKV_NOALLOC_SCRATCH_BYTES the call returns PKV_ERR_UNSUPPORTED and launches
+ * nothing (use larger partition_tokens, fewer sequences per call, or the
+ * regular entry point with your own workspace).
+ *
+ * Every call uses the same array and leaves its contents behind; nothing in it
+ * needs to start at zero. Calls whose kernels overlap on the GPU (two streams,
+ * two host threads) race on it: serialise them.
+ */
+pkv_status pkv_paged_attention_decode_noalloc(
+    void* out, pkv_dtype out_dtype,
+    const void* q, const void* k_cache, const void* v_cache, pkv_dtype kv_dtype,
+    const int32_t* block_tables, const int32_t* context_lens, float scale,
+    int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+    int block_size, int max_blocks_per_seq, int num_blocks,
+    int max_context_len, int partition_tokens, void* stream);
+
 /* ------------------------------------------------------------------------- */
 /* Cache-side kernels                                                        */
 /* ------------------------------------------------------------------------- */

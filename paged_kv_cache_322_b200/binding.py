@@ -38,6 +38,8 @@ _SIGS = {
     "pkv_status_string": (_c.c_char_p, [_i32]),
     "pkv_paged_attention_decode": (_i32, [_vp, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _f32, _i32, _i32, _i32, _i32,
                                           _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp]),
+    "pkv_paged_attention_decode_noalloc": (_i32, [_vp, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _f32, _i32, _i32, _i32,
+                                                  _i32, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pkv_paged_attention_workspace_bytes": (_sz, [_i32] * 8),
     "pkv_paged_attention_partition_tokens": (_i32, [_i32] * 8),
     "pkv_reshape_and_cache": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
@@ -160,6 +162,34 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
         _dtype_code(k_cache), block_tables.data_ptr(), context_lens.data_ptr(), float(scale), B, hq, hkv, d, bs,
         mb, nb, int(max_context_len), int(partition_tokens), ws_ptr, ws_n, _stream(q, stream))
     _check(st, "pkv_paged_attention_decode")
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def paged_attention_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                                   max_context_len: int = 0, partition_tokens: int = 0, stream=None):
+    """paged_attention_decode without a workspace: the split-K scratch is a fixed
+    array inside the library (NOALLOC_SCRATCH_BYTES per GPU), for callers that
+    must not allocate device memory. Raises PkvError(PKV_ERR_UNSUPPORTED) when
+    the sizes need more scratch than that. Concurrent calls on different
+    streams share the array and must be serialised."""
+    torch = _torch()
+    _cuda_contig(out, q, k_cache, v_cache, block_tables, context_lens)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    B, hq, d = q.shape
+    nb, bs, hkv, d2 = k_cache.shape
+    if d2 != d or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != (B, hq, d):
+        raise ValueError("shape mismatch")
+    if q.dtype != k_cache.dtype or v_cache.dtype != k_cache.dtype:
+        raise TypeError("q, k_cache and v_cache must share a dtype")
+    st = _lib().pkv_paged_attention_decode_noalloc(
+        out.data_ptr(), _dtype_code(out), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+        _dtype_code(k_cache), block_tables.data_ptr(), context_lens.data_ptr(), float(scale), B, hq, hkv, d, bs,
+        block_tables.shape[1], nb, int(max_context_len), int(partition_tokens), _stream(q, stream))
+    _check(st, "pkv_paged_attention_decode_noalloc")
     return out
 
 
