@@ -1,0 +1,340 @@
+// Pieces shared by the paged decode attention kernels: parameters, output
+// store, and the two consumer implementations (CUDA-core and tensor-core) that
+// fold one 16-token block of K/V into a running online-softmax state.
+#pragma once
+
+#include <cmath>
+
+#include "common.cuh"
+
+namespace pkv {
+namespace attn {
+
+constexpr int BS = 16;          // tokens per physical block (the only size built)
+constexpr int NCW = 4;          // consumer warps per CTA
+constexpr int NTHREADS = 32 * (NCW + 1);
+constexpr float kNegInf = -INFINITY;
+
+struct Params {
+    void* out;
+    const void* q;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    float* ws_o;        // [B, Hq, C, D] partition outputs (normalised)
+    float* ws_ml;       // [B, Hq, C, 2] partition (m, l), m in log2 units
+    int* err;
+    float scale_log2;   // scale * log2(e)
+    int out_f32;
+    int num_q_heads, num_kv_heads, group;
+    int max_blocks, num_blocks;
+    int ctx_cap;        // clamp for context_lens
+    int part_blocks;    // blocks per partition
+    int num_parts;      // grid.y
+    // persistent schedule
+    int num_seqs;
+    float* ws_part;                 // [2 * CTAs][group][D + 2]: per-piece (o / l, m, l)
+    unsigned long long* counters;   // [B * Hkv]: (epoch << 24) | pieces arrived
+    unsigned long long epoch;       // distinct per call
+    int team_size;                  // CTAs per team (one KV head each), divides Hkv and the grid
+};
+
+__device__ __forceinline__ void consumers_barrier() {
+    asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+}
+
+__device__ __forceinline__ void store_out(const Params& p, int64_t idx, float v) {
+    if (p.out_f32) static_cast<float*>(p.out)[idx] = v;
+    else static_cast<__nv_bfloat16*>(p.out)[idx] = __float2bfloat16_rn(v);
+}
+
+// ---------------------------------------------------------------------------
+// SIMT consumer: HPW query heads per warp, 8 lanes per token, 4 tokens per
+// round, fp32 math. T = float or __nv_bfloat16.
+// ---------------------------------------------------------------------------
+template <typename T, int D, int HPW>
+struct SimtConsumer {
+    static constexpr int RB = D * (int)sizeof(T);          // row bytes
+    static constexpr int NCH = RB / 16;                     // 16-byte chunks per row
+    static constexpr int CPL = NCH / 8;                     // chunks per lane
+    static constexpr int EPC = 16 / (int)sizeof(T);         // elements per chunk
+    static constexpr int EPL = CPL * EPC;                   // elements per lane
+    static constexpr int ROUNDS = BS / 4;
+    static_assert(NCH % 8 == 0, "row must hold a multiple of 8 chunks");
+
+    float q[HPW][EPL];
+    float acc[HPW][EPL];
+    float m[HPW], l[HPW];
+
+    __device__ __forceinline__ static void unpack(const uint4& raw, float* f) {
+        if constexpr (sizeof(T) == 4) {
+            f[0] = __uint_as_float(raw.x); f[1] = __uint_as_float(raw.y);
+            f[2] = __uint_as_float(raw.z); f[3] = __uint_as_float(raw.w);
+        } else {
+            f[0] = bf16lo(raw.x); f[1] = bf16hi(raw.x); f[2] = bf16lo(raw.y); f[3] = bf16hi(raw.y);
+            f[4] = bf16lo(raw.z); f[5] = bf16hi(raw.z); f[6] = bf16lo(raw.w); f[7] = bf16hi(raw.w);
+        }
+    }
+
+    // q_rows points at query head (first head of this warp) of this sequence.
+    __device__ __forceinline__ void init(const T* q_rows, float scale_log2, int lane) {
+        const int li = lane & 7;
+#pragma unroll
+        for (int h = 0; h < HPW; ++h) {
+            const uint4* row = reinterpret_cast<const uint4*>(q_rows + (int64_t)h * D);
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                float f[EPC];
+                unpack(row[c * 8 + li], f);
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) q[h][c * EPC + e] = f[e] * scale_log2;
+            }
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[h][e] = 0.f;
+            m[h] = kNegInf;
+            l[h] = 0.f;
+        }
+    }
+
+    __device__ __forceinline__ void consume(const uint8_t* ks, const uint8_t* vs, int nvalid, int lane) {
+        const int li = lane & 7, tg = lane >> 3;
+        float x[ROUNDS][HPW];
+#pragma unroll
+        for (int r = 0; r < ROUNDS; ++r) {
+            const uint4* row = reinterpret_cast<const uint4*>(ks + (r * 4 + tg) * RB);
+            float part[HPW];
+#pragma unroll
+            for (int h = 0; h < HPW; ++h) part[h] = 0.f;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                float f[EPC];
+                unpack(row[c * 8 + li], f);
+#pragma unroll
+                for (int h = 0; h < HPW; ++h)
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) part[h] = fmaf(q[h][c * EPC + e], f[e], part[h]);
+            }
+#pragma unroll
+            for (int h = 0; h < HPW; ++h) {
+                part[h] += __shfl_xor_sync(0xffffffffu, part[h], 1);
+                part[h] += __shfl_xor_sync(0xffffffffu, part[h], 2);
+                part[h] += __shfl_xor_sync(0xffffffffu, part[h], 4);
+                x[r][h] = (r * 4 + tg < nvalid) ? part[h] : kNegInf;
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < HPW; ++h) {
+            float bm = x[0][h];
+#pragma unroll
+            for (int r = 1; r < ROUNDS; ++r) bm = fmaxf(bm, x[r][h]);
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+            const float mn = fmaxf(m[h], bm);     // finite: every block has a valid token
+            const float alpha = fast_exp2(m[h] - mn);
+            m[h] = mn;
+            float ps = 0.f;
+#pragma unroll
+            for (int r = 0; r < ROUNDS; ++r) {
+                x[r][h] = fast_exp2(x[r][h] - mn);
+                ps += x[r][h];
+            }
+            l[h] = l[h] * alpha + ps;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[h][e] *= alpha;
+        }
+#pragma unroll
+        for (int r = 0; r < ROUNDS; ++r) {
+            if (r * 4 + tg < nvalid) {         // never touch rows past the context
+                const uint4* row = reinterpret_cast<const uint4*>(vs + (r * 4 + tg) * RB);
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) {
+                    float f[EPC];
+                    unpack(row[c * 8 + li], f);
+#pragma unroll
+                    for (int h = 0; h < HPW; ++h)
+#pragma unroll
+                        for (int e = 0; e < EPC; ++e)
+                            acc[h][c * EPC + e] = fmaf(x[r][h], f[e], acc[h][c * EPC + e]);
+                }
+            }
+        }
+    }
+
+    // Sum over the 4 token groups; lanes 0..7 write acc, lane 0 writes m and l.
+    __device__ __forceinline__ void finish(float* red_o, float* red_m, float* red_l, int lane) {
+        const int li = lane & 7;
+#pragma unroll
+        for (int h = 0; h < HPW; ++h) {
+            float lh = l[h];
+            lh += __shfl_xor_sync(0xffffffffu, lh, 8);
+            lh += __shfl_xor_sync(0xffffffffu, lh, 16);
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) {
+                float a = acc[h][e];
+                a += __shfl_xor_sync(0xffffffffu, a, 8);
+                a += __shfl_xor_sync(0xffffffffu, a, 16);
+                acc[h][e] = a;
+            }
+            if (lane < 8) {
+#pragma unroll
+                for (int c = 0; c < CPL; ++c)
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e)
+                        red_o[h * D + (c * 8 + li) * EPC + e] = acc[h][c * EPC + e];
+            }
+            if (lane == 0) {
+                red_m[h] = m[h];
+                red_l[h] = lh;
+            }
+        }
+    }
+};
+
+// ---------------------------------------------------------------------------
+// Tensor-core consumer (bf16, up to 8 query heads per KV head).
+// Stage layout: for K then V, D/64 half-tiles of [16 rows x 128 B], each
+// written by TMA with the 128-byte swizzle (16-byte chunk c of row r lives at
+// chunk c ^ (r & 7)), so ldmatrix reads are bank-conflict free.
+// ---------------------------------------------------------------------------
+template <int D>
+struct MmaConsumer {
+    static constexpr int KS = D / 16;          // k-steps of S^T = K Q^T
+    static constexpr int MT = D / 16;          // m-tiles of O^T
+    static constexpr int HALF = BS * 128;      // bytes of one 64-wide half tile
+
+    uint32_t qb[KS][2];                        // Q^T as B fragments (N = 8 query heads)
+    float o[MT][4];                            // O^T fragments: dims x heads
+    float m0, m1, l0, l1;                      // heads 2t, 2t+1
+
+    __device__ __forceinline__ void init(const __nv_bfloat16* q_rows, int group, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+        const uint32_t* row = reinterpret_cast<const uint32_t*>(q_rows + (int64_t)g * D);
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            if (g < group) {
+                qb[ks][0] = row[(ks * 16 + 2 * t) / 2];
+                qb[ks][1] = row[(ks * 16 + 2 * t + 8) / 2];
+            } else {
+                qb[ks][0] = qb[ks][1] = 0u;
+            }
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+        m0 = m1 = kNegInf;
+        l0 = l1 = 0.f;
+    }
+
+    __device__ __forceinline__ void consume(uint32_t ks_base, uint32_t vs_base, uint8_t* vs_ptr, int nvalid,
+                                            float scale_log2, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+        // Rows past the context may hold anything (NaN included): zero them in V,
+        // so that p = 0 times the row stays 0. K rows are masked by select.
+        if (nvalid < BS) {
+            for (int i = lane; i < (BS - nvalid) * (D / 8); i += 32) {
+                const int r = nvalid + i / (D / 8), cc = i % (D / 8);
+                const int half = cc >> 3, c = cc & 7;
+                *reinterpret_cast<uint4*>(vs_ptr + half * HALF + r * 128 + ((c ^ (r & 7)) << 4)) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+            __syncwarp();
+        }
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            const int r = lane & 15;
+            const int c = ((ks & 3) << 1) + (lane >> 4);
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4(a0, a1, a2, a3, ks_base + (ks >> 2) * HALF + r * 128 + ((c ^ (r & 7)) << 4));
+            mma_bf16_16816(s, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+        }
+        // s[0]: (token g, head 2t)  s[1]: (g, 2t+1)  s[2]: (g+8, 2t)  s[3]: (g+8, 2t+1)
+        float x0 = g < nvalid ? s[0] * scale_log2 : kNegInf;
+        float x1 = g < nvalid ? s[1] * scale_log2 : kNegInf;
+        float x2 = g + 8 < nvalid ? s[2] * scale_log2 : kNegInf;
+        float x3 = g + 8 < nvalid ? s[3] * scale_log2 : kNegInf;
+        float b0 = fmaxf(x0, x2), b1 = fmaxf(x1, x3);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            b0 = fmaxf(b0, __shfl_xor_sync(0xffffffffu, b0, off));
+            b1 = fmaxf(b1, __shfl_xor_sync(0xffffffffu, b1, off));
+        }
+        const float n0 = fmaxf(m0, b0), n1 = fmaxf(m1, b1);
+        const float al0 = fast_exp2(m0 - n0), al1 = fast_exp2(m1 - n1);
+        m0 = n0;
+        m1 = n1;
+        const float p0 = fast_exp2(x0 - n0), p1 = fast_exp2(x1 - n1);
+        const float p2 = fast_exp2(x2 - n0), p3 = fast_exp2(x3 - n1);
+        l0 = l0 * al0 + (p0 + p2);
+        l1 = l1 * al1 + (p1 + p3);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            o[mt][0] *= al0; o[mt][1] *= al1; o[mt][2] *= al0; o[mt][3] *= al1;
+        }
+        // P^T as B fragments (k = token, n = head), high and low bf16 parts.
+        const uint32_t h02 = pack_bf16(p0, p2), h13 = pack_bf16(p1, p3);
+        const uint32_t e02 = pack_bf16(p0 - bf16lo(h02), p2 - bf16hi(h02));
+        const uint32_t e13 = pack_bf16(p1 - bf16lo(h13), p3 - bf16hi(h13));
+        const int srcA = (2 * t) * 4 + (g >> 1), srcB = srcA + 4;
+        const bool odd = g & 1;
+        uint32_t ya, yb, za, zb;
+        {
+            const uint32_t u0 = __shfl_sync(0xffffffffu, h02, srcA), u1 = __shfl_sync(0xffffffffu, h13, srcA);
+            const uint32_t v0 = __shfl_sync(0xffffffffu, h02, srcB), v1 = __shfl_sync(0xffffffffu, h13, srcB);
+            ya = odd ? u1 : u0;
+            yb = odd ? v1 : v0;
+        }
+        {
+            const uint32_t u0 = __shfl_sync(0xffffffffu, e02, srcA), u1 = __shfl_sync(0xffffffffu, e13, srcA);
+            const uint32_t v0 = __shfl_sync(0xffffffffu, e02, srcB), v1 = __shfl_sync(0xffffffffu, e13, srcB);
+            za = odd ? u1 : u0;
+            zb = odd ? v1 : v0;
+        }
+        const uint32_t bh0 = __byte_perm(ya, yb, 0x5410), bh1 = __byte_perm(ya, yb, 0x7632);
+        const uint32_t bl0 = __byte_perm(za, zb, 0x5410), bl1 = __byte_perm(za, zb, 0x7632);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const int mi = lane >> 3;
+            const int tok = (lane & 7) + ((mi >> 1) << 3);
+            const int c = (((mt * 16) & 63) >> 3) + (mi & 1);
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4_trans(a0, a1, a2, a3,
+                              vs_base + ((mt * 16) >> 6) * HALF + tok * 128 + ((c ^ (tok & 7)) << 4));
+            mma_bf16_16816(o[mt], a0, a1, a2, a3, bh0, bh1);
+            mma_bf16_16816(o[mt], a0, a1, a2, a3, bl0, bl1);
+        }
+    }
+
+    __device__ __forceinline__ void finish(float* red_o, float* red_m, float* red_l, int group, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+        }
+        const int h0 = 2 * t, h1 = 2 * t + 1;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            if (h0 < group) {
+                red_o[h0 * D + mt * 16 + g] = o[mt][0];
+                red_o[h0 * D + mt * 16 + g + 8] = o[mt][2];
+            }
+            if (h1 < group) {
+                red_o[h1 * D + mt * 16 + g] = o[mt][1];
+                red_o[h1 * D + mt * 16 + g + 8] = o[mt][3];
+            }
+        }
+        if (g == 0) {
+            if (h0 < group) { red_m[h0] = m0; red_l[h0] = l0; }
+            if (h1 < group) { red_m[h1] = m1; red_l[h1] = l1; }
+        }
+    }
+};
+
+
+// Persistent schedule (paged_attention_persistent.cu).
+cudaError_t launch_persistent(bool bf16, bool use_mma, int head_dim, int group, const CUtensorMap& mk,
+                              const CUtensorMap& mv, const Params& p, int grid, cudaStream_t st);
+int persistent_ctas_per_sm();
+int persistent_max_seqs();
+
+}  // namespace attn
+}  // namespace pkv

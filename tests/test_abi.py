@@ -270,4 +270,9 @@ def test_workspace_and_partition_rule(lib):
     assert n >= rows * 128 * 4 + rows * 2 * 4
     assert binding.workspace_bytes(4, 8, 8, 64, 16, 16, 256, 512) == 0      # one partition
     assert binding.partition_tokens(16, 32, 8, 128, 16, 2048, 32768, 500) == 512
-    assert binding.partition_tokens(64, 32, 32, 128, 16, 128, 2048, 0) in (256, 512)
+    # 0 = the persistent, evenly split schedule: per-CTA pieces + one counter per (sequence, KV head)
+    assert binding.partition_tokens(64, 32, 32, 128, 16, 128, 2048, 0) == 0
+    n = binding.workspace_bytes(64, 32, 32, 128, 16, 128, 2048, 0)
+    assert n >= 64 * 32 * 8 and n < 32 * 2 ** 20
+    # more than 2048 sequences fall back to 512/256-token partitions
+    assert binding.partition_tokens(4096, 32, 8, 128, 16, 64, 1024, 0) == 512

@@ -45,14 +45,18 @@ SMALL = {
 
 @pytest.mark.parametrize("name", list(SMALL))
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
-def test_decode_step_matches_oracle(name, out_dtype):
+@pytest.mark.parametrize("schedule", ["persistent", "partitioned"])
+def test_decode_step_matches_oracle(name, out_dtype, schedule):
+    """schedule: persistent = the evenly split default (partition_tokens 0);
+    partitioned = fixed partitions (the workload's, else 512) + merge kernel."""
     w = SMALL[name]
+    part = 0 if schedule == "persistent" else (w.partition_tokens or 512)
     cache, lens = gpu_problem(w)
     op = OracleProblem(w)
     for step in range(2):
         q, kn, vn = step_inputs(w, step)
         out = cache.decode_step(np.arange(w.num_seqs), q, kn, vn, w.scale, out_dtype=out_dtype,
-                                partition_tokens=w.partition_tokens)
+                                partition_tokens=part)
         ref = op.decode_step(step)
         torch.cuda.synchronize()
         assert binding.get_device_error() == 0
@@ -132,6 +136,7 @@ def _run(dev, out_dtype=torch.float32, partition_tokens=0, max_context_len=0):
 @pytest.mark.parametrize("hq,hkv", [(4, 4), (4, 2), (8, 2), (16, 2)])
 @pytest.mark.parametrize("part", [0, 16, 64, 512])
 def test_edge_contexts(dtype, d, hq, hkv, part):
+    """part 0 = persistent schedule; > 0 = fixed partitions of that many tokens."""
     dev, ref = _edge_problem(hq * 1000 + hkv * 100 + d, hq, hkv, d, dtype, EDGE_LENS)
     out = _run(dev, partition_tokens=part)
     torch.cuda.synchronize()
@@ -145,7 +150,7 @@ def test_edge_contexts(dtype, d, hq, hkv, part):
 
 def test_partition_counts_agree():
     dev, ref = _edge_problem(5, 32, 8, 128, "bf16", [3000, 4097, 17, 8191])
-    outs = [_run(dev, partition_tokens=p).cpu().numpy() for p in (16, 128, 512, 2048, 8192)]
+    outs = [_run(dev, partition_tokens=p).cpu().numpy() for p in (16, 128, 512, 2048, 8192, 0)]
     for o in outs:
         assert np.abs(o - ref).max() <= 2e-3
     for o in outs[1:]:
@@ -157,17 +162,18 @@ def test_bf16_output():
     check_bf16_out(_run(dev, out_dtype=torch.bfloat16), ref)
 
 
-def test_permutation_of_physical_blocks_is_bitwise_invariant():
+@pytest.mark.parametrize("part", [256, 0])
+def test_permutation_of_physical_blocks_is_bitwise_invariant(part):
     """Moving blocks to other physical ids (and the table with them) changes
     nothing: the reduction order depends only on logical positions."""
     dev, _ = _edge_problem(7, 32, 8, 128, "bf16", [700, 33, 1024])
-    out1 = _run(dev, partition_tokens=256)
+    out1 = _run(dev, partition_tokens=part)
     nb = dev["nb"]
     perm = torch.from_numpy(np.random.default_rng(8).permutation(nb)).cuda()
     kc2, vc2 = torch.empty_like(dev["kc"]), torch.empty_like(dev["vc"])
     kc2[perm], vc2[perm] = dev["kc"], dev["vc"]
     dev2 = dict(dev, kc=kc2, vc=vc2, tables=perm[dev["tables"].long()].int().contiguous())
-    out2 = _run(dev2, partition_tokens=256)
+    out2 = _run(dev2, partition_tokens=part)
     assert torch.equal(out1, out2)
 
 
@@ -191,3 +197,26 @@ def test_context_beyond_table_is_clamped_and_flagged():
     assert binding.get_device_error() == 4
     # sequence 0 now reads the unwritten (NaN) tail of its last block; the other is untouched
     assert np.abs(out.cpu().numpy()[1] - ref[1]).max() <= 1e-5
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_persistent_schedule_many_small_and_long_items(seed):
+    """Mixed batch: many 1-3 block items (whole segments), zero lengths, and a
+    few long items that span many CTAs (pieces merged by the last CTA)."""
+    rng = np.random.default_rng(100 + seed)
+    lens = list(rng.integers(0, 48, size=40)) + [9000, 1, 20000, 0, 4096] + list(rng.integers(1, 700, size=20))
+    dev, ref = _edge_problem(200 + seed, 16, 4, 128, "bf16", lens)
+    out = _run(dev, partition_tokens=0, max_context_len=max(lens))
+    torch.cuda.synchronize()
+    assert binding.get_device_error() == 0
+    got = out.cpu().numpy()
+    assert np.isfinite(got).all()
+    assert np.abs(got - ref).max() <= 2e-3
+    # repeated calls reuse the workspace counters (a new epoch each call)
+    ws = torch.empty(binding.workspace_bytes(len(lens), 16, 4, 128, 16, dev["mb"], max(lens), 0),
+                     dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        out2 = torch.empty_like(out)
+        binding.paged_attention_decode(out2, dev["q"], dev["kc"], dev["vc"], dev["tables"], dev["lens"],
+                                       dev["scale"], max_context_len=max(lens), partition_tokens=0, workspace=ws)
+        assert torch.equal(out2, out)

@@ -11,9 +11,12 @@ from tests.paged_problem import OracleProblem, gpu_problem, step_inputs, toleran
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("name", ["llama2_7b", "gqa_70b", "shared_prefix", "long_splitk"])
-def test_full_size_sampled_against_oracle(name):
-    w = wl.WORKLOADS[name]
+@pytest.mark.parametrize("name,part", [("llama2_7b", 0), ("gqa_70b", 0), ("shared_prefix", 0), ("long_splitk", 512),
+                                       ("long_splitk", 0), ("llama2_7b", 512)])
+def test_full_size_sampled_against_oracle(name, part):
+    """part 0: the persistent schedule; 512: fixed 512-token partitions + merge."""
+    import dataclasses
+    w = dataclasses.replace(wl.WORKLOADS[name], partition_tokens=part)
     sample = wl.sample_seqs(w, 6)
     cache, lens = gpu_problem(w, fill_nan=(name == "shared_prefix"))
     op = OracleProblem(w, keep=sample)
