@@ -52,7 +52,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="pkv", choices=["pkv", "reference"])
     ap.add_argument("--workload", default="llama2_7b", choices=list(wl.WORKLOADS))
-    ap.add_argument("--partition-tokens", type=int, default=-1, help="-1: the workload's, 0: library default")
+    ap.add_argument("--partition-tokens", type=int, default=-2,
+                    help="-2: the workload's; 0: library-chosen partitions; -1: persistent schedule; >0: fixed")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
@@ -86,24 +87,38 @@ def barrier(ws):
         dist.barrier()
 
 
-def all_max(x: float, ws: int) -> float:
+def _all_reduce(x: float, ws: int, op: str) -> float:
+    """Reduces a host float over all ranks (CUDA tensor under NCCL, CPU under gloo)."""
     if ws == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def all_max(x: float, ws: int) -> float:
+    return _all_reduce(x, ws, "max")
 
 
 def all_sum(x: float, ws: int) -> float:
-    if ws == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return _all_reduce(x, ws, "sum")
+
+
+def replica_workload(w: wl.Workload, rank: int) -> wl.Workload:
+    """Rank r's replica of the batch: same shapes, its own seed (decode batches
+    are independent, so the replicas exchange no data)."""
+    return w if rank == 0 else dataclasses.replace(w, seed=w.seed + 7919 * rank)
+
+
+def aggregate(ms_local: float, bytes_local: float, tokens_local: float, ws: int):
+    """Whole-job figures: time = max over ranks, bytes and tokens summed."""
+    ms = all_max(ms_local, ws)
+    nbytes = all_sum(bytes_local, ws)
+    tokens = all_sum(tokens_local, ws)
+    return ms, nbytes / (ms * 1e-3) / 1e9, tokens / (ms * 1e-3)
 
 
 # ---------------------------------------------------------------------------
@@ -197,10 +212,16 @@ def traffic_record():
 
 
 def kernel_source_sha1() -> str:
+    """Hash of the partitioned attention kernel's device code (the shared device
+    headers and paged_attention.cu up to its host-side section)."""
+    csrc = os.path.join(ROOT, "paged_kv_cache_322_b200", "csrc")
     h = hashlib.sha1()
-    for name in ("paged_attention.cu", "common.cuh"):
-        with open(os.path.join(ROOT, "paged_kv_cache_322_b200", "csrc", name), "rb") as f:
+    for name in ("common.cuh", "attention_common.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
+    with open(os.path.join(csrc, "paged_attention.cu"), "rb") as f:
+        src = f.read()
+    h.update(src.split(b"// Host side")[0])
     return h.hexdigest()
 
 
@@ -235,9 +256,8 @@ def run_pkv(args, ws, rank, local):
         w = dataclasses.replace(w, num_seqs=args.num_seqs or w.num_seqs, num_blocks=args.num_blocks or w.num_blocks,
                                 description=w.description + f" [override: B={args.num_seqs or w.num_seqs}, "
                                                             f"pool={args.num_blocks or w.num_blocks}]")
-    if rank:
-        w = dataclasses.replace(w, seed=w.seed + 7919 * rank)     # each replica its own batch
-    part = w.partition_tokens if args.partition_tokens < 0 else args.partition_tokens
+    w = replica_workload(w, rank)
+    part = w.partition_tokens if args.partition_tokens == -2 else args.partition_tokens
     K, W = args.steps, args.warmup
     total_steps = 2 * (K + W) + 2
     lens0 = wl.context_lens(w)
@@ -272,10 +292,10 @@ def run_pkv(args, ws, rank, local):
             maxlen=int(lens.max()), bytes_attn=attention_bytes(w, lens, 2)))
     out = torch.empty((w.num_seqs, w.num_q_heads, w.head_dim), dtype=torch.bfloat16, device=dev)
     ws_bytes = binding.workspace_bytes(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, mb,
-                                       max(s["maxlen"] for s in steps), part if part > 0 else 0)
+                                       max(s["maxlen"] for s in steps), part)
     workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     part_used = binding.partition_tokens(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, mb,
-                                         max(s["maxlen"] for s in steps), part if part > 0 else 0)
+                                         max(s["maxlen"] for s in steps), part)
     stream = torch.cuda.current_stream(dev)
     maxctx = max(s["maxlen"] for s in steps)
 
@@ -284,8 +304,7 @@ def run_pkv(args, ws, rank, local):
         if ev0 is not None:
             ev0.record(stream)
         binding.paged_attention_decode(out, st["q"], cache.k_cache, cache.v_cache, st["tables"], st["lens"],
-                                       w.scale, max_context_len=maxctx, partition_tokens=part if part > 0 else 0,
-                                       workspace=workspace)
+                                       w.scale, max_context_len=maxctx, partition_tokens=part, workspace=workspace)
         if ev1 is not None:
             ev1.record(stream)
 
@@ -309,15 +328,12 @@ def run_pkv(args, ws, rank, local):
     timed = steps[W:]
     bytes_step = [s["bytes_attn"] + append_bytes(w) for s in timed]
     local_bytes = float(sum(bytes_step))
-    ms_max = all_max(ms, ws)
-    total_bytes = all_sum(local_bytes, ws)
-    gbs = total_bytes / (ms_max * 1e-3) / 1e9
-    tokens_s = ws * w.num_seqs * K / (ms_max * 1e-3)
+    ms_max, gbs, tokens_s = aggregate(ms, local_bytes, float(w.num_seqs * K), ws)
     peak, peak_kind = measured_peaks()
     attn_avg_ms = statistics.mean(attn_ms)
     attn_bytes_avg = statistics.mean(s["bytes_attn"] for s in timed)
     achieved = attn_bytes_avg / (attn_avg_ms * 1e-3) / 1e9
-    launches_per_step = 2 + (1 if (part_used and maxctx > part_used) else 0)
+    launches_per_step = 2 + (1 if (part_used > 0 and maxctx > part_used) else 0)
     del steps
 
     # ---- end to end through the public API from host buffers ----
@@ -338,7 +354,7 @@ def run_pkv(args, ws, rank, local):
             q_d.copy_(hq, non_blocking=True)
             k_d.copy_(hk, non_blocking=True)
             v_d.copy_(hv, non_blocking=True)
-            o = cache.decode_step(ids, q_d, k_d, v_d, w.scale, out=out, partition_tokens=part if part > 0 else 0)
+            o = cache.decode_step(ids, q_d, k_d, v_d, w.scale, out=out, partition_tokens=part)
             out_host.copy_(o, non_blocking=True)
             stream.synchronize()
 
@@ -357,14 +373,13 @@ def run_pkv(args, ws, rank, local):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(ws)
-        e_ms = all_max(e0.elapsed_time(e1), ws)
-        e_total = all_sum(float(sum(e2e_bytes)), ws)
+        e_ms, e_gbs, e_tok = aggregate(e0.elapsed_time(e1), float(sum(e2e_bytes)), float(w.num_seqs * K), ws)
         eb = w.elt_bytes
         h2d = (w.num_seqs * w.num_q_heads * w.head_dim * eb + 2 * w.num_seqs * w.num_kv_heads * w.head_dim * eb +
                w.num_seqs * 8 + w.num_seqs * mb * 4 + w.num_seqs * 4)
         d2h = w.num_seqs * w.num_q_heads * w.head_dim * 2
-        e2e = {"value": round(e_total / (e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
-               "decode_tokens_per_s": round(ws * w.num_seqs * K / (e_ms * 1e-3), 1),
+        e2e = {"value": round(e_gbs, 1), "unit": "GB/s",
+               "decode_tokens_per_s": round(e_tok, 1),
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e_ms / K, 4)}
 
     cpu = None
@@ -381,7 +396,8 @@ def run_pkv(args, ws, rank, local):
         "decode_tokens_per_s": round(tokens_s, 1),
         "attention_layer_tokens_per_s_per_32_layers": round(tokens_s / 32, 1),
         "config": {"workload": w.description, "global_batch": w.num_seqs * ws, "seq_len": f"U[{w.lo},{w.hi}]",
-                   "block_size": w.block_size, "partition_tokens": part_used,
+                   "block_size": w.block_size,
+                   "schedule": ("persistent" if part == -1 else f"partitions of {part_used} tokens"),
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
                    "l2": f"inputs larger than L2 ({int(lens0.sum()) * w.num_kv_heads * w.head_dim * w.elt_bytes * 2 / 1e9:.2f} GB KV per step vs 126 MB L2); no flush",
                    "seed": w.seed},

@@ -71,6 +71,9 @@ typedef enum pkv_status {
 
 typedef enum pkv_dtype { PKV_F32 = 0, PKV_BF16 = 1 } pkv_dtype;
 
+/* partition_tokens value selecting the persistent schedule of the decode call. */
+#define PKV_SCHEDULE_PERSISTENT (-1)
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* pkv_status_string(int status);
 
@@ -86,10 +89,16 @@ const char* pkv_status_string(int status);
  * is read from physical block block_tables[s][j / block_size], offset
  * j % block_size. A sequence with context length 0 gets a zero output.
  *
- * Long contexts are cut into partitions of `partition_tokens` tokens (a
- * multiple of block_size; 0 picks one from the shapes) that are processed in
- * parallel and merged exactly with a log-sum-exp reduction. Partial results
- * live in `workspace` (device memory, at least
+ * Schedules (`partition_tokens`):
+ *   > 0  contexts are cut into partitions of that many tokens (rounded up to a
+ *        multiple of block_size), processed in parallel and merged exactly with
+ *        a log-sum-exp reduction;
+ *   0    the same, with the partition length picked from the shapes (long
+ *        partitions whenever the batch still fills the GPU);
+ *   -1   PKV_SCHEDULE_PERSISTENT: two CTAs per SM, each streaming an equal
+ *        share of the batch's (sequence, block) tiles, with split sequences
+ *        merged inside the kernel (at most 2048 sequences).
+ * Partial results live in `workspace` (device memory, at least
  * pkv_paged_attention_workspace_bytes(...) bytes, 256-byte aligned; it may be
  * NULL when that size is 0). Its contents need no initialisation and are
  * scratch between calls; two calls in flight at once need two workspaces.
@@ -122,7 +131,8 @@ size_t pkv_paged_attention_workspace_bytes(
     int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
     int max_blocks_per_seq, int max_context_len, int partition_tokens);
 
-/* The partition length (tokens) the decode call uses for these sizes. */
+/* The partition length (tokens) the decode call uses for these sizes, 0 for
+ * the persistent schedule, -1 for invalid sizes. */
 int pkv_paged_attention_partition_tokens(
     int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
     int max_blocks_per_seq, int max_context_len, int partition_tokens);

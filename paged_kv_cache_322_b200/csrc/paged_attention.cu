@@ -318,13 +318,19 @@ struct Plan {
     int team_size;      // CTAs per team (one KV head each)
 };
 
-// Schedule for one call. partition_tokens > 0 asks for fixed partitions (the
-// partitioned kernel + merge kernel); 0 picks the persistent, evenly split
-// schedule whenever it applies (at most 2048 sequences and < 2^31 tiles),
-// else 512/256-token partitions.
+// Schedule for one call.
+//   partition_tokens > 0  : fixed partitions of that many tokens (+ merge kernel).
+//   partition_tokens == 0 : fixed partitions chosen here: the largest of
+//                           2048/1024/512/256 tokens that still gives about two
+//                           waves of work items (estimated from the longest
+//                           context, assuming lengths spread down to ~half of it).
+//                           Measured on B200: fewer, longer partitions stream
+//                           fastest (no merge pass, fewer CTA start-ups).
+//   partition_tokens == -1: the persistent, evenly split schedule (at most 2048
+//                           sequences and < 2^31 tiles).
 bool plan(int num_seqs, int num_kv_heads, int block_size, int max_blocks, int max_context_len,
           int partition_tokens, Plan* pl) {
-    if (num_seqs <= 0 || num_kv_heads <= 0 || block_size != BS || max_blocks <= 0 || partition_tokens < 0)
+    if (num_seqs <= 0 || num_kv_heads <= 0 || block_size != BS || max_blocks <= 0 || partition_tokens < -1)
         return false;
     const int64_t cap_tbl = (int64_t)max_blocks * block_size;
     if (cap_tbl > INT32_MAX) return false;
@@ -333,8 +339,10 @@ bool plan(int num_seqs, int num_kv_heads, int block_size, int max_blocks, int ma
     pl->ctx_cap = cap;
     pl->persistent = false;
     pl->grid = 0;
-    const int64_t max_tiles = (int64_t)num_seqs * num_kv_heads * ((cap + BS - 1) / BS);
-    if (partition_tokens == 0 && num_seqs <= persistent_max_seqs() && max_tiles < INT32_MAX) {
+    pl->team_size = 0;
+    if (partition_tokens == -1) {
+        const int64_t max_tiles = (int64_t)num_seqs * num_kv_heads * ((cap + BS - 1) / BS);
+        if (num_seqs > persistent_max_seqs() || max_tiles >= INT32_MAX) return false;
         pl->persistent = true;
         // teams of Hkv CTAs (one KV head each); as many whole teams as fit two CTAs per SM
         const int slots = num_sms() * persistent_ctas_per_sm();
@@ -345,9 +353,20 @@ bool plan(int num_seqs, int num_kv_heads, int block_size, int max_blocks, int ma
         return true;
     }
     int pt = partition_tokens;
-    if (pt <= 0) {
-        const int64_t items = (int64_t)num_seqs * num_kv_heads;
-        pt = items >= 4 * num_sms() ? 512 : 256;
+    if (pt == 0) {
+        // Fewest partitions of at most kMaxAutoPartition tokens that still give
+        // about two waves of work items (estimated with lengths spread down to
+        // ~half of the longest); never shorter than 256 tokens.
+        constexpr int kMaxAutoPartition = 2560;
+        const int64_t target = 2ll * 3 * num_sms();             // ~two waves of 3 CTAs per SM
+        pt = 256;
+        for (int nparts = 1; nparts <= 65535; ++nparts) {
+            const int cand = (int)(((int64_t)(cap + nparts - 1) / nparts + BS - 1) / BS * BS);
+            if (cand < 256) break;
+            if (cand > kMaxAutoPartition) continue;
+            const int64_t est = (int64_t)num_seqs * num_kv_heads * std::max<int64_t>(1, (nparts + 1) / 2);
+            if (est >= target) { pt = cand; break; }
+        }
     }
     pt = ((pt + BS - 1) / BS) * BS;
     int parts = (cap + pt - 1) / pt;
@@ -447,7 +466,7 @@ pkv_status pkv_paged_attention_decode(void* out, pkv_dtype out_dtype, const void
     using namespace pkv;
     using namespace pkv::attn;
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
-        max_context_len < 0 || !std::isfinite(scale))
+        max_context_len < 0 || partition_tokens < -1 || !std::isfinite(scale))
         return PKV_ERR_INVALID_ARG;
     if ((out_dtype != PKV_F32 && out_dtype != PKV_BF16) || (kv_dtype != PKV_F32 && kv_dtype != PKV_BF16))
         return PKV_ERR_INVALID_ARG;

@@ -270,9 +270,16 @@ def test_workspace_and_partition_rule(lib):
     assert n >= rows * 128 * 4 + rows * 2 * 4
     assert binding.workspace_bytes(4, 8, 8, 64, 16, 16, 256, 512) == 0      # one partition
     assert binding.partition_tokens(16, 32, 8, 128, 16, 2048, 32768, 500) == 512
-    # 0 = the persistent, evenly split schedule: per-CTA pieces + one counter per (sequence, KV head)
-    assert binding.partition_tokens(64, 32, 32, 128, 16, 128, 2048, 0) == 0
-    n = binding.workspace_bytes(64, 32, 32, 128, 16, 128, 2048, 0)
+    # -1 = the persistent, evenly split schedule: per-CTA pieces + one counter per (sequence, KV head)
+    assert binding.partition_tokens(64, 32, 32, 128, 16, 128, 2048, -1) == 0
+    n = binding.workspace_bytes(64, 32, 32, 128, 16, 128, 2048, -1)
     assert n >= 64 * 32 * 8 and n < 32 * 2 ** 20
-    # more than 2048 sequences fall back to 512/256-token partitions
-    assert binding.partition_tokens(4096, 32, 8, 128, 16, 64, 1024, 0) == 512
+    with pytest.raises(binding.PkvError):
+        binding.workspace_bytes(4096, 32, 8, 128, 16, 64, 1024, -1)   # more than 2048 sequences
+    # 0 = library-chosen partitions: long ones while the batch fills the GPU, shorter for small batches
+    p7 = binding.partition_tokens(64, 32, 32, 128, 16, 256, 2158, 0)                # 7B-shaped batch
+    assert p7 >= 2158 and p7 % 16 == 0                                                # one partition, no merge
+    assert binding.workspace_bytes(64, 32, 32, 128, 16, 256, 2158, 0) == 0
+    p70 = binding.partition_tokens(128, 64, 8, 128, 16, 512, 4100, 0)               # 70B-shaped batch
+    assert -(-4100 // p70) == 2 and p70 <= 2560                                       # two partitions
+    assert binding.partition_tokens(1, 32, 8, 128, 16, 2048, 32768, 0) == 256       # one long sequence

@@ -47,10 +47,10 @@ SMALL = {
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("schedule", ["persistent", "partitioned"])
 def test_decode_step_matches_oracle(name, out_dtype, schedule):
-    """schedule: persistent = the evenly split default (partition_tokens 0);
-    partitioned = fixed partitions (the workload's, else 512) + merge kernel."""
+    """schedule: persistent = the evenly split schedule (partition_tokens -1);
+    partitioned = fixed partitions (the workload's, else the library default)."""
     w = SMALL[name]
-    part = 0 if schedule == "persistent" else (w.partition_tokens or 512)
+    part = -1 if schedule == "persistent" else w.partition_tokens
     cache, lens = gpu_problem(w)
     op = OracleProblem(w)
     for step in range(2):
@@ -134,9 +134,9 @@ def _run(dev, out_dtype=torch.float32, partition_tokens=0, max_context_len=0):
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("hq,hkv", [(4, 4), (4, 2), (8, 2), (16, 2)])
-@pytest.mark.parametrize("part", [0, 16, 64, 512])
+@pytest.mark.parametrize("part", [-1, 0, 16, 64, 512])
 def test_edge_contexts(dtype, d, hq, hkv, part):
-    """part 0 = persistent schedule; > 0 = fixed partitions of that many tokens."""
+    """part -1 = persistent schedule; 0 = library-chosen partitions; > 0 = fixed."""
     dev, ref = _edge_problem(hq * 1000 + hkv * 100 + d, hq, hkv, d, dtype, EDGE_LENS)
     out = _run(dev, partition_tokens=part)
     torch.cuda.synchronize()
@@ -150,7 +150,7 @@ def test_edge_contexts(dtype, d, hq, hkv, part):
 
 def test_partition_counts_agree():
     dev, ref = _edge_problem(5, 32, 8, 128, "bf16", [3000, 4097, 17, 8191])
-    outs = [_run(dev, partition_tokens=p).cpu().numpy() for p in (16, 128, 512, 2048, 8192, 0)]
+    outs = [_run(dev, partition_tokens=p).cpu().numpy() for p in (16, 128, 512, 2048, 8192, 0, -1)]
     for o in outs:
         assert np.abs(o - ref).max() <= 2e-3
     for o in outs[1:]:
@@ -162,7 +162,7 @@ def test_bf16_output():
     check_bf16_out(_run(dev, out_dtype=torch.bfloat16), ref)
 
 
-@pytest.mark.parametrize("part", [256, 0])
+@pytest.mark.parametrize("part", [256, 0, -1])
 def test_permutation_of_physical_blocks_is_bitwise_invariant(part):
     """Moving blocks to other physical ids (and the table with them) changes
     nothing: the reduction order depends only on logical positions."""
@@ -206,17 +206,17 @@ def test_persistent_schedule_many_small_and_long_items(seed):
     rng = np.random.default_rng(100 + seed)
     lens = list(rng.integers(0, 48, size=40)) + [9000, 1, 20000, 0, 4096] + list(rng.integers(1, 700, size=20))
     dev, ref = _edge_problem(200 + seed, 16, 4, 128, "bf16", lens)
-    out = _run(dev, partition_tokens=0, max_context_len=max(lens))
+    out = _run(dev, partition_tokens=-1, max_context_len=max(lens))
     torch.cuda.synchronize()
     assert binding.get_device_error() == 0
     got = out.cpu().numpy()
     assert np.isfinite(got).all()
     assert np.abs(got - ref).max() <= 2e-3
     # repeated calls reuse the workspace counters (a new epoch each call)
-    ws = torch.empty(binding.workspace_bytes(len(lens), 16, 4, 128, 16, dev["mb"], max(lens), 0),
+    ws = torch.empty(binding.workspace_bytes(len(lens), 16, 4, 128, 16, dev["mb"], max(lens), -1),
                      dtype=torch.uint8, device="cuda")
     for _ in range(3):
         out2 = torch.empty_like(out)
         binding.paged_attention_decode(out2, dev["q"], dev["kc"], dev["vc"], dev["tables"], dev["lens"],
-                                       dev["scale"], max_context_len=max(lens), partition_tokens=0, workspace=ws)
+                                       dev["scale"], max_context_len=max(lens), partition_tokens=-1, workspace=ws)
         assert torch.equal(out2, out)

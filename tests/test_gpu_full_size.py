@@ -12,9 +12,10 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("name,part", [("llama2_7b", 0), ("gqa_70b", 0), ("shared_prefix", 0), ("long_splitk", 512),
-                                       ("long_splitk", 0), ("llama2_7b", 512)])
+                                       ("long_splitk", -1), ("llama2_7b", -1), ("gqa_70b", -1)])
 def test_full_size_sampled_against_oracle(name, part):
-    """part 0: the persistent schedule; 512: fixed 512-token partitions + merge."""
+    """part 0: library-chosen partitions; 512: fixed 512-token partitions;
+    -1: the persistent schedule."""
     import dataclasses
     w = dataclasses.replace(wl.WORKLOADS[name], partition_tokens=part)
     sample = wl.sample_seqs(w, 6)
