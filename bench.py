@@ -199,16 +199,17 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def traffic_record():
-    """ncu DRAM traffic of the attention kernel, if taken on the current source."""
+def traffic_record(workload: str):
+    """ncu DRAM traffic of the attention kernel for this workload, if it was taken
+    on the current device code (else None)."""
     path = os.path.join(ROOT, "profiles", "attention_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f)
-    if rec.get("source_sha1") != kernel_source_sha1():
+    if rec.get("source_sha1") != kernel_source_sha1() or workload not in rec:
         return None
-    return rec
+    return rec[workload]
 
 
 def kernel_source_sha1() -> str:
@@ -336,7 +337,7 @@ def run_pkv(args, ws, rank, local):
     launches_per_step = 2 + (1 if (part_used > 0 and maxctx > part_used) else 0)
     del steps
 
-    # ---- end to end through the public API from host buffers ----
+    # ---- end to end through the C ABI from host buffers: pkv_decode_step ----
     e2e = None
     if not args.no_e2e:
         host = []
@@ -344,24 +345,19 @@ def run_pkv(args, ws, rank, local):
             q = wl.decode_q(w, 1000 + i)
             kn, vn = wl.decode_kv(w, 1000 + i)
             host.append(tuple(torch.from_numpy(x).to(dt).pin_memory() for x in (q, kn, vn)))
-        out_host = torch.empty(out.shape, dtype=torch.bfloat16, pin_memory=True)
-        q_d = torch.empty(host[0][0].shape, dtype=dt, device=dev)
-        k_d = torch.empty(host[0][1].shape, dtype=dt, device=dev)
-        v_d = torch.empty(host[0][2].shape, dtype=dt, device=dev)
+        out_host = torch.empty((w.num_seqs, w.num_q_heads, w.head_dim), dtype=torch.bfloat16).pin_memory()
+        native = binding.DecodeStep(cache.bm, cache.k_cache, cache.v_cache, max_seqs=w.num_seqs,
+                                    num_q_heads=w.num_q_heads, max_blocks_per_seq=mb, out_dtype=torch.bfloat16,
+                                    partition_tokens=part)
         e2e_bytes = []
 
         def step_host(hq, hk, hv):
-            q_d.copy_(hq, non_blocking=True)
-            k_d.copy_(hk, non_blocking=True)
-            v_d.copy_(hv, non_blocking=True)
-            o = cache.decode_step(ids, q_d, k_d, v_d, w.scale, out=out, partition_tokens=part)
-            out_host.copy_(o, non_blocking=True)
-            stream.synchronize()
+            native(ids, hq, hk, hv, out_host, w.scale, stream=stream)
+            stream.synchronize()                  # the step's result is on the host
 
         lens_now = np.array([cache.bm.seq_len(int(s)) for s in ids])
         for i in range(K):
             e2e_bytes.append(attention_bytes(w, lens_now + W + i + 1, 2) + append_bytes(w))
-
         for i in range(W):
             step_host(*host[i])
         barrier(ws)
@@ -373,20 +369,22 @@ def run_pkv(args, ws, rank, local):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(ws)
+        assert binding.get_device_error() == 0
         e_ms, e_gbs, e_tok = aggregate(e0.elapsed_time(e1), float(sum(e2e_bytes)), float(w.num_seqs * K), ws)
         eb = w.elt_bytes
         h2d = (w.num_seqs * w.num_q_heads * w.head_dim * eb + 2 * w.num_seqs * w.num_kv_heads * w.head_dim * eb +
-               w.num_seqs * 8 + w.num_seqs * mb * 4 + w.num_seqs * 4)
+               w.num_seqs * (3 * 8 + mb * 4 + 4))
         d2h = w.num_seqs * w.num_q_heads * w.head_dim * 2
         e2e = {"value": round(e_gbs, 1), "unit": "GB/s",
                "decode_tokens_per_s": round(e_tok, 1),
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e_ms / K, 4)}
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e_ms / K, 4),
+               "path": "pkv_decode_step (C ABI, host buffers): block manager, H2D, kernels, D2H, stream sync"}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.cpu_seconds)
 
-    tr = traffic_record()
+    tr = traffic_record(args.workload) if part != -1 else None
     result = {
         "metric": "paged decode attention achieved HBM GB/s (% of B200 peak); decode tokens/s",
         "value": round(gbs, 1), "unit": "GB/s", "n_gpus": ws, "steps": K, "warmup": W,

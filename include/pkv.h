@@ -223,6 +223,44 @@ pkv_status pkv_copy_blocks(
 pkv_status pkv_get_device_error(int* code, void* stream);
 
 /* ------------------------------------------------------------------------- */
+/* One decode step from host buffers ([VP] §3.3 decode, §4.1 copy-on-write)  */
+/* ------------------------------------------------------------------------- */
+/*
+ * A step context owns the device buffers one decode step needs for up to
+ * max_seqs sequences (the step's q / new K,V / metadata / output / split-K
+ * workspace) and two pinned staging slots. Creating it allocates (once);
+ * pkv_decode_step allocates nothing. partition_tokens is the schedule the steps
+ * will use (same meaning as in pkv_paged_attention_decode). One context serves
+ * one stream at a time.
+ */
+typedef struct pkv_step_ctx pkv_step_ctx;
+typedef struct pkv_block_manager pkv_block_manager;
+
+pkv_status pkv_step_ctx_create(int max_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                               int max_blocks_per_seq, pkv_dtype kv_dtype, pkv_dtype out_dtype,
+                               int partition_tokens, pkv_step_ctx** out);
+void pkv_step_ctx_destroy(pkv_step_ctx* ctx);
+
+/*
+ * One decode step for the n listed sequences of `bm` (n <= max_seqs):
+ *   1. the block manager appends one token to each sequence (slot mapping,
+ *      copy-on-write pairs, block tables and lengths, in pinned staging);
+ *   2. metadata, q [n, Hq, D], k and v [n, Hkv, D] are copied to the device
+ *      (q_host, k_host, v_host are HOST pointers; pinned memory makes the copies
+ *      asynchronous);
+ *   3. pkv_copy_blocks for the copy-on-write pairs, pkv_reshape_and_cache for
+ *      the new tokens, pkv_paged_attention_decode over the updated contexts;
+ *   4. the output [n, Hq, D] (out_dtype of the context) is copied to out_host.
+ * k_cache / v_cache are the device caches (block_size 16). Everything is
+ * enqueued on `stream`; synchronise it before reading out_host. A block manager
+ * error (PKV_ERR_OUT_OF_BLOCKS) is returned before anything is enqueued.
+ */
+pkv_status pkv_decode_step(pkv_step_ctx* ctx, pkv_block_manager* bm, const int64_t* seq_ids, int n,
+                           const void* q_host, const void* k_host, const void* v_host,
+                           void* k_cache, void* v_cache, int num_blocks, float scale,
+                           int partition_tokens, void* out_host, void* stream);
+
+/* ------------------------------------------------------------------------- */
 /* Host block manager ([ENG] §2.3; [VP] §3.3, §4.1, §4.2; [BT])              */
 /* ------------------------------------------------------------------------- */
 /*
@@ -234,8 +272,6 @@ pkv_status pkv_get_device_error(int* code, void* stream);
  * ([ENG] §2.3). Reference counts: a block shared by k sequences has count k;
  * a block whose count falls to 0 goes back to the free list ([VP] §4.2).
  */
-typedef struct pkv_block_manager pkv_block_manager;
-
 /* free_order: the initial free-list order (a permutation of 0..num_blocks-1),
  * or NULL for 0,1,2,... The manager copies it. */
 pkv_status pkv_bm_create(int num_blocks, int block_size, const int32_t* free_order,

@@ -45,6 +45,9 @@ _SIGS = {
     "pkv_reshape_and_cache": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pkv_copy_blocks": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pkv_get_device_error": (_i32, [_c.POINTER(_c.c_int), _vp]),
+    "pkv_step_ctx_create": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _c.POINTER(_vp)]),
+    "pkv_step_ctx_destroy": (None, [_vp]),
+    "pkv_decode_step": (_i32, [_vp, _vp, _pi64, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _f32, _i32, _vp, _vp]),
     "pkv_bm_create": (_i32, [_i32, _i32, _pi32, _c.POINTER(_vp)]),
     "pkv_bm_destroy": (None, [_vp]),
     "pkv_bm_allocate": (_i32, [_vp, _i64, _i32, _pi64]),
@@ -303,3 +306,42 @@ class BlockManager:
 
     def seq_len(self, seq_id: int) -> int:
         return _lib().pkv_bm_seq_len(self._h, seq_id)
+
+
+class DecodeStep:
+    """The native decode step (pkv_decode_step): block manager append, H2D of the
+    step's q / new K,V / metadata from host buffers, copy-on-write copies, KV
+    append, attention, D2H of the output -- one C call per step."""
+
+    def __init__(self, bm: BlockManager, k_cache, v_cache, max_seqs: int, num_q_heads: int,
+                 max_blocks_per_seq: int, out_dtype, partition_tokens: int = 0):
+        torch = _torch()
+        self.bm, self.k_cache, self.v_cache = bm, k_cache, v_cache
+        nb, bs, hkv, d = k_cache.shape
+        if bs != 16:
+            raise ValueError("block_size 16 only")
+        self.num_blocks, self.hq, self.hkv, self.d = nb, num_q_heads, hkv, d
+        self.partition_tokens = partition_tokens
+        self.out_dtype = out_dtype
+        self._h = ctypes.c_void_p()
+        _check(_lib().pkv_step_ctx_create(max_seqs, num_q_heads, hkv, d, max_blocks_per_seq, _dtype_code(k_cache),
+                                          PKV_F32 if out_dtype == torch.float32 else PKV_BF16,
+                                          partition_tokens, ctypes.byref(self._h)), "pkv_step_ctx_create")
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value and _L is not None:
+            _L.pkv_step_ctx_destroy(h)
+            self._h = None
+
+    def __call__(self, seq_ids: np.ndarray, q_host, k_host, v_host, out_host, scale: float, stream=None):
+        """q_host/k_host/v_host/out_host: CPU tensors (pinned for asynchronous copies).
+        Enqueues the step; synchronise the stream before reading out_host."""
+        torch = _torch()
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        s = stream if stream is not None else torch.cuda.current_stream(self.k_cache.device)
+        st = _lib().pkv_decode_step(self._h, self.bm._h, _ptr(ids, ctypes.c_int64), ids.size, q_host.data_ptr(),
+                                    k_host.data_ptr(), v_host.data_ptr(), self.k_cache.data_ptr(),
+                                    self.v_cache.data_ptr(), self.num_blocks, float(scale), self.partition_tokens,
+                                    out_host.data_ptr(), s.cuda_stream)
+        _check(st, "pkv_decode_step")

@@ -1,0 +1,182 @@
+// One whole decode step from host buffers, in native code.
+//
+// The step follows "vLLM PagedAttention 深度解析" §3.3 (decode: write the new
+// token's K/V into its logical block through the block table, a new block when
+// the last one is full) and §4.1 (a shared partially filled block is copied
+// before the write):
+//   1. block manager: one slot per sequence, copy-on-write pairs, block tables;
+//   2. the metadata goes to the device in one copy from pinned staging, q and
+//      the new K/V in one copy each from the caller's host buffers;
+//   3. copy_blocks (if any pair), reshape_and_cache, paged decode attention;
+//   4. the attention output is copied back to the caller's host buffer.
+// Everything is enqueued on the caller's stream; the call returns without
+// waiting. The step context owns the device-side buffers and two pinned
+// staging slots (so one step's metadata can be written while the previous
+// step's copy is still in flight).
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "common.cuh"
+
+struct pkv_step_ctx {
+    int max_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks;
+    pkv_dtype kv_dtype, out_dtype;
+    size_t meta_bytes, q_bytes, kv_bytes, out_bytes, ws_bytes;
+    // device
+    unsigned char* d_meta = nullptr;   // slots i64[S] | src i64[S] | dst i64[S] | tables i32[S*MB] | lens i32[S]
+    void* d_q = nullptr;
+    void* d_k = nullptr;
+    void* d_v = nullptr;
+    void* d_out = nullptr;
+    void* d_ws = nullptr;
+    // host
+    unsigned char* h_meta[2] = {nullptr, nullptr};
+    cudaEvent_t meta_done[2] = {nullptr, nullptr};
+    int slot = 0;
+    int device = 0;
+};
+
+namespace {
+
+int elt(pkv_dtype t) { return t == PKV_F32 ? 4 : 2; }
+
+void release(pkv_step_ctx* c) {
+    if (!c) return;
+    int prev = 0;
+    cudaGetDevice(&prev);
+    cudaSetDevice(c->device);
+    cudaFree(c->d_meta);
+    cudaFree(c->d_q);
+    cudaFree(c->d_k);
+    cudaFree(c->d_v);
+    cudaFree(c->d_out);
+    cudaFree(c->d_ws);
+    for (int i = 0; i < 2; ++i) {
+        if (c->h_meta[i]) cudaFreeHost(c->h_meta[i]);
+        if (c->meta_done[i]) cudaEventDestroy(c->meta_done[i]);
+    }
+    cudaSetDevice(prev);
+    delete c;
+}
+
+}  // namespace
+
+extern "C" {
+
+pkv_status pkv_step_ctx_create(int max_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                               int max_blocks_per_seq, pkv_dtype kv_dtype, pkv_dtype out_dtype,
+                               int partition_tokens, pkv_step_ctx** out) {
+    if (!out || max_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        max_blocks_per_seq <= 0 || num_q_heads % num_kv_heads != 0 ||
+        (kv_dtype != PKV_F32 && kv_dtype != PKV_BF16) || (out_dtype != PKV_F32 && out_dtype != PKV_BF16))
+        return PKV_ERR_INVALID_ARG;
+    *out = nullptr;
+    pkv_step_ctx* c = new (std::nothrow) pkv_step_ctx();
+    if (!c) return PKV_ERR_INVALID_ARG;
+    cudaGetDevice(&c->device);
+    c->max_seqs = max_seqs;
+    c->num_q_heads = num_q_heads;
+    c->num_kv_heads = num_kv_heads;
+    c->head_dim = head_dim;
+    c->max_blocks = max_blocks_per_seq;
+    c->kv_dtype = kv_dtype;
+    c->out_dtype = out_dtype;
+    const size_t S = (size_t)max_seqs;
+    c->meta_bytes = S * 8 * 3 + S * max_blocks_per_seq * 4 + S * 4;
+    c->q_bytes = S * num_q_heads * head_dim * elt(kv_dtype);
+    c->kv_bytes = S * num_kv_heads * head_dim * elt(kv_dtype);
+    c->out_bytes = S * num_q_heads * head_dim * elt(out_dtype);
+    // Largest workspace any step can ask for: a fixed partition length never needs
+    // more than at max_seqs and full tables; the library-chosen one is >= 256 tokens.
+    const int sizing_part = partition_tokens == 0 ? 256 : partition_tokens;
+    const size_t ws = pkv_paged_attention_workspace_bytes(max_seqs, num_q_heads, num_kv_heads, head_dim, 16,
+                                                          max_blocks_per_seq, 0, sizing_part);
+    if (ws == (size_t)-1) {
+        delete c;
+        return PKV_ERR_INVALID_ARG;
+    }
+    c->ws_bytes = ws;
+    bool ok = cudaMalloc(&c->d_meta, c->meta_bytes) == cudaSuccess && cudaMalloc(&c->d_q, c->q_bytes) == cudaSuccess &&
+              cudaMalloc(&c->d_k, c->kv_bytes) == cudaSuccess && cudaMalloc(&c->d_v, c->kv_bytes) == cudaSuccess &&
+              cudaMalloc(&c->d_out, c->out_bytes) == cudaSuccess &&
+              (ws == 0 || cudaMalloc(&c->d_ws, ws) == cudaSuccess);
+    for (int i = 0; ok && i < 2; ++i)
+        ok = cudaHostAlloc((void**)&c->h_meta[i], c->meta_bytes, cudaHostAllocDefault) == cudaSuccess &&
+             cudaEventCreateWithFlags(&c->meta_done[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+        release(c);
+        return PKV_ERR_CUDA;
+    }
+    *out = c;
+    return PKV_OK;
+}
+
+void pkv_step_ctx_destroy(pkv_step_ctx* ctx) { release(ctx); }
+
+pkv_status pkv_decode_step(pkv_step_ctx* c, pkv_block_manager* bm, const int64_t* seq_ids, int n,
+                           const void* q_host, const void* k_host, const void* v_host, void* k_cache, void* v_cache,
+                           int num_blocks, float scale, int partition_tokens, void* out_host, void* stream) {
+    if (!c || !bm || n < 0 || n > c->max_seqs || (n > 0 && (!seq_ids || !q_host || !k_host || !v_host ||
+                                                            !k_cache || !v_cache || !out_host)))
+        return PKV_ERR_INVALID_ARG;
+    if (n == 0) return PKV_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t S = (size_t)c->max_seqs;
+    // 1. host metadata into a pinned slot whose previous copy has finished
+    const int sl = c->slot;
+    c->slot ^= 1;
+    if (cudaEventSynchronize(c->meta_done[sl]) != cudaSuccess) return PKV_ERR_CUDA;
+    unsigned char* h = c->h_meta[sl];
+    int64_t* slots = reinterpret_cast<int64_t*>(h);
+    int64_t* src = slots + S;
+    int64_t* dst = src + S;
+    int32_t* tables = reinterpret_cast<int32_t*>(dst + S);
+    int32_t* lens = tables + S * c->max_blocks;
+    int ncopy = 0;
+    pkv_status s = pkv_bm_append_slots(bm, seq_ids, n, slots, src, dst, &ncopy, nullptr);
+    if (s != PKV_OK) return s;
+    // tables of the listed sequences, row stride max_blocks
+    s = pkv_bm_block_tables(bm, seq_ids, n, c->max_blocks, tables, lens);
+    if (s != PKV_OK) return s;
+    int max_len = 0;
+    for (int i = 0; i < n; ++i) max_len = lens[i] > max_len ? lens[i] : max_len;
+    // 2. copies to the device
+    if (cudaMemcpyAsync(c->d_meta, h, c->meta_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaEventRecord(c->meta_done[sl], st) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    const size_t qb = (size_t)n * c->num_q_heads * c->head_dim * elt(c->kv_dtype);
+    const size_t kb = (size_t)n * c->num_kv_heads * c->head_dim * elt(c->kv_dtype);
+    if (cudaMemcpyAsync(c->d_q, q_host, qb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(c->d_k, k_host, kb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(c->d_v, v_host, kb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    const int64_t* d_slots = reinterpret_cast<const int64_t*>(c->d_meta);
+    const int64_t* d_src = d_slots + S;
+    const int64_t* d_dst = d_src + S;
+    const int32_t* d_tables = reinterpret_cast<const int32_t*>(d_dst + S);
+    const int32_t* d_lens = d_tables + S * c->max_blocks;
+    // 3. the kernels
+    if (ncopy > 0) {
+        s = pkv_copy_blocks(k_cache, v_cache, c->kv_dtype, d_src, d_dst, ncopy, 16, c->num_kv_heads, c->head_dim,
+                            num_blocks, stream);
+        if (s != PKV_OK) return s;
+    }
+    s = pkv_reshape_and_cache(c->d_k, c->d_v, k_cache, v_cache, c->kv_dtype, d_slots, n, c->num_kv_heads,
+                              c->head_dim, 16, num_blocks, stream);
+    if (s != PKV_OK) return s;
+    // workspace sized at creation for max_seqs and the table capacity; this call asks for the
+    // same schedule over n sequences, which never needs more
+    s = pkv_paged_attention_decode(c->d_out, c->out_dtype, c->d_q, k_cache, v_cache, c->kv_dtype, d_tables, d_lens,
+                                   scale, n, c->num_q_heads, c->num_kv_heads, c->head_dim, 16, c->max_blocks,
+                                   num_blocks, max_len, partition_tokens, c->d_ws, c->ws_bytes, stream);
+    if (s != PKV_OK) return s;
+    // 4. the result back to the host
+    const size_t ob = (size_t)n * c->num_q_heads * c->head_dim * elt(c->out_dtype);
+    if (cudaMemcpyAsync(out_host, c->d_out, ob, cudaMemcpyDeviceToHost, st) != cudaSuccess) return PKV_ERR_CUDA;
+    return PKV_OK;
+}
+
+}  // extern "C"
