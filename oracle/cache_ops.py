@@ -43,3 +43,16 @@ def copy_blocks(k_cache, v_cache, src, dst):
     for i, d in enumerate(dst):
         k_cache[d] = snap_k[i]
         v_cache[d] = snap_v[i]
+
+
+def reshape_and_cache_fp8(k, v, k_codes, v_codes, slot_mapping, k_scale: float, v_scale: float):
+    """KV append into an FP8 (e4m3) cache: token t's K (V) is stored as the
+    codes of float32(k[t] * inv_scale) (see oracle.fp8). Caches hold uint8 codes."""
+    from oracle import fp8
+    bs = int(k_codes.shape[1])
+    for t, slot in enumerate(np.asarray(slot_mapping).tolist()):
+        if slot < 0:
+            continue
+        b, o = divmod(int(slot), bs)
+        k_codes[b, o] = fp8.quantize(k[t], k_scale)
+        v_codes[b, o] = fp8.quantize(v[t], v_scale)

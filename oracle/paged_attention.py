@@ -60,3 +60,24 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
         V = gather_logical(v_cache, block_tables[s], ctx, block_size)
         out[i] = attend(q[s], K, V, float(scale))
     return out
+
+
+def paged_attention_decode_fp8(q, k_codes, v_codes, block_tables, context_lens, scale, block_size: int,
+                               k_scale: float, v_scale: float, seqs=None) -> np.ndarray:
+    """Decode attention over an FP8 (e4m3) cache: the logical K/V are the
+    dequantised cache values decode(code) * scale (oracle.fp8), then the same
+    fp64 attention as paged_attention_decode."""
+    from oracle import fp8
+    q = np.asarray(q)
+    idx = range(q.shape[0]) if seqs is None else [int(s) for s in seqs]
+    out = np.zeros((len(idx), q.shape[1], q.shape[2]), dtype=np.float64)
+    for i, s in enumerate(idx):
+        ctx = int(context_lens[s])
+        n_blk = -(-ctx // int(block_size))
+        ids = np.asarray(block_tables[s][:n_blk], dtype=np.int64)
+        kb = fp8.dequantize(np.asarray(k_codes[ids]), k_scale)
+        vb = fp8.dequantize(np.asarray(v_codes[ids]), v_scale)
+        K = kb.reshape((n_blk * block_size,) + kb.shape[2:])[:ctx]
+        V = vb.reshape((n_blk * block_size,) + vb.shape[2:])[:ctx]
+        out[i] = attend(q[s], K, V, float(scale))
+    return out
