@@ -232,15 +232,15 @@ def kernel_source_sha1() -> str:
 def attention_bytes(w: wl.Workload, lens_after: np.ndarray, out_elt: int) -> int:
     eb = w.elt_bytes
     kv = int(lens_after.sum()) * w.num_kv_heads * w.head_dim * eb * 2
-    q = w.num_seqs * w.num_q_heads * w.head_dim * eb
+    q = w.num_seqs * w.num_q_heads * w.head_dim * w.in_bytes
     out = w.num_seqs * w.num_q_heads * w.head_dim * out_elt
     tables = int(sum(-(-int(n) // w.block_size) for n in lens_after)) * 4
     return kv + q + out + tables + 4 * w.num_seqs
 
 
 def append_bytes(w: wl.Workload) -> int:
-    row = w.num_kv_heads * w.head_dim * w.elt_bytes
-    return w.num_seqs * (2 * row * 2 + 8)          # K and V rows read and written, slot ids
+    n = w.num_kv_heads * w.head_dim
+    return w.num_seqs * (2 * n * (w.in_bytes + w.elt_bytes) + 8)   # K and V rows read and written, slot ids
 
 
 # ---------------------------------------------------------------------------
@@ -262,12 +262,13 @@ def run_pkv(args, ws, rank, local):
     K, W = args.steps, args.warmup
     total_steps = 2 * (K + W) + 2
     lens0 = wl.context_lens(w)
-    dt = torch.float32 if w.kv_dtype == "f32" else torch.bfloat16
+    dt = torch.float32 if w.kv_dtype == "f32" else torch.bfloat16       # q and the appended K/V
+    cdt = torch.uint8 if w.kv_dtype == "fp8" else dt                     # cache storage
     mb = -(-int(lens0.max() + total_steps) // w.block_size)
 
     # ---- set-up (untimed): prompts into the cache through the library ----
-    cache = PagedKVCache(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, dt, dev,
-                         free_order=wl.free_order(w), max_blocks_per_seq=mb)
+    cache = PagedKVCache(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, cdt, dev,
+                         free_order=wl.free_order(w), max_blocks_per_seq=mb, kv_scales=(w.kv_scale, w.kv_scale))
     kvs = wl.prompt_kv_all(w, lens0)
     for s in range(w.num_seqs):
         k, v = kvs[s]
@@ -301,11 +302,11 @@ def run_pkv(args, ws, rank, local):
     maxctx = max(s["maxlen"] for s in steps)
 
     def step_device(st, ev0=None, ev1=None):
-        binding.reshape_and_cache(st["kn"], st["vn"], cache.k_cache, cache.v_cache, st["slots"])
+        cache.append(st["kn"], st["vn"], st["slots"])
         if ev0 is not None:
             ev0.record(stream)
-        binding.paged_attention_decode(out, st["q"], cache.k_cache, cache.v_cache, st["tables"], st["lens"],
-                                       w.scale, max_context_len=maxctx, partition_tokens=part, workspace=workspace)
+        cache.attention(out, st["q"], st["tables"], st["lens"], w.scale, max_context_len=maxctx,
+                        partition_tokens=part, workspace=workspace)
         if ev1 is not None:
             ev1.record(stream)
 
@@ -348,7 +349,7 @@ def run_pkv(args, ws, rank, local):
         out_host = torch.empty((w.num_seqs, w.num_q_heads, w.head_dim), dtype=torch.bfloat16).pin_memory()
         native = binding.DecodeStep(cache.bm, cache.k_cache, cache.v_cache, max_seqs=w.num_seqs,
                                     num_q_heads=w.num_q_heads, max_blocks_per_seq=mb, out_dtype=torch.bfloat16,
-                                    partition_tokens=part)
+                                    partition_tokens=part, kv_scales=(w.kv_scale, w.kv_scale))
         e2e_bytes = []
 
         def step_host(hq, hk, hv):
@@ -371,7 +372,7 @@ def run_pkv(args, ws, rank, local):
         barrier(ws)
         assert binding.get_device_error() == 0
         e_ms, e_gbs, e_tok = aggregate(e0.elapsed_time(e1), float(sum(e2e_bytes)), float(w.num_seqs * K), ws)
-        eb = w.elt_bytes
+        eb = w.in_bytes
         h2d = (w.num_seqs * w.num_q_heads * w.head_dim * eb + 2 * w.num_seqs * w.num_kv_heads * w.head_dim * eb +
                w.num_seqs * (3 * 8 + mb * 4 + 4))
         d2h = w.num_seqs * w.num_q_heads * w.head_dim * 2
@@ -434,11 +435,17 @@ def cpu_baseline(w: wl.Workload, target_s: float):
             kc = np.zeros((nblk, w.block_size, w.num_kv_heads, w.head_dim), np.float32)
             vc = np.zeros_like(kc)
             t0 = time.perf_counter()
-            ocache.reshape_and_cache(k, v, kc, vc, np.asarray(bm.allocate(0, n)))
-            oattn.paged_attention_decode(q[s:s + 1], kc, vc, [bm.block_table(0)], [n], w.scale, w.block_size)
+            if w.kv_dtype == "fp8":
+                kc, vc = kc.astype(np.uint8), vc.astype(np.uint8)
+                ocache.reshape_and_cache_fp8(k, v, kc, vc, np.asarray(bm.allocate(0, n)), w.kv_scale, w.kv_scale)
+                oattn.paged_attention_decode_fp8(q[s:s + 1], kc, vc, [bm.block_table(0)], [n], w.scale,
+                                                 w.block_size, w.kv_scale, w.kv_scale)
+            else:
+                ocache.reshape_and_cache(k, v, kc, vc, np.asarray(bm.allocate(0, n)))
+                oattn.paged_attention_decode(q[s:s + 1], kc, vc, [bm.block_table(0)], [n], w.scale, w.block_size)
             t_total += time.perf_counter() - t0
             done += 1
-            nbytes += n * w.num_kv_heads * w.head_dim * w.elt_bytes * 2 + 2 * w.num_q_heads * w.head_dim * w.elt_bytes
+            nbytes += n * w.num_kv_heads * w.head_dim * w.elt_bytes * 2 + 2 * w.num_q_heads * w.head_dim * w.in_bytes
             if t_total >= target_s:
                 break
         step += 1

@@ -69,7 +69,11 @@ typedef enum pkv_status {
     PKV_ERR_DEVICE_TIMEOUT = 6   /* (device word) a bounded wait inside a kernel gave up */
 } pkv_status;
 
-typedef enum pkv_dtype { PKV_F32 = 0, PKV_BF16 = 1 } pkv_dtype;
+typedef enum pkv_dtype {
+    PKV_F32 = 0,
+    PKV_BF16 = 1,
+    PKV_FP8_E4M3 = 2     /* cache storage only: 8-bit e4m3 codes with a per-tensor scale */
+} pkv_dtype;
 
 /* partition_tokens value selecting the persistent schedule of the decode call. */
 #define PKV_SCHEDULE_PERSISTENT (-1)
@@ -118,6 +122,23 @@ pkv_status pkv_paged_attention_decode(
     void* out, pkv_dtype out_dtype,
     const void* q, const void* k_cache, const void* v_cache, pkv_dtype kv_dtype,
     const int32_t* block_tables, const int32_t* context_lens, float scale,
+    int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+    int block_size, int max_blocks_per_seq, int num_blocks,
+    int max_context_len, int partition_tokens,
+    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Decode attention over an FP8 (e4m3) cache written by pkv_reshape_and_cache_fp8
+ * ("vLLM PagedAttention 深度解析" §7.4). Same computation and arguments as
+ * pkv_paged_attention_decode with K = decode(k code) * k_scale and
+ * V = decode(v code) * v_scale; q is bf16 [num_seqs, num_q_heads, head_dim]
+ * (converted to f16 for the tensor-core path, so |q| should stay below 65504).
+ * head_dim 128; partition_tokens >= 0 (the persistent schedule is not built for
+ * fp8). The workspace rule is pkv_paged_attention_workspace_bytes's.
+ */
+pkv_status pkv_paged_attention_decode_fp8(
+    void* out, pkv_dtype out_dtype, const void* q, const void* k_cache, const void* v_cache,
+    float k_scale, float v_scale, const int32_t* block_tables, const int32_t* context_lens, float scale,
     int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
     int block_size, int max_blocks_per_seq, int num_blocks,
     int max_context_len, int partition_tokens,
@@ -206,7 +227,7 @@ pkv_status pkv_reshape_and_cache(
  * for i < num_pairs, every slot of the block. Destination ids must be distinct
  * and must not appear among the sources of the same call (the copies run in
  * parallel). Ids outside [0, num_blocks) are skipped and flagged
- * PKV_ERR_DEVICE_BOUNDS.
+ * PKV_ERR_DEVICE_BOUNDS. dtype may be PKV_FP8_E4M3 (1-byte elements).
  *
  *   src_block_ids, dst_block_ids  device int64 [num_pairs]
  * num_pairs may be 0 (nothing is launched).
@@ -215,6 +236,21 @@ pkv_status pkv_copy_blocks(
     void* k_cache, void* v_cache, pkv_dtype dtype,
     const int64_t* src_block_ids, const int64_t* dst_block_ids, int num_pairs,
     int block_size, int num_kv_heads, int head_dim, int num_blocks, void* stream);
+
+/*
+ * FP8 KV append ("vLLM PagedAttention 深度解析" §7.4: K/V stored as FP8 so a block
+ * holds twice the tokens). Same addressing as pkv_reshape_and_cache; the caches
+ * hold e4m3 codes (1 byte per element) and the stored code of an element x is
+ * e4m3(float32(x * float32(1 / scale))), rounded to nearest even, finite values
+ * beyond the e4m3 range saturating to +-448. The value a code stands for is
+ * decode(code) * scale. One scale per tensor: k_scale for K, v_scale for V
+ * (finite, > 0). k, v are bf16 or f32 (in_dtype), [num_tokens, Hkv, D];
+ * Hkv * D must be a multiple of 16.
+ */
+pkv_status pkv_reshape_and_cache_fp8(
+    const void* k, const void* v, pkv_dtype in_dtype, void* k_cache, void* v_cache,
+    float k_scale, float v_scale, const int64_t* slot_mapping, int num_tokens,
+    int num_kv_heads, int head_dim, int block_size, int num_blocks, void* stream);
 
 /*
  * Reads and clears the current device's error word (0 or a pkv_status code set
@@ -236,9 +272,12 @@ pkv_status pkv_get_device_error(int* code, void* stream);
 typedef struct pkv_step_ctx pkv_step_ctx;
 typedef struct pkv_block_manager pkv_block_manager;
 
+/* kv_dtype PKV_FP8_E4M3: the caches hold e4m3 codes, the step's q / new K,V
+ * are bf16 on the host, and k_scale / v_scale are the per-tensor scales
+ * (ignored for f32 / bf16 caches). */
 pkv_status pkv_step_ctx_create(int max_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                int max_blocks_per_seq, pkv_dtype kv_dtype, pkv_dtype out_dtype,
-                               int partition_tokens, pkv_step_ctx** out);
+                               int partition_tokens, float k_scale, float v_scale, pkv_step_ctx** out);
 void pkv_step_ctx_destroy(pkv_step_ctx* ctx);
 
 /*

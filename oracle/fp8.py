@@ -86,8 +86,29 @@ def encode(x: float) -> int:
 
 
 def encode_array(x) -> np.ndarray:
-    flat = np.asarray(x, dtype=np.float64).ravel()
-    return np.array([encode(v) for v in flat], dtype=np.uint8).reshape(np.shape(x))
+    """encode() applied elementwise, written with array operations: the binade
+    from frexp (subnormals share the lowest binade's quantum 2^-9), the
+    significand rounded half to even (np.rint), a carry into the next binade,
+    then saturation, zeros, signs and NaN as in encode()."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    with np.errstate(invalid="ignore", over="ignore"):
+        _, e = np.frexp(a)
+        e = np.maximum(e.astype(np.int64) - 1, 1 - _BIAS)        # floor(log2 a), at least -6
+        n = np.rint(a / np.ldexp(1.0, e - 3))                    # significand in quanta
+        carry = n >= 16
+        e = np.where(carry, e + 1, e)
+        n = np.where(carry, 8, n)
+        value = n * np.ldexp(1.0, e - 3)
+        sat = ~(value <= MAX_E4M3) | np.isinf(a)                # beyond 448, infinity
+    n = np.where(np.isfinite(n), n, 0).astype(np.int64)
+    sub = (e == 1 - _BIAS) & (n < 8)
+    code = np.where(sub, n, ((e + _BIAS) << 3) | np.maximum(n - 8, 0))
+    code = np.where(sat, 0x7E, code)
+    code = np.where(a == 0, 0, code)
+    code = code | (np.signbit(x).astype(np.int64) << 7)
+    code = np.where(np.isnan(x), 0x7F, code)
+    return code.astype(np.uint8)
 
 
 def quantize(x, scale: float) -> np.ndarray:

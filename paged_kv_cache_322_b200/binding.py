@@ -17,7 +17,7 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpkv.so")
 
-PKV_F32, PKV_BF16 = 0, 1
+PKV_F32, PKV_BF16, PKV_FP8_E4M3 = 0, 1, 2
 STATUS = {0: "PKV_OK", 1: "PKV_ERR_INVALID_ARG", 2: "PKV_ERR_UNSUPPORTED", 3: "PKV_ERR_CUDA",
           4: "PKV_ERR_DEVICE_BOUNDS", 5: "PKV_ERR_OUT_OF_BLOCKS", 6: "PKV_ERR_DEVICE_TIMEOUT"}
 
@@ -40,12 +40,16 @@ _SIGS = {
                                           _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp]),
     "pkv_paged_attention_decode_noalloc": (_i32, [_vp, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _f32, _i32, _i32, _i32,
                                                   _i32, _i32, _i32, _i32, _i32, _i32, _vp]),
+    "pkv_paged_attention_decode_fp8": (_i32, [_vp, _i32, _vp, _vp, _vp, _f32, _f32, _vp, _vp, _f32, _i32, _i32, _i32,
+                                              _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp]),
+    "pkv_reshape_and_cache_fp8": (_i32, [_vp, _vp, _i32, _vp, _vp, _f32, _f32, _vp, _i32, _i32, _i32, _i32, _i32,
+                                         _vp]),
     "pkv_paged_attention_workspace_bytes": (_sz, [_i32] * 8),
     "pkv_paged_attention_partition_tokens": (_i32, [_i32] * 8),
     "pkv_reshape_and_cache": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pkv_copy_blocks": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pkv_get_device_error": (_i32, [_c.POINTER(_c.c_int), _vp]),
-    "pkv_step_ctx_create": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _c.POINTER(_vp)]),
+    "pkv_step_ctx_create": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _f32, _c.POINTER(_vp)]),
     "pkv_step_ctx_destroy": (None, [_vp]),
     "pkv_decode_step": (_i32, [_vp, _vp, _pi64, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _f32, _i32, _vp, _vp]),
     "pkv_bm_create": (_i32, [_i32, _i32, _pi32, _c.POINTER(_vp)]),
@@ -100,12 +104,15 @@ def _torch():
 
 
 def _dtype_code(t) -> int:
+    """float32 / bfloat16 tensors; uint8 tensors hold FP8 (e4m3) cache codes."""
     torch = _torch()
     if t.dtype == torch.float32:
         return PKV_F32
     if t.dtype == torch.bfloat16:
         return PKV_BF16
-    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+    if t.dtype == torch.uint8:
+        return PKV_FP8_E4M3
+    raise TypeError(f"unsupported dtype {t.dtype} (float32, bfloat16, or uint8 for FP8 codes)")
 
 
 def _stream(t, stream) -> int:
@@ -214,6 +221,53 @@ def reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, stream=None):
     _check(st, "pkv_reshape_and_cache")
 
 
+def reshape_and_cache_fp8(k, v, k_cache, v_cache, slot_mapping, k_scale: float, v_scale: float, stream=None):
+    """FP8 (e4m3) append: k, v [T, Hkv, D] bf16 or f32 are quantised into uint8
+    caches of codes, code = e4m3(x * (1 / scale)), saturating at +-448."""
+    torch = _torch()
+    _cuda_contig(k, v, k_cache, v_cache, slot_mapping)
+    if slot_mapping.dtype != torch.int64 or k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8:
+        raise TypeError("slot_mapping int64, caches uint8 (FP8 codes)")
+    nb, bs, hkv, d = k_cache.shape
+    T = k.shape[0]
+    if tuple(k.shape) != (T, hkv, d) or tuple(v.shape) != (T, hkv, d) or slot_mapping.numel() != T:
+        raise ValueError("shape mismatch")
+    if k.dtype != v.dtype:
+        raise TypeError("k and v must share a dtype")
+    st = _lib().pkv_reshape_and_cache_fp8(k.data_ptr(), v.data_ptr(), _dtype_code(k), k_cache.data_ptr(),
+                                          v_cache.data_ptr(), float(k_scale), float(v_scale), slot_mapping.data_ptr(),
+                                          T, hkv, d, bs, nb, _stream(k_cache, stream))
+    _check(st, "pkv_reshape_and_cache_fp8")
+
+
+def paged_attention_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, scale: float, k_scale: float,
+                               v_scale: float, max_context_len: int = 0, partition_tokens: int = 0, workspace=None,
+                               stream=None):
+    """Decode attention over uint8 FP8 caches (K = code value * k_scale, V likewise); q bf16."""
+    torch = _torch()
+    _cuda_contig(out, q, k_cache, v_cache, block_tables, context_lens)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    if q.dtype != torch.bfloat16 or k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8:
+        raise TypeError("q bfloat16, caches uint8 (FP8 codes)")
+    B, hq, d = q.shape
+    nb, bs, hkv, d2 = k_cache.shape
+    if d2 != d or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != (B, hq, d):
+        raise ValueError("shape mismatch")
+    mb = block_tables.shape[1]
+    need = workspace_bytes(B, hq, hkv, d, bs, mb, max_context_len, partition_tokens)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_n = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = _lib().pkv_paged_attention_decode_fp8(
+        out.data_ptr(), _dtype_code(out), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), float(k_scale),
+        float(v_scale), block_tables.data_ptr(), context_lens.data_ptr(), float(scale), B, hq, hkv, d, bs, mb, nb,
+        int(max_context_len), int(partition_tokens), ws_ptr, ws_n, _stream(q, stream))
+    _check(st, "pkv_paged_attention_decode_fp8")
+    return out
+
+
 def copy_blocks(k_cache, v_cache, src, dst, stream=None):
     """cache[dst[i]] = cache[src[i]] for K and V (src, dst int64 CUDA tensors)."""
     torch = _torch()
@@ -314,7 +368,7 @@ class DecodeStep:
     append, attention, D2H of the output -- one C call per step."""
 
     def __init__(self, bm: BlockManager, k_cache, v_cache, max_seqs: int, num_q_heads: int,
-                 max_blocks_per_seq: int, out_dtype, partition_tokens: int = 0):
+                 max_blocks_per_seq: int, out_dtype, partition_tokens: int = 0, kv_scales=(1.0, 1.0)):
         torch = _torch()
         self.bm, self.k_cache, self.v_cache = bm, k_cache, v_cache
         nb, bs, hkv, d = k_cache.shape
@@ -326,7 +380,8 @@ class DecodeStep:
         self._h = ctypes.c_void_p()
         _check(_lib().pkv_step_ctx_create(max_seqs, num_q_heads, hkv, d, max_blocks_per_seq, _dtype_code(k_cache),
                                           PKV_F32 if out_dtype == torch.float32 else PKV_BF16,
-                                          partition_tokens, ctypes.byref(self._h)), "pkv_step_ctx_create")
+                                          partition_tokens, float(kv_scales[0]), float(kv_scales[1]),
+                                          ctypes.byref(self._h)), "pkv_step_ctx_create")
 
     def __del__(self):
         h = getattr(self, "_h", None)

@@ -23,7 +23,8 @@ struct Params {
     float* ws_o;        // [B, Hq, C, D] partition outputs (normalised)
     float* ws_ml;       // [B, Hq, C, 2] partition (m, l), m in log2 units
     int* err;
-    float scale_log2;   // scale * log2(e)
+    float scale_log2;   // scale * log2(e) (times the K scale for an fp8 cache)
+    float out_scale;    // 1, or the V scale for an fp8 cache
     int out_f32;
     int num_q_heads, num_kv_heads, group;
     int max_blocks, num_blocks;
@@ -43,15 +44,22 @@ __device__ __forceinline__ void consumers_barrier() {
 }
 
 __device__ __forceinline__ void store_out(const Params& p, int64_t idx, float v) {
+    v *= p.out_scale;
     if (p.out_f32) static_cast<float*>(p.out)[idx] = v;
     else static_cast<__nv_bfloat16*>(p.out)[idx] = __float2bfloat16_rn(v);
+}
+
+template <typename TQ>
+__device__ __forceinline__ float to_float(TQ x) {
+    if constexpr (sizeof(TQ) == 4) return x;
+    else return __bfloat162float(x);
 }
 
 // ---------------------------------------------------------------------------
 // SIMT consumer: HPW query heads per warp, 8 lanes per token, 4 tokens per
 // round, fp32 math. T = float or __nv_bfloat16.
 // ---------------------------------------------------------------------------
-template <typename T, int D, int HPW>
+template <typename T, int D, int HPW, typename TQ = T>
 struct SimtConsumer {
     static constexpr int RB = D * (int)sizeof(T);          // row bytes
     static constexpr int NCH = RB / 16;                     // 16-byte chunks per row
@@ -66,7 +74,15 @@ struct SimtConsumer {
     float m[HPW], l[HPW];
 
     __device__ __forceinline__ static void unpack(const uint4& raw, float* f) {
-        if constexpr (sizeof(T) == 4) {
+        if constexpr (sizeof(T) == 1) {          // 16 e4m3 codes
+            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 a = f16x2_to_float2(e4m3x2_to_f16x2(w[i] & 0xffffu));
+                const float2 b = f16x2_to_float2(e4m3x2_to_f16x2(w[i] >> 16));
+                f[4 * i] = a.x; f[4 * i + 1] = a.y; f[4 * i + 2] = b.x; f[4 * i + 3] = b.y;
+            }
+        } else if constexpr (sizeof(T) == 4) {
             f[0] = __uint_as_float(raw.x); f[1] = __uint_as_float(raw.y);
             f[2] = __uint_as_float(raw.z); f[3] = __uint_as_float(raw.w);
         } else {
@@ -76,18 +92,16 @@ struct SimtConsumer {
     }
 
     // q_rows points at query head (first head of this warp) of this sequence.
-    __device__ __forceinline__ void init(const T* q_rows, float scale_log2, int lane) {
+    // Lane li holds dims (c * 8 + li) * EPC + e of each head, the dims it reads of K and V.
+    __device__ __forceinline__ void init(const TQ* q_rows, float scale_log2, int lane) {
         const int li = lane & 7;
 #pragma unroll
         for (int h = 0; h < HPW; ++h) {
-            const uint4* row = reinterpret_cast<const uint4*>(q_rows + (int64_t)h * D);
 #pragma unroll
-            for (int c = 0; c < CPL; ++c) {
-                float f[EPC];
-                unpack(row[c * 8 + li], f);
+            for (int c = 0; c < CPL; ++c)
 #pragma unroll
-                for (int e = 0; e < EPC; ++e) q[h][c * EPC + e] = f[e] * scale_log2;
-            }
+                for (int e = 0; e < EPC; ++e)
+                    q[h][c * EPC + e] = to_float(q_rows[(int64_t)h * D + (c * 8 + li) * EPC + e]) * scale_log2;
 #pragma unroll
             for (int e = 0; e < EPL; ++e) acc[h][e] = 0.f;
             m[h] = kNegInf;
@@ -329,6 +343,167 @@ struct MmaConsumer {
     }
 };
 
+
+// ---------------------------------------------------------------------------
+// Tensor-core consumer for an FP8 (e4m3) cache, D = 128, up to 8 query heads.
+// The K and V tiles are 16 rows x 128 bytes, TMA-written with the 128-byte
+// swizzle. ldmatrix reads the codes as 16-bit pairs and cvt turns each pair
+// into f16x2 exactly; the MMAs run in f16 (q is converted once; P split into
+// f16 high + low parts).
+//   S^T = K Q^T: thread (g, t) gets the codes of dims 4t..4t+3 of a 16-dim
+//   chunk; they serve as the fragment's k slots 2t, 2t+1, 2t+8, 2t+9, and Q's
+//   B fragment is built with the same dim order, so the dot products are
+//   unchanged.
+//   O^T += V^T P^T: ldmatrix.trans gives a thread two dims (2g, 2g+1) of two
+//   tokens; a byte permute splits them into the even-dim row (fragment row g)
+//   and the odd-dim row (fragment row g + 8), so each 16-dim chunk is one MMA
+//   whose output rows are dims 2g and 2g + 1.
+// ---------------------------------------------------------------------------
+struct MmaConsumerFp8 {
+    static constexpr int D = 128;
+    static constexpr int NCHUNK = D / 16;
+
+    uint32_t qb[NCHUNK][2];
+    float o[NCHUNK][4];
+    float m0, m1, l0, l1;
+
+    __device__ __forceinline__ static uint32_t f16pair(float a, float b) {
+        return pack_f16(fminf(fmaxf(a, -65504.f), 65504.f), fminf(fmaxf(b, -65504.f), 65504.f));
+    }
+
+    __device__ __forceinline__ void init(const __nv_bfloat16* q_rows, int group, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+        for (int ks = 0; ks < NCHUNK; ++ks) {
+            if (g < group) {
+                const uint2 w = *reinterpret_cast<const uint2*>(q_rows + (int64_t)g * D + 16 * ks + 4 * t);
+                qb[ks][0] = f16pair(bf16lo(w.x), bf16hi(w.x));
+                qb[ks][1] = f16pair(bf16lo(w.y), bf16hi(w.y));
+            } else {
+                qb[ks][0] = qb[ks][1] = 0u;
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < NCHUNK; ++c) o[c][0] = o[c][1] = o[c][2] = o[c][3] = 0.f;
+        m0 = m1 = kNegInf;
+        l0 = l1 = 0.f;
+    }
+
+    __device__ __forceinline__ void consume(uint32_t ks_base, uint32_t vs_base, uint8_t* vs_ptr, int nvalid,
+                                            float scale_log2, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+        if (nvalid < BS) {          // rows past the context: zero V codes (0 * NaN would poison O)
+            for (int i = lane; i < (BS - nvalid) * 8; i += 32) {
+                const int r = nvalid + i / 8, c = i % 8;
+                *reinterpret_cast<uint4*>(vs_ptr + r * 128 + ((c ^ (r & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            __syncwarp();
+        }
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        const int mi = lane >> 3;
+        const int row = (lane & 7) + ((mi & 1) << 3);
+#pragma unroll
+        for (int kp = 0; kp < NCHUNK / 2; ++kp) {
+            const int chunk = 2 * kp + (mi >> 1);
+            uint32_t r0, r1, r2, r3;
+            ldmatrix_x4(r0, r1, r2, r3, ks_base + row * 128 + ((chunk ^ (row & 7)) << 4));
+            mma_f16_16816(s, e4m3x2_to_f16x2(r0 & 0xffffu), e4m3x2_to_f16x2(r1 & 0xffffu), e4m3x2_to_f16x2(r0 >> 16),
+                          e4m3x2_to_f16x2(r1 >> 16), qb[2 * kp][0], qb[2 * kp][1]);
+            mma_f16_16816(s, e4m3x2_to_f16x2(r2 & 0xffffu), e4m3x2_to_f16x2(r3 & 0xffffu), e4m3x2_to_f16x2(r2 >> 16),
+                          e4m3x2_to_f16x2(r3 >> 16), qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
+        }
+        float x0 = g < nvalid ? s[0] * scale_log2 : kNegInf;
+        float x1 = g < nvalid ? s[1] * scale_log2 : kNegInf;
+        float x2 = g + 8 < nvalid ? s[2] * scale_log2 : kNegInf;
+        float x3 = g + 8 < nvalid ? s[3] * scale_log2 : kNegInf;
+        float b0 = fmaxf(x0, x2), b1 = fmaxf(x1, x3);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            b0 = fmaxf(b0, __shfl_xor_sync(0xffffffffu, b0, off));
+            b1 = fmaxf(b1, __shfl_xor_sync(0xffffffffu, b1, off));
+        }
+        const float n0 = fmaxf(m0, b0), n1 = fmaxf(m1, b1);
+        const float al0 = fast_exp2(m0 - n0), al1 = fast_exp2(m1 - n1);
+        m0 = n0;
+        m1 = n1;
+        const float p0 = fast_exp2(x0 - n0), p1 = fast_exp2(x1 - n1);
+        const float p2 = fast_exp2(x2 - n0), p3 = fast_exp2(x3 - n1);
+        l0 = l0 * al0 + (p0 + p2);
+        l1 = l1 * al1 + (p1 + p3);
+#pragma unroll
+        for (int c = 0; c < NCHUNK; ++c) {
+            o[c][0] *= al0; o[c][1] *= al1; o[c][2] *= al0; o[c][3] *= al1;
+        }
+        const uint32_t h02 = pack_f16(p0, p2), h13 = pack_f16(p1, p3);
+        const float2 f02 = f16x2_to_float2(h02), f13 = f16x2_to_float2(h13);
+        const uint32_t e02 = pack_f16(p0 - f02.x, p2 - f02.y), e13 = pack_f16(p1 - f13.x, p3 - f13.y);
+        const int srcA = (2 * t) * 4 + (g >> 1), srcB = srcA + 4;
+        const bool odd = g & 1;
+        uint32_t ya, yb, za, zb;
+        {
+            const uint32_t u0 = __shfl_sync(0xffffffffu, h02, srcA), u1 = __shfl_sync(0xffffffffu, h13, srcA);
+            const uint32_t v0 = __shfl_sync(0xffffffffu, h02, srcB), v1 = __shfl_sync(0xffffffffu, h13, srcB);
+            ya = odd ? u1 : u0;
+            yb = odd ? v1 : v0;
+        }
+        {
+            const uint32_t u0 = __shfl_sync(0xffffffffu, e02, srcA), u1 = __shfl_sync(0xffffffffu, e13, srcA);
+            const uint32_t v0 = __shfl_sync(0xffffffffu, e02, srcB), v1 = __shfl_sync(0xffffffffu, e13, srcB);
+            za = odd ? u1 : u0;
+            zb = odd ? v1 : v0;
+        }
+        const uint32_t bh0 = __byte_perm(ya, yb, 0x5410), bh1 = __byte_perm(ya, yb, 0x7632);
+        const uint32_t bl0 = __byte_perm(za, zb, 0x5410), bl1 = __byte_perm(za, zb, 0x7632);
+        const int tok = (lane & 7) + ((mi & 1) << 3);
+#pragma unroll
+        for (int cp = 0; cp < NCHUNK / 2; ++cp) {
+            const int chunk = 2 * cp + (mi >> 1);
+            uint32_t r0, r1, r2, r3;
+            ldmatrix_x4_trans(r0, r1, r2, r3, vs_base + tok * 128 + ((chunk ^ (tok & 7)) << 4));
+            // r0: tokens 0-7 of chunk 2cp, r1: tokens 8-15 of it; r2, r3: chunk 2cp + 1
+            {
+                const uint32_t x = __byte_perm(r0, 0u, 0x3120), y = __byte_perm(r1, 0u, 0x3120);
+                const uint32_t a0 = e4m3x2_to_f16x2(x & 0xffffu), a1 = e4m3x2_to_f16x2(x >> 16);
+                const uint32_t a2 = e4m3x2_to_f16x2(y & 0xffffu), a3 = e4m3x2_to_f16x2(y >> 16);
+                mma_f16_16816(o[2 * cp], a0, a1, a2, a3, bh0, bh1);
+                mma_f16_16816(o[2 * cp], a0, a1, a2, a3, bl0, bl1);
+            }
+            {
+                const uint32_t x = __byte_perm(r2, 0u, 0x3120), y = __byte_perm(r3, 0u, 0x3120);
+                const uint32_t a0 = e4m3x2_to_f16x2(x & 0xffffu), a1 = e4m3x2_to_f16x2(x >> 16);
+                const uint32_t a2 = e4m3x2_to_f16x2(y & 0xffffu), a3 = e4m3x2_to_f16x2(y >> 16);
+                mma_f16_16816(o[2 * cp + 1], a0, a1, a2, a3, bh0, bh1);
+                mma_f16_16816(o[2 * cp + 1], a0, a1, a2, a3, bl0, bl1);
+            }
+        }
+    }
+
+    __device__ __forceinline__ void finish(float* red_o, float* red_m, float* red_l, int group, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+        }
+        const int h0 = 2 * t, h1 = 2 * t + 1;
+#pragma unroll
+        for (int c = 0; c < NCHUNK; ++c) {
+            const int de = 16 * c + 2 * g;            // fragment rows g / g + 8 are dims de / de + 1
+            if (h0 < group) {
+                red_o[h0 * D + de] = o[c][0];
+                red_o[h0 * D + de + 1] = o[c][2];
+            }
+            if (h1 < group) {
+                red_o[h1 * D + de] = o[c][1];
+                red_o[h1 * D + de + 1] = o[c][3];
+            }
+        }
+        if (g == 0) {
+            if (h0 < group) { red_m[h0] = m0; red_l[h0] = l0; }
+            if (h1 < group) { red_m[h1] = m1; red_l[h1] = l1; }
+        }
+    }
+};
 
 // Persistent schedule (paged_attention_persistent.cu).
 cudaError_t launch_persistent(bool bf16, bool use_mma, int head_dim, int group, const CUtensorMap& mk,

@@ -6,6 +6,8 @@
 // physical block is one contiguous span of block_size*Hkv*D elements, so the
 // block copy is a span copy. Both move 16-byte vectors, several in flight per
 // thread, with non-allocating loads of the read-once source.
+#include <cmath>
+
 #include "common.cuh"
 
 namespace pkv {
@@ -45,6 +47,54 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     for (; i < row_vecs; i += 256) dst[i] = ld_stream(src + i);
 }
 
+// FP8 append: grid.x = token, grid.y = 0 (K) / 1 (V). Each thread turns 16
+// input elements (bf16 or fp32) into one 16-byte vector of e4m3 codes:
+// code = e4m3(x * inv_scale) with round to nearest even and saturation.
+template <typename TIn>
+__global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(
+    const TIn* __restrict__ k, const TIn* __restrict__ v, uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+    float k_inv, float v_inv, const int64_t* __restrict__ slot_mapping, int row_elems, int64_t num_slots, int* err) {
+    const int t = blockIdx.x;
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) return;
+    if (slot >= num_slots) {
+        if (threadIdx.x == 0) flag_error(err, PKV_ERR_DEVICE_BOUNDS);
+        return;
+    }
+    const bool is_k = blockIdx.y == 0;
+    const TIn* src = (is_k ? k : v) + (int64_t)t * row_elems;
+    uint4* dst = (is_k ? k_cache : v_cache) + slot * (row_elems / 16);
+    const float inv = is_k ? k_inv : v_inv;
+    for (int c = threadIdx.x; c < row_elems / 16; c += 256) {
+        float f[16];
+        if constexpr (sizeof(TIn) == 4) {
+            const float4* s4 = reinterpret_cast<const float4*>(src + c * 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 x = s4[i];
+                f[4 * i] = x.x; f[4 * i + 1] = x.y; f[4 * i + 2] = x.z; f[4 * i + 3] = x.w;
+            }
+        } else {
+            const uint4* s4 = reinterpret_cast<const uint4*>(src + c * 16);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const uint4 x = s4[i];
+                f[8 * i] = bf16lo(x.x); f[8 * i + 1] = bf16hi(x.x); f[8 * i + 2] = bf16lo(x.y);
+                f[8 * i + 3] = bf16hi(x.y); f[8 * i + 4] = bf16lo(x.z); f[8 * i + 5] = bf16hi(x.z);
+                f[8 * i + 6] = bf16lo(x.w); f[8 * i + 7] = bf16hi(x.w);
+            }
+        }
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = float2_to_e4m3x2(__fmul_rn(f[4 * i], inv), __fmul_rn(f[4 * i + 1], inv));
+            const uint32_t hi = float2_to_e4m3x2(__fmul_rn(f[4 * i + 2], inv), __fmul_rn(f[4 * i + 3], inv));
+            w[i] = lo | (hi << 16);
+        }
+        dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
 // grid.x = chunk of the block span (kChunkVecs vectors), grid.y = pair,
 // grid.z = 0 (K) / 1 (V).
 constexpr int kCopyThreads = 256;
@@ -78,7 +128,7 @@ __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int elt_bytes(pkv_dtype t) { return t == PKV_F32 ? 4 : (t == PKV_BF16 ? 2 : 0); }
+int elt_bytes(pkv_dtype t) { return t == PKV_F32 ? 4 : (t == PKV_BF16 ? 2 : (t == PKV_FP8_E4M3 ? 1 : 0)); }
 
 }  // namespace
 }  // namespace pkv
@@ -107,6 +157,35 @@ pkv_status pkv_reshape_and_cache(const void* k, const void* v, void* k_cache, vo
         static_cast<const int4*>(k), static_cast<const int4*>(v), static_cast<int4*>(k_cache),
         static_cast<int4*>(v_cache), slot_mapping, (int)(row_bytes / 16),
         (int64_t)num_blocks * block_size, err);
+    return cuda_status(cudaGetLastError());
+}
+
+pkv_status pkv_reshape_and_cache_fp8(const void* k, const void* v, pkv_dtype in_dtype, void* k_cache, void* v_cache,
+                                     float k_scale, float v_scale, const int64_t* slot_mapping, int num_tokens,
+                                     int num_kv_heads, int head_dim, int block_size, int num_blocks, void* stream) {
+    using namespace pkv;
+    if ((in_dtype != PKV_F32 && in_dtype != PKV_BF16) || num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0 || num_blocks <= 0 || !(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) ||
+        !std::isfinite(v_scale))
+        return PKV_ERR_INVALID_ARG;
+    const int64_t row = (int64_t)num_kv_heads * head_dim;
+    if (row % 16 != 0 || row > INT32_MAX) return PKV_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PKV_OK;
+    if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache)) return PKV_ERR_INVALID_ARG;
+    int* err = device_error_word();
+    if (!err) return PKV_ERR_CUDA;
+    const float k_inv = 1.0f / k_scale, v_inv = 1.0f / v_scale;
+    dim3 grid(num_tokens, 2);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (in_dtype == PKV_F32)
+        reshape_and_cache_fp8_kernel<float><<<grid, 256, 0, st>>>(
+            static_cast<const float*>(k), static_cast<const float*>(v), static_cast<uint4*>(k_cache),
+            static_cast<uint4*>(v_cache), k_inv, v_inv, slot_mapping, (int)row, (int64_t)num_blocks * block_size, err);
+    else
+        reshape_and_cache_fp8_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), static_cast<uint4*>(k_cache),
+            static_cast<uint4*>(v_cache), k_inv, v_inv, slot_mapping, (int)row, (int64_t)num_blocks * block_size, err);
     return cuda_status(cudaGetLastError());
 }
 

@@ -24,6 +24,7 @@
 struct pkv_step_ctx {
     int max_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks;
     pkv_dtype kv_dtype, out_dtype;
+    float k_scale = 1.f, v_scale = 1.f;   // FP8 caches
     size_t meta_bytes, q_bytes, kv_bytes, out_bytes, ws_bytes;
     // device
     unsigned char* d_meta = nullptr;   // slots i64[S] | src i64[S] | dst i64[S] | tables i32[S*MB] | lens i32[S]
@@ -41,7 +42,9 @@ struct pkv_step_ctx {
 
 namespace {
 
-int elt(pkv_dtype t) { return t == PKV_F32 ? 4 : 2; }
+int elt(pkv_dtype t) { return t == PKV_F32 ? 4 : (t == PKV_BF16 ? 2 : 1); }
+// host-side element size of the step's q / new K,V (bf16 for an FP8 cache)
+int in_elt(pkv_dtype t) { return t == PKV_F32 ? 4 : 2; }
 
 void release(pkv_step_ctx* c) {
     if (!c) return;
@@ -68,10 +71,12 @@ extern "C" {
 
 pkv_status pkv_step_ctx_create(int max_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                int max_blocks_per_seq, pkv_dtype kv_dtype, pkv_dtype out_dtype,
-                               int partition_tokens, pkv_step_ctx** out) {
+                               int partition_tokens, float k_scale, float v_scale, pkv_step_ctx** out) {
     if (!out || max_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
         max_blocks_per_seq <= 0 || num_q_heads % num_kv_heads != 0 ||
-        (kv_dtype != PKV_F32 && kv_dtype != PKV_BF16) || (out_dtype != PKV_F32 && out_dtype != PKV_BF16))
+        (kv_dtype != PKV_F32 && kv_dtype != PKV_BF16 && kv_dtype != PKV_FP8_E4M3) ||
+        (out_dtype != PKV_F32 && out_dtype != PKV_BF16) ||
+        (kv_dtype == PKV_FP8_E4M3 && !(k_scale > 0.f && v_scale > 0.f)))
         return PKV_ERR_INVALID_ARG;
     *out = nullptr;
     pkv_step_ctx* c = new (std::nothrow) pkv_step_ctx();
@@ -84,10 +89,12 @@ pkv_status pkv_step_ctx_create(int max_seqs, int num_q_heads, int num_kv_heads, 
     c->max_blocks = max_blocks_per_seq;
     c->kv_dtype = kv_dtype;
     c->out_dtype = out_dtype;
+    c->k_scale = k_scale;
+    c->v_scale = v_scale;
     const size_t S = (size_t)max_seqs;
     c->meta_bytes = S * 8 * 3 + S * max_blocks_per_seq * 4 + S * 4;
-    c->q_bytes = S * num_q_heads * head_dim * elt(kv_dtype);
-    c->kv_bytes = S * num_kv_heads * head_dim * elt(kv_dtype);
+    c->q_bytes = S * num_q_heads * head_dim * in_elt(kv_dtype);
+    c->kv_bytes = S * num_kv_heads * head_dim * in_elt(kv_dtype);
     c->out_bytes = S * num_q_heads * head_dim * elt(out_dtype);
     // Largest workspace any step can ask for: a fixed partition length never needs
     // more than at max_seqs and full tables; the library-chosen one is >= 256 tokens.
@@ -147,8 +154,8 @@ pkv_status pkv_decode_step(pkv_step_ctx* c, pkv_block_manager* bm, const int64_t
     if (cudaMemcpyAsync(c->d_meta, h, c->meta_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaEventRecord(c->meta_done[sl], st) != cudaSuccess)
         return PKV_ERR_CUDA;
-    const size_t qb = (size_t)n * c->num_q_heads * c->head_dim * elt(c->kv_dtype);
-    const size_t kb = (size_t)n * c->num_kv_heads * c->head_dim * elt(c->kv_dtype);
+    const size_t qb = (size_t)n * c->num_q_heads * c->head_dim * in_elt(c->kv_dtype);
+    const size_t kb = (size_t)n * c->num_kv_heads * c->head_dim * in_elt(c->kv_dtype);
     if (cudaMemcpyAsync(c->d_q, q_host, qb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(c->d_k, k_host, kb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(c->d_v, v_host, kb, cudaMemcpyHostToDevice, st) != cudaSuccess)
@@ -164,14 +171,22 @@ pkv_status pkv_decode_step(pkv_step_ctx* c, pkv_block_manager* bm, const int64_t
                             num_blocks, stream);
         if (s != PKV_OK) return s;
     }
-    s = pkv_reshape_and_cache(c->d_k, c->d_v, k_cache, v_cache, c->kv_dtype, d_slots, n, c->num_kv_heads,
-                              c->head_dim, 16, num_blocks, stream);
+    const bool fp8 = c->kv_dtype == PKV_FP8_E4M3;
+    s = fp8 ? pkv_reshape_and_cache_fp8(c->d_k, c->d_v, PKV_BF16, k_cache, v_cache, c->k_scale, c->v_scale, d_slots,
+                                        n, c->num_kv_heads, c->head_dim, 16, num_blocks, stream)
+            : pkv_reshape_and_cache(c->d_k, c->d_v, k_cache, v_cache, c->kv_dtype, d_slots, n, c->num_kv_heads,
+                                    c->head_dim, 16, num_blocks, stream);
     if (s != PKV_OK) return s;
     // workspace sized at creation for max_seqs and the table capacity; this call asks for the
     // same schedule over n sequences, which never needs more
-    s = pkv_paged_attention_decode(c->d_out, c->out_dtype, c->d_q, k_cache, v_cache, c->kv_dtype, d_tables, d_lens,
-                                   scale, n, c->num_q_heads, c->num_kv_heads, c->head_dim, 16, c->max_blocks,
-                                   num_blocks, max_len, partition_tokens, c->d_ws, c->ws_bytes, stream);
+    s = fp8 ? pkv_paged_attention_decode_fp8(c->d_out, c->out_dtype, c->d_q, k_cache, v_cache, c->k_scale,
+                                             c->v_scale, d_tables, d_lens, scale, n, c->num_q_heads, c->num_kv_heads,
+                                             c->head_dim, 16, c->max_blocks, num_blocks, max_len, partition_tokens,
+                                             c->d_ws, c->ws_bytes, stream)
+            : pkv_paged_attention_decode(c->d_out, c->out_dtype, c->d_q, k_cache, v_cache, c->kv_dtype, d_tables,
+                                         d_lens, scale, n, c->num_q_heads, c->num_kv_heads, c->head_dim, 16,
+                                         c->max_blocks, num_blocks, max_len, partition_tokens, c->d_ws, c->ws_bytes,
+                                         stream);
     if (s != PKV_OK) return s;
     // 4. the result back to the host
     const size_t ob = (size_t)n * c->num_q_heads * c->head_dim * elt(c->out_dtype);

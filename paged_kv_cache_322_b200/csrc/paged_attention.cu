@@ -36,6 +36,7 @@
 #include <atomic>
 #include <cmath>
 #include <mutex>
+#include <type_traits>
 
 #include "attention_common.cuh"
 
@@ -52,6 +53,8 @@ template <typename T, int D, int PATH, int HPW, int STAGES>
 struct Kern {
     static constexpr bool kMma = PATH == 2;
     static constexpr int TILE = BS * D * (int)sizeof(T);              // one block, one head, K or V
+    static constexpr int BOX = 128 / (int)sizeof(T);                   // elements per swizzled 128-byte box row
+    static constexpr int NBOX = D * (int)sizeof(T) / 128;              // boxes per row (tensor-core path)
     static constexpr int STAGE_BYTES = 2 * TILE;
     static constexpr int RING = STAGES * STAGE_BYTES;
     static constexpr int NSLOT = PATH == 1 ? 1 : NCW;                  // partial states to merge
@@ -139,9 +142,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                         uint8_t* dst = smem + st * K::STAGE_BYTES;
                         if constexpr (K::kMma) {
 #pragma unroll
-                            for (int h = 0; h < D / 64; ++h) {
-                                tma_load_4d(dst + h * (BS * 128), &tm_k, &full[st], h * 64, kvh, 0, pb, pol);
-                                tma_load_4d(dst + K::TILE + h * (BS * 128), &tm_v, &full[st], h * 64, kvh, 0, pb, pol);
+                            for (int h = 0; h < K::NBOX; ++h) {
+                                tma_load_4d(dst + h * (BS * 128), &tm_k, &full[st], h * K::BOX, kvh, 0, pb, pol);
+                                tma_load_4d(dst + K::TILE + h * (BS * 128), &tm_v, &full[st], h * K::BOX, kvh, 0, pb,
+                                            pol);
                             }
                         } else {
                             tma_load_4d(dst, &tm_k, &full[st], 0, kvh, 0, pb, pol);
@@ -162,9 +166,11 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     } else {
         // ---------------- consumers ----------------
         const int cw = warp - 1;
-        const T* qbase = static_cast<const T*>(p.q) + ((int64_t)seq * p.num_q_heads + qh0) * D;
+        using TQ = std::conditional_t<sizeof(T) == 1, __nv_bfloat16, T>;   // an fp8 cache takes bf16 queries
+        const TQ* qbase = static_cast<const TQ*>(p.q) + ((int64_t)seq * p.num_q_heads + qh0) * D;
         if constexpr (PATH == 2) {
-            MmaConsumer<D> c;
+            using Cons = std::conditional_t<sizeof(T) == 1, MmaConsumerFp8, MmaConsumer<D>>;
+            Cons c;
             c.init(reinterpret_cast<const __nv_bfloat16*>(qbase), group, lane);
             for (int j = cw; j < nblk; j += NCW) {
                 const int st = j % STAGES;
@@ -185,7 +191,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         } else {
             constexpr int HPWc = HPW;
             const int hbase = PATH == 1 ? cw * HPWc : 0;
-            SimtConsumer<T, D, HPWc> c;
+            SimtConsumer<T, D, HPWc, TQ> c;
             c.init(qbase + (int64_t)hbase * D, p.scale_log2, lane);
             const int jstart = PATH == 1 ? 0 : cw, jstep = PATH == 1 ? 1 : NCW;
             for (int j = jstart; j < nblk; j += jstep) {
@@ -284,18 +290,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// Tensor map over a cache [NB, BS, Hkv, D]: box = one block of one head, the
-// whole row (SIMT) or a 64-element half row with the 128-byte swizzle (MMA).
-bool make_cache_map(CUtensorMap* map, const void* base, bool bf16, int nb, int hkv, int d, bool mma) {
+// Tensor map over a cache [NB, BS, Hkv, D] of 4-, 2- or 1-byte elements: box =
+// one block of one head, the whole row (SIMT) or 128-byte box rows with the
+// 128-byte swizzle (tensor-core path).
+bool make_cache_map(CUtensorMap* map, const void* base, pkv_dtype dt, int nb, int hkv, int d, bool mma) {
     auto fn = encode_fn();
     if (!fn) return false;
-    const cuuint64_t eb = bf16 ? 2 : 4;
+    const cuuint64_t eb = dt == PKV_F32 ? 4 : (dt == PKV_BF16 ? 2 : 1);
+    const CUtensorMapDataType ty = dt == PKV_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                   : dt == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_UINT8;
     cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)hkv, (cuuint64_t)BS, (cuuint64_t)nb};
     cuuint64_t strides[3] = {d * eb, (cuuint64_t)hkv * d * eb, (cuuint64_t)BS * hkv * d * eb};
-    cuuint32_t box[4] = {(cuuint32_t)(mma ? 64 : d), 1, (cuuint32_t)BS, 1};
+    cuuint32_t box[4] = {(cuuint32_t)(mma ? 128 / eb : d), 1, (cuuint32_t)BS, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
-                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+    CUresult r = fn(map, ty, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     mma ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -457,22 +466,28 @@ int pkv_paged_attention_partition_tokens(int num_seqs, int num_q_heads, int num_
     return pl.part_tokens;
 }
 
-pkv_status pkv_paged_attention_decode(void* out, pkv_dtype out_dtype, const void* q, const void* k_cache,
-                                      const void* v_cache, pkv_dtype kv_dtype, const int32_t* block_tables,
-                                      const int32_t* context_lens, float scale, int num_seqs, int num_q_heads,
-                                      int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
-                                      int num_blocks, int max_context_len, int partition_tokens,
-                                      void* workspace, size_t workspace_bytes, void* stream) {
-    using namespace pkv;
-    using namespace pkv::attn;
+}  // extern "C"
+
+namespace pkv {
+namespace attn {
+
+// One decode call. kv_dtype: the cache storage (f32, bf16 or fp8 e4m3); q is
+// kv_dtype for f32 / bf16 caches and bf16 for an fp8 cache, whose K and V
+// scales fold into the logit scale and the output.
+pkv_status decode_impl(void* out, pkv_dtype out_dtype, const void* q, const void* k_cache, const void* v_cache,
+                       pkv_dtype kv_dtype, float k_scale, float v_scale, const int32_t* block_tables,
+                       const int32_t* context_lens, float scale, int num_seqs, int num_q_heads, int num_kv_heads,
+                       int head_dim, int block_size, int max_blocks_per_seq, int num_blocks, int max_context_len,
+                       int partition_tokens, void* workspace, size_t workspace_bytes, void* stream) {
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
         max_context_len < 0 || partition_tokens < -1 || !std::isfinite(scale))
         return PKV_ERR_INVALID_ARG;
-    if ((out_dtype != PKV_F32 && out_dtype != PKV_BF16) || (kv_dtype != PKV_F32 && kv_dtype != PKV_BF16))
-        return PKV_ERR_INVALID_ARG;
+    if (out_dtype != PKV_F32 && out_dtype != PKV_BF16) return PKV_ERR_INVALID_ARG;
     if (num_q_heads % num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
     const int group = num_q_heads / num_kv_heads;
+    const bool fp8 = kv_dtype == PKV_FP8_E4M3;
     if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
+    if (fp8 && (head_dim != 128 || partition_tokens == -1)) return PKV_ERR_UNSUPPORTED;
     if (block_size != BS) return PKV_ERR_UNSUPPORTED;
     if (group != 1 && group != 2 && group != 4 && group != 8) return PKV_ERR_UNSUPPORTED;
     if (num_seqs == 0) return PKV_OK;
@@ -492,10 +507,10 @@ pkv_status pkv_paged_attention_decode(void* out, pkv_dtype out_dtype, const void
     if (!err) return PKV_ERR_CUDA;
 
     const bool bf16 = kv_dtype == PKV_BF16;
-    const bool use_mma = bf16 && group >= 2;
+    const bool use_mma = (bf16 || fp8) && group >= 2;
     CUtensorMap mk, mv;
-    if (!make_cache_map(&mk, k_cache, bf16, num_blocks, num_kv_heads, head_dim, use_mma) ||
-        !make_cache_map(&mv, v_cache, bf16, num_blocks, num_kv_heads, head_dim, use_mma))
+    if (!make_cache_map(&mk, k_cache, kv_dtype, num_blocks, num_kv_heads, head_dim, use_mma) ||
+        !make_cache_map(&mv, v_cache, kv_dtype, num_blocks, num_kv_heads, head_dim, use_mma))
         return PKV_ERR_CUDA;
 
     Params p{};
@@ -504,7 +519,8 @@ pkv_status pkv_paged_attention_decode(void* out, pkv_dtype out_dtype, const void
     p.block_tables = block_tables;
     p.context_lens = context_lens;
     p.err = err;
-    p.scale_log2 = scale * 1.4426950408889634f;
+    p.scale_log2 = scale * 1.4426950408889634f * (fp8 ? k_scale : 1.0f);
+    p.out_scale = fp8 ? v_scale : 1.0f;
     p.out_f32 = out_dtype == PKV_F32;
     p.num_q_heads = num_q_heads;
     p.num_kv_heads = num_kv_heads;
@@ -537,7 +553,10 @@ pkv_status pkv_paged_attention_decode(void* out, pkv_dtype out_dtype, const void
 
     dim3 grid(num_kv_heads, pl.num_parts, num_seqs);
     cudaError_t e;
-    if (use_mma) {
+    if (fp8) {
+        e = use_mma ? launch_decode<uint8_t, 128, 2, 8, stages_for<uint8_t, 128>()>(mk, mv, p, grid, st)
+                    : dispatch_simt<uint8_t, 128>(group, mk, mv, p, grid, st);
+    } else if (use_mma) {
         e = head_dim == 128
                 ? launch_decode<__nv_bfloat16, 128, 2, 8, stages_for<__nv_bfloat16, 128>()>(mk, mv, p, grid, st)
                 : launch_decode<__nv_bfloat16, 64, 2, 8, stages_for<__nv_bfloat16, 64>()>(mk, mv, p, grid, st);
@@ -556,6 +575,39 @@ pkv_status pkv_paged_attention_decode(void* out, pkv_dtype out_dtype, const void
         if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
     }
     return PKV_OK;
+}
+
+}  // namespace attn
+}  // namespace pkv
+
+extern "C" {
+
+pkv_status pkv_paged_attention_decode(void* out, pkv_dtype out_dtype, const void* q, const void* k_cache,
+                                      const void* v_cache, pkv_dtype kv_dtype, const int32_t* block_tables,
+                                      const int32_t* context_lens, float scale, int num_seqs, int num_q_heads,
+                                      int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                                      int num_blocks, int max_context_len, int partition_tokens,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
+    if (kv_dtype != PKV_F32 && kv_dtype != PKV_BF16) return PKV_ERR_INVALID_ARG;
+    return pkv::attn::decode_impl(out, out_dtype, q, k_cache, v_cache, kv_dtype, 1.0f, 1.0f, block_tables,
+                                  context_lens, scale, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                  max_blocks_per_seq, num_blocks, max_context_len, partition_tokens, workspace,
+                                  workspace_bytes, stream);
+}
+
+pkv_status pkv_paged_attention_decode_fp8(void* out, pkv_dtype out_dtype, const void* q, const void* k_cache,
+                                          const void* v_cache, float k_scale, float v_scale,
+                                          const int32_t* block_tables, const int32_t* context_lens, float scale,
+                                          int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                          int block_size, int max_blocks_per_seq, int num_blocks,
+                                          int max_context_len, int partition_tokens, void* workspace,
+                                          size_t workspace_bytes, void* stream) {
+    if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+        return PKV_ERR_INVALID_ARG;
+    return pkv::attn::decode_impl(out, out_dtype, q, k_cache, v_cache, PKV_FP8_E4M3, k_scale, v_scale, block_tables,
+                                  context_lens, scale, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                  max_blocks_per_seq, num_blocks, max_context_len, partition_tokens, workspace,
+                                  workspace_bytes, stream);
 }
 
 }  // extern "C"

@@ -23,19 +23,26 @@ from . import binding
 
 
 class PagedKVCache:
+    """dtype float32 / bfloat16 caches, or torch.uint8 for an FP8 (e4m3) cache
+    with per-tensor scales kv_scales = (k_scale, v_scale); FP8 caches take bf16
+    K/V on append and bf16 queries."""
+
     def __init__(self, num_blocks: int, block_size: int, num_kv_heads: int, head_dim: int,
                  dtype: torch.dtype, device, free_order=None, max_blocks_per_seq: int = 0,
-                 fill_value: float | None = None):
+                 fill_value: float | None = None, kv_scales=(1.0, 1.0)):
         self.num_blocks, self.block_size = num_blocks, block_size
         self.num_kv_heads, self.head_dim, self.dtype = num_kv_heads, head_dim, dtype
+        self.fp8 = dtype == torch.uint8
+        self.kv_scales = (float(kv_scales[0]), float(kv_scales[1]))
         self.device = torch.device(device)
         shape = (num_blocks, block_size, num_kv_heads, head_dim)
         if fill_value is None:
             self.k_cache = torch.empty(shape, dtype=dtype, device=self.device)
             self.v_cache = torch.empty(shape, dtype=dtype, device=self.device)
         else:
-            self.k_cache = torch.full(shape, fill_value, dtype=dtype, device=self.device)
-            self.v_cache = torch.full(shape, fill_value, dtype=dtype, device=self.device)
+            fill = 0x7F if (self.fp8 and fill_value != fill_value) else fill_value    # NaN -> the e4m3 NaN code
+            self.k_cache = torch.full(shape, fill, dtype=dtype, device=self.device)
+            self.v_cache = torch.full(shape, fill, dtype=dtype, device=self.device)
         self.bm = binding.BlockManager(num_blocks, block_size, free_order)
         self.max_blocks_per_seq = max_blocks_per_seq or num_blocks
         self._pinned = {}
@@ -68,9 +75,27 @@ class PagedKVCache:
         its blocks and writes the prompt into them."""
         slots = self.bm.allocate(seq_id, k.shape[0])
         if k.shape[0]:
-            binding.reshape_and_cache(k, v, self.k_cache, self.v_cache, self._to_device("slots", slots, stream),
-                                      stream=stream)
+            self.append(k, v, self._to_device("slots", slots, stream), stream=stream)
         return slots
+
+    def append(self, k, v, slot_mapping, stream=None):
+        """reshape_and_cache (quantising for an FP8 cache)."""
+        if self.fp8:
+            binding.reshape_and_cache_fp8(k, v, self.k_cache, self.v_cache, slot_mapping, *self.kv_scales,
+                                          stream=stream)
+        else:
+            binding.reshape_and_cache(k, v, self.k_cache, self.v_cache, slot_mapping, stream=stream)
+
+    def attention(self, out, q, tables, lens, scale, max_context_len=0, partition_tokens=0, workspace=None,
+                  stream=None):
+        if self.fp8:
+            return binding.paged_attention_decode_fp8(out, q, self.k_cache, self.v_cache, tables, lens, scale,
+                                                      *self.kv_scales, max_context_len=max_context_len,
+                                                      partition_tokens=partition_tokens, workspace=workspace,
+                                                      stream=stream)
+        return binding.paged_attention_decode(out, q, self.k_cache, self.v_cache, tables, lens, scale,
+                                              max_context_len=max_context_len, partition_tokens=partition_tokens,
+                                              workspace=workspace, stream=stream)
 
     def fork(self, parent: int, child: int):
         self.bm.fork(parent, child)
@@ -101,13 +126,11 @@ class PagedKVCache:
         if src.size:
             binding.copy_blocks(self.k_cache, self.v_cache, self._to_device("src", src, stream),
                                 self._to_device("dst", dst, stream), stream=stream)
-        binding.reshape_and_cache(k_new, v_new, self.k_cache, self.v_cache, self._to_device("slots", slots, stream),
-                                  stream=stream)
+        self.append(k_new, v_new, self._to_device("slots", slots, stream), stream=stream)
         tables, lens = self.block_tables(seq_ids)
         if out is None:
             out = torch.empty(q.shape, dtype=out_dtype, device=self.device)
-        binding.paged_attention_decode(out, q, self.k_cache, self.v_cache, self._to_device("tables", tables, stream),
-                                       self._to_device("lens", lens, stream), scale,
-                                       max_context_len=int(lens.max()) if lens.size else 0,
-                                       partition_tokens=partition_tokens, stream=stream)
+        self.attention(out, q, self._to_device("tables", tables, stream), self._to_device("lens", lens, stream),
+                       scale, max_context_len=int(lens.max()) if lens.size else 0, partition_tokens=partition_tokens,
+                       stream=stream)
         return out

@@ -37,7 +37,7 @@ class Workload:
     head_dim: int
     block_size: int
     num_blocks: int
-    kv_dtype: str                 # "f32" or "bf16": storage type of q, k, v and the caches
+    kv_dtype: str                 # "f32", "bf16" or "fp8" (e4m3 cache codes; q, k, v in bf16)
     ctx: str                      # "fixed" | "uniform" | "loguniform" | "shared_prefix"
     lo: int = 0
     hi: int = 0
@@ -45,6 +45,7 @@ class Workload:
     shared_prefix: int = 0        # tokens of the shared prompt (shared_prefix workloads)
     partition_tokens: int = 0     # split-K partition the workload asks for (0 = library default)
     seed: int = 0
+    kv_scale: float = 1.0         # per-tensor K and V scale of an fp8 cache
     description: str = field(default="", compare=False)
 
     @property
@@ -53,6 +54,12 @@ class Workload:
 
     @property
     def elt_bytes(self) -> int:
+        """Bytes per cache element."""
+        return {"f32": 4, "bf16": 2, "fp8": 1}[self.kv_dtype]
+
+    @property
+    def in_bytes(self) -> int:
+        """Bytes per element of q and of the new K/V the step appends."""
         return 4 if self.kv_dtype == "f32" else 2
 
     @property
@@ -75,6 +82,14 @@ WORKLOADS = {
         shared_prefix=1024, seed=1003,
         description="parallel sampling: 32 seqs share a 1024-token prefix (64 blocks, ref 32) + private tails U[64,512]; "
                     "32/32 heads, D=128, bf16, bs=16"),
+    "llama2_7b_fp8": Workload(
+        "llama2_7b_fp8", 64, 32, 32, 128, 16, 16384, "fp8", "uniform", lo=512, hi=2048, seed=1001, kv_scale=1 / 64,
+        description="Llama-2-7B-shaped decode over an FP8 (e4m3, scale 1/64) cache: B=64, 32/32 heads, D=128, "
+                    "bs=16, ctx U[512,2048], 16384-block pool"),
+    "gqa_70b_fp8": Workload(
+        "gqa_70b_fp8", 128, 64, 8, 128, 16, 65536, "fp8", "uniform", lo=1024, hi=4096, seed=1002, kv_scale=1 / 64,
+        description="70B-shaped GQA decode over an FP8 (e4m3, scale 1/64) cache: B=128, 64/8 heads, D=128, bs=16, "
+                    "ctx U[1024,4096], 65536-block pool"),
     "long_splitk": Workload(
         "long_splitk", 16, 32, 8, 128, 16, 65536, "bf16", "loguniform", lo=16, hi=32768,
         partition_tokens=512, seed=1004,
@@ -102,7 +117,7 @@ def _normal(w: Workload, rng: np.random.Generator, shape) -> np.ndarray:
     """N(0,1) samples stored in the workload's dtype; returned as float32 values
     exactly representable in that dtype (bf16-rounded for bf16 workloads)."""
     x = rng.standard_normal(shape, dtype=np.float32)
-    if w.kv_dtype == "bf16":
+    if w.kv_dtype in ("bf16", "fp8"):
         x = bf16_bits_to_f32(round_to_bf16(x))
     return x
 

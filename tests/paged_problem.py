@@ -13,16 +13,19 @@ from paged_kv_cache_322_b200 import workloads as wl
 
 class SparsePool:
     """A cache [num_blocks, bs, Hkv, D] that stores only written blocks; unwritten
-    blocks read as NaN (like the sentinel-filled device pool)."""
+    blocks read as NaN (like the sentinel-filled device pool; the NaN code 0x7F
+    for an FP8 pool of uint8 codes)."""
 
-    def __init__(self, num_blocks, bs, hkv, d):
+    def __init__(self, num_blocks, bs, hkv, d, dtype=np.float32):
         self.shape = (num_blocks, bs, hkv, d)
+        self.dtype = dtype
         self.blocks = {}
 
     def _blk(self, b):
         b = int(b)
         if b not in self.blocks:
-            self.blocks[b] = np.full(self.shape[1:], np.nan, dtype=np.float32)
+            fill = 0x7F if self.dtype == np.uint8 else np.nan
+            self.blocks[b] = np.full(self.shape[1:], fill, dtype=self.dtype)
         return self.blocks[b]
 
     def __getitem__(self, key):
@@ -31,7 +34,7 @@ class SparsePool:
         if isinstance(key, (int, np.integer)):
             return self._blk(key)
         return np.stack([self._blk(b) for b in np.asarray(key).tolist()]) if len(key) else \
-            np.zeros((0,) + self.shape[1:], np.float32)
+            np.zeros((0,) + self.shape[1:], self.dtype)
 
     def __setitem__(self, key, val):
         if isinstance(key, tuple):
@@ -49,12 +52,14 @@ class OracleProblem:
         self.lens = wl.context_lens(w)
         self.bm = OracleBM(w.num_blocks, w.block_size, wl.free_order(w))
         shape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
+        self.fp8 = w.kv_dtype == "fp8"
+        dt, fill = (np.uint8, 0x7F) if self.fp8 else (np.float32, np.nan)
         if dense:
-            self.kc = np.full(shape, np.nan, np.float32)
-            self.vc = np.full(shape, np.nan, np.float32)
+            self.kc = np.full(shape, fill, dt)
+            self.vc = np.full(shape, fill, dt)
         else:
-            self.kc = SparsePool(*shape)
-            self.vc = SparsePool(*shape)
+            self.kc = SparsePool(*shape, dtype=dt)
+            self.vc = SparsePool(*shape, dtype=dt)
         self.keep = set(range(w.num_seqs)) if keep is None else set(int(s) for s in keep)
         if w.ctx == "shared_prefix":
             self._build_shared()
@@ -63,15 +68,21 @@ class OracleProblem:
                 slots = self.bm.allocate(s, int(self.lens[s]))
                 if s in self.keep:
                     k, v = wl.prompt_kv(w, s, int(self.lens[s]))
-                    ocache.reshape_and_cache(k, v, self.kc, self.vc, np.asarray(slots))
+                    self._scatter(k, v, np.asarray(slots))
         self.cow_pairs = []
+
+    def _scatter(self, k, v, slots):
+        if self.fp8:
+            ocache.reshape_and_cache_fp8(k, v, self.kc, self.vc, slots, self.w.kv_scale, self.w.kv_scale)
+        else:
+            ocache.reshape_and_cache(k, v, self.kc, self.vc, slots)
 
     def _build_shared(self):
         w = self.w
         p = w.shared_prefix
         slots = self.bm.allocate(-1, p)
         k0, v0 = wl.prompt_kv(w, 0, int(self.lens[0]))
-        ocache.reshape_and_cache(k0[:p], v0[:p], self.kc, self.vc, np.asarray(slots))
+        self._scatter(k0[:p], v0[:p], np.asarray(slots))
         for s in range(w.num_seqs):
             self.bm.fork(-1, s)
         self.bm.free_seq(-1)
@@ -80,7 +91,7 @@ class OracleProblem:
             tail = [self.bm.append_slot(s)[0] for _ in range(n - p)]
             if s in self.keep:
                 k, v = wl.prompt_kv(w, s, n)
-                ocache.reshape_and_cache(k[p:], v[p:], self.kc, self.vc, np.asarray(tail))
+                self._scatter(k[p:], v[p:], np.asarray(tail))
 
     def fork_last_shared_block(self):
         """Copy-on-write of the last shared prefix block for every sequence
@@ -104,16 +115,19 @@ class OracleProblem:
             slot, copy = self.bm.append_slot(s)
             assert copy is None
             slots.append(slot if s in self.keep else -1)
-        ocache.reshape_and_cache(kn, vn, self.kc, self.vc, np.asarray(slots))
+        self._scatter(kn, vn, np.asarray(slots))
         return self.attend(q, seqs)
 
     def attend(self, q, seqs=None):
         seqs = sorted(self.keep) if seqs is None else list(seqs)
         tables = {s: self.bm.block_table(s) for s in seqs}
         lens = {s: self.bm.lens[s] for s in seqs}
-        out = oattn.paged_attention_decode(q, self.kc, self.vc, _TableView(tables), _TableView(lens),
-                                           self.w.scale, self.w.block_size, seqs=seqs)
-        return out
+        if self.fp8:
+            return oattn.paged_attention_decode_fp8(q, self.kc, self.vc, _TableView(tables), _TableView(lens),
+                                                    self.w.scale, self.w.block_size, self.w.kv_scale,
+                                                    self.w.kv_scale, seqs=seqs)
+        return oattn.paged_attention_decode(q, self.kc, self.vc, _TableView(tables), _TableView(lens),
+                                            self.w.scale, self.w.block_size, seqs=seqs)
 
 
 class _TableView:
@@ -130,11 +144,12 @@ def gpu_problem(w: wl.Workload, device="cuda", fill_nan=True, max_new_tokens=4):
     import torch
     from paged_kv_cache_322_b200.engine import PagedKVCache
     lens = wl.context_lens(w)
-    dt = torch.float32 if w.kv_dtype == "f32" else torch.bfloat16
+    dt = torch.float32 if w.kv_dtype == "f32" else torch.bfloat16          # q / k / v
+    cdt = torch.uint8 if w.kv_dtype == "fp8" else dt                        # caches
     mb = -(-int(lens.max() + max_new_tokens) // w.block_size)
-    cache = PagedKVCache(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, dt, device,
+    cache = PagedKVCache(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, cdt, device,
                          free_order=wl.free_order(w), max_blocks_per_seq=mb,
-                         fill_value=float("nan") if fill_nan else None)
+                         fill_value=float("nan") if fill_nan else None, kv_scales=(w.kv_scale, w.kv_scale))
     def dev(x):
         return torch.from_numpy(x).to(device=device, dtype=dt)
     if w.ctx == "shared_prefix":
@@ -149,9 +164,7 @@ def gpu_problem(w: wl.Workload, device="cuda", fill_nan=True, max_new_tokens=4):
             k, v = wl.prompt_kv(w, s, n)
             kt, vt = dev(k[p:]), dev(v[p:])
             slots = np.concatenate([cache.bm.append_slots([s])[0] for _ in range(n - p)])
-            from paged_kv_cache_322_b200 import binding
-            binding.reshape_and_cache(kt, vt, cache.k_cache, cache.v_cache,
-                                      torch.from_numpy(slots).to(device))
+            cache.append(kt, vt, torch.from_numpy(slots).to(device))
     else:
         kvs = wl.prompt_kv_all(w, lens)
         for s in range(w.num_seqs):
@@ -170,5 +183,6 @@ def step_inputs(w: wl.Workload, step: int, device="cuda"):
 
 def tolerance(w: wl.Workload) -> float:
     """Max abs error allowed against the fp64 oracle: 1e-5 for fp32 inputs,
-    2e-3 for bf16-rounded inputs (fp32 accumulation, fp32 output)."""
+    2e-3 for bf16-rounded inputs and for FP8 caches (the oracle attends over the
+    same dequantised values; fp32 accumulation, fp32 output)."""
     return 1e-5 if w.kv_dtype == "f32" else 2e-3

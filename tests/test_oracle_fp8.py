@@ -96,3 +96,14 @@ def test_planted_encoder_mistakes_are_caught(mistake):
         return 0x7F if abs(x) > 448 else c
     xs = [1.0625, 0.3, -2.7, 500.0, 100.0]
     assert any(bad(x) != fp8.encode(x) for x in xs)
+
+
+def test_array_encoder_equals_scalar_definition():
+    rng = np.random.default_rng(9)
+    vals = fp8.decode_array(np.arange(256))
+    fin = np.sort(np.unique(vals[np.isfinite(vals)]))
+    mids = (fin[1:] + fin[:-1]) / 2
+    x = np.concatenate([fin, -fin, mids, -mids, np.nextafter(mids, 0), np.nextafter(mids, 1e9),
+                        rng.standard_normal(5000) * 50, [0.0, -0.0, 1e-300, 464.0, 480.0, 1e9, -1e9, math.inf,
+                                                          -math.inf, math.nan]])
+    assert np.array_equal(fp8.encode_array(x), np.array([fp8.encode(v) for v in x], dtype=np.uint8))
