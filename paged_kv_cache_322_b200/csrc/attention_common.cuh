@@ -59,14 +59,14 @@ __device__ __forceinline__ float to_float(TQ x) {
 // SIMT consumer: HPW query heads per warp, 8 lanes per token, 4 tokens per
 // round, fp32 math. T = float or __nv_bfloat16.
 // ---------------------------------------------------------------------------
-template <typename T, int D, int HPW, typename TQ = T>
+template <typename T, int D, int HPW, typename TQ = T, int TOK = BS>
 struct SimtConsumer {
     static constexpr int RB = D * (int)sizeof(T);          // row bytes
     static constexpr int NCH = RB / 16;                     // 16-byte chunks per row
     static constexpr int CPL = NCH / 8;                     // chunks per lane
     static constexpr int EPC = 16 / (int)sizeof(T);         // elements per chunk
     static constexpr int EPL = CPL * EPC;                   // elements per lane
-    static constexpr int ROUNDS = BS / 4;
+    static constexpr int ROUNDS = TOK / 4;                 // 4 tokens per round (8 lanes each)
     static_assert(NCH % 8 == 0, "row must hold a multiple of 8 chunks");
 
     float q[HPW][EPL];
@@ -359,9 +359,11 @@ struct MmaConsumer {
 //   and the odd-dim row (fragment row g + 8), so each 16-dim chunk is one MMA
 //   whose output rows are dims 2g and 2g + 1.
 // ---------------------------------------------------------------------------
+template <int NT>      // 16-token tiles per stage (1 or 2)
 struct MmaConsumerFp8 {
     static constexpr int D = 128;
     static constexpr int NCHUNK = D / 16;
+    static constexpr int TOK = 16 * NT;
 
     uint32_t qb[NCHUNK][2];
     float o[NCHUNK][4];
@@ -389,51 +391,10 @@ struct MmaConsumerFp8 {
         l0 = l1 = 0.f;
     }
 
-    __device__ __forceinline__ void consume(uint32_t ks_base, uint32_t vs_base, uint8_t* vs_ptr, int nvalid,
-                                            float scale_log2, int lane) {
+    // P^T of one 16-token tile as f16 B fragments (high and low parts).
+    __device__ __forceinline__ static void p_fragments(float p0, float p1, float p2, float p3, int lane,
+                                                       uint32_t& bh0, uint32_t& bh1, uint32_t& bl0, uint32_t& bl1) {
         const int g = lane >> 2, t = lane & 3;
-        if (nvalid < BS) {          // rows past the context: zero V codes (0 * NaN would poison O)
-            for (int i = lane; i < (BS - nvalid) * 8; i += 32) {
-                const int r = nvalid + i / 8, c = i % 8;
-                *reinterpret_cast<uint4*>(vs_ptr + r * 128 + ((c ^ (r & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
-            }
-            __syncwarp();
-        }
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
-        const int mi = lane >> 3;
-        const int row = (lane & 7) + ((mi & 1) << 3);
-#pragma unroll
-        for (int kp = 0; kp < NCHUNK / 2; ++kp) {
-            const int chunk = 2 * kp + (mi >> 1);
-            uint32_t r0, r1, r2, r3;
-            ldmatrix_x4(r0, r1, r2, r3, ks_base + row * 128 + ((chunk ^ (row & 7)) << 4));
-            mma_f16_16816(s, e4m3x2_to_f16x2(r0 & 0xffffu), e4m3x2_to_f16x2(r1 & 0xffffu), e4m3x2_to_f16x2(r0 >> 16),
-                          e4m3x2_to_f16x2(r1 >> 16), qb[2 * kp][0], qb[2 * kp][1]);
-            mma_f16_16816(s, e4m3x2_to_f16x2(r2 & 0xffffu), e4m3x2_to_f16x2(r3 & 0xffffu), e4m3x2_to_f16x2(r2 >> 16),
-                          e4m3x2_to_f16x2(r3 >> 16), qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
-        }
-        float x0 = g < nvalid ? s[0] * scale_log2 : kNegInf;
-        float x1 = g < nvalid ? s[1] * scale_log2 : kNegInf;
-        float x2 = g + 8 < nvalid ? s[2] * scale_log2 : kNegInf;
-        float x3 = g + 8 < nvalid ? s[3] * scale_log2 : kNegInf;
-        float b0 = fmaxf(x0, x2), b1 = fmaxf(x1, x3);
-#pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-            b0 = fmaxf(b0, __shfl_xor_sync(0xffffffffu, b0, off));
-            b1 = fmaxf(b1, __shfl_xor_sync(0xffffffffu, b1, off));
-        }
-        const float n0 = fmaxf(m0, b0), n1 = fmaxf(m1, b1);
-        const float al0 = fast_exp2(m0 - n0), al1 = fast_exp2(m1 - n1);
-        m0 = n0;
-        m1 = n1;
-        const float p0 = fast_exp2(x0 - n0), p1 = fast_exp2(x1 - n1);
-        const float p2 = fast_exp2(x2 - n0), p3 = fast_exp2(x3 - n1);
-        l0 = l0 * al0 + (p0 + p2);
-        l1 = l1 * al1 + (p1 + p3);
-#pragma unroll
-        for (int c = 0; c < NCHUNK; ++c) {
-            o[c][0] *= al0; o[c][1] *= al1; o[c][2] *= al0; o[c][3] *= al1;
-        }
         const uint32_t h02 = pack_f16(p0, p2), h13 = pack_f16(p1, p3);
         const float2 f02 = f16x2_to_float2(h02), f13 = f16x2_to_float2(h13);
         const uint32_t e02 = pack_f16(p0 - f02.x, p2 - f02.y), e13 = pack_f16(p1 - f13.x, p3 - f13.y);
@@ -452,28 +413,108 @@ struct MmaConsumerFp8 {
             za = odd ? u1 : u0;
             zb = odd ? v1 : v0;
         }
-        const uint32_t bh0 = __byte_perm(ya, yb, 0x5410), bh1 = __byte_perm(ya, yb, 0x7632);
-        const uint32_t bl0 = __byte_perm(za, zb, 0x5410), bl1 = __byte_perm(za, zb, 0x7632);
-        const int tok = (lane & 7) + ((mi & 1) << 3);
-#pragma unroll
-        for (int cp = 0; cp < NCHUNK / 2; ++cp) {
-            const int chunk = 2 * cp + (mi >> 1);
-            uint32_t r0, r1, r2, r3;
-            ldmatrix_x4_trans(r0, r1, r2, r3, vs_base + tok * 128 + ((chunk ^ (tok & 7)) << 4));
-            // r0: tokens 0-7 of chunk 2cp, r1: tokens 8-15 of it; r2, r3: chunk 2cp + 1
-            {
-                const uint32_t x = __byte_perm(r0, 0u, 0x3120), y = __byte_perm(r1, 0u, 0x3120);
-                const uint32_t a0 = e4m3x2_to_f16x2(x & 0xffffu), a1 = e4m3x2_to_f16x2(x >> 16);
-                const uint32_t a2 = e4m3x2_to_f16x2(y & 0xffffu), a3 = e4m3x2_to_f16x2(y >> 16);
-                mma_f16_16816(o[2 * cp], a0, a1, a2, a3, bh0, bh1);
-                mma_f16_16816(o[2 * cp], a0, a1, a2, a3, bl0, bl1);
+        bh0 = __byte_perm(ya, yb, 0x5410);
+        bh1 = __byte_perm(ya, yb, 0x7632);
+        bl0 = __byte_perm(za, zb, 0x5410);
+        bl1 = __byte_perm(za, zb, 0x7632);
+    }
+
+    // One even/odd-dim MMA pair input from two ldmatrix.trans registers (tokens 0-7, 8-15 of a tile).
+    __device__ __forceinline__ void pv(int c, uint32_t rlo, uint32_t rhi, uint32_t bh0, uint32_t bh1, uint32_t bl0,
+                                       uint32_t bl1) {
+        const uint32_t x = __byte_perm(rlo, 0u, 0x3120), y = __byte_perm(rhi, 0u, 0x3120);
+        const uint32_t a0 = e4m3x2_to_f16x2(x & 0xffffu), a1 = e4m3x2_to_f16x2(x >> 16);
+        const uint32_t a2 = e4m3x2_to_f16x2(y & 0xffffu), a3 = e4m3x2_to_f16x2(y >> 16);
+        mma_f16_16816(o[c], a0, a1, a2, a3, bh0, bh1);
+        mma_f16_16816(o[c], a0, a1, a2, a3, bl0, bl1);
+    }
+
+    __device__ __forceinline__ void consume(uint32_t ks_base, uint32_t vs_base, uint8_t* vs_ptr, int nvalid,
+                                            float scale_log2, int lane) {
+        const int g = lane >> 2;
+        if (nvalid < TOK) {         // rows past the context: zero V codes (0 * NaN would poison O)
+            for (int i = lane; i < (TOK - nvalid) * 8; i += 32) {
+                const int r = nvalid + i / 8, c = i % 8;
+                *reinterpret_cast<uint4*>(vs_ptr + r * 128 + ((c ^ (r & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
             }
-            {
-                const uint32_t x = __byte_perm(r2, 0u, 0x3120), y = __byte_perm(r3, 0u, 0x3120);
-                const uint32_t a0 = e4m3x2_to_f16x2(x & 0xffffu), a1 = e4m3x2_to_f16x2(x >> 16);
-                const uint32_t a2 = e4m3x2_to_f16x2(y & 0xffffu), a3 = e4m3x2_to_f16x2(y >> 16);
-                mma_f16_16816(o[2 * cp + 1], a0, a1, a2, a3, bh0, bh1);
-                mma_f16_16816(o[2 * cp + 1], a0, a1, a2, a3, bl0, bl1);
+            __syncwarp();
+        }
+        float s[NT][4];
+#pragma unroll
+        for (int tt = 0; tt < NT; ++tt) s[tt][0] = s[tt][1] = s[tt][2] = s[tt][3] = 0.f;
+        const int mi = lane >> 3;
+        const int row = (lane & 7) + ((mi & 1) << 3);
+#pragma unroll
+        for (int kp = 0; kp < NCHUNK / 2; ++kp) {
+            const int chunk = 2 * kp + (mi >> 1);
+#pragma unroll
+            for (int tt = 0; tt < NT; ++tt) {
+                const int r = tt * 16 + row;
+                uint32_t r0, r1, r2, r3;
+                ldmatrix_x4(r0, r1, r2, r3, ks_base + r * 128 + ((chunk ^ (r & 7)) << 4));
+                mma_f16_16816(s[tt], e4m3x2_to_f16x2(r0 & 0xffffu), e4m3x2_to_f16x2(r1 & 0xffffu),
+                              e4m3x2_to_f16x2(r0 >> 16), e4m3x2_to_f16x2(r1 >> 16), qb[2 * kp][0], qb[2 * kp][1]);
+                mma_f16_16816(s[tt], e4m3x2_to_f16x2(r2 & 0xffffu), e4m3x2_to_f16x2(r3 & 0xffffu),
+                              e4m3x2_to_f16x2(r2 >> 16), e4m3x2_to_f16x2(r3 >> 16), qb[2 * kp + 1][0],
+                              qb[2 * kp + 1][1]);
+            }
+        }
+        float x[NT][4];
+        float b0 = kNegInf, b1 = kNegInf;
+#pragma unroll
+        for (int tt = 0; tt < NT; ++tt) {
+            x[tt][0] = tt * 16 + g < nvalid ? s[tt][0] * scale_log2 : kNegInf;
+            x[tt][1] = tt * 16 + g < nvalid ? s[tt][1] * scale_log2 : kNegInf;
+            x[tt][2] = tt * 16 + g + 8 < nvalid ? s[tt][2] * scale_log2 : kNegInf;
+            x[tt][3] = tt * 16 + g + 8 < nvalid ? s[tt][3] * scale_log2 : kNegInf;
+            b0 = fmaxf(b0, fmaxf(x[tt][0], x[tt][2]));
+            b1 = fmaxf(b1, fmaxf(x[tt][1], x[tt][3]));
+        }
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            b0 = fmaxf(b0, __shfl_xor_sync(0xffffffffu, b0, off));
+            b1 = fmaxf(b1, __shfl_xor_sync(0xffffffffu, b1, off));
+        }
+        const float n0 = fmaxf(m0, b0), n1 = fmaxf(m1, b1);
+        const float al0 = fast_exp2(m0 - n0), al1 = fast_exp2(m1 - n1);
+        m0 = n0;
+        m1 = n1;
+        float ps0 = 0.f, ps1 = 0.f;
+        uint32_t bh[NT][2], bl[NT][2];
+#pragma unroll
+        for (int tt = 0; tt < NT; ++tt) {
+            const float p0 = fast_exp2(x[tt][0] - n0), p1 = fast_exp2(x[tt][1] - n1);
+            const float p2 = fast_exp2(x[tt][2] - n0), p3 = fast_exp2(x[tt][3] - n1);
+            ps0 += p0 + p2;
+            ps1 += p1 + p3;
+            p_fragments(p0, p1, p2, p3, lane, bh[tt][0], bh[tt][1], bl[tt][0], bl[tt][1]);
+        }
+        l0 = l0 * al0 + ps0;
+        l1 = l1 * al1 + ps1;
+#pragma unroll
+        for (int c = 0; c < NCHUNK; ++c) {
+            o[c][0] *= al0; o[c][1] *= al1; o[c][2] *= al0; o[c][3] *= al1;
+        }
+        if constexpr (NT == 1) {
+            const int tok = (lane & 7) + ((mi & 1) << 3);
+#pragma unroll
+            for (int cp = 0; cp < NCHUNK / 2; ++cp) {
+                const int chunk = 2 * cp + (mi >> 1);
+                uint32_t r0, r1, r2, r3;
+                ldmatrix_x4_trans(r0, r1, r2, r3, vs_base + tok * 128 + ((chunk ^ (tok & 7)) << 4));
+                // r0: tokens 0-7 of chunk 2cp, r1: tokens 8-15 of it; r2, r3: chunk 2cp + 1
+                pv(2 * cp, r0, r1, bh[0][0], bh[0][1], bl[0][0], bl[0][1]);
+                pv(2 * cp + 1, r2, r3, bh[0][0], bh[0][1], bl[0][0], bl[0][1]);
+            }
+        } else {
+            // one ldmatrix.x4.trans per chunk: tokens 0-7, 8-15 (tile 0) and 16-23, 24-31 (tile 1)
+            const int tok = (mi >> 1) * 16 + (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+            for (int c = 0; c < NCHUNK; ++c) {
+                uint32_t r0, r1, r2, r3;
+                ldmatrix_x4_trans(r0, r1, r2, r3, vs_base + tok * 128 + ((c ^ (tok & 7)) << 4));
+                pv(c, r0, r1, bh[0][0], bh[0][1], bl[0][0], bl[0][1]);
+                pv(c, r2, r3, bh[1][0], bh[1][1], bl[1][0], bl[1][1]);
             }
         }
     }

@@ -55,7 +55,12 @@ struct Kern {
     static constexpr int TILE = BS * D * (int)sizeof(T);              // one block, one head, K or V
     static constexpr int BOX = 128 / (int)sizeof(T);                   // elements per swizzled 128-byte box row
     static constexpr int NBOX = D * (int)sizeof(T) / 128;              // boxes per row (tensor-core path)
-    static constexpr int STAGE_BYTES = 2 * TILE;
+    // FP8 tiles are half the size: two physical blocks share a stage, so a stage
+    // is 8 KB and a consumer folds 32 tokens per step (K rows of both blocks
+    // first, then V rows).
+    static constexpr int BPS = sizeof(T) == 1 ? 2 : 1;                  // blocks per stage
+    static constexpr int TOK = BS * BPS;
+    static constexpr int STAGE_BYTES = 2 * BPS * TILE;
     static constexpr int RING = STAGES * STAGE_BYTES;
     static constexpr int NSLOT = PATH == 1 ? 1 : NCW;                  // partial states to merge
     static constexpr int MAXG = PATH == 2 ? 8 : (PATH == 1 ? HPW * NCW : HPW);
@@ -133,25 +138,29 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             for (int jj = 0; jj < jn; ++jj) {
                 const int pb = __shfl_sync(0xffffffffu, id, jj);
                 if (lane == 0 && ok) {
-                    const int j = j0 + jj, st = j % STAGES;
-                    if (!mbar_wait_bounded(&empty[st], ((j / STAGES) & 1) ^ 1, p.err)) {
-                        ok = false;
-                        s_abort = 1;
-                    } else {
-                        mbar_arrive_expect_tx(&full[st], K::STAGE_BYTES);
-                        uint8_t* dst = smem + st * K::STAGE_BYTES;
+                    const int j = j0 + jj, si = j / K::BPS, b = j - si * K::BPS, st = si % STAGES;
+                    if (b == 0) {                                 // first block of a stage: claim it
+                        if (!mbar_wait_bounded(&empty[st], ((si / STAGES) & 1) ^ 1, p.err)) {
+                            ok = false;
+                            s_abort = 1;
+                        } else {
+                            mbar_arrive_expect_tx(&full[st], min(K::BPS, nblk - j) * 2 * K::TILE);
+                            ++issued;
+                        }
+                    }
+                    if (ok) {
+                        uint8_t* dst = smem + st * K::STAGE_BYTES + b * K::TILE;
+                        uint8_t* vdst = dst + K::BPS * K::TILE;
                         if constexpr (K::kMma) {
 #pragma unroll
                             for (int h = 0; h < K::NBOX; ++h) {
                                 tma_load_4d(dst + h * (BS * 128), &tm_k, &full[st], h * K::BOX, kvh, 0, pb, pol);
-                                tma_load_4d(dst + K::TILE + h * (BS * 128), &tm_v, &full[st], h * K::BOX, kvh, 0, pb,
-                                            pol);
+                                tma_load_4d(vdst + h * (BS * 128), &tm_v, &full[st], h * K::BOX, kvh, 0, pb, pol);
                             }
                         } else {
                             tma_load_4d(dst, &tm_k, &full[st], 0, kvh, 0, pb, pol);
-                            tma_load_4d(dst + K::TILE, &tm_v, &full[st], 0, kvh, 0, pb, pol);
+                            tma_load_4d(vdst, &tm_v, &full[st], 0, kvh, 0, pb, pol);
                         }
-                        ++issued;
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -168,11 +177,12 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         const int cw = warp - 1;
         using TQ = std::conditional_t<sizeof(T) == 1, __nv_bfloat16, T>;   // an fp8 cache takes bf16 queries
         const TQ* qbase = static_cast<const TQ*>(p.q) + ((int64_t)seq * p.num_q_heads + qh0) * D;
+        const int nstage = (nblk + K::BPS - 1) / K::BPS;
         if constexpr (PATH == 2) {
-            using Cons = std::conditional_t<sizeof(T) == 1, MmaConsumerFp8, MmaConsumer<D>>;
+            using Cons = std::conditional_t<sizeof(T) == 1, MmaConsumerFp8<K::BPS>, MmaConsumer<D>>;
             Cons c;
             c.init(reinterpret_cast<const __nv_bfloat16*>(qbase), group, lane);
-            for (int j = cw; j < nblk; j += NCW) {
+            for (int j = cw; j < nstage; j += NCW) {
                 const int st = j % STAGES;
                 const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err);
                 if (__any_sync(0xffffffffu, !got || s_abort != 0)) {   // warp-uniform exit
@@ -180,9 +190,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     break;
                 }
                 uint8_t* stage = smem + st * K::STAGE_BYTES;
-                const int nvalid = min(BS, ctx - (blk0 + j) * BS);
-                c.consume(smem_u32(stage), smem_u32(stage + K::TILE), stage + K::TILE, nvalid, p.scale_log2, lane);
-                if (nvalid < BS) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                const int nvalid = min(K::TOK, ctx - (blk0 + j * K::BPS) * BS);
+                uint8_t* vst = stage + K::BPS * K::TILE;
+                c.consume(smem_u32(stage), smem_u32(vst), vst, nvalid, p.scale_log2, lane);
+                if (nvalid < K::TOK) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[st]);
             }
@@ -191,10 +202,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         } else {
             constexpr int HPWc = HPW;
             const int hbase = PATH == 1 ? cw * HPWc : 0;
-            SimtConsumer<T, D, HPWc, TQ> c;
+            SimtConsumer<T, D, HPWc, TQ, K::TOK> c;
             c.init(qbase + (int64_t)hbase * D, p.scale_log2, lane);
             const int jstart = PATH == 1 ? 0 : cw, jstep = PATH == 1 ? 1 : NCW;
-            for (int j = jstart; j < nblk; j += jstep) {
+            for (int j = jstart; j < nstage; j += jstep) {
                 const int st = j % STAGES;
                 const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err);
                 if (__any_sync(0xffffffffu, !got || s_abort != 0)) {
@@ -202,7 +213,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     break;
                 }
                 const uint8_t* stage = smem + st * K::STAGE_BYTES;
-                c.consume(stage, stage + K::TILE, min(BS, ctx - (blk0 + j) * BS), lane);
+                c.consume(stage, stage + K::BPS * K::TILE, min(K::TOK, ctx - (blk0 + j * K::BPS) * BS), lane);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[st]);
             }
@@ -421,7 +432,7 @@ cudaError_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const Pa
 // so three CTAs fit on an SM with ~190 KB of KV in flight.
 template <typename T, int D>
 constexpr int stages_for() {
-    constexpr int sb = 2 * BS * D * (int)sizeof(T);
+    constexpr int sb = 2 * (sizeof(T) == 1 ? 2 : 1) * BS * D * (int)sizeof(T);   // bytes of one stage (Kern::STAGE_BYTES)
     constexpr int n = 65536 / sb;
     return n < 4 ? 4 : (n > 16 ? 16 : n);
 }
