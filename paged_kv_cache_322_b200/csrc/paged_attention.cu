@@ -49,7 +49,7 @@ namespace attn {
 //   PATH 1: SIMT, head-split (every warp reads every block, HPW = group / NCW)
 //   PATH 2: tensor cores, block-split (group <= 8)
 // ---------------------------------------------------------------------------
-template <typename T, int D, int PATH, int HPW, int STAGES>
+template <typename T, int D, int PATH, int HPW, int STAGES, int KPC = 1>
 struct Kern {
     static constexpr bool kMma = PATH == 2;
     static constexpr int TILE = BS * D * (int)sizeof(T);              // one block, one head, K or V
@@ -60,7 +60,12 @@ struct Kern {
     // first, then V rows).
     static constexpr int BPS = sizeof(T) == 1 ? 2 : 1;                  // blocks per stage
     static constexpr int TOK = BS * BPS;
-    static constexpr int STAGE_BYTES = 2 * BPS * TILE;
+    // KPC KV heads per CTA: their tiles are loaded back to back, so a token row's
+    // neighbouring heads (adjacent in HBM) are read together; consumer warps split
+    // by head (WPH warps per head). Stage layout: K [head][block][tile], then V.
+    static constexpr int WPH = NCW / KPC;
+    static constexpr int STAGE_BYTES = 2 * BPS * KPC * TILE;
+    static_assert(PATH != 1 || KPC == 1, "head-split consumers serve one KV head");
     static constexpr int RING = STAGES * STAGE_BYTES;
     static constexpr int NSLOT = PATH == 1 ? 1 : NCW;                  // partial states to merge
     static constexpr int MAXG = PATH == 2 ? 8 : (PATH == 1 ? HPW * NCW : HPW);
@@ -71,21 +76,21 @@ struct Kern {
     // Block-split consumers take tiles round-robin; with STAGES a multiple of NCW
     // every round of a stage goes to the same warp, so no warp can wait on a ring
     // phase two rounds ahead of the producer (the parity wait would pass early).
-    static_assert(PATH == 1 || STAGES % NCW == 0, "ring depth must be a multiple of the consumer warps");
+    static_assert(PATH == 1 || STAGES % WPH == 0, "ring depth must be a multiple of the warps per head");
 };
 
-template <typename T, int D, int PATH, int HPW, int STAGES>
+template <typename T, int D, int PATH, int HPW, int STAGES, int KPC>
 __global__ void __launch_bounds__(NTHREADS, 3)
 paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const Params p) {
-    using K = Kern<T, D, PATH, HPW, STAGES>;
+    using K = Kern<T, D, PATH, HPW, STAGES, KPC>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + K::BODY);
     uint64_t* empty = full + STAGES;
     __shared__ volatile int s_abort;
 
-    const int kvh = blockIdx.x, part = blockIdx.y, seq = blockIdx.z;
+    const int kvh = blockIdx.x * KPC, part = blockIdx.y, seq = blockIdx.z;   // first KV head of this CTA
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     int ctx = p.context_lens[seq];
@@ -104,7 +109,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], PATH == 1 ? NCW : 1);
+            mbar_init(&empty[i], PATH == 1 ? NCW : KPC);
         }
         s_abort = 0;
         fence_barrier_init();
@@ -144,22 +149,27 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                             ok = false;
                             s_abort = 1;
                         } else {
-                            mbar_arrive_expect_tx(&full[st], min(K::BPS, nblk - j) * 2 * K::TILE);
+                            mbar_arrive_expect_tx(&full[st], min(K::BPS, nblk - j) * 2 * KPC * K::TILE);
                             ++issued;
                         }
                     }
                     if (ok) {
-                        uint8_t* dst = smem + st * K::STAGE_BYTES + b * K::TILE;
-                        uint8_t* vdst = dst + K::BPS * K::TILE;
-                        if constexpr (K::kMma) {
 #pragma unroll
-                            for (int h = 0; h < K::NBOX; ++h) {
-                                tma_load_4d(dst + h * (BS * 128), &tm_k, &full[st], h * K::BOX, kvh, 0, pb, pol);
-                                tma_load_4d(vdst + h * (BS * 128), &tm_v, &full[st], h * K::BOX, kvh, 0, pb, pol);
+                        for (int hd = 0; hd < KPC; ++hd) {
+                            uint8_t* dst = smem + st * K::STAGE_BYTES + (hd * K::BPS + b) * K::TILE;
+                            uint8_t* vdst = dst + KPC * K::BPS * K::TILE;
+                            if constexpr (K::kMma) {
+#pragma unroll
+                                for (int h = 0; h < K::NBOX; ++h) {
+                                    tma_load_4d(dst + h * (BS * 128), &tm_k, &full[st], h * K::BOX, kvh + hd, 0, pb,
+                                                pol);
+                                    tma_load_4d(vdst + h * (BS * 128), &tm_v, &full[st], h * K::BOX, kvh + hd, 0, pb,
+                                                pol);
+                                }
+                            } else {
+                                tma_load_4d(dst, &tm_k, &full[st], 0, kvh + hd, 0, pb, pol);
+                                tma_load_4d(vdst, &tm_v, &full[st], 0, kvh + hd, 0, pb, pol);
                             }
-                        } else {
-                            tma_load_4d(dst, &tm_k, &full[st], 0, kvh, 0, pb, pol);
-                            tma_load_4d(vdst, &tm_v, &full[st], 0, kvh, 0, pb, pol);
                         }
                     }
                 }
@@ -175,14 +185,16 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     } else {
         // ---------------- consumers ----------------
         const int cw = warp - 1;
+        const int hd = cw / K::WPH, sub = cw - hd * K::WPH;               // this warp's KV head, and its turn
         using TQ = std::conditional_t<sizeof(T) == 1, __nv_bfloat16, T>;   // an fp8 cache takes bf16 queries
-        const TQ* qbase = static_cast<const TQ*>(p.q) + ((int64_t)seq * p.num_q_heads + qh0) * D;
+        const TQ* qbase = static_cast<const TQ*>(p.q) + ((int64_t)seq * p.num_q_heads + qh0 + hd * group) * D;
         const int nstage = (nblk + K::BPS - 1) / K::BPS;
+        const int kofs = hd * K::BPS * K::TILE, vofs = (KPC + hd) * K::BPS * K::TILE;
         if constexpr (PATH == 2) {
             using Cons = std::conditional_t<sizeof(T) == 1, MmaConsumerFp8<K::BPS>, MmaConsumer<D>>;
             Cons c;
             c.init(reinterpret_cast<const __nv_bfloat16*>(qbase), group, lane);
-            for (int j = cw; j < nstage; j += NCW) {
+            for (int j = sub; j < nstage; j += K::WPH) {
                 const int st = j % STAGES;
                 const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err);
                 if (__any_sync(0xffffffffu, !got || s_abort != 0)) {   // warp-uniform exit
@@ -191,8 +203,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 }
                 uint8_t* stage = smem + st * K::STAGE_BYTES;
                 const int nvalid = min(K::TOK, ctx - (blk0 + j * K::BPS) * BS);
-                uint8_t* vst = stage + K::BPS * K::TILE;
-                c.consume(smem_u32(stage), smem_u32(vst), vst, nvalid, p.scale_log2, lane);
+                uint8_t* vst = stage + vofs;
+                c.consume(smem_u32(stage + kofs), smem_u32(vst), vst, nvalid, p.scale_log2, lane);
                 if (nvalid < K::TOK) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[st]);
@@ -204,7 +216,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             const int hbase = PATH == 1 ? cw * HPWc : 0;
             SimtConsumer<T, D, HPWc, TQ, K::TOK> c;
             c.init(qbase + (int64_t)hbase * D, p.scale_log2, lane);
-            const int jstart = PATH == 1 ? 0 : cw, jstep = PATH == 1 ? 1 : NCW;
+            const int jstart = PATH == 1 ? 0 : sub, jstep = PATH == 1 ? 1 : K::WPH;
             for (int j = jstart; j < nstage; j += jstep) {
                 const int st = j % STAGES;
                 const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err);
@@ -213,7 +225,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     break;
                 }
                 const uint8_t* stage = smem + st * K::STAGE_BYTES;
-                c.consume(stage, stage + K::BPS * K::TILE, min(K::TOK, ctx - (blk0 + j * K::BPS) * BS), lane);
+                c.consume(stage + kofs, stage + vofs, min(K::TOK, ctx - (blk0 + j * K::BPS) * BS), lane);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[st]);
             }
@@ -227,17 +239,19 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     if (s_abort) return;
 
     // ---------------- merge consumer states, write output or partial ----------------
-    const int nheads = group;
+    // KV head hd of this CTA: its states are in warp slots [hd * NSLOT / KPC, (hd + 1) * NSLOT / KPC).
+    constexpr int SPH = K::NSLOT / KPC;
     const int C = p.num_parts;
-    for (int idx = threadIdx.x; idx < nheads * D; idx += NTHREADS) {
-        const int h = idx / D, d = idx - h * D;
+    for (int idx = threadIdx.x; idx < KPC * group * D; idx += NTHREADS) {
+        const int hd = idx / (group * D), rem = idx - hd * group * D;
+        const int h = rem / D, d = rem - h * D;
         float M = kNegInf;
 #pragma unroll
-        for (int w = 0; w < K::NSLOT; ++w) M = fmaxf(M, red_m[w * K::MAXG + h]);
+        for (int w = hd * SPH; w < (hd + 1) * SPH; ++w) M = fmaxf(M, red_m[w * K::MAXG + h]);
         float L = 0.f, O = 0.f;
         if (M != kNegInf) {
 #pragma unroll
-            for (int w = 0; w < K::NSLOT; ++w) {
+            for (int w = hd * SPH; w < (hd + 1) * SPH; ++w) {
                 const float mw = red_m[w * K::MAXG + h];
                 if (mw == kNegInf) continue;
                 const float sc = fast_exp2(mw - M);
@@ -246,7 +260,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
         }
         const float val = L > 0.f ? O / L : 0.f;
-        const int64_t qh = (int64_t)seq * p.num_q_heads + qh0 + h;
+        const int64_t qh = (int64_t)seq * p.num_q_heads + qh0 + hd * group + h;
         if (nparts <= 1) {
             store_out(p, qh * D + d, val);
         } else {
@@ -409,11 +423,12 @@ size_t ws_bytes_for(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
     return o_bytes + rows * 2 * 4;
 }
 
-template <typename T, int D, int PATH, int HPW, int STAGES>
+template <typename T, int D, int PATH, int HPW, int STAGES, int KPC = 1>
 cudaError_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, dim3 grid,
                           cudaStream_t stream) {
-    using K = Kern<T, D, PATH, HPW, STAGES>;
-    auto kern = paged_decode_kernel<T, D, PATH, HPW, STAGES>;
+    using K = Kern<T, D, PATH, HPW, STAGES, KPC>;
+    auto kern = paged_decode_kernel<T, D, PATH, HPW, STAGES, KPC>;
+    grid.x /= KPC;
     // Opt in to >48 KB dynamic shared memory once per device.
     static std::atomic<uint64_t> done_mask{0};
     int dev = 0;
@@ -430,21 +445,23 @@ cudaError_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const Pa
 
 // Ring depth: about 64 KB of stages per CTA (8 KB per stage for bf16 D=128),
 // so three CTAs fit on an SM with ~190 KB of KV in flight.
-template <typename T, int D>
+template <typename T, int D, int KPC = 1>
 constexpr int stages_for() {
-    constexpr int sb = 2 * (sizeof(T) == 1 ? 2 : 1) * BS * D * (int)sizeof(T);   // bytes of one stage (Kern::STAGE_BYTES)
+    constexpr int sb = 2 * (sizeof(T) == 1 ? 2 : 1) * KPC * BS * D * (int)sizeof(T);   // Kern::STAGE_BYTES
     constexpr int n = 65536 / sb;
     return n < 4 ? 4 : (n > 16 ? 16 : n);
 }
 
-template <typename T, int D>
+template <typename T, int D, int KPC = 1>
 cudaError_t dispatch_simt(int group, const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, dim3 grid,
                           cudaStream_t st) {
     switch (group) {
-        case 1: return launch_decode<T, D, 0, 1, stages_for<T, D>()>(mk, mv, p, grid, st);
-        case 2: return launch_decode<T, D, 0, 2, stages_for<T, D>()>(mk, mv, p, grid, st);
-        case 4: return launch_decode<T, D, 1, 1, stages_for<T, D>()>(mk, mv, p, grid, st);
-        case 8: return launch_decode<T, D, 1, 2, stages_for<T, D>()>(mk, mv, p, grid, st);
+        case 1: return launch_decode<T, D, 0, 1, stages_for<T, D, KPC>(), KPC>(mk, mv, p, grid, st);
+        case 2: return launch_decode<T, D, 0, 2, stages_for<T, D, KPC>(), KPC>(mk, mv, p, grid, st);
+        case 4: return KPC == 1 ? launch_decode<T, D, 1, 1, stages_for<T, D>()>(mk, mv, p, grid, st)
+                                : cudaErrorInvalidValue;
+        case 8: return KPC == 1 ? launch_decode<T, D, 1, 2, stages_for<T, D>()>(mk, mv, p, grid, st)
+                                : cudaErrorInvalidValue;
         default: return cudaErrorInvalidValue;
     }
 }
@@ -565,8 +582,16 @@ pkv_status decode_impl(void* out, pkv_dtype out_dtype, const void* q, const void
     dim3 grid(num_kv_heads, pl.num_parts, num_seqs);
     cudaError_t e;
     if (fp8) {
-        e = use_mma ? launch_decode<uint8_t, 128, 2, 8, stages_for<uint8_t, 128>()>(mk, mv, p, grid, st)
-                    : dispatch_simt<uint8_t, 128>(group, mk, mv, p, grid, st);
+        // Two KV heads per CTA where the SIMT path splits by block (groups 1, 2)
+        // or on tensor cores: each token's 256 contiguous bytes of K (and of V)
+        // are fetched in one go instead of two 128-byte halves by different CTAs.
+        const bool pair = num_kv_heads % 2 == 0 && (use_mma || group <= 2);
+        if (use_mma)
+            e = pair ? launch_decode<uint8_t, 128, 2, 8, stages_for<uint8_t, 128, 2>(), 2>(mk, mv, p, grid, st)
+                     : launch_decode<uint8_t, 128, 2, 8, stages_for<uint8_t, 128>()>(mk, mv, p, grid, st);
+        else
+            e = pair ? dispatch_simt<uint8_t, 128, 2>(group, mk, mv, p, grid, st)
+                     : dispatch_simt<uint8_t, 128>(group, mk, mv, p, grid, st);
     } else if (use_mma) {
         e = head_dim == 128
                 ? launch_decode<__nv_bfloat16, 128, 2, 8, stages_for<__nv_bfloat16, 128>()>(mk, mv, p, grid, st)
