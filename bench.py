@@ -56,6 +56,8 @@ def parse():
                     help="-2: the workload's; 0: library-chosen partitions; -1: persistent schedule; >0: fixed")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-paging-overhead", action="store_true",
+                    help="skip the random- vs identity-placement timing of the attention call")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     ap.add_argument("--num-seqs", type=int, default=0, help="override the batch size (profiling a small case)")
     ap.add_argument("--num-blocks", type=int, default=0, help="override the pool size (profiling a small case)")
@@ -207,9 +209,10 @@ def traffic_record(workload: str):
         return None
     with open(path) as f:
         rec = json.load(f)
-    if rec.get("source_sha1") != kernel_source_sha1() or workload not in rec:
+    entry = rec.get(workload)
+    if not isinstance(entry, dict) or entry.get("source_sha1") != kernel_source_sha1():
         return None
-    return rec[workload]
+    return entry
 
 
 def kernel_source_sha1() -> str:
@@ -273,11 +276,14 @@ def run_pkv(args, ws, rank, local):
     for s in range(w.num_seqs):
         k, v = kvs[s]
         cache.add_sequence(s, torch.from_numpy(k).to(dev, dt), torch.from_numpy(v).to(dev, dt))
-    del kvs
     ids = np.arange(w.num_seqs, dtype=np.int64)
     if w.ctx == "shared_prefix":
         raise SystemExit("the shared-prefix workload is a parity case; bench the decode workloads")
     torch.cuda.synchronize()
+    paging = None
+    if not args.no_paging_overhead and part != -1:
+        paging = paging_overhead(w, cache, kvs, dev, dt, cdt, mb, part, K, W)
+    del kvs
 
     # ---- per-step inputs, resident in HBM before timing ----
     steps = []
@@ -407,11 +413,56 @@ def run_pkv(args, ws, rank, local):
                      "traffic": (int(tr["traffic_per_algorithmic_byte"] * attn_bytes_avg) if tr else None),
                      "traffic_source": (tr["captured_on"] if tr else None)},
         "e2e": e2e,
+        "paging_overhead": paging,
         "gpu_launches": launches_per_step * K,
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,
     }
     return result
+
+
+def paging_overhead(w, cache, kvs, dev, dt, cdt, mb, part, K, W):
+    """The same attention call over the same prompts stored twice: blocks in the
+    workload's random physical placement (the bench cache) and in identity
+    placement (each sequence's blocks consecutive in the pool). Calls alternate,
+    each timed with CUDA events; ratio = random / identity time."""
+    import torch
+    from paged_kv_cache_322_b200 import binding
+    from paged_kv_cache_322_b200.engine import PagedKVCache
+    ident = PagedKVCache(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, cdt, dev,
+                         free_order=np.arange(w.num_blocks, dtype=np.int32), max_blocks_per_seq=mb,
+                         kv_scales=(w.kv_scale, w.kv_scale))
+    for s in range(w.num_seqs):
+        k, v = kvs[s]
+        ident.add_sequence(s, torch.from_numpy(k).to(dev, dt), torch.from_numpy(v).to(dev, dt))
+    ids = np.arange(w.num_seqs, dtype=np.int64)
+    legs = []
+    for c in (cache, ident):
+        tables, lens = c.block_tables(ids)
+        legs.append((c, torch.from_numpy(tables).to(dev), torch.from_numpy(lens).to(dev), int(lens.max())))
+    q = torch.from_numpy(wl.decode_q(w, 0)).to(dev, dt)
+    out = torch.empty((w.num_seqs, w.num_q_heads, w.head_dim), dtype=torch.bfloat16, device=dev)
+    ws_bytes = binding.workspace_bytes(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, mb,
+                                       legs[0][3], part)
+    workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    times = ([], [])
+    for i in range(W + K):
+        for j, (c, t, l, mx) in enumerate(legs):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            c.attention(out, q, t, l, w.scale, max_context_len=mx, partition_tokens=part, workspace=workspace)
+            e1.record(stream)
+            if i >= W:
+                times[j].append((e0, e1))
+    torch.cuda.synchronize()
+    assert binding.get_device_error() == 0
+    r_ms, i_ms = (statistics.median(a.elapsed_time(b) for a, b in t) for t in times)
+    del ident
+    torch.cuda.empty_cache()
+    return {"random_placement_ms": round(r_ms, 5), "identity_placement_ms": round(i_ms, 5),
+            "ratio": round(r_ms / i_ms, 4),
+            "what": "median attention-call time over the prompts (no append), random vs identity block placement"}
 
 
 def cpu_baseline(w: wl.Workload, target_s: float):
