@@ -45,6 +45,16 @@ def copy_blocks(k_cache, v_cache, src, dst):
         v_cache[d] = snap_v[i]
 
 
+def swap_blocks(src_k, src_v, dst_k, dst_v, src, dst):
+    """dst_pool[dst[i]] = src_pool[src[i]] for every pair, K and V: the block
+    moves of a swap between the GPU pool and the CPU pool ("vLLM PagedAttention
+    深度解析" §5.2 Swapping; "LLM 推理引擎内部原理" §3.1 blocks_to_swap_in/out).
+    The two pools are different arrays, so pairs cannot alias. In place on dst."""
+    for s, d in zip(np.asarray(src).tolist(), np.asarray(dst).tolist()):
+        dst_k[int(d)] = np.array(src_k[int(s)], copy=True)
+        dst_v[int(d)] = np.array(src_v[int(s)], copy=True)
+
+
 def reshape_and_cache_fp8(k, v, k_codes, v_codes, slot_mapping, k_scale: float, v_scale: float):
     """KV append into an FP8 (e4m3) cache: token t's K (V) is stored as the
     codes of float32(k[t] * inv_scale) (see oracle.fp8). Caches hold uint8 codes."""
