@@ -51,6 +51,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="pkv", choices=["pkv", "reference"])
+    ap.add_argument("--op", default="decode", choices=["decode", "swap"],
+                    help="decode: the decode step (append + attention); swap: preemption by swapping half the "
+                         "workload's sequences to a page-locked host pool and back")
     ap.add_argument("--workload", default="llama2_7b", choices=list(wl.WORKLOADS))
     ap.add_argument("--partition-tokens", type=int, default=-2,
                     help="-2: the workload's; 0: library-chosen partitions; -1: persistent schedule; >0: fixed")
@@ -421,6 +424,124 @@ def run_pkv(args, ws, rank, local):
     return result
 
 
+def run_swap(args, ws, rank, local):
+    """Swap-out and swap-in of every other sequence of the workload through the
+    cache's public calls (block manager + block-id staging + one swap kernel per
+    direction), timed with CUDA events; the kernel alone on the same block sets;
+    and, as the host-link roofline, one contiguous page-locked copy of the same
+    bytes per direction by the copy engine."""
+    import torch
+    from paged_kv_cache_322_b200 import binding
+    from paged_kv_cache_322_b200.engine import PagedKVCache
+
+    dev = torch.device("cuda", local)
+    w = replica_workload(wl.WORKLOADS[args.workload], rank)
+    if args.num_seqs or args.num_blocks:
+        w = dataclasses.replace(w, num_seqs=args.num_seqs or w.num_seqs, num_blocks=args.num_blocks or w.num_blocks)
+    K, W = args.steps, args.warmup
+    lens = wl.context_lens(w)
+    bs = w.block_size
+    group = list(range(0, w.num_seqs, 2))
+    nblk = int(sum(-(-int(lens[s]) // bs) for s in group))
+    cdt = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.uint8}[w.kv_dtype]
+    cache = PagedKVCache(w.num_blocks, bs, w.num_kv_heads, w.head_dim, cdt, dev, free_order=wl.free_order(w),
+                         host_blocks=nblk)
+    for s in range(w.num_seqs):
+        cache.bm.allocate(s, int(lens[s]))
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed)
+    for c in (cache.k_cache, cache.v_cache):           # synthetic pool contents (a copy does not read values)
+        c.view(torch.uint8).copy_(torch.randint(0, 256, c.view(torch.uint8).shape, device=dev, dtype=torch.uint8,
+                                                generator=g))
+    stream = torch.cuda.current_stream(dev)
+    block_bytes = bs * w.num_kv_heads * w.head_dim * w.elt_bytes
+    moved = 2 * nblk * block_bytes                       # K and V, one direction
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    # ---- through the cache's calls ----
+    t_out, t_in = [], []
+    for i in range(W + K):
+        e0, e1, e2 = ev(), ev(), ev()
+        e0.record(stream)
+        pairs_out = cache.swap_out(group)
+        e1.record(stream)
+        pairs_in = cache.swap_in(group)
+        e2.record(stream)
+        if i >= W:
+            t_out.append((e0, e1))
+            t_in.append((e1, e2))
+    torch.cuda.synchronize()
+    assert binding.get_device_error() == 0 and len(pairs_out) == nblk and len(pairs_in) == nblk
+    api_out = statistics.median(a.elapsed_time(b) for a, b in t_out)
+    api_in = statistics.median(a.elapsed_time(b) for a, b in t_in)
+
+    # ---- the kernel alone, same block sets (device ids of the last swap-in) ----
+    dblk = torch.tensor([d for _, d in pairs_in], dtype=torch.int64, device=dev)
+    hblk = torch.tensor([h for h, _ in pairs_in], dtype=torch.int64, device=dev)
+    k_out, k_in = [], []
+    for i in range(W + K):
+        e0, e1, e2 = ev(), ev(), ev()
+        e0.record(stream)
+        binding.swap_blocks(cache.k_cache, cache.v_cache, cache.k_host, cache.v_host, dblk, hblk)
+        e1.record(stream)
+        binding.swap_blocks(cache.k_host, cache.v_host, cache.k_cache, cache.v_cache, hblk, dblk)
+        e2.record(stream)
+        if i >= W:
+            k_out.append((e0, e1))
+            k_in.append((e1, e2))
+    torch.cuda.synchronize()
+    assert binding.get_device_error() == 0
+    kern_out = statistics.median(a.elapsed_time(b) for a, b in k_out)
+    kern_in = statistics.median(a.elapsed_time(b) for a, b in k_in)
+
+    # ---- roofline: one contiguous page-locked copy of the same bytes per direction ----
+    hbuf = torch.empty(moved, dtype=torch.uint8, pin_memory=True)
+    dbuf = torch.empty(moved, dtype=torch.uint8, device=dev)
+    c_out, c_in = [], []
+    for i in range(W + K):
+        e0, e1, e2 = ev(), ev(), ev()
+        e0.record(stream)
+        hbuf.copy_(dbuf, non_blocking=True)
+        e1.record(stream)
+        dbuf.copy_(hbuf, non_blocking=True)
+        e2.record(stream)
+        if i >= W:
+            c_out.append((e0, e1))
+            c_in.append((e1, e2))
+    torch.cuda.synchronize()
+    copy_out = statistics.median(a.elapsed_time(b) for a, b in c_out)
+    copy_in = statistics.median(a.elapsed_time(b) for a, b in c_in)
+
+    def gbs(ms):
+        return round(moved / (ms * 1e-3) / 1e9, 2)
+
+    ms_step = api_out + api_in
+    ms_max, total_gbs, _ = aggregate(ms_step * K, 2.0 * moved * K, float(len(group) * K), ws)
+    ach = 2.0 * moved / ((kern_out + kern_in) * 1e-3) / 1e9
+    peak = 2.0 * moved / ((copy_out + copy_in) * 1e-3) / 1e9
+    return {
+        "metric": "swap_blocks: preemption swap-out + swap-in GB/s over the host link (device <-> page-locked host)",
+        "value": round(total_gbs, 2), "unit": "GB/s", "n_gpus": ws, "steps": K, "warmup": W,
+        "ms_per_step": round(ms_max / K, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.kv_dtype, "data": "synthetic",
+        "config": {"workload": f"swap every other sequence of: {w.description}", "sequences_swapped": len(group),
+                   "blocks_per_direction": nblk, "bytes_per_direction": moved,
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+        "api": {"swap_out_ms": round(api_out, 4), "swap_in_ms": round(api_in, 4), "swap_out_gbs": gbs(api_out),
+                "swap_in_gbs": gbs(api_in)},
+        "kernel": {"swap_out_ms": round(kern_out, 4), "swap_in_ms": round(kern_in, 4),
+                   "swap_out_gbs": gbs(kern_out), "swap_in_gbs": gbs(kern_in)},
+        "roofline": {"bound": "host_link", "achieved": round(ach, 2), "peak": round(peak, 2), "unit": "GB/s",
+                     "frac": round(ach / peak, 4),
+                     "peak_source": "measured in this run: one contiguous page-locked copy of the same bytes per "
+                                    f"direction (copy engine; out {gbs(copy_out)} GB/s, in {gbs(copy_in)} GB/s)",
+                     "traffic": None},
+        "gpu_launches": 2 * K,
+    }
+
+
 def paging_overhead(w, cache, kvs, dev, dt, cdt, mb, part, K, W):
     """The same attention call over the same prompts stored twice: blocks in the
     workload's random physical placement (the bench cache) and in identity
@@ -539,7 +660,7 @@ def main():
         return
     ws, rank, local = dist_init(args)
     try:
-        r = run_pkv(args, ws, rank, local)
+        r = run_swap(args, ws, rank, local) if args.op == "swap" else run_pkv(args, ws, rank, local)
         if rank == 0:
             print(json.dumps(r), flush=True)
     finally:

@@ -7,6 +7,8 @@
  *     reached through per-sequence block tables (MHA and grouped-query).
  *   - pkv_reshape_and_cache      : the per-token KV append into the cache.
  *   - pkv_copy_blocks            : physical block copies for copy-on-write forks.
+ *   - pkv_swap_blocks            : block moves between the device pool and a
+ *     page-locked host pool (preemption by swapping).
  *   - pkv_bm_*                   : a host-side block manager (free list, block
  *     tables, slot mapping, reference counts, copy-on-write) that produces the
  *     block tables, slot mappings and copy lists the kernels consume.
@@ -21,7 +23,8 @@
  *         two-level addressing block table -> physical block -> in-block offset).
  *   [VP]  "vLLM PagedAttention 深度解析" (cyqw.cn), §3.3 (single-request prefill and
  *         decode flow), §4.1 (parallel sampling, reference counts, copy-on-write),
- *         §4.2 (beam search, blocks freed when their count reaches 0).
+ *         §4.2 (beam search, blocks freed when their count reaches 0), §5.2
+ *         (preemption: a request's KV blocks swapped out to CPU memory and back).
  *
  * Conventions shared by every call:
  *   - Every data pointer passed to a kernel entry point is a DEVICE pointer
@@ -238,6 +241,34 @@ pkv_status pkv_copy_blocks(
     int block_size, int num_kv_heads, int head_dim, int num_blocks, void* stream);
 
 /*
+ * Block moves of a swap ([VP] §5.2: a preempted request's KV blocks go out to
+ * CPU memory, freeing their GPU blocks, and come back when it resumes; [ENG]
+ * §3.1 hands them to the cache engine as blocks_to_swap_out / blocks_to_swap_in):
+ *     dst_k[dst[i]] = src_k[src[i]],  dst_v[dst[i]] = src_v[src[i]]
+ * for i < num_pairs, every slot of the block, between two pools of the same
+ * block shape [*, block_size, num_kv_heads, head_dim] and dtype.
+ *
+ *   src_k_cache, src_v_cache  [src_num_blocks, ...]: device memory, or page-locked
+ *                             host memory (cudaHostAlloc / cudaHostRegister; the
+ *                             kernel reads it through its mapped device address)
+ *   dst_k_cache, dst_v_cache  [dst_num_blocks, ...]: the same choice
+ *   src_block_ids, dst_block_ids  int64 [num_pairs], device or page-locked host
+ * Swap-out is device -> host, swap-in host -> device; one kernel moves all pairs
+ * over the host link, so scattered blocks need no per-block copy calls. Pageable
+ * host memory, or K and V of one side in different kinds of memory, return
+ * PKV_ERR_INVALID_ARG. Destination ids must be distinct; if both sides are the
+ * same pool the rules of pkv_copy_blocks apply. Ids outside their pool are
+ * skipped and flagged PKV_ERR_DEVICE_BOUNDS. The caller owns all memory and keeps
+ * the host buffers alive until the stream has passed the call. num_pairs may be
+ * 0 (nothing is launched); at most 65535 pairs per call.
+ */
+pkv_status pkv_swap_blocks(
+    const void* src_k_cache, const void* src_v_cache, int src_num_blocks,
+    void* dst_k_cache, void* dst_v_cache, int dst_num_blocks, pkv_dtype dtype,
+    const int64_t* src_block_ids, const int64_t* dst_block_ids, int num_pairs,
+    int block_size, int num_kv_heads, int head_dim, void* stream);
+
+/*
  * FP8 KV append ("vLLM PagedAttention 深度解析" §7.4: K/V stored as FP8 so a block
  * holds twice the tokens). Same addressing as pkv_reshape_and_cache; the caches
  * hold e4m3 codes (1 byte per element) and the stored code of an element x is
@@ -353,6 +384,38 @@ pkv_status pkv_bm_free(pkv_block_manager* bm, int64_t seq_id);
  * sequence has more than max_blocks blocks. context_lens_out may be NULL. */
 pkv_status pkv_bm_block_tables(const pkv_block_manager* bm, const int64_t* seq_ids, int n,
                                int max_blocks, int32_t* tables_out, int32_t* context_lens_out);
+
+/*
+ * Host (CPU) block pool for swapping ([VP] §5.2). Set once, before any swap:
+ * num_host_blocks ids with their own FIFO free list (free_order or NULL for
+ * 0,1,2,...) and reference counts.
+ */
+pkv_status pkv_bm_set_host_pool(pkv_block_manager* bm, int num_host_blocks, const int32_t* free_order);
+
+/*
+ * Swap-out of a group of resident sequences: every distinct device block their
+ * tables reference gets one host block (taken in order of first appearance,
+ * sequences in the given order, tables in order), written as the pair
+ * (dev_blocks_out[i], host_blocks_out[i]) for the copy; each reference moves its
+ * count from the device block (freed at 0, so blocks still used by a sequence
+ * left behind stay) to the host block. The sequences become swapped out: their
+ * tables hold host ids, and append, fork, make_writable and block_tables refuse
+ * them (PKV_ERR_INVALID_ARG); pkv_bm_free releases their host blocks.
+ * capacity: room in each output array (the group's total block count always
+ * suffices). All or nothing: PKV_ERR_OUT_OF_BLOCKS if the host pool has too few
+ * free blocks; PKV_ERR_INVALID_ARG for an unknown, repeated or swapped-out id.
+ */
+pkv_status pkv_bm_swap_out(pkv_block_manager* bm, const int64_t* seq_ids, int n, int64_t* dev_blocks_out,
+                           int64_t* host_blocks_out, int capacity, int* num_pairs_out);
+
+/* The mirror image for swapped-out sequences: pairs (host, device). */
+pkv_status pkv_bm_swap_in(pkv_block_manager* bm, const int64_t* seq_ids, int n, int64_t* host_blocks_out,
+                          int64_t* dev_blocks_out, int capacity, int* num_pairs_out);
+
+int pkv_bm_num_free_host(const pkv_block_manager* bm);
+int pkv_bm_host_ref_count(const pkv_block_manager* bm, int block);
+/* 1 swapped out, 0 resident, -1 unknown. */
+int pkv_bm_is_swapped(const pkv_block_manager* bm, int64_t seq_id);
 
 int pkv_bm_num_free(const pkv_block_manager* bm);
 int pkv_bm_ref_count(const pkv_block_manager* bm, int block);

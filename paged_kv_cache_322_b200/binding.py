@@ -48,6 +48,7 @@ _SIGS = {
     "pkv_paged_attention_partition_tokens": (_i32, [_i32] * 8),
     "pkv_reshape_and_cache": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pkv_copy_blocks": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
+    "pkv_swap_blocks": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp]),
     "pkv_get_device_error": (_i32, [_c.POINTER(_c.c_int), _vp]),
     "pkv_step_ctx_create": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _f32, _c.POINTER(_vp)]),
     "pkv_step_ctx_destroy": (None, [_vp]),
@@ -64,6 +65,12 @@ _SIGS = {
     "pkv_bm_num_free": (_i32, [_vp]),
     "pkv_bm_ref_count": (_i32, [_vp, _i32]),
     "pkv_bm_seq_len": (_i32, [_vp, _i64]),
+    "pkv_bm_set_host_pool": (_i32, [_vp, _i32, _pi32]),
+    "pkv_bm_swap_out": (_i32, [_vp, _pi64, _i32, _pi64, _pi64, _i32, _c.POINTER(_c.c_int)]),
+    "pkv_bm_swap_in": (_i32, [_vp, _pi64, _i32, _pi64, _pi64, _i32, _c.POINTER(_c.c_int)]),
+    "pkv_bm_num_free_host": (_i32, [_vp]),
+    "pkv_bm_host_ref_count": (_i32, [_vp, _i32]),
+    "pkv_bm_is_swapped": (_i32, [_vp, _i64]),
 }
 
 
@@ -280,6 +287,32 @@ def copy_blocks(k_cache, v_cache, src, dst, stream=None):
     _check(st, "pkv_copy_blocks")
 
 
+def swap_blocks(src_k, src_v, dst_k, dst_v, src, dst, stream=None):
+    """dst_pool[dst[i]] = src_pool[src[i]] for K and V between two pools of the
+    same block shape: CUDA tensors or page-locked (pin_memory) CPU tensors, e.g.
+    device -> host for a swap-out. src, dst: int64 tensors (CUDA or pinned)."""
+    torch = _torch()
+    for t in (src_k, src_v, dst_k, dst_v, src, dst):
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+        if not (t.is_cuda or t.is_pinned()):
+            raise ValueError("swap_blocks takes CUDA tensors or page-locked CPU tensors")
+    if src.dtype != torch.int64 or dst.dtype != torch.int64 or src.numel() != dst.numel():
+        raise TypeError("src and dst must be int64 tensors of equal length")
+    if src_k.shape[1:] != dst_k.shape[1:] or src_k.dtype != dst_k.dtype:
+        raise ValueError("both pools must have the same block shape and dtype")
+    dev = next((t.device for t in (src_k, dst_k, src, dst) if t.is_cuda), None)
+    if dev is None:
+        raise ValueError("one side of the swap must be on the device")
+    st = stream.cuda_stream if stream is not None else torch.cuda.current_stream(dev).cuda_stream
+    _, bs, hkv, d = src_k.shape
+    with torch.cuda.device(dev):
+        r = _lib().pkv_swap_blocks(src_k.data_ptr(), src_v.data_ptr(), src_k.shape[0], dst_k.data_ptr(),
+                                   dst_v.data_ptr(), dst_k.shape[0], _dtype_code(src_k), src.data_ptr(),
+                                   dst.data_ptr(), src.numel(), bs, hkv, d, st)
+    _check(r, "pkv_swap_blocks")
+
+
 def get_device_error(stream=None) -> int:
     """Reads and clears the current device's error word (synchronises the stream)."""
     torch = _torch()
@@ -360,6 +393,48 @@ class BlockManager:
 
     def seq_len(self, seq_id: int) -> int:
         return _lib().pkv_bm_seq_len(self._h, seq_id)
+
+    # -- swapping ------------------------------------------------------------
+    def set_host_pool(self, num_host_blocks: int, free_order=None):
+        order = None
+        if free_order is not None:
+            order = np.ascontiguousarray(free_order, dtype=np.int32)
+            if order.size != num_host_blocks:
+                raise ValueError("free_order must list every host block")
+        _check(_lib().pkv_bm_set_host_pool(self._h, num_host_blocks,
+                                           _ptr(order, ctypes.c_int32) if order is not None else None),
+               "pkv_bm_set_host_pool")
+        self.num_host_blocks = num_host_blocks
+
+    def _swap(self, fn, seq_ids):
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        cap = sum(max(0, -(-max(self.seq_len(int(s)), 0) // self.block_size)) for s in ids.tolist())
+        a = np.empty(max(cap, 1), np.int64)
+        b = np.empty(max(cap, 1), np.int64)
+        n = ctypes.c_int(0)
+        _check(getattr(_lib(), fn)(self._h, _ptr(ids, ctypes.c_int64), ids.size, _ptr(a, ctypes.c_int64),
+                                   _ptr(b, ctypes.c_int64), cap, ctypes.byref(n)), fn)
+        return a[:n.value], b[:n.value]
+
+    def swap_out(self, seq_ids):
+        """Moves the group to host blocks -> (device_blocks, host_blocks) to copy."""
+        return self._swap("pkv_bm_swap_out", seq_ids)
+
+    def swap_in(self, seq_ids):
+        """Brings the group back -> (host_blocks, device_blocks) to copy."""
+        return self._swap("pkv_bm_swap_in", seq_ids)
+
+    def num_free_host(self) -> int:
+        return _lib().pkv_bm_num_free_host(self._h)
+
+    def host_ref_count(self, block: int) -> int:
+        return _lib().pkv_bm_host_ref_count(self._h, block)
+
+    def is_swapped(self, seq_id: int) -> bool:
+        r = _lib().pkv_bm_is_swapped(self._h, seq_id)
+        if r < 0:
+            raise KeyError(seq_id)
+        return bool(r)
 
 
 class DecodeStep:

@@ -10,7 +10,15 @@
 // writer (old count - 1, new count 1); §4.2: a block returns to the pool when its
 // count reaches 0.
 //
-// The free list is a ring buffer of capacity num_blocks (each id is either in
+// Swapping ("为什么PagedAttention能让大模型推理吞吐量提升数倍", section on
+// scheduling and preemption; "vLLM PagedAttention 深度解析" §5.2): a second pool
+// of host (CPU) blocks with its own free list and counts. swap_out moves a set of
+// sequences' blocks to host blocks (each distinct block once, counts moved per
+// reference, device blocks freed at 0) and yields the (device, host) block map
+// for the copy; swap_in is the mirror image. All or nothing: a move that does
+// not fit in the destination pool changes nothing.
+//
+// Each free list is a ring buffer of capacity num_blocks (each id is either in
 // the ring or referenced, never both), so every call is O(1) per block.
 #include <cstdint>
 #include <cstring>
@@ -25,18 +33,33 @@ namespace {
 struct Seq {
     std::vector<int32_t> table;
     int64_t len = 0;
+    bool swapped = false;           // table holds host block ids
 };
 
-}  // namespace
-
-struct pkv_block_manager {
-    int num_blocks = 0;
-    int block_size = 0;
+struct Pool {
     std::vector<int32_t> ring;      // free list, FIFO
     size_t head = 0, count = 0;
     std::vector<int32_t> ref;
-    std::unordered_map<int64_t, Seq> seqs;
 
+    bool init(int n, const int32_t* order) {
+        ring.resize(n);
+        ref.assign(n, 0);
+        if (order) {
+            std::vector<char> seen(n, 0);
+            for (int i = 0; i < n; ++i) {
+                const int32_t b = order[i];
+                if (b < 0 || b >= n || seen[b]) return false;
+                seen[b] = 1;
+                ring[i] = b;
+            }
+        } else {
+            for (int i = 0; i < n; ++i) ring[i] = i;
+        }
+        head = 0;
+        count = n;
+        return true;
+    }
+    int size() const { return (int)ref.size(); }
     bool take(int32_t* b) {
         if (count == 0) return false;
         *b = ring[head];
@@ -52,8 +75,64 @@ struct pkv_block_manager {
     void release(int32_t b) {
         if (--ref[b] == 0) give_back(b);
     }
+};
+
+}  // namespace
+
+struct pkv_block_manager {
+    int num_blocks = 0;
+    int block_size = 0;
+    Pool dev, host;
+    std::unordered_map<int64_t, Seq> seqs;
+
+    bool take(int32_t* b) { return dev.take(b); }
+    void release(int32_t b) { dev.release(b); }
+    size_t free_count() const { return dev.count; }
     int64_t slot(const Seq& s, int64_t pos) const {
         return (int64_t)s.table[pos / block_size] * block_size + pos % block_size;
+    }
+    // A resident sequence, or nullptr (unknown or swapped out).
+    Seq* resident(int64_t id) {
+        auto it = seqs.find(id);
+        return (it == seqs.end() || it->second.swapped) ? nullptr : &it->second;
+    }
+
+    // Moves the listed sequences' blocks from pool `from` to pool `to`.
+    pkv_status move(const int64_t* ids, int n, bool out, int64_t* src_out, int64_t* dst_out, int capacity,
+                    int* num_pairs) {
+        Pool& from = out ? dev : host;
+        Pool& to = out ? host : dev;
+        std::unordered_map<int32_t, int32_t> fresh;       // source block -> destination block
+        std::unordered_map<int64_t, char> listed;
+        for (int i = 0; i < n; ++i) {
+            auto it = seqs.find(ids[i]);
+            if (it == seqs.end() || it->second.swapped != !out || listed.count(ids[i]))
+                return PKV_ERR_INVALID_ARG;
+            listed[ids[i]] = 1;
+            for (int32_t b : it->second.table) fresh.emplace(b, -1);
+        }
+        if (fresh.size() > (size_t)capacity) return PKV_ERR_INVALID_ARG;
+        if (fresh.size() > to.count) return PKV_ERR_OUT_OF_BLOCKS;
+        int np = 0;
+        for (int i = 0; i < n; ++i) {
+            Seq& s = seqs[ids[i]];
+            for (int32_t& b : s.table) {
+                int32_t& d = fresh[b];
+                if (d < 0) {                                  // first sight: one copy
+                    to.take(&d);
+                    to.ref[d] = 0;
+                    src_out[np] = b;
+                    dst_out[np] = d;
+                    ++np;
+                }
+                to.ref[d] += 1;
+                from.release(b);
+                b = d;
+            }
+            s.swapped = out;
+        }
+        *num_pairs = np;
+        return PKV_OK;
     }
 };
 
@@ -67,23 +146,49 @@ pkv_status pkv_bm_create(int num_blocks, int block_size, const int32_t* free_ord
     if (!bm) return PKV_ERR_INVALID_ARG;
     bm->num_blocks = num_blocks;
     bm->block_size = block_size;
-    bm->ring.resize(num_blocks);
-    bm->ref.assign(num_blocks, 0);
-    if (free_order) {
-        std::vector<char> seen(num_blocks, 0);
-        for (int i = 0; i < num_blocks; ++i) {
-            int32_t b = free_order[i];
-            if (b < 0 || b >= num_blocks || seen[b]) { delete bm; return PKV_ERR_INVALID_ARG; }
-            seen[b] = 1;
-            bm->ring[i] = b;
-        }
-    } else {
-        for (int i = 0; i < num_blocks; ++i) bm->ring[i] = i;
-    }
-    bm->head = 0;
-    bm->count = num_blocks;
+    if (!bm->dev.init(num_blocks, free_order)) { delete bm; return PKV_ERR_INVALID_ARG; }
     *out = bm;
     return PKV_OK;
+}
+
+pkv_status pkv_bm_set_host_pool(pkv_block_manager* bm, int num_host_blocks, const int32_t* free_order) {
+    if (!bm || num_host_blocks < 0 || bm->host.size() > 0) return PKV_ERR_INVALID_ARG;
+    if (num_host_blocks == 0) return PKV_OK;
+    Pool p;
+    if (!p.init(num_host_blocks, free_order)) return PKV_ERR_INVALID_ARG;
+    bm->host = std::move(p);
+    return PKV_OK;
+}
+
+pkv_status pkv_bm_swap_out(pkv_block_manager* bm, const int64_t* seq_ids, int n, int64_t* dev_blocks_out,
+                           int64_t* host_blocks_out, int capacity, int* num_pairs_out) {
+    if (num_pairs_out) *num_pairs_out = 0;
+    if (!bm || n < 0 || capacity < 0 || !num_pairs_out ||
+        (n > 0 && (!seq_ids || (capacity > 0 && (!dev_blocks_out || !host_blocks_out)))))
+        return PKV_ERR_INVALID_ARG;
+    return bm->move(seq_ids, n, true, dev_blocks_out, host_blocks_out, capacity, num_pairs_out);
+}
+
+pkv_status pkv_bm_swap_in(pkv_block_manager* bm, const int64_t* seq_ids, int n, int64_t* host_blocks_out,
+                          int64_t* dev_blocks_out, int capacity, int* num_pairs_out) {
+    if (num_pairs_out) *num_pairs_out = 0;
+    if (!bm || n < 0 || capacity < 0 || !num_pairs_out ||
+        (n > 0 && (!seq_ids || (capacity > 0 && (!dev_blocks_out || !host_blocks_out)))))
+        return PKV_ERR_INVALID_ARG;
+    return bm->move(seq_ids, n, false, host_blocks_out, dev_blocks_out, capacity, num_pairs_out);
+}
+
+int pkv_bm_num_free_host(const pkv_block_manager* bm) { return bm ? (int)bm->host.count : -1; }
+
+int pkv_bm_host_ref_count(const pkv_block_manager* bm, int block) {
+    if (!bm || block < 0 || block >= bm->host.size()) return -1;
+    return bm->host.ref[block];
+}
+
+int pkv_bm_is_swapped(const pkv_block_manager* bm, int64_t seq_id) {
+    if (!bm) return -1;
+    auto it = bm->seqs.find(seq_id);
+    return it == bm->seqs.end() ? -1 : (it->second.swapped ? 1 : 0);
 }
 
 void pkv_bm_destroy(pkv_block_manager* bm) { delete bm; }
@@ -92,7 +197,7 @@ pkv_status pkv_bm_allocate(pkv_block_manager* bm, int64_t seq_id, int num_tokens
     if (!bm || num_tokens < 0) return PKV_ERR_INVALID_ARG;
     if (bm->seqs.count(seq_id)) return PKV_ERR_INVALID_ARG;
     const int64_t nblk = ((int64_t)num_tokens + bm->block_size - 1) / bm->block_size;
-    if ((size_t)nblk > bm->count) return PKV_ERR_OUT_OF_BLOCKS;
+    if ((size_t)nblk > bm->free_count()) return PKV_ERR_OUT_OF_BLOCKS;
     Seq s;
     s.table.resize(nblk);
     for (int64_t i = 0; i < nblk; ++i) bm->take(&s.table[i]);
@@ -112,17 +217,17 @@ pkv_status pkv_bm_append_slots(pkv_block_manager* bm, const int64_t* seq_ids, in
                                    !copy_dst_out || !num_copies_out)))
         return PKV_ERR_INVALID_ARG;
     for (int i = 0; i < n; ++i)
-        if (!bm->seqs.count(seq_ids[i])) return PKV_ERR_INVALID_ARG;
+        if (!bm->resident(seq_ids[i])) return PKV_ERR_INVALID_ARG;
     int ncopy = 0;
     for (int i = 0; i < n; ++i) {
         Seq& s = bm->seqs[seq_ids[i]];
         const int64_t len = s.len;
         if (len % bm->block_size != 0) {
             int32_t last = s.table.back();
-            if (bm->ref[last] > 1) {             // shared partially filled block: copy-on-write
+            if (bm->dev.ref[last] > 1) {         // shared partially filled block: copy-on-write
                 int32_t fresh;
                 if (!bm->take(&fresh)) { *num_copies_out = ncopy; return PKV_ERR_OUT_OF_BLOCKS; }
-                bm->ref[last] -= 1;
+                bm->dev.ref[last] -= 1;
                 s.table.back() = fresh;
                 copy_src_out[ncopy] = last;
                 copy_dst_out[ncopy] = fresh;
@@ -145,15 +250,15 @@ pkv_status pkv_bm_make_writable(pkv_block_manager* bm, int64_t seq_id, int logic
                                 int64_t* src, int64_t* dst) {
     if (!bm || !src || !dst) return PKV_ERR_INVALID_ARG;
     *src = *dst = -1;
-    auto it = bm->seqs.find(seq_id);
-    if (it == bm->seqs.end()) return PKV_ERR_INVALID_ARG;
-    Seq& s = it->second;
+    Seq* sp = bm->resident(seq_id);
+    if (!sp) return PKV_ERR_INVALID_ARG;
+    Seq& s = *sp;
     if (logical_block < 0 || (size_t)logical_block >= s.table.size()) return PKV_ERR_INVALID_ARG;
     int32_t old = s.table[logical_block];
-    if (bm->ref[old] <= 1) return PKV_OK;
+    if (bm->dev.ref[old] <= 1) return PKV_OK;
     int32_t fresh;
     if (!bm->take(&fresh)) return PKV_ERR_OUT_OF_BLOCKS;
-    bm->ref[old] -= 1;
+    bm->dev.ref[old] -= 1;
     s.table[logical_block] = fresh;
     *src = old;
     *dst = fresh;
@@ -162,10 +267,10 @@ pkv_status pkv_bm_make_writable(pkv_block_manager* bm, int64_t seq_id, int logic
 
 pkv_status pkv_bm_fork(pkv_block_manager* bm, int64_t parent, int64_t child) {
     if (!bm) return PKV_ERR_INVALID_ARG;
-    auto it = bm->seqs.find(parent);
-    if (it == bm->seqs.end() || bm->seqs.count(child)) return PKV_ERR_INVALID_ARG;
-    Seq c = it->second;
-    for (int32_t b : c.table) bm->ref[b] += 1;
+    Seq* p = bm->resident(parent);
+    if (!p || bm->seqs.count(child)) return PKV_ERR_INVALID_ARG;
+    Seq c = *p;
+    for (int32_t b : c.table) bm->dev.ref[b] += 1;
     bm->seqs.emplace(child, std::move(c));
     return PKV_OK;
 }
@@ -174,7 +279,8 @@ pkv_status pkv_bm_free(pkv_block_manager* bm, int64_t seq_id) {
     if (!bm) return PKV_ERR_INVALID_ARG;
     auto it = bm->seqs.find(seq_id);
     if (it == bm->seqs.end()) return PKV_ERR_INVALID_ARG;
-    for (int32_t b : it->second.table) bm->release(b);
+    Pool& pool = it->second.swapped ? bm->host : bm->dev;
+    for (int32_t b : it->second.table) pool.release(b);
     bm->seqs.erase(it);
     return PKV_OK;
 }
@@ -185,7 +291,7 @@ pkv_status pkv_bm_block_tables(const pkv_block_manager* bm, const int64_t* seq_i
         return PKV_ERR_INVALID_ARG;
     for (int i = 0; i < n; ++i) {
         auto it = bm->seqs.find(seq_ids[i]);
-        if (it == bm->seqs.end()) return PKV_ERR_INVALID_ARG;
+        if (it == bm->seqs.end() || it->second.swapped) return PKV_ERR_INVALID_ARG;
         const Seq& s = it->second;
         if (s.table.size() > (size_t)max_blocks || s.len > INT32_MAX) return PKV_ERR_INVALID_ARG;
         int32_t* row = tables_out + (size_t)i * max_blocks;
@@ -196,11 +302,11 @@ pkv_status pkv_bm_block_tables(const pkv_block_manager* bm, const int64_t* seq_i
     return PKV_OK;
 }
 
-int pkv_bm_num_free(const pkv_block_manager* bm) { return bm ? (int)bm->count : -1; }
+int pkv_bm_num_free(const pkv_block_manager* bm) { return bm ? (int)bm->dev.count : -1; }
 
 int pkv_bm_ref_count(const pkv_block_manager* bm, int block) {
     if (!bm || block < 0 || block >= bm->num_blocks) return -1;
-    return bm->ref[block];
+    return bm->dev.ref[block];
 }
 
 int pkv_bm_seq_len(const pkv_block_manager* bm, int64_t seq_id) {

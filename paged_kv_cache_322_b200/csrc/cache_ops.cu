@@ -1,4 +1,5 @@
-// Cache-side kernels: KV append (reshape_and_cache) and block copy (copy_blocks).
+// Cache-side kernels: KV append (reshape_and_cache), block copy (copy_blocks)
+// and block swap between a device pool and a page-locked host pool (swap_blocks).
 //
 // Layout ("LLM 推理引擎内部原理" §2.4): cache[num_blocks, block_size, Hkv, D].
 // One token's K (or V) for all heads is one contiguous row of Hkv*D elements
@@ -96,34 +97,58 @@ __global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(
 }
 
 // grid.x = chunk of the block span (kChunkVecs vectors), grid.y = pair,
-// grid.z = 0 (K) / 1 (V).
+// grid.z = 0 (K) / 1 (V). Copies block src_ids[y] of the source pool to block
+// dst_ids[y] of the destination pool (the same pool for copy-on-write copies).
+// A source in device memory is read through the non-coherent streaming path; a
+// source in mapped host memory (swap-in) with plain loads, several 16-byte
+// vectors in flight per thread to cover the host link's latency.
 constexpr int kCopyThreads = 256;
 constexpr int kCopyUnroll = 4;
 constexpr int kChunkVecs = kCopyThreads * kCopyUnroll;
 
-__global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
-    int4* __restrict__ k_cache, int4* __restrict__ v_cache, const int64_t* __restrict__ src_ids,
-    const int64_t* __restrict__ dst_ids, int64_t block_vecs, int64_t num_blocks, int* err) {
+template <bool kDeviceSrc>
+__global__ void __launch_bounds__(kCopyThreads) block_copy_kernel(
+    const int4* __restrict__ src_k, const int4* __restrict__ src_v, int4* __restrict__ dst_k,
+    int4* __restrict__ dst_v, const int64_t* __restrict__ src_ids, const int64_t* __restrict__ dst_ids,
+    int64_t block_vecs, int64_t src_blocks, int64_t dst_blocks, int* err) {
     const int64_t s = src_ids[blockIdx.y], d = dst_ids[blockIdx.y];
-    if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks) {
+    if (s < 0 || s >= src_blocks || d < 0 || d >= dst_blocks) {
         if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0) flag_error(err, PKV_ERR_DEVICE_BOUNDS);
         return;
     }
-    int4* cache = blockIdx.z == 0 ? k_cache : v_cache;
-    const int4* src = cache + s * block_vecs;
-    int4* dst = cache + d * block_vecs;
+    const int4* src = (blockIdx.z == 0 ? src_k : src_v) + s * block_vecs;
+    int4* dst = (blockIdx.z == 0 ? dst_k : dst_v) + d * block_vecs;
     const int64_t base = (int64_t)blockIdx.x * kChunkVecs + threadIdx.x;
     int4 r[kCopyUnroll];
 #pragma unroll
     for (int u = 0; u < kCopyUnroll; ++u) {
         const int64_t i = base + u * kCopyThreads;
-        if (i < block_vecs) r[u] = ld_stream(src + i);
+        if (i < block_vecs) r[u] = kDeviceSrc ? ld_stream(src + i) : src[i];
     }
 #pragma unroll
     for (int u = 0; u < kCopyUnroll; ++u) {
         const int64_t i = base + u * kCopyThreads;
         if (i < block_vecs) dst[i] = r[u];
     }
+}
+
+// A pointer the kernels can use for p: device (or managed) memory as is, page-
+// locked host memory through its mapped device address. Pageable host memory
+// and unknown pointers give nullptr. *host tells which.
+void* device_view(const void* p, bool* host) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    *host = a.type == cudaMemoryTypeHost;
+    if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) return const_cast<void*>(p);
+    if (a.type == cudaMemoryTypeHost && a.devicePointer) {
+        // the mapped address of p itself (p may point inside the allocation)
+        const char* base_h = static_cast<const char*>(a.hostPointer);
+        return static_cast<char*>(a.devicePointer) + (static_cast<const char*>(p) - base_h);
+    }
+    return nullptr;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -209,9 +234,48 @@ pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, pkv_dtype dtype,
     const int64_t chunks = (block_vecs + kChunkVecs - 1) / kChunkVecs;
     if (chunks > INT32_MAX) return PKV_ERR_UNSUPPORTED;
     dim3 grid((unsigned)chunks, num_pairs, 2);
-    copy_blocks_kernel<<<grid, kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<int4*>(k_cache), static_cast<int4*>(v_cache), src_block_ids, dst_block_ids,
-        block_vecs, num_blocks, err);
+    block_copy_kernel<true><<<grid, kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const int4*>(k_cache), static_cast<const int4*>(v_cache), static_cast<int4*>(k_cache),
+        static_cast<int4*>(v_cache), src_block_ids, dst_block_ids, block_vecs, num_blocks, num_blocks, err);
+    return cuda_status(cudaGetLastError());
+}
+
+pkv_status pkv_swap_blocks(const void* src_k_cache, const void* src_v_cache, int src_num_blocks, void* dst_k_cache,
+                           void* dst_v_cache, int dst_num_blocks, pkv_dtype dtype, const int64_t* src_block_ids,
+                           const int64_t* dst_block_ids, int num_pairs, int block_size, int num_kv_heads,
+                           int head_dim, void* stream) {
+    using namespace pkv;
+    const int eb = elt_bytes(dtype);
+    if (eb == 0 || num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        src_num_blocks <= 0 || dst_num_blocks <= 0 || num_pairs > 65535)
+        return PKV_ERR_INVALID_ARG;
+    const int64_t block_bytes = (int64_t)block_size * num_kv_heads * head_dim * eb;
+    if (block_bytes % 16 != 0) return PKV_ERR_UNSUPPORTED;
+    if (num_pairs == 0) return PKV_OK;
+    if (!src_k_cache || !src_v_cache || !dst_k_cache || !dst_v_cache || !src_block_ids || !dst_block_ids)
+        return PKV_ERR_INVALID_ARG;
+    if (!aligned16(src_k_cache) || !aligned16(src_v_cache) || !aligned16(dst_k_cache) || !aligned16(dst_v_cache))
+        return PKV_ERR_INVALID_ARG;
+    bool hk, hv, dk_host, dv_host, hs, hd;
+    const void* sk = device_view(src_k_cache, &hk);
+    const void* sv = device_view(src_v_cache, &hv);
+    void* dk = device_view(dst_k_cache, &dk_host);
+    void* dv = device_view(dst_v_cache, &dv_host);
+    const void* ids_s = device_view(src_block_ids, &hs);
+    const void* ids_d = device_view(dst_block_ids, &hd);
+    if (!sk || !sv || !dk || !dv || !ids_s || !ids_d || hk != hv || dk_host != dv_host) return PKV_ERR_INVALID_ARG;
+    int* err = device_error_word();
+    if (!err) return PKV_ERR_CUDA;
+    const int64_t block_vecs = block_bytes / 16;
+    const int64_t chunks = (block_vecs + kChunkVecs - 1) / kChunkVecs;
+    if (chunks > INT32_MAX) return PKV_ERR_UNSUPPORTED;
+    dim3 grid((unsigned)chunks, num_pairs, 2);
+    auto st = static_cast<cudaStream_t>(stream);
+    auto kern = hk ? block_copy_kernel<false> : block_copy_kernel<true>;
+    kern<<<grid, kCopyThreads, 0, st>>>(static_cast<const int4*>(sk), static_cast<const int4*>(sv),
+                                        static_cast<int4*>(dk), static_cast<int4*>(dv),
+                                        static_cast<const int64_t*>(ids_s), static_cast<const int64_t*>(ids_d),
+                                        block_vecs, src_num_blocks, dst_num_blocks, err);
     return cuda_status(cudaGetLastError());
 }
 

@@ -29,7 +29,8 @@ class PagedKVCache:
 
     def __init__(self, num_blocks: int, block_size: int, num_kv_heads: int, head_dim: int,
                  dtype: torch.dtype, device, free_order=None, max_blocks_per_seq: int = 0,
-                 fill_value: float | None = None, kv_scales=(1.0, 1.0)):
+                 fill_value: float | None = None, kv_scales=(1.0, 1.0), host_blocks: int = 0,
+                 host_free_order=None):
         self.num_blocks, self.block_size = num_blocks, block_size
         self.num_kv_heads, self.head_dim, self.dtype = num_kv_heads, head_dim, dtype
         self.fp8 = dtype == torch.uint8
@@ -44,6 +45,17 @@ class PagedKVCache:
             self.k_cache = torch.full(shape, fill, dtype=dtype, device=self.device)
             self.v_cache = torch.full(shape, fill, dtype=dtype, device=self.device)
         self.bm = binding.BlockManager(num_blocks, block_size, free_order)
+        # page-locked host pool for swapped-out sequences (same block shape)
+        self.host_blocks = int(host_blocks)
+        self.k_host = self.v_host = None
+        if self.host_blocks:
+            hshape = (self.host_blocks,) + shape[1:]
+            self.k_host = torch.empty(hshape, dtype=dtype, pin_memory=True)
+            self.v_host = torch.empty(hshape, dtype=dtype, pin_memory=True)
+            if fill_value is not None:
+                self.k_host.fill_(fill)
+                self.v_host.fill_(fill)
+            self.bm.set_host_pool(self.host_blocks, host_free_order)
         self.max_blocks_per_seq = max_blocks_per_seq or num_blocks
         self._pinned = {}
 
@@ -112,6 +124,32 @@ class PagedKVCache:
 
     def free(self, seq_id: int):
         self.bm.free(seq_id)
+
+    # -- preemption by swapping ---------------------------------------------
+    def swap_out(self, seq_ids, stream=None):
+        """Moves a group of sequences' blocks to the host pool and frees their
+        device blocks; the copies run on `stream` before anything queued after
+        them reuses the blocks. Returns the (device, host) block pairs."""
+        if not self.host_blocks:
+            raise RuntimeError("no host pool (host_blocks=0)")
+        dev_b, host_b = self.bm.swap_out(seq_ids)
+        if dev_b.size:
+            binding.swap_blocks(self.k_cache, self.v_cache, self.k_host, self.v_host,
+                                self._to_device("swap_src", dev_b, stream), self._to_device("swap_dst", host_b, stream),
+                                stream=stream)
+        return list(zip(dev_b.tolist(), host_b.tolist()))
+
+    def swap_in(self, seq_ids, stream=None):
+        """Brings a swapped-out group back into fresh device blocks. Returns the
+        (host, device) block pairs."""
+        if not self.host_blocks:
+            raise RuntimeError("no host pool (host_blocks=0)")
+        host_b, dev_b = self.bm.swap_in(seq_ids)
+        if dev_b.size:
+            binding.swap_blocks(self.k_host, self.v_host, self.k_cache, self.v_cache,
+                                self._to_device("swap_src", host_b, stream), self._to_device("swap_dst", dev_b, stream),
+                                stream=stream)
+        return list(zip(host_b.tolist(), dev_b.tolist()))
 
     def block_tables(self, seq_ids):
         return self.bm.block_tables(seq_ids, self.max_blocks_per_seq)

@@ -47,10 +47,10 @@ class OracleProblem:
     """Oracle side of a workload: block tables from the oracle block manager,
     cache contents for the listed sequences only (`keep`, default all)."""
 
-    def __init__(self, w: wl.Workload, keep=None, dense=False):
+    def __init__(self, w: wl.Workload, keep=None, dense=False, cpu_blocks=0):
         self.w = w
         self.lens = wl.context_lens(w)
-        self.bm = OracleBM(w.num_blocks, w.block_size, wl.free_order(w))
+        self.bm = OracleBM(w.num_blocks, w.block_size, wl.free_order(w), num_cpu_blocks=cpu_blocks)
         shape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
         self.fp8 = w.kv_dtype == "fp8"
         dt, fill = (np.uint8, 0x7F) if self.fp8 else (np.float32, np.nan)
@@ -60,6 +60,9 @@ class OracleProblem:
         else:
             self.kc = SparsePool(*shape, dtype=dt)
             self.vc = SparsePool(*shape, dtype=dt)
+        hshape = (cpu_blocks,) + shape[1:]
+        self.kc_host = np.full(hshape, fill, dt)       # CPU pool of swapped-out blocks
+        self.vc_host = np.full(hshape, fill, dt)
         self.keep = set(range(w.num_seqs)) if keep is None else set(int(s) for s in keep)
         if w.ctx == "shared_prefix":
             self._build_shared()
@@ -138,7 +141,7 @@ class _TableView:
         return self.d[int(s)]
 
 
-def gpu_problem(w: wl.Workload, device="cuda", fill_nan=True, max_new_tokens=4):
+def gpu_problem(w: wl.Workload, device="cuda", fill_nan=True, max_new_tokens=4, host_blocks=0):
     """Library side: a PagedKVCache with the workload's prompts written by
     reshape_and_cache through the library's block manager."""
     import torch
@@ -149,7 +152,8 @@ def gpu_problem(w: wl.Workload, device="cuda", fill_nan=True, max_new_tokens=4):
     mb = -(-int(lens.max() + max_new_tokens) // w.block_size)
     cache = PagedKVCache(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, cdt, device,
                          free_order=wl.free_order(w), max_blocks_per_seq=mb,
-                         fill_value=float("nan") if fill_nan else None, kv_scales=(w.kv_scale, w.kv_scale))
+                         fill_value=float("nan") if fill_nan else None, kv_scales=(w.kv_scale, w.kv_scale),
+                         host_blocks=host_blocks)
     def dev(x):
         return torch.from_numpy(x).to(device=device, dtype=dt)
     if w.ctx == "shared_prefix":

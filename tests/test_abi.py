@@ -283,3 +283,112 @@ def test_workspace_and_partition_rule(lib):
     p70 = binding.partition_tokens(128, 64, 8, 128, 16, 512, 4100, 0)               # 70B-shaped batch
     assert -(-4100 // p70) == 2 and p70 <= 2560                                       # two partitions
     assert binding.partition_tokens(1, 32, 8, 128, 16, 2048, 32768, 0) == 256       # one long sequence
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_swap_ops_bit_exact_vs_oracle(lib, seed):
+    """Random allocate / append / fork / free / swap-out / swap-in through the
+    C++ block manager and the oracle: the same block pairs, tables, counts and
+    free lists on both pools, and the same all-or-nothing refusals."""
+    rng = random.Random(100 + seed)
+    bs = rng.choice([1, 4, 16])
+    nb, nh = 48, 40
+    order = rng.sample(range(nb), nb)
+    horder = rng.sample(range(nh), nh)
+    o = OracleBM(nb, bs, order, num_cpu_blocks=nh, cpu_free_order=horder)
+    p = binding.BlockManager(nb, bs, order)
+    p.set_host_pool(nh, horder)
+    alive, nxt = [], 0
+    for _ in range(200):
+        x = rng.random()
+        resident = [s for s in alive if s not in o.swapped]
+        out = [s for s in alive if s in o.swapped]
+        if x < 0.2 or not alive:
+            n = rng.randint(0, 3 * bs)
+            r = o.allocate(nxt, n)
+            if r is None:
+                with pytest.raises(binding.PkvError):
+                    p.allocate(nxt, n)
+            else:
+                assert p.allocate(nxt, n).tolist() == r
+                alive.append(nxt)
+            nxt += 1
+        elif x < 0.3 and resident:
+            s = rng.choice(resident)
+            o.fork(s, nxt)
+            p.fork(s, nxt)
+            alive.append(nxt)
+            nxt += 1
+        elif x < 0.5 and resident:
+            s = rng.choice(resident)
+            r = o.append_slot(s)
+            if r is None:
+                with pytest.raises(binding.PkvError):
+                    p.append_slots([s])
+                break
+            slots, src, dst = p.append_slots([s])
+            assert slots.tolist() == [r[0]]
+            assert list(zip(src.tolist(), dst.tolist())) == ([r[1]] if r[1] else [])
+        elif x < 0.6 and alive:
+            s = alive.pop(rng.randrange(len(alive)))
+            o.free_seq(s)
+            p.free(s)
+        elif x < 0.8 and resident:
+            group = rng.sample(resident, rng.randint(1, min(3, len(resident))))
+            r = o.swap_out(group)
+            if r is None:
+                with pytest.raises(binding.PkvError) as e:
+                    p.swap_out(group)
+                assert e.value.status == 5
+            else:
+                a, b = p.swap_out(group)
+                assert list(zip(a.tolist(), b.tolist())) == r
+        elif out:
+            group = rng.sample(out, rng.randint(1, min(3, len(out))))
+            r = o.swap_in(group)
+            if r is None:
+                with pytest.raises(binding.PkvError) as e:
+                    p.swap_in(group)
+                assert e.value.status == 5
+            else:
+                a, b = p.swap_in(group)
+                assert list(zip(a.tolist(), b.tolist())) == r
+        assert o.num_free() == p.num_free() and len(o.cpu_free) == p.num_free_host()
+        for s in alive:
+            assert p.is_swapped(s) == (s in o.swapped)
+            if s not in o.swapped:
+                t = o.block_table(s)
+                tables, lens = p.block_tables([s], max(len(t), 1))
+                assert tables[0, :len(t)].tolist() == t and lens[0] == o.lens[s]
+        assert [p.ref_count(b) for b in range(nb)] == o.ref
+        assert [p.host_ref_count(b) for b in range(nh)] == o.cpu_ref
+
+
+def test_swap_errors(lib):
+    bm = binding.BlockManager(8, 4)
+    bm.allocate(0, 5)
+    with pytest.raises(binding.PkvError):
+        bm.swap_out([0])                                    # no host pool: 0 free host blocks
+    bm.set_host_pool(4)
+    with pytest.raises(binding.PkvError):
+        bm.set_host_pool(4)                                 # set once
+    a, b = bm.swap_out([0])
+    assert a.size == 2 and bm.is_swapped(0) and bm.num_free() == 8 and bm.num_free_host() == 2
+    for call in (lambda: bm.append_slots([0]), lambda: bm.fork(0, 1), lambda: bm.make_writable(0, 0),
+                 lambda: bm.block_tables([0], 4), lambda: bm.swap_out([0])):
+        with pytest.raises(binding.PkvError) as e:
+            call()
+        assert e.value.status == 1
+    with pytest.raises(binding.PkvError):
+        bm.swap_in([0, 0])                                  # repeated id
+    bm.free(0)
+    assert bm.num_free_host() == 4
+    with pytest.raises(KeyError):
+        bm.is_swapped(0)
+    # host-side checks of the copy entry point
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.pkv_swap_blocks(None, None, 1, None, None, 1, 1, None, None, 0, 16, 8, 128, None) == 0
+    assert lib.pkv_swap_blocks(fake, fake, 4, fake, fake, 4, 9, fake, fake, 1, 16, 8, 128, None) == 1
+    assert lib.pkv_swap_blocks(fake, fake, 0, fake, fake, 4, 1, fake, fake, 1, 16, 8, 128, None) == 1
+    assert lib.pkv_swap_blocks(fake, fake, 4, fake, fake, 4, 1, fake, fake, -1, 16, 8, 128, None) == 1
+    assert lib.pkv_swap_blocks(fake, fake, 4, fake, fake, 4, 2, fake, fake, 1, 1, 1, 8, None) == 2  # 8-byte block
