@@ -64,6 +64,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     ap.add_argument("--num-seqs", type=int, default=0, help="override the batch size (profiling a small case)")
     ap.add_argument("--num-blocks", type=int, default=0, help="override the pool size (profiling a small case)")
+    ap.add_argument("--block-size", type=int, default=0,
+                    help="tokens per block (8, 16, 32, 64); the pool keeps the workload's token capacity")
     return ap.parse_args()
 
 
@@ -110,6 +112,23 @@ def all_max(x: float, ws: int) -> float:
 
 def all_sum(x: float, ws: int) -> float:
     return _all_reduce(x, ws, "sum")
+
+
+def override_workload(w: wl.Workload, args) -> wl.Workload:
+    """--num-seqs / --num-blocks / --block-size applied to a workload (a block
+    size change keeps the pool's token capacity)."""
+    notes = []
+    if args.block_size and args.block_size != w.block_size:
+        nb = (args.num_blocks or w.num_blocks) * w.block_size // args.block_size
+        w = dataclasses.replace(w, block_size=args.block_size, num_blocks=nb)
+        notes.append(f"block_size={args.block_size}, pool={nb} blocks")
+    if args.num_seqs or args.num_blocks:
+        w = dataclasses.replace(w, num_seqs=args.num_seqs or w.num_seqs,
+                                num_blocks=w.num_blocks if args.block_size else (args.num_blocks or w.num_blocks))
+        notes.append(f"B={w.num_seqs}, pool={w.num_blocks}")
+    if notes:
+        w = dataclasses.replace(w, description=w.description + " [override: " + "; ".join(notes) + "]")
+    return w
 
 
 def replica_workload(w: wl.Workload, rank: int) -> wl.Workload:
@@ -220,10 +239,11 @@ def traffic_record(workload: str):
 
 def kernel_source_sha1() -> str:
     """Hash of the partitioned attention kernel's device code (the shared device
-    headers and paged_attention.cu up to its host-side section)."""
+    headers, the kernel template and paged_attention.cu up to its host-side
+    section)."""
     csrc = os.path.join(ROOT, "paged_kv_cache_322_b200", "csrc")
     h = hashlib.sha1()
-    for name in ("common.cuh", "attention_common.cuh"):
+    for name in ("common.cuh", "attention_common.cuh", "paged_attention_kernel.cuh"):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     with open(os.path.join(csrc, "paged_attention.cu"), "rb") as f:
@@ -259,10 +279,7 @@ def run_pkv(args, ws, rank, local):
 
     dev = torch.device("cuda", local)
     w = wl.WORKLOADS[args.workload]
-    if args.num_seqs or args.num_blocks:
-        w = dataclasses.replace(w, num_seqs=args.num_seqs or w.num_seqs, num_blocks=args.num_blocks or w.num_blocks,
-                                description=w.description + f" [override: B={args.num_seqs or w.num_seqs}, "
-                                                            f"pool={args.num_blocks or w.num_blocks}]")
+    w = override_workload(w, args)
     w = replica_workload(w, rank)
     part = w.partition_tokens if args.partition_tokens == -2 else args.partition_tokens
     K, W = args.steps, args.warmup
@@ -436,8 +453,7 @@ def run_swap(args, ws, rank, local):
 
     dev = torch.device("cuda", local)
     w = replica_workload(wl.WORKLOADS[args.workload], rank)
-    if args.num_seqs or args.num_blocks:
-        w = dataclasses.replace(w, num_seqs=args.num_seqs or w.num_seqs, num_blocks=args.num_blocks or w.num_blocks)
+    w = override_workload(w, args)
     K, W = args.steps, args.warmup
     lens = wl.context_lens(w)
     bs = w.block_size

@@ -40,7 +40,9 @@
  *                       physical block holding tokens [j*block_size, (j+1)*block_size)
  *       context_lens    int32 [num_seqs]
  *       slot_mapping    int64 [num_tokens]; slot = physical_block*block_size + offset
- *   - Supported: head_dim 64 or 128; block_size 16; num_q_heads a multiple of
+ *   - Supported: head_dim 64 or 128; block_size 8, 16, 32 or 64 ("vLLM
+ *     PagedAttention 深度解析" §8.1 names powers of two with 16 the default;
+ *     the persistent schedule takes 16 only); num_q_heads a multiple of
  *     num_kv_heads with group size num_q_heads/num_kv_heads in {1, 2, 4, 8};
  *     kv dtype f32 or bf16 (q has the kv dtype). Query head h reads KV head
  *     h / group (a reading: the pages do not discuss grouped-query attention).
@@ -104,7 +106,8 @@ const char* pkv_status_string(int status);
  *        partitions whenever the batch still fills the GPU);
  *   -1   PKV_SCHEDULE_PERSISTENT: two CTAs per SM, each streaming an equal
  *        share of the batch's (sequence, block) tiles, with split sequences
- *        merged inside the kernel (at most 2048 sequences).
+ *        merged inside the kernel (at most 2048 sequences; block_size 16,
+ *        f32 / bf16 caches).
  * Partial results live in `workspace` (device memory, at least
  * pkv_paged_attention_workspace_bytes(...) bytes, 256-byte aligned; it may be
  * NULL when that size is 0). Its contents need no initialisation and are
@@ -305,9 +308,11 @@ typedef struct pkv_block_manager pkv_block_manager;
 
 /* kv_dtype PKV_FP8_E4M3: the caches hold e4m3 codes, the step's q / new K,V
  * are bf16 on the host, and k_scale / v_scale are the per-tensor scales
- * (ignored for f32 / bf16 caches). */
+ * (ignored for f32 / bf16 caches). block_size: tokens per block of the caches
+ * and of the block manager the steps will use (pkv_decode_step refuses a
+ * manager with another block size). */
 pkv_status pkv_step_ctx_create(int max_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                               int max_blocks_per_seq, pkv_dtype kv_dtype, pkv_dtype out_dtype,
+                               int max_blocks_per_seq, int block_size, pkv_dtype kv_dtype, pkv_dtype out_dtype,
                                int partition_tokens, float k_scale, float v_scale, pkv_step_ctx** out);
 void pkv_step_ctx_destroy(pkv_step_ctx* ctx);
 
@@ -321,7 +326,7 @@ void pkv_step_ctx_destroy(pkv_step_ctx* ctx);
  *   3. pkv_copy_blocks for the copy-on-write pairs, pkv_reshape_and_cache for
  *      the new tokens, pkv_paged_attention_decode over the updated contexts;
  *   4. the output [n, Hq, D] (out_dtype of the context) is copied to out_host.
- * k_cache / v_cache are the device caches (block_size 16). Everything is
+ * k_cache / v_cache are the device caches (the context's block_size). Everything is
  * enqueued on `stream`; synchronise it before reading out_host. A block manager
  * error (PKV_ERR_OUT_OF_BLOCKS) is returned before anything is enqueued.
  */
@@ -417,6 +422,8 @@ int pkv_bm_host_ref_count(const pkv_block_manager* bm, int block);
 /* 1 swapped out, 0 resident, -1 unknown. */
 int pkv_bm_is_swapped(const pkv_block_manager* bm, int64_t seq_id);
 
+/* Tokens per block of the manager, or -1 for NULL. */
+int pkv_bm_block_size(const pkv_block_manager* bm);
 int pkv_bm_num_free(const pkv_block_manager* bm);
 int pkv_bm_ref_count(const pkv_block_manager* bm, int block);
 /* Number of tokens of a sequence, or -1 if unknown. */

@@ -50,7 +50,8 @@ _SIGS = {
     "pkv_copy_blocks": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pkv_swap_blocks": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp]),
     "pkv_get_device_error": (_i32, [_c.POINTER(_c.c_int), _vp]),
-    "pkv_step_ctx_create": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _f32, _c.POINTER(_vp)]),
+    "pkv_step_ctx_create": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _f32,
+                                   _c.POINTER(_vp)]),
     "pkv_step_ctx_destroy": (None, [_vp]),
     "pkv_decode_step": (_i32, [_vp, _vp, _pi64, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _f32, _i32, _vp, _vp]),
     "pkv_bm_create": (_i32, [_i32, _i32, _pi32, _c.POINTER(_vp)]),
@@ -65,6 +66,7 @@ _SIGS = {
     "pkv_bm_num_free": (_i32, [_vp]),
     "pkv_bm_ref_count": (_i32, [_vp, _i32]),
     "pkv_bm_seq_len": (_i32, [_vp, _i64]),
+    "pkv_bm_block_size": (_i32, [_vp]),
     "pkv_bm_set_host_pool": (_i32, [_vp, _i32, _pi32]),
     "pkv_bm_swap_out": (_i32, [_vp, _pi64, _i32, _pi64, _pi64, _i32, _c.POINTER(_c.c_int)]),
     "pkv_bm_swap_in": (_i32, [_vp, _pi64, _i32, _pi64, _pi64, _i32, _c.POINTER(_c.c_int)]),
@@ -447,13 +449,13 @@ class DecodeStep:
         torch = _torch()
         self.bm, self.k_cache, self.v_cache = bm, k_cache, v_cache
         nb, bs, hkv, d = k_cache.shape
-        if bs != 16:
-            raise ValueError("block_size 16 only")
+        if bs != bm.block_size:
+            raise ValueError("the caches' block size differs from the block manager's")
         self.num_blocks, self.hq, self.hkv, self.d = nb, num_q_heads, hkv, d
         self.partition_tokens = partition_tokens
         self.out_dtype = out_dtype
         self._h = ctypes.c_void_p()
-        _check(_lib().pkv_step_ctx_create(max_seqs, num_q_heads, hkv, d, max_blocks_per_seq, _dtype_code(k_cache),
+        _check(_lib().pkv_step_ctx_create(max_seqs, num_q_heads, hkv, d, max_blocks_per_seq, bs, _dtype_code(k_cache),
                                           PKV_F32 if out_dtype == torch.float32 else PKV_BF16,
                                           partition_tokens, float(kv_scales[0]), float(kv_scales[1]),
                                           ctypes.byref(self._h)), "pkv_step_ctx_create")

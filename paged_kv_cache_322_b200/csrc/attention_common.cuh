@@ -10,8 +10,16 @@
 namespace pkv {
 namespace attn {
 
-constexpr int BS = 16;          // tokens per physical block (the only size built)
+constexpr int TILE_ROWS = 16;   // tokens of one tensor-core tile
 constexpr int NCW = 4;          // consumer warps per CTA
+
+// Block sizes built (tokens per physical block). A ring stage always holds a
+// fixed number of tokens: 16 for 4- and 2-byte caches, 32 for FP8 caches. A
+// stage is filled with "pieces" of piece_rows(bs) tokens: several whole blocks
+// when bs is smaller than a stage, one slice of a block when it is larger.
+constexpr bool block_size_built(int bs) { return bs == 8 || bs == 16 || bs == 32 || bs == 64; }
+constexpr int stage_tokens(int elt_bytes) { return elt_bytes == 1 ? 32 : 16; }
+constexpr int piece_rows(int bs, int elt_bytes) { return bs < stage_tokens(elt_bytes) ? bs : stage_tokens(elt_bytes); }
 constexpr int NTHREADS = 32 * (NCW + 1);
 constexpr float kNegInf = -INFINITY;
 
@@ -29,6 +37,7 @@ struct Params {
     int num_q_heads, num_kv_heads, group;
     int max_blocks, num_blocks;
     int ctx_cap;        // clamp for context_lens
+    int block_size;     // tokens per physical block
     int part_blocks;    // blocks per partition
     int num_parts;      // grid.y
     // persistent schedule
@@ -59,7 +68,7 @@ __device__ __forceinline__ float to_float(TQ x) {
 // SIMT consumer: HPW query heads per warp, 8 lanes per token, 4 tokens per
 // round, fp32 math. T = float or __nv_bfloat16.
 // ---------------------------------------------------------------------------
-template <typename T, int D, int HPW, typename TQ = T, int TOK = BS>
+template <typename T, int D, int HPW, typename TQ = T, int TOK = TILE_ROWS>
 struct SimtConsumer {
     static constexpr int RB = D * (int)sizeof(T);          // row bytes
     static constexpr int NCH = RB / 16;                     // 16-byte chunks per row
@@ -213,7 +222,7 @@ template <int D>
 struct MmaConsumer {
     static constexpr int KS = D / 16;          // k-steps of S^T = K Q^T
     static constexpr int MT = D / 16;          // m-tiles of O^T
-    static constexpr int HALF = BS * 128;      // bytes of one 64-wide half tile
+    static constexpr int HALF = TILE_ROWS * 128;   // bytes of one 64-wide half tile
 
     uint32_t qb[KS][2];                        // Q^T as B fragments (N = 8 query heads)
     float o[MT][4];                            // O^T fragments: dims x heads
@@ -242,8 +251,8 @@ struct MmaConsumer {
         const int g = lane >> 2, t = lane & 3;
         // Rows past the context may hold anything (NaN included): zero them in V,
         // so that p = 0 times the row stays 0. K rows are masked by select.
-        if (nvalid < BS) {
-            for (int i = lane; i < (BS - nvalid) * (D / 8); i += 32) {
+        if (nvalid < TILE_ROWS) {
+            for (int i = lane; i < (TILE_ROWS - nvalid) * (D / 8); i += 32) {
                 const int r = nvalid + i / (D / 8), cc = i % (D / 8);
                 const int half = cc >> 3, c = cc & 7;
                 *reinterpret_cast<uint4*>(vs_ptr + half * HALF + r * 128 + ((c ^ (r & 7)) << 4)) =
@@ -545,6 +554,14 @@ struct MmaConsumerFp8 {
         }
     }
 };
+
+// Partitioned schedule, one instantiation per block size (paged_attention_bs*.cu):
+// picks the consumer path for the cache dtype, head size and group and launches
+// the pipelined kernel over grid (Hkv, partitions, sequences).
+template <int BSZ>
+cudaError_t dispatch_partitioned(pkv_dtype kv_dtype, bool use_mma, int head_dim, int group, int num_kv_heads,
+                                 const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, dim3 grid,
+                                 cudaStream_t st);
 
 // Persistent schedule (paged_attention_persistent.cu).
 cudaError_t launch_persistent(bool bf16, bool use_mma, int head_dim, int group, const CUtensorMap& mk,

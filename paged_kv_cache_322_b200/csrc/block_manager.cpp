@@ -302,6 +302,8 @@ pkv_status pkv_bm_block_tables(const pkv_block_manager* bm, const int64_t* seq_i
     return PKV_OK;
 }
 
+int pkv_bm_block_size(const pkv_block_manager* bm) { return bm ? bm->block_size : -1; }
+
 int pkv_bm_num_free(const pkv_block_manager* bm) { return bm ? (int)bm->dev.count : -1; }
 
 int pkv_bm_ref_count(const pkv_block_manager* bm, int block) {

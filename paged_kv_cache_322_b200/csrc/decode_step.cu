@@ -22,7 +22,7 @@
 #include "common.cuh"
 
 struct pkv_step_ctx {
-    int max_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks;
+    int max_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks, block_size;
     pkv_dtype kv_dtype, out_dtype;
     float k_scale = 1.f, v_scale = 1.f;   // FP8 caches
     size_t meta_bytes, q_bytes, kv_bytes, out_bytes, ws_bytes;
@@ -70,10 +70,10 @@ void release(pkv_step_ctx* c) {
 extern "C" {
 
 pkv_status pkv_step_ctx_create(int max_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                               int max_blocks_per_seq, pkv_dtype kv_dtype, pkv_dtype out_dtype,
+                               int max_blocks_per_seq, int block_size, pkv_dtype kv_dtype, pkv_dtype out_dtype,
                                int partition_tokens, float k_scale, float v_scale, pkv_step_ctx** out) {
     if (!out || max_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
-        max_blocks_per_seq <= 0 || num_q_heads % num_kv_heads != 0 ||
+        max_blocks_per_seq <= 0 || block_size <= 0 || num_q_heads % num_kv_heads != 0 ||
         (kv_dtype != PKV_F32 && kv_dtype != PKV_BF16 && kv_dtype != PKV_FP8_E4M3) ||
         (out_dtype != PKV_F32 && out_dtype != PKV_BF16) ||
         (kv_dtype == PKV_FP8_E4M3 && !(k_scale > 0.f && v_scale > 0.f)))
@@ -87,6 +87,7 @@ pkv_status pkv_step_ctx_create(int max_seqs, int num_q_heads, int num_kv_heads, 
     c->num_kv_heads = num_kv_heads;
     c->head_dim = head_dim;
     c->max_blocks = max_blocks_per_seq;
+    c->block_size = block_size;
     c->kv_dtype = kv_dtype;
     c->out_dtype = out_dtype;
     c->k_scale = k_scale;
@@ -99,7 +100,7 @@ pkv_status pkv_step_ctx_create(int max_seqs, int num_q_heads, int num_kv_heads, 
     // Largest workspace any step can ask for: a fixed partition length never needs
     // more than at max_seqs and full tables; the library-chosen one is >= 256 tokens.
     const int sizing_part = partition_tokens == 0 ? 256 : partition_tokens;
-    const size_t ws = pkv_paged_attention_workspace_bytes(max_seqs, num_q_heads, num_kv_heads, head_dim, 16,
+    const size_t ws = pkv_paged_attention_workspace_bytes(max_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                                                           max_blocks_per_seq, 0, sizing_part);
     if (ws == (size_t)-1) {
         delete c;
@@ -129,6 +130,7 @@ pkv_status pkv_decode_step(pkv_step_ctx* c, pkv_block_manager* bm, const int64_t
     if (!c || !bm || n < 0 || n > c->max_seqs || (n > 0 && (!seq_ids || !q_host || !k_host || !v_host ||
                                                             !k_cache || !v_cache || !out_host)))
         return PKV_ERR_INVALID_ARG;
+    if (pkv_bm_block_size(bm) != c->block_size) return PKV_ERR_INVALID_ARG;
     if (n == 0) return PKV_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t S = (size_t)c->max_seqs;
@@ -167,24 +169,24 @@ pkv_status pkv_decode_step(pkv_step_ctx* c, pkv_block_manager* bm, const int64_t
     const int32_t* d_lens = d_tables + S * c->max_blocks;
     // 3. the kernels
     if (ncopy > 0) {
-        s = pkv_copy_blocks(k_cache, v_cache, c->kv_dtype, d_src, d_dst, ncopy, 16, c->num_kv_heads, c->head_dim,
+        s = pkv_copy_blocks(k_cache, v_cache, c->kv_dtype, d_src, d_dst, ncopy, c->block_size, c->num_kv_heads, c->head_dim,
                             num_blocks, stream);
         if (s != PKV_OK) return s;
     }
     const bool fp8 = c->kv_dtype == PKV_FP8_E4M3;
     s = fp8 ? pkv_reshape_and_cache_fp8(c->d_k, c->d_v, PKV_BF16, k_cache, v_cache, c->k_scale, c->v_scale, d_slots,
-                                        n, c->num_kv_heads, c->head_dim, 16, num_blocks, stream)
+                                        n, c->num_kv_heads, c->head_dim, c->block_size, num_blocks, stream)
             : pkv_reshape_and_cache(c->d_k, c->d_v, k_cache, v_cache, c->kv_dtype, d_slots, n, c->num_kv_heads,
-                                    c->head_dim, 16, num_blocks, stream);
+                                    c->head_dim, c->block_size, num_blocks, stream);
     if (s != PKV_OK) return s;
     // workspace sized at creation for max_seqs and the table capacity; this call asks for the
     // same schedule over n sequences, which never needs more
     s = fp8 ? pkv_paged_attention_decode_fp8(c->d_out, c->out_dtype, c->d_q, k_cache, v_cache, c->k_scale,
                                              c->v_scale, d_tables, d_lens, scale, n, c->num_q_heads, c->num_kv_heads,
-                                             c->head_dim, 16, c->max_blocks, num_blocks, max_len, partition_tokens,
+                                             c->head_dim, c->block_size, c->max_blocks, num_blocks, max_len, partition_tokens,
                                              c->d_ws, c->ws_bytes, stream)
             : pkv_paged_attention_decode(c->d_out, c->out_dtype, c->d_q, k_cache, v_cache, c->kv_dtype, d_tables,
-                                         d_lens, scale, n, c->num_q_heads, c->num_kv_heads, c->head_dim, 16,
+                                         d_lens, scale, n, c->num_q_heads, c->num_kv_heads, c->head_dim, c->block_size,
                                          c->max_blocks, num_blocks, max_len, partition_tokens, c->d_ws, c->ws_bytes,
                                          stream);
     if (s != PKV_OK) return s;

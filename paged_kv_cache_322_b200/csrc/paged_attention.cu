@@ -43,243 +43,13 @@
 namespace pkv {
 namespace attn {
 
-// ---------------------------------------------------------------------------
-// The pipelined kernel.
-//   PATH 0: SIMT, block-split (each consumer warp takes whole blocks, HPW = group)
-//   PATH 1: SIMT, head-split (every warp reads every block, HPW = group / NCW)
-//   PATH 2: tensor cores, block-split (group <= 8)
-// ---------------------------------------------------------------------------
-template <typename T, int D, int PATH, int HPW, int STAGES, int KPC = 1>
-struct Kern {
-    static constexpr bool kMma = PATH == 2;
-    static constexpr int TILE = BS * D * (int)sizeof(T);              // one block, one head, K or V
-    static constexpr int BOX = 128 / (int)sizeof(T);                   // elements per swizzled 128-byte box row
-    static constexpr int NBOX = D * (int)sizeof(T) / 128;              // boxes per row (tensor-core path)
-    // FP8 tiles are half the size: two physical blocks share a stage, so a stage
-    // is 8 KB and a consumer folds 32 tokens per step (K rows of both blocks
-    // first, then V rows).
-    static constexpr int BPS = sizeof(T) == 1 ? 2 : 1;                  // blocks per stage
-    static constexpr int TOK = BS * BPS;
-    // KPC KV heads per CTA: their tiles are loaded back to back, so a token row's
-    // neighbouring heads (adjacent in HBM) are read together; consumer warps split
-    // by head (WPH warps per head). Stage layout: K [head][block][tile], then V.
-    static constexpr int WPH = NCW / KPC;
-    static constexpr int STAGE_BYTES = 2 * BPS * KPC * TILE;
-    static_assert(PATH != 1 || KPC == 1, "head-split consumers serve one KV head");
-    static constexpr int RING = STAGES * STAGE_BYTES;
-    static constexpr int NSLOT = PATH == 1 ? 1 : NCW;                  // partial states to merge
-    static constexpr int MAXG = PATH == 2 ? 8 : (PATH == 1 ? HPW * NCW : HPW);
-    static constexpr int RED = NSLOT * MAXG * (D + 2) * 4;
-    static constexpr int BODY = RING > RED ? RING : RED;
-    static constexpr int SMEM = 1024 /*align slack*/ + BODY + 2 * STAGES * 8;
-    static_assert(RED <= BODY, "reduction scratch must fit");
-    // Block-split consumers take tiles round-robin; with STAGES a multiple of NCW
-    // every round of a stage goes to the same warp, so no warp can wait on a ring
-    // phase two rounds ahead of the producer (the parity wait would pass early).
-    static_assert(PATH == 1 || STAGES % WPH == 0, "ring depth must be a multiple of the warps per head");
-};
-
-template <typename T, int D, int PATH, int HPW, int STAGES, int KPC>
-__global__ void __launch_bounds__(NTHREADS, 3)
-paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                    const Params p) {
-    using K = Kern<T, D, PATH, HPW, STAGES, KPC>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + K::BODY);
-    uint64_t* empty = full + STAGES;
-    __shared__ volatile int s_abort;
-
-    const int kvh = blockIdx.x * KPC, part = blockIdx.y, seq = blockIdx.z;   // first KV head of this CTA
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    int ctx = p.context_lens[seq];
-    if (ctx < 0 || ctx > p.ctx_cap) {
-        if (threadIdx.x == 0 && part == 0 && kvh == 0) flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
-        ctx = ctx < 0 ? 0 : p.ctx_cap;
-    }
-    const int nblk_seq = (ctx + BS - 1) / BS;
-    const int nparts = (nblk_seq + p.part_blocks - 1) / p.part_blocks;
-    if (part > 0 && part >= nparts) return;                       // beyond this sequence's context
-    const int blk0 = part * p.part_blocks;
-    const int nblk = max(0, min(p.part_blocks, nblk_seq - blk0));
-    const int group = p.group;
-    const int64_t qh0 = (int64_t)kvh * group;                     // first query head of this KV head
-
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < STAGES; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], PATH == 1 ? NCW : KPC);
-        }
-        s_abort = 0;
-        fence_barrier_init();
-    }
-    if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_v);
-    }
-    __syncthreads();
-
-    float* red_o = reinterpret_cast<float*>(smem);
-    float* red_m = red_o + K::NSLOT * K::MAXG * D;
-    float* red_l = red_m + K::NSLOT * K::MAXG;
-
-    if (warp == 0) {
-        // ---------------- producer ----------------
-        const uint64_t pol = l2_policy_evict_first();
-        const int32_t* bt = p.block_tables + (int64_t)seq * p.max_blocks + blk0;
-        int issued = 0;
-        bool ok = true;
-        for (int j0 = 0; j0 < nblk && ok; j0 += 32) {
-            int id = 0;
-            if (j0 + lane < nblk) {
-                id = __ldg(bt + j0 + lane);
-                if (id < 0 || id >= p.num_blocks) {
-                    flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
-                    id = p.num_blocks;                            // TMA fills an out-of-range tile with zeros
-                }
-            }
-            const int jn = min(32, nblk - j0);
-            for (int jj = 0; jj < jn; ++jj) {
-                const int pb = __shfl_sync(0xffffffffu, id, jj);
-                if (lane == 0 && ok) {
-                    const int j = j0 + jj, si = j / K::BPS, b = j - si * K::BPS, st = si % STAGES;
-                    if (b == 0) {                                 // first block of a stage: claim it
-                        if (!mbar_wait_bounded(&empty[st], ((si / STAGES) & 1) ^ 1, p.err)) {
-                            ok = false;
-                            s_abort = 1;
-                        } else {
-                            mbar_arrive_expect_tx(&full[st], min(K::BPS, nblk - j) * 2 * KPC * K::TILE);
-                            ++issued;
-                        }
-                    }
-                    if (ok) {
-#pragma unroll
-                        for (int hd = 0; hd < KPC; ++hd) {
-                            uint8_t* dst = smem + st * K::STAGE_BYTES + (hd * K::BPS + b) * K::TILE;
-                            uint8_t* vdst = dst + KPC * K::BPS * K::TILE;
-                            if constexpr (K::kMma) {
-#pragma unroll
-                                for (int h = 0; h < K::NBOX; ++h) {
-                                    tma_load_4d(dst + h * (BS * 128), &tm_k, &full[st], h * K::BOX, kvh + hd, 0, pb,
-                                                pol);
-                                    tma_load_4d(vdst + h * (BS * 128), &tm_v, &full[st], h * K::BOX, kvh + hd, 0, pb,
-                                                pol);
-                                }
-                            } else {
-                                tma_load_4d(dst, &tm_k, &full[st], 0, kvh + hd, 0, pb, pol);
-                                tma_load_4d(vdst, &tm_v, &full[st], 0, kvh + hd, 0, pb, pol);
-                            }
-                        }
-                    }
-                }
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-                if (!ok) break;
-            }
-        }
-        if (lane == 0 && !ok) {
-            // Drain: wait (bounded) for every copy still in flight before the CTA exits.
-            for (int j = max(0, issued - STAGES); j < issued; ++j)
-                mbar_wait_bounded(&full[j % STAGES], (j / STAGES) & 1, p.err);
-        }
-    } else {
-        // ---------------- consumers ----------------
-        const int cw = warp - 1;
-        const int hd = cw / K::WPH, sub = cw - hd * K::WPH;               // this warp's KV head, and its turn
-        using TQ = std::conditional_t<sizeof(T) == 1, __nv_bfloat16, T>;   // an fp8 cache takes bf16 queries
-        const TQ* qbase = static_cast<const TQ*>(p.q) + ((int64_t)seq * p.num_q_heads + qh0 + hd * group) * D;
-        const int nstage = (nblk + K::BPS - 1) / K::BPS;
-        const int kofs = hd * K::BPS * K::TILE, vofs = (KPC + hd) * K::BPS * K::TILE;
-        if constexpr (PATH == 2) {
-            using Cons = std::conditional_t<sizeof(T) == 1, MmaConsumerFp8<K::BPS>, MmaConsumer<D>>;
-            Cons c;
-            c.init(reinterpret_cast<const __nv_bfloat16*>(qbase), group, lane);
-            for (int j = sub; j < nstage; j += K::WPH) {
-                const int st = j % STAGES;
-                const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err);
-                if (__any_sync(0xffffffffu, !got || s_abort != 0)) {   // warp-uniform exit
-                    s_abort = 1;
-                    break;
-                }
-                uint8_t* stage = smem + st * K::STAGE_BYTES;
-                const int nvalid = min(K::TOK, ctx - (blk0 + j * K::BPS) * BS);
-                uint8_t* vst = stage + vofs;
-                c.consume(smem_u32(stage + kofs), smem_u32(vst), vst, nvalid, p.scale_log2, lane);
-                if (nvalid < K::TOK) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[st]);
-            }
-            consumers_barrier();      // every consumer is done with the stage ring it aliases
-            c.finish(red_o + cw * K::MAXG * D, red_m + cw * K::MAXG, red_l + cw * K::MAXG, group, lane);
-        } else {
-            constexpr int HPWc = HPW;
-            const int hbase = PATH == 1 ? cw * HPWc : 0;
-            SimtConsumer<T, D, HPWc, TQ, K::TOK> c;
-            c.init(qbase + (int64_t)hbase * D, p.scale_log2, lane);
-            const int jstart = PATH == 1 ? 0 : sub, jstep = PATH == 1 ? 1 : K::WPH;
-            for (int j = jstart; j < nstage; j += jstep) {
-                const int st = j % STAGES;
-                const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err);
-                if (__any_sync(0xffffffffu, !got || s_abort != 0)) {
-                    s_abort = 1;
-                    break;
-                }
-                const uint8_t* stage = smem + st * K::STAGE_BYTES;
-                c.consume(stage + kofs, stage + vofs, min(K::TOK, ctx - (blk0 + j * K::BPS) * BS), lane);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[st]);
-            }
-            consumers_barrier();
-            const int slot = PATH == 1 ? 0 : cw;
-            c.finish(red_o + (slot * K::MAXG + hbase) * D, red_m + slot * K::MAXG + hbase,
-                     red_l + slot * K::MAXG + hbase, lane);
-        }
-    }
-    __syncthreads();
-    if (s_abort) return;
-
-    // ---------------- merge consumer states, write output or partial ----------------
-    // KV head hd of this CTA: its states are in warp slots [hd * NSLOT / KPC, (hd + 1) * NSLOT / KPC).
-    constexpr int SPH = K::NSLOT / KPC;
-    const int C = p.num_parts;
-    for (int idx = threadIdx.x; idx < KPC * group * D; idx += NTHREADS) {
-        const int hd = idx / (group * D), rem = idx - hd * group * D;
-        const int h = rem / D, d = rem - h * D;
-        float M = kNegInf;
-#pragma unroll
-        for (int w = hd * SPH; w < (hd + 1) * SPH; ++w) M = fmaxf(M, red_m[w * K::MAXG + h]);
-        float L = 0.f, O = 0.f;
-        if (M != kNegInf) {
-#pragma unroll
-            for (int w = hd * SPH; w < (hd + 1) * SPH; ++w) {
-                const float mw = red_m[w * K::MAXG + h];
-                if (mw == kNegInf) continue;
-                const float sc = fast_exp2(mw - M);
-                L += red_l[w * K::MAXG + h] * sc;
-                O += red_o[(w * K::MAXG + h) * D + d] * sc;
-            }
-        }
-        const float val = L > 0.f ? O / L : 0.f;
-        const int64_t qh = (int64_t)seq * p.num_q_heads + qh0 + hd * group + h;
-        if (nparts <= 1) {
-            store_out(p, qh * D + d, val);
-        } else {
-            p.ws_o[(qh * C + part) * D + d] = val;
-            if (d == 0) {
-                p.ws_ml[(qh * C + part) * 2 + 0] = M;
-                p.ws_ml[(qh * C + part) * 2 + 1] = L;
-            }
-        }
-    }
-}
-
 // Log-sum-exp merge of partition results. grid = (Hq, B), block = D threads.
 template <int D>
 __global__ void __launch_bounds__(D) merge_partitions_kernel(const Params p) {
     const int qhead = blockIdx.x, seq = blockIdx.y, d = threadIdx.x;
     int ctx = p.context_lens[seq];
     ctx = ctx < 0 ? 0 : (ctx > p.ctx_cap ? p.ctx_cap : ctx);
-    const int nparts = ((ctx + BS - 1) / BS + p.part_blocks - 1) / p.part_blocks;
+    const int nparts = ((ctx + p.block_size - 1) / p.block_size + p.part_blocks - 1) / p.part_blocks;
     if (nparts <= 1) return;
     const int64_t qh = (int64_t)seq * p.num_q_heads + qhead;
     const float* ml = p.ws_ml + qh * p.num_parts * 2;
@@ -315,19 +85,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// Tensor map over a cache [NB, BS, Hkv, D] of 4-, 2- or 1-byte elements: box =
-// one block of one head, the whole row (SIMT) or 128-byte box rows with the
-// 128-byte swizzle (tensor-core path).
-bool make_cache_map(CUtensorMap* map, const void* base, pkv_dtype dt, int nb, int hkv, int d, bool mma) {
+// Tensor map over a cache [NB, bs, Hkv, D] of 4-, 2- or 1-byte elements: box =
+// piece_rows(bs) tokens of one head (a whole block, or a slice of a block longer
+// than a ring stage), the whole row (SIMT) or 128-byte box rows with the 128-byte
+// swizzle (tensor-core path).
+bool make_cache_map(CUtensorMap* map, const void* base, pkv_dtype dt, int nb, int bs, int hkv, int d, bool mma) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t eb = dt == PKV_F32 ? 4 : (dt == PKV_BF16 ? 2 : 1);
     const CUtensorMapDataType ty = dt == PKV_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                                    : dt == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                     : CU_TENSOR_MAP_DATA_TYPE_UINT8;
-    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)hkv, (cuuint64_t)BS, (cuuint64_t)nb};
-    cuuint64_t strides[3] = {d * eb, (cuuint64_t)hkv * d * eb, (cuuint64_t)BS * hkv * d * eb};
-    cuuint32_t box[4] = {(cuuint32_t)(mma ? 128 / eb : d), 1, (cuuint32_t)BS, 1};
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)hkv, (cuuint64_t)bs, (cuuint64_t)nb};
+    cuuint64_t strides[3] = {d * eb, (cuuint64_t)hkv * d * eb, (cuuint64_t)bs * hkv * d * eb};
+    cuuint32_t box[4] = {(cuuint32_t)(mma ? 128 / eb : d), 1, (cuuint32_t)piece_rows(bs, (int)eb), 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(map, ty, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     mma ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -364,8 +135,10 @@ struct Plan {
 //                           sequences and < 2^31 tiles).
 bool plan(int num_seqs, int num_kv_heads, int block_size, int max_blocks, int max_context_len,
           int partition_tokens, Plan* pl) {
-    if (num_seqs <= 0 || num_kv_heads <= 0 || block_size != BS || max_blocks <= 0 || partition_tokens < -1)
+    if (num_seqs <= 0 || num_kv_heads <= 0 || !block_size_built(block_size) || max_blocks <= 0 ||
+        partition_tokens < -1 || (partition_tokens == -1 && block_size != 16))
         return false;
+    const int BS = block_size;
     const int64_t cap_tbl = (int64_t)max_blocks * block_size;
     if (cap_tbl > INT32_MAX) return false;
     int cap = (int)cap_tbl;
@@ -423,49 +196,6 @@ size_t ws_bytes_for(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
     return o_bytes + rows * 2 * 4;
 }
 
-template <typename T, int D, int PATH, int HPW, int STAGES, int KPC = 1>
-cudaError_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, dim3 grid,
-                          cudaStream_t stream) {
-    using K = Kern<T, D, PATH, HPW, STAGES, KPC>;
-    auto kern = paged_decode_kernel<T, D, PATH, HPW, STAGES, KPC>;
-    grid.x /= KPC;
-    // Opt in to >48 KB dynamic shared memory once per device.
-    static std::atomic<uint64_t> done_mask{0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    const uint64_t bit = 1ull << (dev & 63);
-    if (!(done_mask.load() & bit)) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
-        if (e != cudaSuccess) return e;
-        done_mask.fetch_or(bit);
-    }
-    kern<<<grid, NTHREADS, K::SMEM, stream>>>(mk, mv, p);
-    return cudaGetLastError();
-}
-
-// Ring depth: about 64 KB of stages per CTA (8 KB per stage for bf16 D=128),
-// so three CTAs fit on an SM with ~190 KB of KV in flight.
-template <typename T, int D, int KPC = 1>
-constexpr int stages_for() {
-    constexpr int sb = 2 * (sizeof(T) == 1 ? 2 : 1) * KPC * BS * D * (int)sizeof(T);   // Kern::STAGE_BYTES
-    constexpr int n = 65536 / sb;
-    return n < 4 ? 4 : (n > 16 ? 16 : n);
-}
-
-template <typename T, int D, int KPC = 1>
-cudaError_t dispatch_simt(int group, const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, dim3 grid,
-                          cudaStream_t st) {
-    switch (group) {
-        case 1: return launch_decode<T, D, 0, 1, stages_for<T, D, KPC>(), KPC>(mk, mv, p, grid, st);
-        case 2: return launch_decode<T, D, 0, 2, stages_for<T, D, KPC>(), KPC>(mk, mv, p, grid, st);
-        case 4: return KPC == 1 ? launch_decode<T, D, 1, 1, stages_for<T, D>()>(mk, mv, p, grid, st)
-                                : cudaErrorInvalidValue;
-        case 8: return KPC == 1 ? launch_decode<T, D, 1, 2, stages_for<T, D>()>(mk, mv, p, grid, st)
-                                : cudaErrorInvalidValue;
-        default: return cudaErrorInvalidValue;
-    }
-}
-
 }  // namespace attn
 }  // namespace pkv
 
@@ -516,7 +246,7 @@ pkv_status decode_impl(void* out, pkv_dtype out_dtype, const void* q, const void
     const bool fp8 = kv_dtype == PKV_FP8_E4M3;
     if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
     if (fp8 && (head_dim != 128 || partition_tokens == -1)) return PKV_ERR_UNSUPPORTED;
-    if (block_size != BS) return PKV_ERR_UNSUPPORTED;
+    if (!block_size_built(block_size) || (partition_tokens == -1 && block_size != 16)) return PKV_ERR_UNSUPPORTED;
     if (group != 1 && group != 2 && group != 4 && group != 8) return PKV_ERR_UNSUPPORTED;
     if (num_seqs == 0) return PKV_OK;
     if (num_seqs > 65535) return PKV_ERR_UNSUPPORTED;
@@ -537,8 +267,8 @@ pkv_status decode_impl(void* out, pkv_dtype out_dtype, const void* q, const void
     const bool bf16 = kv_dtype == PKV_BF16;
     const bool use_mma = (bf16 || fp8) && group >= 2;
     CUtensorMap mk, mv;
-    if (!make_cache_map(&mk, k_cache, kv_dtype, num_blocks, num_kv_heads, head_dim, use_mma) ||
-        !make_cache_map(&mv, v_cache, kv_dtype, num_blocks, num_kv_heads, head_dim, use_mma))
+    if (!make_cache_map(&mk, k_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim, use_mma) ||
+        !make_cache_map(&mv, v_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim, use_mma))
         return PKV_ERR_CUDA;
 
     Params p{};
@@ -556,7 +286,8 @@ pkv_status decode_impl(void* out, pkv_dtype out_dtype, const void* q, const void
     p.max_blocks = max_blocks_per_seq;
     p.num_blocks = num_blocks;
     p.ctx_cap = pl.ctx_cap;
-    p.part_blocks = pl.part_tokens / BS;
+    p.block_size = block_size;
+    p.part_blocks = pl.part_tokens / block_size;
     p.num_parts = pl.num_parts;
     p.num_seqs = num_seqs;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -581,27 +312,11 @@ pkv_status decode_impl(void* out, pkv_dtype out_dtype, const void* q, const void
 
     dim3 grid(num_kv_heads, pl.num_parts, num_seqs);
     cudaError_t e;
-    if (fp8) {
-        // Two KV heads per CTA where the SIMT path splits by block (groups 1, 2)
-        // or on tensor cores: each token's 256 contiguous bytes of K (and of V)
-        // are fetched in one go instead of two 128-byte halves by different CTAs.
-        const bool pair = num_kv_heads % 2 == 0 && (use_mma || group <= 2);
-        if (use_mma)
-            e = pair ? launch_decode<uint8_t, 128, 2, 8, stages_for<uint8_t, 128, 2>(), 2>(mk, mv, p, grid, st)
-                     : launch_decode<uint8_t, 128, 2, 8, stages_for<uint8_t, 128>()>(mk, mv, p, grid, st);
-        else
-            e = pair ? dispatch_simt<uint8_t, 128, 2>(group, mk, mv, p, grid, st)
-                     : dispatch_simt<uint8_t, 128>(group, mk, mv, p, grid, st);
-    } else if (use_mma) {
-        e = head_dim == 128
-                ? launch_decode<__nv_bfloat16, 128, 2, 8, stages_for<__nv_bfloat16, 128>()>(mk, mv, p, grid, st)
-                : launch_decode<__nv_bfloat16, 64, 2, 8, stages_for<__nv_bfloat16, 64>()>(mk, mv, p, grid, st);
-    } else if (bf16) {
-        e = head_dim == 128 ? dispatch_simt<__nv_bfloat16, 128>(group, mk, mv, p, grid, st)
-                            : dispatch_simt<__nv_bfloat16, 64>(group, mk, mv, p, grid, st);
-    } else {
-        e = head_dim == 128 ? dispatch_simt<float, 128>(group, mk, mv, p, grid, st)
-                            : dispatch_simt<float, 64>(group, mk, mv, p, grid, st);
+    switch (block_size) {
+        case 8: e = dispatch_partitioned<8>(kv_dtype, use_mma, head_dim, group, num_kv_heads, mk, mv, p, grid, st); break;
+        case 16: e = dispatch_partitioned<16>(kv_dtype, use_mma, head_dim, group, num_kv_heads, mk, mv, p, grid, st); break;
+        case 32: e = dispatch_partitioned<32>(kv_dtype, use_mma, head_dim, group, num_kv_heads, mk, mv, p, grid, st); break;
+        default: e = dispatch_partitioned<64>(kv_dtype, use_mma, head_dim, group, num_kv_heads, mk, mv, p, grid, st); break;
     }
     if (e != cudaSuccess) return PKV_ERR_CUDA;
     if (pl.num_parts > 1) {

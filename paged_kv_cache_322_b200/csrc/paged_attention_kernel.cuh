@@ -1,0 +1,335 @@
+// The pipelined paged decode kernel (partitioned schedule), templated on the
+// cache element type, head size, consumer path, ring depth, KV heads per CTA
+// and block size. Included by one translation unit per block size
+// (paged_attention_bs*.cu), which instantiates dispatch_partitioned<BSZ>; the
+// host side (tensor maps, schedule, argument checks, merge) is in
+// paged_attention.cu. The design is described at the top of that file.
+#pragma once
+
+#include <atomic>
+#include <type_traits>
+
+#include "attention_common.cuh"
+
+namespace pkv {
+namespace attn {
+
+// ---------------------------------------------------------------------------
+// The pipelined kernel.
+//   PATH 0: SIMT, block-split (each consumer warp takes whole blocks, HPW = group)
+//   PATH 1: SIMT, head-split (every warp reads every block, HPW = group / NCW)
+//   PATH 2: tensor cores, block-split (group <= 8)
+// ---------------------------------------------------------------------------
+template <typename T, int D, int PATH, int HPW, int STAGES, int KPC, int BSZ>
+struct Kern {
+    static constexpr bool kMma = PATH == 2;
+    static constexpr int EB = (int)sizeof(T);
+    static constexpr int BOX = 128 / EB;                               // elements per swizzled 128-byte box row
+    static constexpr int NBOX = D * EB / 128;                          // boxes per row (tensor-core path)
+    // A stage holds TOK tokens (16, or 32 for FP8 whose rows are half as long),
+    // filled with BPS pieces of R rows: whole blocks when BSZ < TOK, else one
+    // R-row slice of a block (a block then spans PPB pieces).
+    static constexpr int TOK = stage_tokens(EB);
+    static constexpr int R = piece_rows(BSZ, EB);
+    static constexpr int BPS = TOK / R;                                // pieces per stage
+    static constexpr int PPB = BSZ / R;                                // pieces per block
+    static constexpr int PIECE = R * D * EB;                           // one piece, one head, K or V
+    static constexpr int REGION = TOK * D * EB;                        // one head's K (or V) in a stage
+    static_assert(BPS * R == TOK && PPB * R == BSZ, "block size must be a power of two >= 8");
+    // KPC KV heads per CTA: their tiles are loaded back to back, so a token row's
+    // neighbouring heads (adjacent in HBM) are read together; consumer warps split
+    // by head (WPH warps per head). Stage layout: K [head][TOK rows], then V; on
+    // the tensor-core path each head's rows are split in 128-byte box columns.
+    static constexpr int WPH = NCW / KPC;
+    static constexpr int STAGE_BYTES = 2 * KPC * REGION;
+    // Byte offset of piece b (of BPS), box column h, inside one head's region.
+    __device__ __forceinline__ static int piece_offset(int b, int h) {
+        return kMma ? h * (TOK * 128) + b * (R * 128) : b * PIECE;
+    }
+    static_assert(PATH != 1 || KPC == 1, "head-split consumers serve one KV head");
+    static constexpr int RING = STAGES * STAGE_BYTES;
+    static constexpr int NSLOT = PATH == 1 ? 1 : NCW;                  // partial states to merge
+    static constexpr int MAXG = PATH == 2 ? 8 : (PATH == 1 ? HPW * NCW : HPW);
+    static constexpr int RED = NSLOT * MAXG * (D + 2) * 4;
+    static constexpr int BODY = RING > RED ? RING : RED;
+    static constexpr int SMEM = 1024 /*align slack*/ + BODY + 2 * STAGES * 8;
+    static_assert(RED <= BODY, "reduction scratch must fit");
+    // Block-split consumers take tiles round-robin; with STAGES a multiple of NCW
+    // every round of a stage goes to the same warp, so no warp can wait on a ring
+    // phase two rounds ahead of the producer (the parity wait would pass early).
+    static_assert(PATH == 1 || STAGES % WPH == 0, "ring depth must be a multiple of the warps per head");
+};
+
+template <typename T, int D, int PATH, int HPW, int STAGES, int KPC, int BSZ>
+__global__ void __launch_bounds__(NTHREADS, 3)
+paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const Params p) {
+    using K = Kern<T, D, PATH, HPW, STAGES, KPC, BSZ>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + K::BODY);
+    uint64_t* empty = full + STAGES;
+    __shared__ volatile int s_abort;
+
+    const int kvh = blockIdx.x * KPC, part = blockIdx.y, seq = blockIdx.z;   // first KV head of this CTA
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    int ctx = p.context_lens[seq];
+    if (ctx < 0 || ctx > p.ctx_cap) {
+        if (threadIdx.x == 0 && part == 0 && kvh == 0) flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
+        ctx = ctx < 0 ? 0 : p.ctx_cap;
+    }
+    const int nblk_seq = (ctx + BSZ - 1) / BSZ;
+    const int nparts = (nblk_seq + p.part_blocks - 1) / p.part_blocks;
+    if (part > 0 && part >= nparts) return;                       // beyond this sequence's context
+    const int blk0 = part * p.part_blocks;
+    const int nblk = max(0, min(p.part_blocks, nblk_seq - blk0));
+    const int ntok = max(0, min(p.part_blocks * BSZ, ctx - blk0 * BSZ));   // tokens of this partition
+    const int npiece = (ntok + K::R - 1) / K::R;
+    const int group = p.group;
+    const int64_t qh0 = (int64_t)kvh * group;                     // first query head of this KV head
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], PATH == 1 ? NCW : KPC);
+        }
+        s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    __syncthreads();
+
+    float* red_o = reinterpret_cast<float*>(smem);
+    float* red_m = red_o + K::NSLOT * K::MAXG * D;
+    float* red_l = red_m + K::NSLOT * K::MAXG;
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        const uint64_t pol = l2_policy_evict_first();
+        const int32_t* bt = p.block_tables + (int64_t)seq * p.max_blocks + blk0;
+        int issued = 0;
+        bool ok = true;
+        // 32 blocks' ids per coalesced load; each block gives PPB pieces, the
+        // pieces past the partition's last token are not loaded.
+        for (int q0 = 0; q0 < npiece && ok; q0 += 32 * K::PPB) {
+            const int j0 = q0 / K::PPB;
+            int id = 0;
+            if (j0 + lane < nblk) {
+                id = __ldg(bt + j0 + lane);
+                if (id < 0 || id >= p.num_blocks) {
+                    flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
+                    id = p.num_blocks;                            // TMA fills an out-of-range tile with zeros
+                }
+            }
+            const int qn = min(32 * K::PPB, npiece - q0);
+            for (int qq = 0; qq < qn; ++qq) {
+                const int pb = __shfl_sync(0xffffffffu, id, qq / K::PPB);
+                if (lane == 0 && ok) {
+                    const int q = q0 + qq, sub = qq % K::PPB;     // piece q is rows [sub*R, sub*R + R) of its block
+                    const int si = q / K::BPS, b = q - si * K::BPS, st = si % STAGES;
+                    if (b == 0) {                                 // first piece of a stage: claim it
+                        if (!mbar_wait_bounded(&empty[st], ((si / STAGES) & 1) ^ 1, p.err)) {
+                            ok = false;
+                            s_abort = 1;
+                        } else {
+                            mbar_arrive_expect_tx(&full[st], min(K::BPS, npiece - q) * 2 * KPC * K::PIECE);
+                            ++issued;
+                        }
+                    }
+                    if (ok) {
+#pragma unroll
+                        for (int hd = 0; hd < KPC; ++hd) {
+                            uint8_t* dst = smem + st * K::STAGE_BYTES + hd * K::REGION;
+                            uint8_t* vdst = dst + KPC * K::REGION;
+#pragma unroll
+                            for (int h = 0; h < (K::kMma ? K::NBOX : 1); ++h) {
+                                const int off = K::piece_offset(b, h);
+                                tma_load_4d(dst + off, &tm_k, &full[st], h * K::BOX, kvh + hd, sub * K::R, pb, pol);
+                                tma_load_4d(vdst + off, &tm_v, &full[st], h * K::BOX, kvh + hd, sub * K::R, pb, pol);
+                            }
+                        }
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) break;
+            }
+        }
+        if (lane == 0 && !ok) {
+            // Drain: wait (bounded) for every copy still in flight before the CTA exits.
+            for (int j = max(0, issued - STAGES); j < issued; ++j)
+                mbar_wait_bounded(&full[j % STAGES], (j / STAGES) & 1, p.err);
+        }
+    } else {
+        // ---------------- consumers ----------------
+        const int cw = warp - 1;
+        const int hd = cw / K::WPH, sub = cw - hd * K::WPH;               // this warp's KV head, and its turn
+        using TQ = std::conditional_t<sizeof(T) == 1, __nv_bfloat16, T>;   // an fp8 cache takes bf16 queries
+        const TQ* qbase = static_cast<const TQ*>(p.q) + ((int64_t)seq * p.num_q_heads + qh0 + hd * group) * D;
+        const int nstage = (npiece + K::BPS - 1) / K::BPS;
+        const int kofs = hd * K::REGION, vofs = (KPC + hd) * K::REGION;
+        if constexpr (PATH == 2) {
+            using Cons = std::conditional_t<sizeof(T) == 1, MmaConsumerFp8<K::TOK / TILE_ROWS>, MmaConsumer<D>>;
+            Cons c;
+            c.init(reinterpret_cast<const __nv_bfloat16*>(qbase), group, lane);
+            for (int j = sub; j < nstage; j += K::WPH) {
+                const int st = j % STAGES;
+                const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err);
+                if (__any_sync(0xffffffffu, !got || s_abort != 0)) {   // warp-uniform exit
+                    s_abort = 1;
+                    break;
+                }
+                uint8_t* stage = smem + st * K::STAGE_BYTES;
+                const int nvalid = min(K::TOK, ntok - j * K::TOK);
+                uint8_t* vst = stage + vofs;
+                c.consume(smem_u32(stage + kofs), smem_u32(vst), vst, nvalid, p.scale_log2, lane);
+                if (nvalid < K::TOK) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[st]);
+            }
+            consumers_barrier();      // every consumer is done with the stage ring it aliases
+            c.finish(red_o + cw * K::MAXG * D, red_m + cw * K::MAXG, red_l + cw * K::MAXG, group, lane);
+        } else {
+            constexpr int HPWc = HPW;
+            const int hbase = PATH == 1 ? cw * HPWc : 0;
+            SimtConsumer<T, D, HPWc, TQ, K::TOK> c;
+            c.init(qbase + (int64_t)hbase * D, p.scale_log2, lane);
+            const int jstart = PATH == 1 ? 0 : sub, jstep = PATH == 1 ? 1 : K::WPH;
+            for (int j = jstart; j < nstage; j += jstep) {
+                const int st = j % STAGES;
+                const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err);
+                if (__any_sync(0xffffffffu, !got || s_abort != 0)) {
+                    s_abort = 1;
+                    break;
+                }
+                const uint8_t* stage = smem + st * K::STAGE_BYTES;
+                c.consume(stage + kofs, stage + vofs, min(K::TOK, ntok - j * K::TOK), lane);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[st]);
+            }
+            consumers_barrier();
+            const int slot = PATH == 1 ? 0 : cw;
+            c.finish(red_o + (slot * K::MAXG + hbase) * D, red_m + slot * K::MAXG + hbase,
+                     red_l + slot * K::MAXG + hbase, lane);
+        }
+    }
+    __syncthreads();
+    if (s_abort) return;
+
+    // ---------------- merge consumer states, write output or partial ----------------
+    // KV head hd of this CTA: its states are in warp slots [hd * NSLOT / KPC, (hd + 1) * NSLOT / KPC).
+    constexpr int SPH = K::NSLOT / KPC;
+    const int C = p.num_parts;
+    for (int idx = threadIdx.x; idx < KPC * group * D; idx += NTHREADS) {
+        const int hd = idx / (group * D), rem = idx - hd * group * D;
+        const int h = rem / D, d = rem - h * D;
+        float M = kNegInf;
+#pragma unroll
+        for (int w = hd * SPH; w < (hd + 1) * SPH; ++w) M = fmaxf(M, red_m[w * K::MAXG + h]);
+        float L = 0.f, O = 0.f;
+        if (M != kNegInf) {
+#pragma unroll
+            for (int w = hd * SPH; w < (hd + 1) * SPH; ++w) {
+                const float mw = red_m[w * K::MAXG + h];
+                if (mw == kNegInf) continue;
+                const float sc = fast_exp2(mw - M);
+                L += red_l[w * K::MAXG + h] * sc;
+                O += red_o[(w * K::MAXG + h) * D + d] * sc;
+            }
+        }
+        const float val = L > 0.f ? O / L : 0.f;
+        const int64_t qh = (int64_t)seq * p.num_q_heads + qh0 + hd * group + h;
+        if (nparts <= 1) {
+            store_out(p, qh * D + d, val);
+        } else {
+            p.ws_o[(qh * C + part) * D + d] = val;
+            if (d == 0) {
+                p.ws_ml[(qh * C + part) * 2 + 0] = M;
+                p.ws_ml[(qh * C + part) * 2 + 1] = L;
+            }
+        }
+    }
+}
+
+template <typename T, int D, int PATH, int HPW, int STAGES, int KPC, int BSZ>
+cudaError_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, dim3 grid,
+                          cudaStream_t stream) {
+    using K = Kern<T, D, PATH, HPW, STAGES, KPC, BSZ>;
+    auto kern = paged_decode_kernel<T, D, PATH, HPW, STAGES, KPC, BSZ>;
+    grid.x /= KPC;
+    // Opt in to >48 KB dynamic shared memory once per device.
+    static std::atomic<uint64_t> done_mask{0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(done_mask.load() & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
+        if (e != cudaSuccess) return e;
+        done_mask.fetch_or(bit);
+    }
+    kern<<<grid, NTHREADS, K::SMEM, stream>>>(mk, mv, p);
+    return cudaGetLastError();
+}
+
+// Ring depth: about 64 KB of stages per CTA (8 KB per stage for bf16 D=128),
+// so three CTAs fit on an SM with ~190 KB of KV in flight.
+template <typename T, int D, int KPC = 1>
+constexpr int stages_for() {
+    constexpr int sb = 2 * KPC * stage_tokens((int)sizeof(T)) * D * (int)sizeof(T);   // Kern::STAGE_BYTES
+    constexpr int n = 65536 / sb;
+    return n < 4 ? 4 : (n > 16 ? 16 : n);
+}
+
+template <typename T, int D, int BSZ, int KPC = 1>
+cudaError_t dispatch_simt(int group, const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, dim3 grid,
+                          cudaStream_t st) {
+    switch (group) {
+        case 1: return launch_decode<T, D, 0, 1, stages_for<T, D, KPC>(), KPC, BSZ>(mk, mv, p, grid, st);
+        case 2: return launch_decode<T, D, 0, 2, stages_for<T, D, KPC>(), KPC, BSZ>(mk, mv, p, grid, st);
+        case 4: return KPC == 1 ? launch_decode<T, D, 1, 1, stages_for<T, D>(), 1, BSZ>(mk, mv, p, grid, st)
+                                : cudaErrorInvalidValue;
+        case 8: return KPC == 1 ? launch_decode<T, D, 1, 2, stages_for<T, D>(), 1, BSZ>(mk, mv, p, grid, st)
+                                : cudaErrorInvalidValue;
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int BSZ>
+cudaError_t dispatch_partitioned(pkv_dtype kv_dtype, bool use_mma, int head_dim, int group, int num_kv_heads,
+                                 const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, dim3 grid,
+                                 cudaStream_t st) {
+    if (kv_dtype == PKV_FP8_E4M3) {
+        // Two KV heads per CTA where the SIMT path splits by block (groups 1, 2)
+        // or on tensor cores: each token's 256 contiguous bytes of K (and of V)
+        // are fetched in one go instead of two 128-byte halves by different CTAs.
+        const bool pair = num_kv_heads % 2 == 0 && (use_mma || group <= 2);
+        if (use_mma)
+            return pair ? launch_decode<uint8_t, 128, 2, 8, stages_for<uint8_t, 128, 2>(), 2, BSZ>(mk, mv, p, grid, st)
+                        : launch_decode<uint8_t, 128, 2, 8, stages_for<uint8_t, 128>(), 1, BSZ>(mk, mv, p, grid, st);
+        return pair ? dispatch_simt<uint8_t, 128, BSZ, 2>(group, mk, mv, p, grid, st)
+                    : dispatch_simt<uint8_t, 128, BSZ>(group, mk, mv, p, grid, st);
+    }
+    // bf16 on tensor cores: 8-token blocks make 1 KB copies per head, so two KV
+    // heads per CTA (measured on B200, 70B-shaped GQA: +16% at block size 8,
+    // within 3% at 16-64 where halving the CTA count costs long-context, small
+    // batches far more).
+    if (use_mma && BSZ < 16 && head_dim == 128 && num_kv_heads % 2 == 0)
+        return launch_decode<__nv_bfloat16, 128, 2, 8, stages_for<__nv_bfloat16, 128, 2>(), 2, BSZ>(mk, mv, p, grid, st);
+    if (use_mma)
+        return head_dim == 128
+                   ? launch_decode<__nv_bfloat16, 128, 2, 8, stages_for<__nv_bfloat16, 128>(), 1, BSZ>(mk, mv, p, grid,
+                                                                                                     st)
+                   : launch_decode<__nv_bfloat16, 64, 2, 8, stages_for<__nv_bfloat16, 64>(), 1, BSZ>(mk, mv, p, grid,
+                                                                                                   st);
+    if (kv_dtype == PKV_BF16)
+        return head_dim == 128 ? dispatch_simt<__nv_bfloat16, 128, BSZ>(group, mk, mv, p, grid, st)
+                               : dispatch_simt<__nv_bfloat16, 64, BSZ>(group, mk, mv, p, grid, st);
+    return head_dim == 128 ? dispatch_simt<float, 128, BSZ>(group, mk, mv, p, grid, st)
+                           : dispatch_simt<float, 64, BSZ>(group, mk, mv, p, grid, st);
+}
+
+}  // namespace attn
+}  // namespace pkv

@@ -31,6 +31,8 @@
 namespace pkv {
 namespace attn {
 
+constexpr int PBS = 16;     // the persistent schedule serves 16-token blocks only
+
 constexpr int kPersistCtasPerSm = 2;
 constexpr int kQStages = 4;
 constexpr int kMaxSeqsPersistent = 2048;
@@ -39,7 +41,7 @@ constexpr unsigned long long kCountMask = (1ull << 24) - 1;
 template <typename T, int D, int PATH, int HPW, int STAGES>
 struct PKern {
     static constexpr bool kMma = PATH == 2;
-    static constexpr int TILE = BS * D * (int)sizeof(T);
+    static constexpr int TILE = PBS * D * (int)sizeof(T);
     static constexpr int STAGE_BYTES = 2 * TILE;
     static constexpr int RING = STAGES * STAGE_BYTES;
     static constexpr int MAXG = PATH == 2 ? 8 : (PATH == 1 ? HPW * NCW : HPW);
@@ -70,7 +72,7 @@ struct Walker {
     __device__ __forceinline__ bool next(const int* prefix, const int* ctxs, int ts, int member, Seg& sg) {
         if (t >= t1) return false;
         while (prefix[s + 1] <= t) ++s;
-        const int nblk = (ctxs[s] + BS - 1) / BS;
+        const int nblk = (ctxs[s] + PBS - 1) / PBS;
         const long long off = t - prefix[s];
         sg.s = s;
         sg.gg = (int)(off / nblk);
@@ -155,7 +157,7 @@ paged_decode_persistent_kernel(const __grid_constant__ CUtensorMap tm_k, const _
                 ctx = ctx < 0 ? 0 : p.ctx_cap;
             }
             ctxs[s] = ctx;
-            sum += ((ctx + BS - 1) / BS) * upr;
+            sum += ((ctx + PBS - 1) / PBS) * upr;
             if (ctx == 0 && (s % gridDim.x) == c) {             // empty context: zero output
                 for (int i = 0; i < hq * D; ++i) store_out(p, (int64_t)s * hq * D + i, 0.f);
             }
@@ -173,7 +175,7 @@ paged_decode_persistent_kernel(const __grid_constant__ CUtensorMap tm_k, const _
         int run = base + incl - sum;                             // exclusive prefix of this thread
         for (int s = s_lo; s < s_hi; ++s) {
             prefix[s] = run;
-            run += ((ctxs[s] + BS - 1) / BS) * upr;
+            run += ((ctxs[s] + PBS - 1) / PBS) * upr;
         }
         if (threadIdx.x == NTHREADS - 1) prefix[B] = run;
         __syncthreads();
@@ -231,8 +233,8 @@ paged_decode_persistent_kernel(const __grid_constant__ CUtensorMap tm_k, const _
                             if constexpr (K::kMma) {
 #pragma unroll
                                 for (int h = 0; h < D / 64; ++h) {
-                                    tma_load_4d(dst + h * (BS * 128), &tm_k, &full[st], h * 64, sg.g, 0, pb, pol);
-                                    tma_load_4d(dst + K::TILE + h * (BS * 128), &tm_v, &full[st], h * 64, sg.g, 0, pb,
+                                    tma_load_4d(dst + h * (PBS * 128), &tm_k, &full[st], h * 64, sg.g, 0, pb, pol);
+                                    tma_load_4d(dst + K::TILE + h * (PBS * 128), &tm_v, &full[st], h * 64, sg.g, 0, pb,
                                                 pol);
                                 }
                             } else {
@@ -276,10 +278,10 @@ paged_decode_persistent_kernel(const __grid_constant__ CUtensorMap tm_k, const _
                     if (__any_sync(0xffffffffu, !got)) { s_abort = 1; ok = false; break; }
                     uint8_t* stage = ring + st * K::STAGE_BYTES;
                     const int j = sg.j0 + (int)(ii - i);
-                    const int nvalid = min(BS, sg.ctx - j * BS);
+                    const int nvalid = min(PBS, sg.ctx - j * PBS);
                     cons.consume(smem_u32(stage), smem_u32(stage + K::TILE), stage + K::TILE, nvalid, p.scale_log2,
                                  lane);
-                    if (nvalid < BS) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    if (nvalid < PBS) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&empty[st]);
                 }
@@ -296,7 +298,7 @@ paged_decode_persistent_kernel(const __grid_constant__ CUtensorMap tm_k, const _
                     if (__any_sync(0xffffffffu, !got)) { s_abort = 1; ok = false; break; }
                     const uint8_t* stage = ring + st * K::STAGE_BYTES;
                     const int j = sg.j0 + (int)(ii - i);
-                    cons.consume(stage, stage + K::TILE, min(BS, sg.ctx - j * BS), lane);
+                    cons.consume(stage, stage + K::TILE, min(PBS, sg.ctx - j * PBS), lane);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&empty[st]);
                 }
@@ -463,7 +465,7 @@ cudaError_t launch_persistent_t(const CUtensorMap& mk, const CUtensorMap& mv, co
 
 template <typename T, int D>
 constexpr int persistent_stages() {
-    constexpr int sb = 2 * BS * D * (int)sizeof(T);
+    constexpr int sb = 2 * PBS * D * (int)sizeof(T);
     constexpr int n = 65536 / sb;
     return n < 4 ? 4 : (n > 16 ? 16 : n);
 }

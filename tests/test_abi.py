@@ -231,13 +231,16 @@ def test_block_manager_errors(lib):
 
 def test_kernel_entry_points_reject_bad_arguments_on_host(lib):
     fake = ctypes.c_void_p(1 << 20)
-    # head_dim 96 is not built; group 3 is not built; block size 8 not built
+    # head_dim 96 is not built; group 3 is not built; block size 12 is not built
     assert lib.pkv_paged_attention_decode(fake, 0, fake, fake, fake, 1, fake, fake, 1.0, 2, 8, 8, 96, 16, 4, 64,
                                           0, 0, None, 0, None) == 2
     assert lib.pkv_paged_attention_decode(fake, 0, fake, fake, fake, 1, fake, fake, 1.0, 2, 12, 4, 128, 16, 4, 64,
                                           0, 0, None, 0, None) == 2
-    assert lib.pkv_paged_attention_decode(fake, 0, fake, fake, fake, 1, fake, fake, 1.0, 2, 8, 8, 128, 8, 4, 64,
+    assert lib.pkv_paged_attention_decode(fake, 0, fake, fake, fake, 1, fake, fake, 1.0, 2, 8, 8, 128, 12, 4, 64,
                                           0, 0, None, 0, None) == 2
+    # the persistent schedule serves 16-token blocks only
+    assert lib.pkv_paged_attention_decode(fake, 0, fake, fake, fake, 1, fake, fake, 1.0, 2, 8, 8, 128, 32, 4, 64,
+                                          0, -1, None, 0, None) == 2
     # Hq not a multiple of Hkv, negative sizes, bad dtype, NaN scale, misalignment
     assert lib.pkv_paged_attention_decode(fake, 0, fake, fake, fake, 1, fake, fake, 1.0, 2, 6, 4, 128, 16, 4, 64,
                                           0, 0, None, 0, None) == 1

@@ -87,9 +87,8 @@ def test_tiny_listed_lengths_without_append():
 EDGE_LENS = [0, 1, 2, 15, 16, 17, 31, 33, 255, 256, 257, 511, 512, 513, 1000]
 
 
-def _edge_problem(seed, hq, hkv, d, dtype, lens, nb=None):
+def _edge_problem(seed, hq, hkv, d, dtype, lens, nb=None, bs=16):
     rng = np.random.default_rng(seed)
-    bs = 16
     need = sum(-(-n // bs) for n in lens)
     nb = nb or need + 37
     order = rng.permutation(nb).astype(np.int32)

@@ -75,8 +75,13 @@ EDGE = [1, 2, 15, 16, 17, 33, 255, 513, 1000]
 @pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 4), (16, 4), (16, 2)])
 @pytest.mark.parametrize("part", [0, 64])
 def test_fp8_edge_contexts(hq, hkv, part):
-    rng = np.random.default_rng(hq * 10 + hkv)
-    bs, d, scale = 16, 128, 1 / 32
+    fp8_edge_case(hq, hkv, part)
+
+
+def fp8_edge_case(hq, hkv, part, bs=16):
+    """Ragged contexts through the FP8 append and attention, against the oracle."""
+    rng = np.random.default_rng(hq * 10 + hkv + bs)
+    d, scale = 128, 1 / 32
     nb = sum(-(-n // bs) for n in EDGE) + 9
     order = rng.permutation(nb).astype(np.int32)
     mb = max(-(-n // bs) for n in EDGE)
