@@ -81,3 +81,36 @@ def paged_attention_decode_fp8(q, k_codes, v_codes, block_tables, context_lens, 
         V = vb.reshape((n_blk * block_size,) + vb.shape[2:])[:ctx]
         out[i] = attend(q[s], K, V, float(scale))
     return out
+
+
+def paged_attention_multi_query(q, k_cache, v_cache, block_tables, context_lens, query_start, scale,
+                                block_size: int) -> np.ndarray:
+    """Several new query tokens per sequence over the paged cache, with a
+    causal mask: chunked prefill ("vLLM PagedAttention 深度解析" §7.2: a long
+    prompt is cut into chunks that join the batch; each chunk's K/V go into the
+    sequence's blocks and the chunk attends over everything cached so far) and
+    speculative verification (§7.5; "LLM 推理引擎内部原理" §5.2: the target model
+    checks the draft tokens, whose K/V sit in the same blocks).
+
+    Reading (the pages describe the idea, not the indexing): the chunk's K/V
+    are already in the cache, so context_lens[s] counts them; sequence s's
+    queries are rows query_start[s] .. query_start[s+1]-1 of q ([T, Hq, D]);
+    its i-th query sits at position context_lens[s] - n_s + i and sees the
+    cache tokens 0 .. that position (itself included, none after it).
+    Returns [T, Hq, D] fp64; rows of no sequence stay zero."""
+    q = np.asarray(q)
+    out = np.zeros(q.shape, dtype=np.float64)
+    qs = [int(x) for x in np.asarray(query_start).tolist()]
+    for s in range(len(qs) - 1):
+        n = qs[s + 1] - qs[s]
+        ctx = int(context_lens[s])
+        if n == 0:
+            continue
+        if n > ctx:
+            raise ValueError("a sequence has more queries than cached tokens")
+        K = gather_logical(k_cache, block_tables[s], ctx, block_size)
+        V = gather_logical(v_cache, block_tables[s], ctx, block_size)
+        for i in range(n):
+            visible = ctx - n + i + 1
+            out[qs[s] + i] = attend(q[qs[s] + i], K[:visible], V[:visible], float(scale))
+    return out
