@@ -5,6 +5,8 @@
  *   - pkv_paged_attention_decode : decode attention of one query token per
  *     sequence over a KV cache split into fixed-size physical blocks and
  *     reached through per-sequence block tables (MHA and grouped-query).
+ *   - pkv_paged_attention_multi_query : several causal query tokens per
+ *     sequence (chunked prefill, speculative verification) over the same cache.
  *   - pkv_reshape_and_cache      : the per-token KV append into the cache.
  *   - pkv_copy_blocks            : physical block copies for copy-on-write forks.
  *   - pkv_swap_blocks            : block moves between the device pool and a
@@ -270,6 +272,50 @@ pkv_status pkv_swap_blocks(
     void* dst_k_cache, void* dst_v_cache, int dst_num_blocks, pkv_dtype dtype,
     const int64_t* src_block_ids, const int64_t* dst_block_ids, int num_pairs,
     int block_size, int num_kv_heads, int head_dim, void* stream);
+
+/*
+ * Multi-query paged attention with a causal mask: several new query tokens per
+ * sequence attend over the paged cache ([VP] §7.2 chunked prefill: a long
+ * prompt joins the batch chunk by chunk, each chunk's K/V going into the
+ * sequence's blocks; [VP] §7.5 and [ENG] §5.2 speculative decoding: the target
+ * model checks the draft tokens, whose K/V sit in the same blocks).
+ * The queries' own K/V must already be in the cache (pkv_reshape_and_cache), so
+ * context_lens[s] counts them. Sequence s owns rows query_start[s] ..
+ * query_start[s+1]-1 of q; with n_s = query_start[s+1] - query_start[s] and
+ * c_s = context_lens[s], its i-th query sits at position c_s - n_s + i and
+ *     out[row, h, :] = sum_{j <= c_s - n_s + i} softmax_j(scale q[row,h] . K_s[j,g]) V_s[j,g]
+ * (g = h / group). n_s = 1 with c_s the context is a decode step.
+ *
+ *   out            device, [num_tokens, num_q_heads, head_dim], out_dtype (f32 or bf16)
+ *   q              device, [num_tokens, num_q_heads, head_dim], bf16
+ *   k_cache,v_cache device, [num_blocks, block_size, num_kv_heads, head_dim], kv_dtype (bf16)
+ *   block_tables   device int32 [num_seqs, max_blocks_per_seq]
+ *   context_lens   device int32 [num_seqs]
+ *   query_start    device int32 [num_seqs + 1], non-decreasing, query_start[0] >= 0,
+ *                  query_start[num_seqs] <= num_tokens
+ *   max_query_len  host upper bound of n_s (sizes the grid); max_context_len as in
+ *                  pkv_paged_attention_decode (0 = the table capacity)
+ *   partition_tokens  > 0 fixed KV partitions, 0 chosen from the shapes (no
+ *                  persistent schedule); the workspace is sized by
+ *                  pkv_paged_attention_multi_query_workspace_bytes.
+ * Supported: bf16 caches, head_dim 64 or 128, groups 1, 2, 4, 8, block sizes 8-64
+ * (PKV_ERR_UNSUPPORTED otherwise). A sequence whose n_s, c_s or rows break the
+ * rules above (n_s > c_s, n_s > max_query_len, c_s above the capacity, rows
+ * outside q) is skipped and flagged PKV_ERR_DEVICE_BOUNDS in the device word; its
+ * output rows are not written. Rows of q that belong to no sequence are not
+ * written either.
+ */
+size_t pkv_paged_attention_multi_query_workspace_bytes(
+    int num_seqs, int num_tokens, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+    int max_blocks_per_seq, int max_query_len, int max_context_len, int partition_tokens);
+
+pkv_status pkv_paged_attention_multi_query(
+    void* out, pkv_dtype out_dtype, const void* q, const void* k_cache, const void* v_cache,
+    pkv_dtype kv_dtype, const int32_t* block_tables, const int32_t* context_lens,
+    const int32_t* query_start, float scale, int num_seqs, int num_tokens, int num_q_heads,
+    int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
+    int max_query_len, int max_context_len, int partition_tokens, void* workspace,
+    size_t workspace_bytes, void* stream);
 
 /*
  * FP8 KV append ("vLLM PagedAttention 深度解析" §7.4: K/V stored as FP8 so a block

@@ -45,6 +45,9 @@ _SIGS = {
     "pkv_reshape_and_cache_fp8": (_i32, [_vp, _vp, _i32, _vp, _vp, _f32, _f32, _vp, _i32, _i32, _i32, _i32, _i32,
                                          _vp]),
     "pkv_paged_attention_workspace_bytes": (_sz, [_i32] * 8),
+    "pkv_paged_attention_multi_query_workspace_bytes": (_sz, [_i32] * 10),
+    "pkv_paged_attention_multi_query": (_i32, [_vp, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _f32, _i32, _i32, _i32,
+                                               _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp]),
     "pkv_paged_attention_partition_tokens": (_i32, [_i32] * 8),
     "pkv_reshape_and_cache": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pkv_copy_blocks": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
@@ -287,6 +290,49 @@ def copy_blocks(k_cache, v_cache, src, dst, stream=None):
     st = _lib().pkv_copy_blocks(k_cache.data_ptr(), v_cache.data_ptr(), _dtype_code(k_cache), src.data_ptr(),
                                 dst.data_ptr(), src.numel(), bs, hkv, d, nb, _stream(k_cache, stream))
     _check(st, "pkv_copy_blocks")
+
+
+def multi_query_workspace_bytes(num_seqs, num_tokens, num_q_heads, num_kv_heads, head_dim, block_size,
+                                max_blocks_per_seq, max_query_len, max_context_len=0, partition_tokens=0) -> int:
+    n = _lib().pkv_paged_attention_multi_query_workspace_bytes(num_seqs, num_tokens, num_q_heads, num_kv_heads,
+                                                               head_dim, block_size, max_blocks_per_seq,
+                                                               max_query_len, max_context_len, partition_tokens)
+    if n == ctypes.c_size_t(-1).value:
+        raise PkvError(1, "pkv_paged_attention_multi_query_workspace_bytes")
+    return n
+
+
+def paged_attention_multi_query(out, q, k_cache, v_cache, block_tables, context_lens, query_start, scale: float,
+                                max_query_len: int, max_context_len: int = 0, partition_tokens: int = 0,
+                                workspace=None, stream=None):
+    """Causal multi-query attention: q / out [T, Hq, D] (rows of all sequences,
+    sequence s owning rows query_start[s]..query_start[s+1]-1), bf16 caches
+    [NB, bs, Hkv, D] already holding the queries' K/V, context_lens counting
+    them; query_start int32 [B + 1]."""
+    torch = _torch()
+    _cuda_contig(out, q, k_cache, v_cache, block_tables, context_lens, query_start)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32 or query_start.dtype != torch.int32:
+        raise TypeError("block_tables, context_lens and query_start must be int32")
+    T, hq, d = q.shape
+    nb, bs, hkv, d2 = k_cache.shape
+    B = context_lens.shape[0]
+    if d2 != d or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != (T, hq, d) or \
+            query_start.shape[0] != B + 1:
+        raise ValueError("shape mismatch")
+    if q.dtype != k_cache.dtype or v_cache.dtype != k_cache.dtype:
+        raise TypeError("q, k_cache and v_cache must share a dtype")
+    mb = block_tables.shape[1]
+    need = multi_query_workspace_bytes(B, T, hq, hkv, d, bs, mb, max_query_len, max_context_len, partition_tokens)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_n = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = _lib().pkv_paged_attention_multi_query(
+        out.data_ptr(), _dtype_code(out), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), _dtype_code(k_cache),
+        block_tables.data_ptr(), context_lens.data_ptr(), query_start.data_ptr(), float(scale), B, T, hq, hkv, d, bs,
+        mb, nb, int(max_query_len), int(max_context_len), int(partition_tokens), ws_ptr, ws_n, _stream(q, stream))
+    _check(st, "pkv_paged_attention_multi_query")
+    return out
 
 
 def swap_blocks(src_k, src_v, dst_k, dst_v, src, dst, stream=None):

@@ -563,6 +563,10 @@ cudaError_t dispatch_partitioned(pkv_dtype kv_dtype, bool use_mma, int head_dim,
                                  const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, dim3 grid,
                                  cudaStream_t st);
 
+// Tensor map over a cache [nb, bs, hkv, d] (paged_attention.cu): box = piece_rows(bs)
+// tokens of one head, whole rows (SIMT) or 128-byte swizzled box rows (tensor cores).
+bool make_cache_map(CUtensorMap* map, const void* base, pkv_dtype dt, int nb, int bs, int hkv, int d, bool mma);
+
 // Persistent schedule (paged_attention_persistent.cu).
 cudaError_t launch_persistent(bool bf16, bool use_mma, int head_dim, int group, const CUtensorMap& mk,
                               const CUtensorMap& mv, const Params& p, int grid, cudaStream_t st);

@@ -1,0 +1,599 @@
+// Multi-query paged attention with a causal mask, for sm_100a: several new
+// query tokens per sequence (a chunk of a long prompt, "vLLM PagedAttention 深度
+// 解析" §7.2 Chunked Prefill; or the draft tokens a target model verifies, §7.5
+// and "LLM 推理引擎内部原理" §5.2) attend over the paged cache, which already holds
+// their own K/V. Query i of a sequence with n queries and context c sits at
+// position c - n + i and sees cache tokens 0 .. c - n + i.
+//
+// B200 design (bf16 caches, head_dim 64 / 128, groups 1-8, block sizes 8-64):
+//   * A CTA serves one KV head of one sequence and 64 "query rows" (query
+//     token x query head of the group: row r = token r / G, head r % G), one
+//     partition of the KV range. Grid (Hkv, partitions, sequences x row tiles).
+//   * The producer warp streams the partition's K/V with 4-D TMA pieces into a
+//     ring of 16-token stages (the decode kernel's scheme); the KV range stops at
+//     the CTA's last visible position. L2 evict-normal: the KV of a sequence is
+//     re-read by each of its row tiles.
+//   * Each of the 4 consumer warps owns 16 rows (two 8-row MMA n-tiles) and
+//     folds EVERY stage: S^T = K Q^T with mma.m16n8k16 (16 tokens x 16 rows),
+//     the causal / context mask, online softmax per row, O^T += V^T P^T with P
+//     split into bf16 high + low parts. Rows are disjoint, so no cross-warp
+//     merge: each warp writes its rows (out, or the partition's partial).
+//   * Partitions: as in decode, partial (o / l, m, l) per row and partition, and
+//     an exact log-sum-exp merge over the partitions a row can see.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+
+#include "attention_common.cuh"
+
+namespace pkv {
+namespace attn {
+namespace {
+
+constexpr int MQ_ROWS_PER_WARP = 16;
+constexpr int MQ_ROWS = NCW * MQ_ROWS_PER_WARP;     // query rows per CTA
+
+struct MqParams {
+    void* out;                    // [T, Hq, D]
+    const __nv_bfloat16* q;       // [T, Hq, D]
+    const int32_t* block_tables;
+    const int32_t* context_lens;  // cache tokens per sequence, the queries' own included
+    const int32_t* query_start;   // [B + 1]
+    float* ws_o;                  // [T * Hq, C, D]
+    float* ws_ml;                 // [T * Hq, C, 2]
+    int* err;
+    float scale_log2;
+    int out_f32;
+    int num_seqs, num_tokens, num_q_heads, num_kv_heads, group;
+    int max_blocks, num_blocks, ctx_cap, max_query_len;
+    int block_size, part_blocks, num_parts, row_tiles;
+};
+
+__device__ __forceinline__ uint64_t l2_policy_evict_normal() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// Sequence s's query count n and context c, both checked: 0 <= n <= c <= cap and
+// the queries inside [0, T). A bad entry flags PKV_ERR_DEVICE_BOUNDS and the
+// sequence is skipped (n = 0).
+__device__ __forceinline__ void mq_sequence(const MqParams& p, int s, int& q0, int& n, int& c) {
+    q0 = p.query_start[s];
+    const int q1 = p.query_start[s + 1];
+    c = p.context_lens[s];
+    n = q1 - q0;
+    if (q0 < 0 || n < 0 || q1 > p.num_tokens || n > p.max_query_len || c < n || c > p.ctx_cap) {
+        if (threadIdx.x == 0) flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
+        n = 0;
+        c = 0;
+        q0 = 0;
+    }
+}
+
+// One warp's 16 query rows (two n-tiles of 8) against 16-token K/V tiles.
+template <int D>
+struct MqConsumer {
+    static constexpr int KS = D / 16;
+    static constexpr int MT = D / 16;
+    static constexpr int HALF = TILE_ROWS * 128;
+
+    uint32_t qb[KS][2][2];        // Q^T B fragments per k-step and n-tile
+    float o[MT][2][4];            // O^T fragments
+    float m[2][2], l[2][2];       // [n-tile][column 2t / 2t+1]
+    int pos[2][2];                // position of each of the thread's columns (-1: padding row)
+
+    // rows: this warp's first row (sequence-relative); q0, n, c: the sequence.
+    __device__ __forceinline__ void init(const MqParams& p, int row0, int kvh, int q0, int n, int c, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+        const int G = p.group;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const int r = row0 + nt * 8 + g;                    // the row whose Q this thread loads
+            const int i = r / G, h = r - (r / G) * G;
+            const bool live = i < n;
+            const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+                p.q + ((int64_t)(q0 + (live ? i : 0)) * p.num_q_heads + kvh * G + h) * D);
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                qb[ks][nt][0] = live ? qrow[(ks * 16 + 2 * t) / 2] : 0u;
+                qb[ks][nt][1] = live ? qrow[(ks * 16 + 2 * t + 8) / 2] : 0u;
+            }
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int rc = row0 + nt * 8 + 2 * t + cc;      // the row of fragment column 2t + cc
+                const int ic = rc / G;
+                pos[nt][cc] = ic < n ? c - n + ic : -1;
+                m[nt][cc] = kNegInf;
+                l[nt][cc] = 0.f;
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+        }
+    }
+
+    // tok0: position of the tile's first token; nvalid: tokens of the tile inside the range.
+    __device__ __forceinline__ void consume(uint32_t ks_base, uint32_t vs_base, int tok0, int nvalid,
+                                            float scale_log2, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+        float s[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            const int r = lane & 15;
+            const int c = ((ks & 3) << 1) + (lane >> 4);
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4(a0, a1, a2, a3, ks_base + (ks >> 2) * HALF + r * 128 + ((c ^ (r & 7)) << 4));
+            mma_bf16_16816(s[0], a0, a1, a2, a3, qb[ks][0][0], qb[ks][0][1]);
+            mma_bf16_16816(s[1], a0, a1, a2, a3, qb[ks][1][0], qb[ks][1][1]);
+        }
+        const int ja = tok0 + g, jb = tok0 + g + 8;             // positions of the thread's two tokens
+        const bool va = g < nvalid, vb = g + 8 < nvalid;
+        uint32_t bh[2][2], bl[2][2];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            // s[nt][0]: (token g, col 2t)  [1]: (g, 2t+1)  [2]: (g+8, 2t)  [3]: (g+8, 2t+1)
+            const float x0 = (va && ja <= pos[nt][0]) ? s[nt][0] * scale_log2 : kNegInf;
+            const float x1 = (va && ja <= pos[nt][1]) ? s[nt][1] * scale_log2 : kNegInf;
+            const float x2 = (vb && jb <= pos[nt][0]) ? s[nt][2] * scale_log2 : kNegInf;
+            const float x3 = (vb && jb <= pos[nt][1]) ? s[nt][3] * scale_log2 : kNegInf;
+            float b0 = fmaxf(x0, x2), b1 = fmaxf(x1, x3);
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                b0 = fmaxf(b0, __shfl_xor_sync(0xffffffffu, b0, off));
+                b1 = fmaxf(b1, __shfl_xor_sync(0xffffffffu, b1, off));
+            }
+            const float n0 = fmaxf(m[nt][0], b0), n1 = fmaxf(m[nt][1], b1);
+            // a column that has seen no visible token yet keeps m = -inf: use 0 as
+            // the reference so that no -inf - -inf appears (its o and l stay 0)
+            const float r0 = n0 == kNegInf ? 0.f : n0, r1 = n1 == kNegInf ? 0.f : n1;
+            const float al0 = fast_exp2(m[nt][0] - r0), al1 = fast_exp2(m[nt][1] - r1);
+            m[nt][0] = n0;
+            m[nt][1] = n1;
+            const float p0 = fast_exp2(x0 - r0), p1 = fast_exp2(x1 - r1);
+            const float p2 = fast_exp2(x2 - r0), p3 = fast_exp2(x3 - r1);
+            l[nt][0] = l[nt][0] * al0 + (p0 + p2);
+            l[nt][1] = l[nt][1] * al1 + (p1 + p3);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                o[mt][nt][0] *= al0; o[mt][nt][1] *= al1; o[mt][nt][2] *= al0; o[mt][nt][3] *= al1;
+            }
+            // P^T as B fragments (k = token, n = row), high and low bf16 parts
+            const uint32_t h02 = pack_bf16(p0, p2), h13 = pack_bf16(p1, p3);
+            const uint32_t e02 = pack_bf16(p0 - bf16lo(h02), p2 - bf16hi(h02));
+            const uint32_t e13 = pack_bf16(p1 - bf16lo(h13), p3 - bf16hi(h13));
+            const int srcA = (2 * t) * 4 + (g >> 1), srcB = srcA + 4;
+            const bool odd = g & 1;
+            const uint32_t u0 = __shfl_sync(0xffffffffu, h02, srcA), u1 = __shfl_sync(0xffffffffu, h13, srcA);
+            const uint32_t w0 = __shfl_sync(0xffffffffu, h02, srcB), w1 = __shfl_sync(0xffffffffu, h13, srcB);
+            const uint32_t y0 = __shfl_sync(0xffffffffu, e02, srcA), y1 = __shfl_sync(0xffffffffu, e13, srcA);
+            const uint32_t z0 = __shfl_sync(0xffffffffu, e02, srcB), z1 = __shfl_sync(0xffffffffu, e13, srcB);
+            const uint32_t ya = odd ? u1 : u0, yb = odd ? w1 : w0;
+            const uint32_t za = odd ? y1 : y0, zb = odd ? z1 : z0;
+            bh[nt][0] = __byte_perm(ya, yb, 0x5410);
+            bh[nt][1] = __byte_perm(ya, yb, 0x7632);
+            bl[nt][0] = __byte_perm(za, zb, 0x5410);
+            bl[nt][1] = __byte_perm(za, zb, 0x7632);
+        }
+        // V rows past the range may hold anything (NaN included) and every warp
+        // reads this stage, so nothing is zeroed in shared memory: the V^T
+        // fragment's token columns 2t, 2t+1 (a0, a1) and 2t+8, 2t+9 (a2, a3) are
+        // masked in registers instead (p = 0 there, but 0 * NaN would not be 0).
+        const uint32_t m01 = (2 * t < nvalid ? 0x0000ffffu : 0u) | (2 * t + 1 < nvalid ? 0xffff0000u : 0u);
+        const uint32_t m23 = (2 * t + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * t + 9 < nvalid ? 0xffff0000u : 0u);
+        const bool partial = nvalid < TILE_ROWS;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const int mi = lane >> 3;
+            const int tok = (lane & 7) + ((mi >> 1) << 3);
+            const int c = (((mt * 16) & 63) >> 3) + (mi & 1);
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4_trans(a0, a1, a2, a3, vs_base + ((mt * 16) >> 6) * HALF + tok * 128 + ((c ^ (tok & 7)) << 4));
+            if (partial) {
+                a0 &= m01; a1 &= m01; a2 &= m23; a3 &= m23;
+            }
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                mma_bf16_16816(o[mt][nt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
+                mma_bf16_16816(o[mt][nt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
+            }
+        }
+    }
+
+    // Writes the warp's rows: the output (one partition) or the partition's partial.
+    __device__ __forceinline__ void finish(const MqParams& p, int row0, int kvh, int q0, int n, int part,
+                                           bool direct, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+        const int G = p.group;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                float lsum = l[nt][cc];
+                lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
+                lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
+                lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
+                const int r = row0 + nt * 8 + 2 * t + cc;
+                const int i = r / G, h = r - (r / G) * G;
+                if (i >= n) continue;
+                const int64_t qh = (int64_t)(q0 + i) * p.num_q_heads + kvh * G + h;
+                const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    const float va = o[mt][nt][cc] * inv, vb = o[mt][nt][2 + cc] * inv;
+                    const int d0 = mt * 16 + g, d1 = d0 + 8;
+                    if (direct) {
+                        if (p.out_f32) {
+                            static_cast<float*>(p.out)[qh * D + d0] = va;
+                            static_cast<float*>(p.out)[qh * D + d1] = vb;
+                        } else {
+                            static_cast<__nv_bfloat16*>(p.out)[qh * D + d0] = __float2bfloat16_rn(va);
+                            static_cast<__nv_bfloat16*>(p.out)[qh * D + d1] = __float2bfloat16_rn(vb);
+                        }
+                    } else {
+                        p.ws_o[(qh * p.num_parts + part) * D + d0] = va;
+                        p.ws_o[(qh * p.num_parts + part) * D + d1] = vb;
+                    }
+                }
+                if (!direct && g == 0) {
+                    p.ws_ml[(qh * p.num_parts + part) * 2 + 0] = m[nt][cc];
+                    p.ws_ml[(qh * p.num_parts + part) * 2 + 1] = lsum;
+                }
+            }
+        }
+    }
+};
+
+template <int D, int BSZ, int STAGES>
+struct MqKern {
+    static constexpr int TOK = TILE_ROWS;                       // tokens per stage
+    static constexpr int R = piece_rows(BSZ, 2);
+    static constexpr int BPS = TOK / R;
+    static constexpr int PPB = BSZ / R;
+    static constexpr int NBOX = D * 2 / 128;
+    static constexpr int PIECE = R * D * 2;
+    static constexpr int REGION = TOK * D * 2;                  // K (or V) of one stage
+    static constexpr int STAGE_BYTES = 2 * REGION;
+    static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 2 * STAGES * 8;
+    static_assert(BPS * R == TOK && PPB * R == BSZ, "block size must be a power of two >= 8");
+};
+
+template <int D, int BSZ, int STAGES>
+__global__ void __launch_bounds__(NTHREADS, 2)
+paged_mq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                const MqParams p) {
+    using K = MqKern<D, BSZ, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * K::STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+    __shared__ volatile int s_abort;
+
+    const int kvh = blockIdx.x, part = blockIdx.y;
+    const int seq = blockIdx.z / p.row_tiles, tile = blockIdx.z - seq * p.row_tiles;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int q0, n, c;
+    mq_sequence(p, seq, q0, n, c);
+    const int row_begin = tile * MQ_ROWS;
+    if (row_begin >= n * p.group) return;                          // no live rows in this tile
+    // last visible position of the tile's rows, and this partition's KV range
+    const int last_tok = min(n - 1, (row_begin + MQ_ROWS - 1) / p.group);
+    const int kv_end = c - n + last_tok + 1;                       // tokens [0, kv_end) are visible to some row
+    const int pt = p.part_blocks * BSZ;
+    const int kv0 = part * pt;
+    if (kv0 >= kv_end) return;                                     // no row of the tile sees this partition
+    const int ntok = min(pt, kv_end - kv0);
+    const int npiece = (ntok + K::R - 1) / K::R;
+    const int nblk = (ntok + BSZ - 1) / BSZ;
+    const int blk0 = part * p.part_blocks;
+    const bool direct = (c + pt - 1) / pt <= 1;                    // the whole context is one partition
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], NCW);
+        }
+        s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        // ---------------- producer: the decode kernel's piece walk ----------------
+        const uint64_t pol = l2_policy_evict_normal();
+        const int32_t* bt = p.block_tables + (int64_t)seq * p.max_blocks + blk0;
+        int issued = 0;
+        bool ok = true;
+        for (int q0p = 0; q0p < npiece && ok; q0p += 32 * K::PPB) {
+            const int j0 = q0p / K::PPB;
+            int id = 0;
+            if (j0 + lane < nblk) {
+                id = __ldg(bt + j0 + lane);
+                if (id < 0 || id >= p.num_blocks) {
+                    flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
+                    id = p.num_blocks;                              // TMA fills an out-of-range tile with zeros
+                }
+            }
+            const int qn = min(32 * K::PPB, npiece - q0p);
+            for (int qq = 0; qq < qn; ++qq) {
+                const int pb = __shfl_sync(0xffffffffu, id, qq / K::PPB);
+                if (lane == 0 && ok) {
+                    const int q = q0p + qq, sub = qq % K::PPB;
+                    const int si = q / K::BPS, b = q - si * K::BPS, st = si % STAGES;
+                    if (b == 0) {
+                        if (!mbar_wait_bounded(&empty[st], ((si / STAGES) & 1) ^ 1, p.err)) {
+                            ok = false;
+                            s_abort = 1;
+                        } else {
+                            mbar_arrive_expect_tx(&full[st], min(K::BPS, npiece - q) * 2 * K::PIECE);
+                            ++issued;
+                        }
+                    }
+                    if (ok) {
+                        uint8_t* dst = smem + st * K::STAGE_BYTES;
+                        uint8_t* vdst = dst + K::REGION;
+#pragma unroll
+                        for (int h = 0; h < K::NBOX; ++h) {
+                            const int off = h * (K::TOK * 128) + b * (K::R * 128);
+                            tma_load_4d(dst + off, &tm_k, &full[st], h * 64, kvh, sub * K::R, pb, pol);
+                            tma_load_4d(vdst + off, &tm_v, &full[st], h * 64, kvh, sub * K::R, pb, pol);
+                        }
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) break;
+            }
+        }
+        if (lane == 0 && !ok) {
+            for (int j = max(0, issued - STAGES); j < issued; ++j)
+                mbar_wait_bounded(&full[j % STAGES], (j / STAGES) & 1, p.err);
+        }
+    } else {
+        // ---------------- consumers: every warp folds every stage ----------------
+        const int cw = warp - 1;
+        const int row0 = row_begin + cw * MQ_ROWS_PER_WARP;
+        MqConsumer<D> cons;
+        cons.init(p, row0, kvh, q0, n, c, lane);
+        const int nstage = (npiece + K::BPS - 1) / K::BPS;
+        for (int j = 0; j < nstage; ++j) {
+            const int st = j % STAGES;
+            const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err);
+            if (__any_sync(0xffffffffu, !got || s_abort != 0)) {
+                s_abort = 1;
+                break;
+            }
+            uint8_t* stage = smem + st * K::STAGE_BYTES;
+            const int nvalid = min(K::TOK, ntok - j * K::TOK);
+            cons.consume(smem_u32(stage), smem_u32(stage + K::REGION), kv0 + j * K::TOK, nvalid, p.scale_log2, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
+        if (!s_abort) cons.finish(p, row0, kvh, q0, n, part, direct, lane);
+    }
+}
+
+// Log-sum-exp merge over the partitions each row sees. grid = (Hq, T), block = D.
+template <int D>
+__global__ void __launch_bounds__(D) merge_mq_kernel(const MqParams p) {
+    const int head = blockIdx.x, tok = blockIdx.y, d = threadIdx.x;
+    // the sequence of token `tok`: last s with query_start[s] <= tok
+    int lo = 0, hi = p.num_seqs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.query_start[mid] <= tok) lo = mid;
+        else hi = mid - 1;
+    }
+    int q0, n, c;
+    mq_sequence(p, lo, q0, n, c);
+    const int i = tok - q0;
+    if (i < 0 || i >= n) return;
+    const int pt = p.part_blocks * p.block_size;
+    if ((c + pt - 1) / pt <= 1) return;                            // written directly
+    const int pos = c - n + i;
+    const int nparts = pos / pt + 1;                               // partitions holding tokens 0..pos
+    const int64_t qh = (int64_t)tok * p.num_q_heads + head;
+    const float* ml = p.ws_ml + qh * p.num_parts * 2;
+    const float* o = p.ws_o + qh * p.num_parts * D;
+    float M = kNegInf;
+    for (int k = 0; k < nparts; ++k) M = fmaxf(M, ml[2 * k]);
+    float L = 0.f, O = 0.f;
+    if (M != kNegInf) {
+        for (int k = 0; k < nparts; ++k) {
+            const float mk = ml[2 * k];
+            if (mk == kNegInf) continue;
+            const float w = ml[2 * k + 1] * fast_exp2(mk - M);
+            L += w;
+            O += w * o[(int64_t)k * D + d];
+        }
+    }
+    const float v = L > 0.f ? O / L : 0.f;
+    if (p.out_f32) static_cast<float*>(p.out)[qh * D + d] = v;
+    else static_cast<__nv_bfloat16*>(p.out)[qh * D + d] = __float2bfloat16_rn(v);
+}
+
+template <int D, int BSZ>
+cudaError_t launch_mq(const CUtensorMap& mk, const CUtensorMap& mv, const MqParams& p, dim3 grid, cudaStream_t st) {
+    constexpr int STAGES = 8;
+    using K = MqKern<D, BSZ, STAGES>;
+    auto kern = paged_mq_kernel<D, BSZ, STAGES>;
+    static std::atomic<uint64_t> done_mask{0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(done_mask.load() & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
+        if (e != cudaSuccess) return e;
+        done_mask.fetch_or(bit);
+    }
+    kern<<<grid, NTHREADS, K::SMEM, st>>>(mk, mv, p);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_mq_bs(int bs, const CUtensorMap& mk, const CUtensorMap& mv, const MqParams& p, dim3 grid,
+                         cudaStream_t st) {
+    switch (bs) {
+        case 8: return launch_mq<D, 8>(mk, mv, p, grid, st);
+        case 16: return launch_mq<D, 16>(mk, mv, p, grid, st);
+        case 32: return launch_mq<D, 32>(mk, mv, p, grid, st);
+        default: return launch_mq<D, 64>(mk, mv, p, grid, st);
+    }
+}
+
+struct MqPlan {
+    int ctx_cap, part_tokens, num_parts, row_tiles;
+};
+
+// KV partitions: fixed (partition_tokens > 0, rounded up to whole blocks), or
+// chosen (0): the fewest partitions of at most 2560 tokens that give about two
+// waves of CTAs, counting each sequence's row tiles.
+bool plan_mq(int num_seqs, int num_q_heads, int num_kv_heads, int block_size, int max_blocks, int max_query_len,
+             int max_context_len, int partition_tokens, MqPlan* pl) {
+    if (num_seqs <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || !block_size_built(block_size) ||
+        max_blocks <= 0 || max_query_len <= 0 || partition_tokens < 0)
+        return false;
+    const int64_t cap_tbl = (int64_t)max_blocks * block_size;
+    if (cap_tbl > INT32_MAX) return false;
+    int cap = (int)cap_tbl;
+    if (max_context_len > 0) cap = std::min(cap, max_context_len);
+    if (max_query_len > cap) return false;
+    const int group = num_q_heads / num_kv_heads;
+    pl->ctx_cap = cap;
+    pl->row_tiles = (int)(((int64_t)max_query_len * group + MQ_ROWS - 1) / MQ_ROWS);
+    int pt = partition_tokens;
+    if (pt == 0) {
+        constexpr int kMaxAutoPartition = 2560;
+        int sms = 148, dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int64_t target = 2ll * 2 * sms;                      // ~two waves of 2 CTAs per SM
+        pt = std::max(256, ((cap + block_size - 1) / block_size) * block_size);
+        for (int nparts = 1; nparts <= 65535; ++nparts) {
+            const int cand = (int)(((int64_t)(cap + nparts - 1) / nparts + block_size - 1) / block_size * block_size);
+            if (cand < 256) break;
+            pt = cand;
+            if (cand > kMaxAutoPartition) continue;
+            const int64_t est = (int64_t)num_seqs * num_kv_heads * pl->row_tiles * std::max<int64_t>(1, (nparts + 1) / 2);
+            if (est >= target) break;
+        }
+    }
+    pt = ((pt + block_size - 1) / block_size) * block_size;
+    const int parts = std::max(1, (cap + pt - 1) / pt);
+    if (parts > 65535 || (int64_t)num_seqs * pl->row_tiles > 65535) return false;
+    pl->part_tokens = pt;
+    pl->num_parts = parts;
+    return true;
+}
+
+size_t mq_ws_bytes(int num_tokens, int num_q_heads, int head_dim, const MqPlan& pl) {
+    if (pl.num_parts <= 1) return 0;
+    const size_t rows = (size_t)num_tokens * num_q_heads * pl.num_parts;
+    return (((rows * head_dim * 4) + 255) & ~size_t(255)) + rows * 2 * 4;
+}
+
+}  // namespace
+}  // namespace attn
+}  // namespace pkv
+
+extern "C" {
+
+size_t pkv_paged_attention_multi_query_workspace_bytes(int num_seqs, int num_tokens, int num_q_heads,
+                                                       int num_kv_heads, int head_dim, int block_size,
+                                                       int max_blocks_per_seq, int max_query_len, int max_context_len,
+                                                       int partition_tokens) {
+    pkv::attn::MqPlan pl;
+    if (num_tokens < 0 || head_dim <= 0 ||
+        !pkv::attn::plan_mq(num_seqs, num_q_heads, num_kv_heads, block_size, max_blocks_per_seq, max_query_len,
+                            max_context_len, partition_tokens, &pl))
+        return (size_t)-1;
+    return pkv::attn::mq_ws_bytes(num_tokens, num_q_heads, head_dim, pl);
+}
+
+pkv_status pkv_paged_attention_multi_query(void* out, pkv_dtype out_dtype, const void* q, const void* k_cache,
+                                           const void* v_cache, pkv_dtype kv_dtype, const int32_t* block_tables,
+                                           const int32_t* context_lens, const int32_t* query_start, float scale,
+                                           int num_seqs, int num_tokens, int num_q_heads, int num_kv_heads,
+                                           int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
+                                           int max_query_len, int max_context_len, int partition_tokens,
+                                           void* workspace, size_t workspace_bytes, void* stream) {
+    using namespace pkv;
+    using namespace pkv::attn;
+    if (num_seqs < 0 || num_tokens < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
+        max_blocks_per_seq <= 0 || max_query_len < 0 || max_context_len < 0 || partition_tokens < 0 ||
+        !std::isfinite(scale))
+        return PKV_ERR_INVALID_ARG;
+    if (out_dtype != PKV_F32 && out_dtype != PKV_BF16) return PKV_ERR_INVALID_ARG;
+    if (kv_dtype != PKV_BF16 && kv_dtype != PKV_F32 && kv_dtype != PKV_FP8_E4M3) return PKV_ERR_INVALID_ARG;
+    if (num_q_heads % num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
+    const int group = num_q_heads / num_kv_heads;
+    if (kv_dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+    if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
+    if (!block_size_built(block_size)) return PKV_ERR_UNSUPPORTED;
+    if (group != 1 && group != 2 && group != 4 && group != 8) return PKV_ERR_UNSUPPORTED;
+    if (num_seqs == 0 || num_tokens == 0 || max_query_len == 0) return PKV_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start)
+        return PKV_ERR_INVALID_ARG;
+    auto al = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) == 0; };
+    if (!al(out) || !al(q) || !al(k_cache) || !al(v_cache)) return PKV_ERR_INVALID_ARG;
+    MqPlan pl;
+    if (!plan_mq(num_seqs, num_q_heads, num_kv_heads, block_size, max_blocks_per_seq, max_query_len, max_context_len,
+                 partition_tokens, &pl))
+        return PKV_ERR_INVALID_ARG;
+    const size_t need = mq_ws_bytes(num_tokens, num_q_heads, head_dim, pl);
+    if (need > 0 && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)))
+        return PKV_ERR_INVALID_ARG;
+    int* err = device_error_word();
+    if (!err) return PKV_ERR_CUDA;
+    CUtensorMap mk, mv;
+    if (!make_cache_map(&mk, k_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim, true) ||
+        !make_cache_map(&mv, v_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim, true))
+        return PKV_ERR_CUDA;
+    MqParams p{};
+    p.out = out;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.query_start = query_start;
+    p.err = err;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.out_f32 = out_dtype == PKV_F32;
+    p.num_seqs = num_seqs;
+    p.num_tokens = num_tokens;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.group = group;
+    p.max_blocks = max_blocks_per_seq;
+    p.num_blocks = num_blocks;
+    p.ctx_cap = pl.ctx_cap;
+    p.max_query_len = max_query_len;
+    p.block_size = block_size;
+    p.part_blocks = pl.part_tokens / block_size;
+    p.num_parts = pl.num_parts;
+    p.row_tiles = pl.row_tiles;
+    if (need > 0) {
+        const size_t rows = (size_t)num_tokens * num_q_heads * pl.num_parts;
+        p.ws_o = static_cast<float*>(workspace);
+        p.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + (((rows * head_dim * 4) + 255) & ~size_t(255)));
+    }
+    if (pl.num_parts > 1 && num_tokens > 65535) return PKV_ERR_UNSUPPORTED;   // merge grid
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    dim3 grid(num_kv_heads, pl.num_parts, num_seqs * pl.row_tiles);
+    cudaError_t e = head_dim == 128 ? launch_mq_bs<128>(block_size, mk, mv, p, grid, st)
+                                    : launch_mq_bs<64>(block_size, mk, mv, p, grid, st);
+    if (e != cudaSuccess) return PKV_ERR_CUDA;
+    if (pl.num_parts > 1) {
+        dim3 g2(num_q_heads, num_tokens);
+        if (head_dim == 128) merge_mq_kernel<128><<<g2, 128, 0, st>>>(p);
+        else merge_mq_kernel<64><<<g2, 64, 0, st>>>(p);
+        if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
+    }
+    return PKV_OK;
+}
+
+}  // extern "C"

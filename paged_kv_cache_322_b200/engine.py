@@ -154,6 +154,35 @@ class PagedKVCache:
     def block_tables(self, seq_ids):
         return self.bm.block_tables(seq_ids, self.max_blocks_per_seq)
 
+    # -- several tokens per sequence: chunked prefill, speculative verify -----
+    def extend(self, seq_ids, counts, q, k_new, v_new, scale: float, out=None, out_dtype=torch.float32,
+               partition_tokens: int = 0, stream=None):
+        """Appends counts[i] tokens to sequence seq_ids[i] (k_new, v_new [T, Hkv, D],
+        rows grouped by sequence in the listed order) and returns causal
+        attention of their queries q [T, Hq, D] over each sequence's cache."""
+        seq_ids = np.asarray(seq_ids, dtype=np.int64)
+        counts = np.asarray(counts, dtype=np.int64)
+        if seq_ids.shape != counts.shape or (counts < 0).any() or int(counts.sum()) != q.shape[0]:
+            raise ValueError("counts must match the rows of q, one count per sequence")
+        order = np.repeat(seq_ids, counts)
+        slots, src, dst = self.bm.append_slots(order)
+        if src.size:
+            binding.copy_blocks(self.k_cache, self.v_cache, self._to_device("src", src, stream),
+                                self._to_device("dst", dst, stream), stream=stream)
+        if order.size:
+            self.append(k_new, v_new, self._to_device("slots", slots, stream), stream=stream)
+        tables, lens = self.block_tables(seq_ids)
+        qs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=self.device)
+        if q.shape[0]:
+            binding.paged_attention_multi_query(
+                out, q, self.k_cache, self.v_cache, self._to_device("tables", tables, stream),
+                self._to_device("lens", lens, stream), self._to_device("qstart", qs, stream), scale,
+                max_query_len=int(counts.max()), max_context_len=int(lens.max()), partition_tokens=partition_tokens,
+                stream=stream)
+        return out
+
     # -- the decode step -----------------------------------------------------
     def decode_step(self, seq_ids, q, k_new, v_new, scale: float, out=None, out_dtype=torch.float32,
                     partition_tokens: int = 0, stream=None):
