@@ -51,9 +51,11 @@ def parse():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="pkv", choices=["pkv", "reference"])
-    ap.add_argument("--op", default="decode", choices=["decode", "swap"],
+    ap.add_argument("--op", default="decode", choices=["decode", "swap", "mq"],
                     help="decode: the decode step (append + attention); swap: preemption by swapping half the "
-                         "workload's sequences to a page-locked host pool and back")
+                         "workload's sequences to a page-locked host pool and back; mq: several causal query "
+                         "tokens per sequence (--query-len: 512 = a chunked-prefill chunk, 5 = speculative verify)")
+    ap.add_argument("--query-len", type=int, default=512, help="query tokens per sequence and step (--op mq)")
     ap.add_argument("--workload", default="llama2_7b", choices=list(wl.WORKLOADS))
     ap.add_argument("--partition-tokens", type=int, default=-2,
                     help="-2: the workload's; 0: library-chosen partitions; -1: persistent schedule; >0: fixed")
@@ -221,6 +223,15 @@ def measured_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def measured_tflops() -> float:
+    """Measured dense bf16 TFLOP/s (burst), or the fallback figure."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"])
+    return 1590.0
 
 
 def traffic_record(workload: str):
@@ -558,6 +569,166 @@ def run_swap(args, ws, rank, local):
     }
 
 
+def run_mq(args, ws, rank, local):
+    """Causal multi-query steps: every sequence appends --query-len tokens (a
+    prefill chunk, or draft tokens to verify) and attends with them over its
+    cache. Device-timed: the append kernel + the multi-query attention over
+    inputs already in HBM; the attention launches alone give the roofline
+    (tensor FLOP/s when the step's FLOP per algorithmic byte is above the
+    measured ridge, HBM GB/s otherwise). e2e: the same steps through
+    PagedKVCache.extend from page-locked host buffers, output read back."""
+    import torch
+    from paged_kv_cache_322_b200 import binding
+    from paged_kv_cache_322_b200.engine import PagedKVCache
+
+    dev = torch.device("cuda", local)
+    w = replica_workload(override_workload(wl.WORKLOADS[args.workload], args), rank)
+    if w.kv_dtype != "bf16":
+        raise SystemExit("--op mq runs bf16 caches")
+    n, K, W = args.query_len, args.steps, args.warmup
+    part = 0 if args.partition_tokens in (-2, -1) else args.partition_tokens
+    lens0 = wl.context_lens(w)
+    bs, B = w.block_size, w.num_seqs
+    grow = 2 * (K + W) * n                              # device loop, then the e2e loop
+    mb = -(-int(lens0.max() + grow) // bs)
+    nb = max(w.num_blocks, int(sum(-(-(int(c) + grow) // bs) for c in lens0)) + 64)
+    cache = PagedKVCache(nb, bs, w.num_kv_heads, w.head_dim, torch.bfloat16, dev, free_order=wl.free_order(
+        dataclasses.replace(w, num_blocks=nb)), max_blocks_per_seq=mb)
+    kvs = wl.prompt_kv_all(w, lens0)
+    for s in range(B):
+        cache.add_sequence(s, torch.from_numpy(kvs[s][0]).to(dev, torch.bfloat16),
+                           torch.from_numpy(kvs[s][1]).to(dev, torch.bfloat16))
+    del kvs
+    ids = np.arange(B, dtype=np.int64)
+    hq, hkv, d = w.num_q_heads, w.num_kv_heads, w.head_dim
+    T = B * n
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed)
+
+    def rnd(shape):
+        return torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+
+    def flops_and_bytes(lens_after):
+        fl = sum(4 * hq * d * (n * (int(c) - n) + n * (n + 1) // 2) for c in lens_after)
+        # the attention launch: K and V of every cached token once, q in, out, block tables
+        by = (int(lens_after.sum()) * hkv * d * 2 * 2 + T * hq * d * 2 * 2 +
+              int(sum(-(-int(c) // bs) for c in lens_after)) * 4)
+        return fl, by
+
+    steps = []
+    order = np.repeat(ids, n)
+    for i in range(K + W):
+        slots, src, dst = cache.bm.append_slots(order)
+        assert src.size == 0
+        tables, lens = cache.block_tables(ids)
+        fl, by = flops_and_bytes(lens)
+        steps.append(dict(q=rnd((T, hq, d)), k=rnd((T, hkv, d)), v=rnd((T, hkv, d)),
+                          slots=torch.from_numpy(slots).to(dev), tables=torch.from_numpy(tables).to(dev),
+                          lens=torch.from_numpy(lens).to(dev), maxlen=int(lens.max()), flops=fl, bytes=by))
+    qs = torch.from_numpy(np.arange(0, T + 1, n, dtype=np.int32)).to(dev)
+    out = torch.empty((T, hq, d), dtype=torch.bfloat16, device=dev)
+    maxctx = max(st["maxlen"] for st in steps)
+    wsb = binding.multi_query_workspace_bytes(B, T, hq, hkv, d, bs, mb, n, maxctx, part)
+    workspace = torch.empty(max(wsb, 256), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step_device(st, e0=None, e1=None):
+        cache.append(st["k"], st["v"], st["slots"])
+        if e0 is not None:
+            e0.record(stream)
+        binding.paged_attention_multi_query(out, st["q"], cache.k_cache, cache.v_cache, st["tables"], st["lens"], qs,
+                                            w.scale, max_query_len=n, max_context_len=maxctx, partition_tokens=part,
+                                            workspace=workspace)
+        if e1 is not None:
+            e1.record(stream)
+
+    for i in range(W):
+        step_device(steps[i])
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t0.record(stream)
+        for i in range(K):
+            step_device(steps[W + i], *ev[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    assert binding.get_device_error() == 0
+    ms = t0.elapsed_time(t1)
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    timed = steps[W:]
+    fl = statistics.mean(st["flops"] for st in timed)
+    by = statistics.mean(st["bytes"] for st in timed)
+    ms_max, _, tok_s = aggregate(ms, 0.0, float(T * K), ws)
+    flop_total = all_sum(float(sum(st["flops"] for st in timed)), ws)
+    peak_gbs, peak_kind = measured_peaks()
+    peak_tf = measured_tflops()
+    ridge = peak_tf * 1e12 / (peak_gbs * 1e9)
+    tensor = fl / by > ridge
+    ach = (fl / (attn_ms * 1e-3) / 1e12) if tensor else (by / (attn_ms * 1e-3) / 1e9)
+    peak = peak_tf if tensor else peak_gbs
+    del steps
+
+    # ---- e2e: PagedKVCache.extend from page-locked host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        host = [tuple(torch.empty(shape, dtype=torch.bfloat16).normal_().pin_memory()
+                      for shape in ((T, hq, d), (T, hkv, d), (T, hkv, d))) for _ in range(2)]
+        dq, dk, dv = (torch.empty(x.shape, dtype=torch.bfloat16, device=dev) for x in host[0])
+        out_h = torch.empty((T, hq, d), dtype=torch.bfloat16).pin_memory()
+
+        def step_host(hb):
+            for dst_t, src_t in zip((dq, dk, dv), hb):
+                dst_t.copy_(src_t, non_blocking=True)
+            cache.extend(ids, [n] * B, dq, dk, dv, w.scale, out=out, partition_tokens=part, stream=stream)
+            out_h.copy_(out, non_blocking=True)
+            stream.synchronize()
+
+        for i in range(W):
+            step_host(host[i % 2])
+        barrier(ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(K):
+            step_host(host[i % 2])
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(ws)
+        assert binding.get_device_error() == 0
+        e_ms, _, e_tok_s = aggregate(e0.elapsed_time(e1), 0.0, float(T * K), ws)
+        e2e = {"value": round(e_tok_s, 1), "unit": "query tokens/s",
+               "h2d_bytes_per_step": int(T * (hq + 2 * hkv) * d * 2 + T * 8 + B * (mb * 4 + 8)),
+               "d2h_bytes_per_step": int(T * hq * d * 2), "ms_per_step": round(e_ms / K, 4),
+               "path": "PagedKVCache.extend (block manager, H2D, append, multi-query attention), D2H, sync"}
+
+    return {
+        "metric": f"multi-query paged attention ({'chunked prefill' if n >= 64 else 'speculative verify'}): "
+                  "query tokens/s per step (append + causal attention)",
+        "value": round(tok_s, 1), "unit": "query tokens/s", "n_gpus": ws, "steps": K,
+        "warmup": W, "ms_per_step": round(ms_max / K, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "attention_tflops": round(flop_total / (ms_max * 1e-3) / 1e12, 2),
+        "config": {"workload": w.description, "query_len": n, "global_batch": B * ws, "block_size": bs,
+                   "partition_tokens": part or "library-chosen",
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                   "l2": "KV per step larger than L2; no flush", "seed": w.seed},
+        "roofline": {"bound": "tensor" if tensor else "hbm",
+                     "kernel": "paged_mq_kernel (+ merge_mq_kernel when partitioned)",
+                     "achieved": round(ach, 2), "peak": peak, "unit": "TFLOP/s" if tensor else "GB/s",
+                     "frac": round(ach / peak, 4), "avg_launch_ms": round(attn_ms, 5),
+                     "flops_per_launch": int(fl), "algorithmic_bytes_per_launch": int(by),
+                     "flop_per_byte": round(fl / by, 1), "ridge_flop_per_byte": round(ridge, 1),
+                     "peak_source": ("measured bf16 dense (cuBLAS burst)" if tensor else peak_kind), "traffic": None},
+        "e2e": e2e,
+        "gpu_launches": 2 * K + (K if part and maxctx > part else 0),
+        "clocks": clocks.summary(),
+    }
+
+
 def paging_overhead(w, cache, kvs, dev, dt, cdt, mb, part, K, W):
     """The same attention call over the same prompts stored twice: blocks in the
     workload's random physical placement (the bench cache) and in identity
@@ -676,7 +847,8 @@ def main():
         return
     ws, rank, local = dist_init(args)
     try:
-        r = run_swap(args, ws, rank, local) if args.op == "swap" else run_pkv(args, ws, rank, local)
+        run = {"swap": run_swap, "mq": run_mq}.get(args.op, run_pkv)
+        r = run(args, ws, rank, local)
         if rank == 0:
             print(json.dumps(r), flush=True)
     finally:

@@ -33,7 +33,11 @@ namespace attn {
 namespace {
 
 constexpr int MQ_ROWS_PER_WARP = 16;
-constexpr int MQ_ROWS = NCW * MQ_ROWS_PER_WARP;     // query rows per CTA
+// Consumer warps form NCW / wpr row groups of 16 rows; the wpr warps of a group
+// share its rows and split the KV stages among them (wpr = 1: every warp has
+// its own rows and folds every stage; wpr = 4: one group of 16 rows, the KV
+// range split 4 ways, as a decode step with few query rows wants).
+__host__ __device__ constexpr int mq_rows_per_tile(int wpr) { return NCW / wpr * MQ_ROWS_PER_WARP; }
 
 struct MqParams {
     void* out;                    // [T, Hq, D]
@@ -49,7 +53,24 @@ struct MqParams {
     int num_seqs, num_tokens, num_q_heads, num_kv_heads, group;
     int max_blocks, num_blocks, ctx_cap, max_query_len;
     int block_size, part_blocks, num_parts, row_tiles;
+    int wpr;                      // warps per row group: 1, 2 or 4
 };
+
+// One normalised output value of row qh (sequence-level token row x head),
+// written to out (one partition) or to the partition's partial.
+template <int D>
+__device__ __forceinline__ void mq_store(const MqParams& p, int64_t qh, int part, bool direct, int d, float v) {
+    if (direct) {
+        if (p.out_f32) static_cast<float*>(p.out)[qh * D + d] = v;
+        else static_cast<__nv_bfloat16*>(p.out)[qh * D + d] = __float2bfloat16_rn(v);
+    } else {
+        p.ws_o[(qh * p.num_parts + part) * D + d] = v;
+    }
+}
+
+__device__ __forceinline__ void mq_consumers_barrier() {
+    asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+}
 
 __device__ __forceinline__ uint64_t l2_policy_evict_normal() {
     uint64_t pol;
@@ -223,24 +244,38 @@ struct MqConsumer {
                 const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt) {
-                    const float va = o[mt][nt][cc] * inv, vb = o[mt][nt][2 + cc] * inv;
-                    const int d0 = mt * 16 + g, d1 = d0 + 8;
-                    if (direct) {
-                        if (p.out_f32) {
-                            static_cast<float*>(p.out)[qh * D + d0] = va;
-                            static_cast<float*>(p.out)[qh * D + d1] = vb;
-                        } else {
-                            static_cast<__nv_bfloat16*>(p.out)[qh * D + d0] = __float2bfloat16_rn(va);
-                            static_cast<__nv_bfloat16*>(p.out)[qh * D + d1] = __float2bfloat16_rn(vb);
-                        }
-                    } else {
-                        p.ws_o[(qh * p.num_parts + part) * D + d0] = va;
-                        p.ws_o[(qh * p.num_parts + part) * D + d1] = vb;
-                    }
+                    mq_store<D>(p, qh, part, direct, mt * 16 + g, o[mt][nt][cc] * inv);
+                    mq_store<D>(p, qh, part, direct, mt * 16 + g + 8, o[mt][nt][2 + cc] * inv);
                 }
                 if (!direct && g == 0) {
                     p.ws_ml[(qh * p.num_parts + part) * 2 + 0] = m[nt][cc];
                     p.ws_ml[(qh * p.num_parts + part) * 2 + 1] = lsum;
+                }
+            }
+        }
+    }
+
+    // The warp's unnormalised state for a cross-warp merge: so [16 rows][D],
+    // sm / sl [16 rows] (m and the full l of each row).
+    __device__ __forceinline__ void spill(float* so, float* sm, float* sl, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                float lsum = l[nt][cc];
+                lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
+                lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
+                lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
+                const int r = nt * 8 + 2 * t + cc;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    so[r * D + mt * 16 + g] = o[mt][nt][cc];
+                    so[r * D + mt * 16 + g + 8] = o[mt][nt][2 + cc];
+                }
+                if (g == 0) {
+                    sm[r] = m[nt][cc];
+                    sl[r] = lsum;
                 }
             }
         }
@@ -257,7 +292,10 @@ struct MqKern {
     static constexpr int PIECE = R * D * 2;
     static constexpr int REGION = TOK * D * 2;                  // K (or V) of one stage
     static constexpr int STAGE_BYTES = 2 * REGION;
+    static constexpr int MERGE = NCW * MQ_ROWS_PER_WARP * (D + 2) * 4;   // cross-warp merge scratch
     static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 2 * STAGES * 8;
+    static_assert(MERGE <= STAGES * STAGE_BYTES, "the merge scratch reuses the ring");
+    static_assert(STAGES % 4 == 0, "ring depth must be a multiple of every warps-per-group choice");
     static_assert(BPS * R == TOK && PPB * R == BSZ, "block size must be a power of two >= 8");
 };
 
@@ -277,10 +315,11 @@ paged_mq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int q0, n, c;
     mq_sequence(p, seq, q0, n, c);
-    const int row_begin = tile * MQ_ROWS;
+    const int wpr = p.wpr, rows_per_tile = mq_rows_per_tile(wpr);
+    const int row_begin = tile * rows_per_tile;
     if (row_begin >= n * p.group) return;                          // no live rows in this tile
     // last visible position of the tile's rows, and this partition's KV range
-    const int last_tok = min(n - 1, (row_begin + MQ_ROWS - 1) / p.group);
+    const int last_tok = min(n - 1, (row_begin + rows_per_tile - 1) / p.group);
     const int kv_end = c - n + last_tok + 1;                       // tokens [0, kv_end) are visible to some row
     const int pt = p.part_blocks * BSZ;
     const int kv0 = part * pt;
@@ -294,7 +333,7 @@ paged_mq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], NCW);
+            mbar_init(&empty[i], NCW / wpr);                       // one warp of each row group
         }
         s_abort = 0;
         fence_barrier_init();
@@ -356,13 +395,16 @@ paged_mq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 mbar_wait_bounded(&full[j % STAGES], (j / STAGES) & 1, p.err);
         }
     } else {
-        // ---------------- consumers: every warp folds every stage ----------------
+        // ---------------- consumers: row group rg, turn sub of its wpr warps ----------------
         const int cw = warp - 1;
-        const int row0 = row_begin + cw * MQ_ROWS_PER_WARP;
+        const int rg = cw / wpr, sub = cw - rg * wpr;
+        const int row0 = row_begin + rg * MQ_ROWS_PER_WARP;
         MqConsumer<D> cons;
         cons.init(p, row0, kvh, q0, n, c, lane);
         const int nstage = (npiece + K::BPS - 1) / K::BPS;
-        for (int j = 0; j < nstage; ++j) {
+        // With STAGES a multiple of wpr, every round of a stage goes to the same
+        // warp of each group, so no warp can run a ring phase ahead of the producer.
+        for (int j = sub; j < nstage; j += wpr) {
             const int st = j % STAGES;
             const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err);
             if (__any_sync(0xffffffffu, !got || s_abort != 0)) {
@@ -375,7 +417,47 @@ paged_mq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
         }
-        if (!s_abort) cons.finish(p, row0, kvh, q0, n, part, direct, lane);
+        if (wpr == 1) {
+            if (!s_abort) cons.finish(p, row0, kvh, q0, n, part, direct, lane);
+        } else {
+            // merge the wpr partial states of each row group through shared memory
+            // (the ring is free once every consumer is past its last stage)
+            mq_consumers_barrier();
+            if (!s_abort) {
+                float* so = reinterpret_cast<float*>(smem);
+                float* sm = so + NCW * MQ_ROWS_PER_WARP * D;
+                float* sl = sm + NCW * MQ_ROWS_PER_WARP;
+                cons.spill(so + cw * MQ_ROWS_PER_WARP * D, sm + cw * MQ_ROWS_PER_WARP, sl + cw * MQ_ROWS_PER_WARP,
+                           lane);
+                mq_consumers_barrier();
+                const int G = p.group;
+                for (int idx = threadIdx.x - 32; idx < NCW / wpr * MQ_ROWS_PER_WARP * D; idx += NCW * 32) {
+                    const int grp = idx / (MQ_ROWS_PER_WARP * D), rem = idx - grp * MQ_ROWS_PER_WARP * D;
+                    const int rr = rem / D, d = rem - rr * D;
+                    const int r = row_begin + grp * MQ_ROWS_PER_WARP + rr;
+                    const int i = r / G, h = r - i * G;
+                    if (i >= n) continue;
+                    float M = kNegInf;
+                    for (int w = grp * wpr; w < (grp + 1) * wpr; ++w) M = fmaxf(M, sm[w * MQ_ROWS_PER_WARP + rr]);
+                    float L = 0.f, O = 0.f;
+                    if (M != kNegInf) {
+                        for (int w = grp * wpr; w < (grp + 1) * wpr; ++w) {
+                            const float mw = sm[w * MQ_ROWS_PER_WARP + rr];
+                            if (mw == kNegInf) continue;
+                            const float sc = fast_exp2(mw - M);
+                            L += sl[w * MQ_ROWS_PER_WARP + rr] * sc;
+                            O += so[(w * MQ_ROWS_PER_WARP + rr) * D + d] * sc;
+                        }
+                    }
+                    const int64_t qh = (int64_t)(q0 + i) * p.num_q_heads + kvh * G + h;
+                    mq_store<D>(p, qh, part, direct, d, L > 0.f ? O / L : 0.f);
+                    if (!direct && d == 0) {
+                        p.ws_ml[(qh * p.num_parts + part) * 2 + 0] = M;
+                        p.ws_ml[(qh * p.num_parts + part) * 2 + 1] = L;
+                    }
+                }
+            }
+        }
     }
 }
 
@@ -448,7 +530,7 @@ cudaError_t launch_mq_bs(int bs, const CUtensorMap& mk, const CUtensorMap& mv, c
 }
 
 struct MqPlan {
-    int ctx_cap, part_tokens, num_parts, row_tiles;
+    int ctx_cap, part_tokens, num_parts, row_tiles, wpr;
 };
 
 // KV partitions: fixed (partition_tokens > 0, rounded up to whole blocks), or
@@ -466,7 +548,10 @@ bool plan_mq(int num_seqs, int num_q_heads, int num_kv_heads, int block_size, in
     if (max_query_len > cap) return false;
     const int group = num_q_heads / num_kv_heads;
     pl->ctx_cap = cap;
-    pl->row_tiles = (int)(((int64_t)max_query_len * group + MQ_ROWS - 1) / MQ_ROWS);
+    // few rows (speculative verify, decode): fewer row groups, the KV range split among their warps
+    const int64_t rows = (int64_t)max_query_len * group;
+    pl->wpr = rows <= MQ_ROWS_PER_WARP ? 4 : (rows <= 2 * MQ_ROWS_PER_WARP ? 2 : 1);
+    pl->row_tiles = (int)((rows + mq_rows_per_tile(pl->wpr) - 1) / mq_rows_per_tile(pl->wpr));
     int pt = partition_tokens;
     if (pt == 0) {
         constexpr int kMaxAutoPartition = 2560;
@@ -576,6 +661,7 @@ pkv_status pkv_paged_attention_multi_query(void* out, pkv_dtype out_dtype, const
     p.part_blocks = pl.part_tokens / block_size;
     p.num_parts = pl.num_parts;
     p.row_tiles = pl.row_tiles;
+    p.wpr = pl.wpr;
     if (need > 0) {
         const size_t rows = (size_t)num_tokens * num_q_heads * pl.num_parts;
         p.ws_o = static_cast<float*>(workspace);
