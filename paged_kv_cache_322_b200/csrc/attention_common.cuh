@@ -565,7 +565,9 @@ cudaError_t dispatch_partitioned(pkv_dtype kv_dtype, bool use_mma, int head_dim,
 
 // Tensor map over a cache [nb, bs, hkv, d] (paged_attention.cu): box = piece_rows(bs)
 // tokens of one head, whole rows (SIMT) or 128-byte swizzled box rows (tensor cores).
-bool make_cache_map(CUtensorMap* map, const void* base, pkv_dtype dt, int nb, int bs, int hkv, int d, bool mma);
+// box_rows > 0 overrides the piece height (a divisor of bs, at most 256).
+bool make_cache_map(CUtensorMap* map, const void* base, pkv_dtype dt, int nb, int bs, int hkv, int d, bool mma,
+                    int box_rows = 0);
 
 // Persistent schedule (paged_attention_persistent.cu).
 cudaError_t launch_persistent(bool bf16, bool use_mma, int head_dim, int group, const CUtensorMap& mk,

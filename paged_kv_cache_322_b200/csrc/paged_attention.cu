@@ -89,7 +89,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // piece_rows(bs) tokens of one head (a whole block, or a slice of a block longer
 // than a ring stage), the whole row (SIMT) or 128-byte box rows with the 128-byte
 // swizzle (tensor-core path).
-bool make_cache_map(CUtensorMap* map, const void* base, pkv_dtype dt, int nb, int bs, int hkv, int d, bool mma) {
+bool make_cache_map(CUtensorMap* map, const void* base, pkv_dtype dt, int nb, int bs, int hkv, int d, bool mma,
+                    int box_rows) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t eb = dt == PKV_F32 ? 4 : (dt == PKV_BF16 ? 2 : 1);
@@ -98,7 +99,9 @@ bool make_cache_map(CUtensorMap* map, const void* base, pkv_dtype dt, int nb, in
                                                     : CU_TENSOR_MAP_DATA_TYPE_UINT8;
     cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)hkv, (cuuint64_t)bs, (cuuint64_t)nb};
     cuuint64_t strides[3] = {d * eb, (cuuint64_t)hkv * d * eb, (cuuint64_t)bs * hkv * d * eb};
-    cuuint32_t box[4] = {(cuuint32_t)(mma ? 128 / eb : d), 1, (cuuint32_t)piece_rows(bs, (int)eb), 1};
+    const int rows = box_rows > 0 ? box_rows : piece_rows(bs, (int)eb);
+    if (rows > 256 || bs % rows != 0) return false;
+    cuuint32_t box[4] = {(cuuint32_t)(mma ? 128 / eb : d), 1, (cuuint32_t)rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(map, ty, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     mma ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,

@@ -500,6 +500,62 @@ __global__ void __launch_bounds__(D) merge_mq_kernel(const MqParams p) {
     else static_cast<__nv_bfloat16*>(p.out)[qh * D + d] = __float2bfloat16_rn(v);
 }
 
+}  // namespace
+}  // namespace attn
+}  // namespace pkv
+
+#include "paged_attention_mq_tc.cuh"
+
+namespace pkv {
+namespace attn {
+namespace {
+
+template <int BSZ>
+cudaError_t launch_mq_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const MqParams& p,
+                         dim3 grid, cudaStream_t st) {
+    auto kern = tc::paged_mq_tc_kernel<BSZ>;
+    static std::atomic<uint64_t> done_mask{0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(done_mask.load() & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM);
+        if (e != cudaSuccess) return e;
+        done_mask.fetch_or(bit);
+    }
+    kern<<<grid, tc::THREADS, tc::SMEM, st>>>(mq, mk, mv, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mq_tc_bs(int bs, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                            const MqParams& p, dim3 grid, cudaStream_t st) {
+    switch (bs) {
+        case 8: return launch_mq_tc<8>(mq, mk, mv, p, grid, st);
+        case 16: return launch_mq_tc<16>(mq, mk, mv, p, grid, st);
+        case 32: return launch_mq_tc<32>(mq, mk, mv, p, grid, st);
+        default: return launch_mq_tc<64>(mq, mk, mv, p, grid, st);
+    }
+}
+
+// Tensor map over q [T, Hq, D] (bf16): box (64 dims, G heads, 128 / G tokens),
+// 128-byte swizzle, so one 128-row query tile lands as the K-major operand of
+// the tcgen05 kernel (row = token x G + head).
+bool make_q_map(CUtensorMap* map, const void* q, int T, int hq, int d, int group) {
+    cudaDriverEntryPointQueryResult qr;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &qr) != cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess || !f)
+        return false;
+    auto fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)hq, (cuuint64_t)T};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)hq * d * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)group, (cuuint32_t)(tc::ROWS / group)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, int BSZ>
 cudaError_t launch_mq(const CUtensorMap& mk, const CUtensorMap& mv, const MqParams& p, dim3 grid, cudaStream_t st) {
     constexpr int STAGES = 8;
@@ -531,13 +587,14 @@ cudaError_t launch_mq_bs(int bs, const CUtensorMap& mk, const CUtensorMap& mv, c
 
 struct MqPlan {
     int ctx_cap, part_tokens, num_parts, row_tiles, wpr;
+    bool tc;            // the tcgen05 kernel (128-row tiles)
 };
 
 // KV partitions: fixed (partition_tokens > 0, rounded up to whole blocks), or
 // chosen (0): the fewest partitions of at most 2560 tokens that give about two
 // waves of CTAs, counting each sequence's row tiles.
-bool plan_mq(int num_seqs, int num_q_heads, int num_kv_heads, int block_size, int max_blocks, int max_query_len,
-             int max_context_len, int partition_tokens, MqPlan* pl) {
+bool plan_mq(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks,
+             int max_query_len, int max_context_len, int partition_tokens, MqPlan* pl) {
     if (num_seqs <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || !block_size_built(block_size) ||
         max_blocks <= 0 || max_query_len <= 0 || partition_tokens < 0)
         return false;
@@ -551,13 +608,16 @@ bool plan_mq(int num_seqs, int num_q_heads, int num_kv_heads, int block_size, in
     // few rows (speculative verify, decode): fewer row groups, the KV range split among their warps
     const int64_t rows = (int64_t)max_query_len * group;
     pl->wpr = rows <= MQ_ROWS_PER_WARP ? 4 : (rows <= 2 * MQ_ROWS_PER_WARP ? 2 : 1);
-    pl->row_tiles = (int)((rows + mq_rows_per_tile(pl->wpr) - 1) / mq_rows_per_tile(pl->wpr));
+    // prefill-sized query tiles go to the tcgen05 kernel (head_dim 128)
+    pl->tc = head_dim == 128 && rows >= tc::ROWS;
+    const int tile_rows = pl->tc ? tc::ROWS : mq_rows_per_tile(pl->wpr);
+    pl->row_tiles = (int)((rows + tile_rows - 1) / tile_rows);
     int pt = partition_tokens;
     if (pt == 0) {
         constexpr int kMaxAutoPartition = 2560;
         int sms = 148, dev = 0;
         if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        const int64_t target = 2ll * 2 * sms;                      // ~two waves of 2 CTAs per SM
+        const int64_t target = 2ll * (pl->tc ? 1 : 2) * sms;       // ~two waves (1 or 2 CTAs per SM)
         pt = std::max(256, ((cap + block_size - 1) / block_size) * block_size);
         for (int nparts = 1; nparts <= 65535; ++nparts) {
             const int cand = (int)(((int64_t)(cap + nparts - 1) / nparts + block_size - 1) / block_size * block_size);
@@ -594,8 +654,8 @@ size_t pkv_paged_attention_multi_query_workspace_bytes(int num_seqs, int num_tok
                                                        int partition_tokens) {
     pkv::attn::MqPlan pl;
     if (num_tokens < 0 || head_dim <= 0 ||
-        !pkv::attn::plan_mq(num_seqs, num_q_heads, num_kv_heads, block_size, max_blocks_per_seq, max_query_len,
-                            max_context_len, partition_tokens, &pl))
+        !pkv::attn::plan_mq(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                            max_query_len, max_context_len, partition_tokens, &pl))
         return (size_t)-1;
     return pkv::attn::mq_ws_bytes(num_tokens, num_q_heads, head_dim, pl);
 }
@@ -627,18 +687,20 @@ pkv_status pkv_paged_attention_multi_query(void* out, pkv_dtype out_dtype, const
     auto al = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) == 0; };
     if (!al(out) || !al(q) || !al(k_cache) || !al(v_cache)) return PKV_ERR_INVALID_ARG;
     MqPlan pl;
-    if (!plan_mq(num_seqs, num_q_heads, num_kv_heads, block_size, max_blocks_per_seq, max_query_len, max_context_len,
-                 partition_tokens, &pl))
+    if (!plan_mq(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, max_query_len,
+                 max_context_len, partition_tokens, &pl))
         return PKV_ERR_INVALID_ARG;
     const size_t need = mq_ws_bytes(num_tokens, num_q_heads, head_dim, pl);
     if (need > 0 && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)))
         return PKV_ERR_INVALID_ARG;
     int* err = device_error_word();
     if (!err) return PKV_ERR_CUDA;
-    CUtensorMap mk, mv;
-    if (!make_cache_map(&mk, k_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim, true) ||
-        !make_cache_map(&mv, v_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim, true))
+    CUtensorMap mk, mv, mqm;
+    const int box_rows = pl.tc ? std::min(block_size, tc::TOK) : 0;   // 0: the decode pieces
+    if (!make_cache_map(&mk, k_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim, true, box_rows) ||
+        !make_cache_map(&mv, v_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim, true, box_rows))
         return PKV_ERR_CUDA;
+    if (pl.tc && !make_q_map(&mqm, q, num_tokens, num_q_heads, head_dim, group)) return PKV_ERR_CUDA;
     MqParams p{};
     p.out = out;
     p.q = static_cast<const __nv_bfloat16*>(q);
@@ -670,8 +732,9 @@ pkv_status pkv_paged_attention_multi_query(void* out, pkv_dtype out_dtype, const
     if (pl.num_parts > 1 && num_tokens > 65535) return PKV_ERR_UNSUPPORTED;   // merge grid
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     dim3 grid(num_kv_heads, pl.num_parts, num_seqs * pl.row_tiles);
-    cudaError_t e = head_dim == 128 ? launch_mq_bs<128>(block_size, mk, mv, p, grid, st)
-                                    : launch_mq_bs<64>(block_size, mk, mv, p, grid, st);
+    cudaError_t e = pl.tc ? launch_mq_tc_bs(block_size, mqm, mk, mv, p, grid, st)
+                    : head_dim == 128 ? launch_mq_bs<128>(block_size, mk, mv, p, grid, st)
+                                      : launch_mq_bs<64>(block_size, mk, mv, p, grid, st);
     if (e != cudaSuccess) return PKV_ERR_CUDA;
     if (pl.num_parts > 1) {
         dim3 g2(num_q_heads, num_tokens);

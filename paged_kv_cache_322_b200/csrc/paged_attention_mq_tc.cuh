@@ -1,0 +1,407 @@
+// Multi-query paged attention on the 5th-generation tensor cores (tcgen05) for
+// prefill-sized query tiles: bf16 caches, head_dim 128, 128 query rows per CTA.
+// Included by paged_attention_mq.cu, which routes a call here when every
+// sequence brings at least one full 128-row tile's worth of query rows.
+//
+//   S  = Q K^T   M = 128 query rows, N = 128 KV tokens, K = 128 dims  (TMEM, fp32)
+//   O += P V     M = 128 rows, N = 128 dims, K = 128 tokens            (TMEM, fp32)
+//
+// Roles (192 threads): warp 0 streams Q once and K/V tiles (TMA, 128-byte
+// swizzle, two stages); warp 1 owns the TMEM allocation and one of its threads
+// issues every tcgen05.mma; warps 2-5 run the softmax, one query row per thread
+// (its TMEM lane), so row max and row sum need no shuffles. The S accumulator
+// is double-buffered, so S of tile t+1 is computed while the softmax of tile t
+// runs. P goes to shared memory as two bf16 parts (high, and the rounding
+// residue) that both multiply V, so the probabilities keep ~16 bits. The online
+// softmax rescales O in TMEM only when a row's running maximum grows by more
+// than 2^8 over the reference it uses (p <= 2^8 stays exact enough in bf16 and
+// fp32), so most tiles skip the O round trip.
+#pragma once
+
+namespace pkv {
+namespace attn {
+namespace tc {
+
+constexpr int ROWS = 128;          // query rows per CTA (UMMA M)
+constexpr int TOK = 128;           // KV tokens per tile
+constexpr int D = 128;
+constexpr int THREADS = 192;
+constexpr int HALF = 128 * 128;    // one 64-element-wide half of a 128-row operand, bytes
+constexpr int Q_OFF = 0;
+constexpr int KV_OFF = 2 * HALF;                  // two stages of K (2 halves) + V (2 halves)
+constexpr int STAGE = 4 * HALF;
+constexpr int P_OFF = KV_OFF + 2 * STAGE;         // P high (2 halves), then P low (2 halves)
+constexpr int BAR_OFF = P_OFF + 4 * HALF;
+constexpr int NBAR = 13;
+constexpr int SMEM = 1024 + BAR_OFF + NBAR * 8 + 16;
+constexpr int TMEM_COLS = 512;                    // S0 [0,128) S1 [128,256) O [256,384)
+static_assert(SMEM <= 232448, "shared memory per CTA");
+
+// Barrier indices.
+enum { B_Q = 0, B_FULL = 1, B_EMPTY = 3, B_SFULL = 5, B_SFREE = 7, B_PREADY = 9, B_ODONE = 10, B_DRAIN = 11 };
+
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= 1ull << 46;                              // descriptor version of sm_100
+    d |= 2ull << 61;                              // 128-byte swizzle
+    return d;
+}
+
+// kind::f16 instruction descriptor: bf16 A and B, fp32 D, A K-major, B K- or MN-major.
+constexpr uint32_t idesc_bf16(int m, int n, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major ? (1u << 16) : 0u) | ((uint32_t)(n >> 3) << 17) |
+           ((uint32_t)(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+        ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+          "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+          "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+          "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+          "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+          "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+          "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+          "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+          "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+          "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+          "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// tm_q: q as [T, Hq, D] with box (64, G, 128 / G); tm_k / tm_v: the caches with
+// box (64, 1, R, 1), R = min(block_size, 128) rows (one whole block per piece).
+template <int BSZ>
+__global__ void __launch_bounds__(THREADS, 1)
+paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const MqParams p) {
+    constexpr int R = BSZ < TOK ? BSZ : TOK;                    // rows of one TMA piece (a whole block)
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + BAR_OFF + NBAR * 8);
+    __shared__ volatile int s_abort;
+
+    const int kvh = blockIdx.x, part = blockIdx.y;
+    const int seq = blockIdx.z / p.row_tiles, tile = blockIdx.z - seq * p.row_tiles;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = p.group;
+    int q0, n, c;
+    mq_sequence(p, seq, q0, n, c);
+    const int row_begin = tile * ROWS;
+    if (row_begin >= n * G) return;                             // no live rows (uniform over the CTA)
+    const int last_tok = min(n - 1, (row_begin + ROWS - 1) / G);
+    const int kv_end = c - n + last_tok + 1;
+    const int pt = p.part_blocks * BSZ;
+    const int kv0 = part * pt;
+    if (kv0 >= kv_end) return;
+    const int ntok = min(pt, kv_end - kv0);
+    const int ntiles = (ntok + TOK - 1) / TOK;
+    const int blk0 = part * p.part_blocks;
+    const bool direct = (c + pt - 1) / pt <= 1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bar[B_Q], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bar[B_FULL + s], 1);
+            mbar_init(&bar[B_EMPTY + s], 1);
+            mbar_init(&bar[B_SFULL + s], 1);
+            mbar_init(&bar[B_SFREE + s], 128);
+        }
+        mbar_init(&bar[B_PREADY], 128);
+        mbar_init(&bar[B_ODONE], 1);
+        mbar_init(&bar[B_DRAIN], 1);
+        s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {                                            // TMEM: S0, S1, O
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    fence_before();
+    __syncthreads();
+    fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- producer: Q once, then K/V tiles ----------------
+        if (lane == 0) {
+            bool ok = true;
+            int issued = 0;
+            mbar_arrive_expect_tx(&bar[B_Q], 2 * HALF);
+            for (int h = 0; h < 2; ++h)
+                tma_load_3d(smem + Q_OFF + h * HALF, &tm_q, &bar[B_Q], h * 64, kvh * G, q0 + row_begin / G);
+            const uint64_t pol = l2_policy_evict_normal();
+            const int32_t* bt = p.block_tables + (int64_t)seq * p.max_blocks + blk0;
+            for (int t = 0; t < ntiles && ok; ++t) {
+                const int s = t & 1;
+                if (!mbar_wait_bounded(&bar[B_EMPTY + s], ((t >> 1) & 1) ^ 1, p.err)) {
+                    ok = false;
+                    s_abort = 1;
+                    break;
+                }
+                const int tok_here = min(TOK, ntok - t * TOK);
+                const int np = (tok_here + R - 1) / R;
+                mbar_arrive_expect_tx(&bar[B_FULL + s], np * 2 * 2 * R * 128);
+                ++issued;
+                uint8_t* kst = smem + KV_OFF + s * STAGE;
+                uint8_t* vst = kst + 2 * HALF;
+                for (int b = 0; b < np; ++b) {
+                    const int j = (t * TOK + b * R) / BSZ;      // block of the partition
+                    const int sub = (t * TOK + b * R) % BSZ;    // first row inside it (0 when R = BSZ)
+                    int id = __ldg(bt + j);
+                    if (id < 0 || id >= p.num_blocks) {
+                        flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
+                        id = p.num_blocks;                      // zero-filled tile
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        tma_load_4d(kst + h * HALF + b * R * 128, &tm_k, &bar[B_FULL + s], h * 64, kvh, sub, id, pol);
+                        tma_load_4d(vst + h * HALF + b * R * 128, &tm_v, &bar[B_FULL + s], h * 64, kvh, sub, id, pol);
+                    }
+                }
+            }
+            if (!ok) {
+                for (int t = max(0, issued - 2); t < issued; ++t)
+                    mbar_wait_bounded(&bar[B_FULL + (t & 1)], (t >> 1) & 1, p.err);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (one thread) ----------------
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16(ROWS, TOK, false);
+            constexpr uint32_t IDESC_PV = idesc_bf16(ROWS, D, true);
+            const uint32_t q_addr = smem_u32(smem + Q_OFF);
+            const uint32_t p_addr = smem_u32(smem + P_OFF);
+            bool ok = mbar_wait_bounded(&bar[B_Q], 0, p.err);
+            int issued_pv = 0;
+            // PV of tile u: O += P_hi V + P_lo V over the tile's 128 tokens, 8 k-steps of 16
+            auto pv = [&](int u) -> bool {
+                if (!mbar_wait_bounded(&bar[B_PREADY], u & 1, p.err)) return false;
+                fence_after();
+                const uint32_t v_addr = smem_u32(smem + KV_OFF + (u & 1) * STAGE + 2 * HALF);
+#pragma unroll
+                for (int part_lo = 0; part_lo < 2; ++part_lo) {
+#pragma unroll
+                    for (int k = 0; k < TOK / 16; ++k) {
+                        // A = P: K-major rows, tokens 16k..16k+15 -> half k/4, 32 bytes per k-step inside it
+                        const uint64_t a = desc_sw128(p_addr + part_lo * 2 * HALF + (k >> 2) * HALF + (k & 3) * 32,
+                                                      16, 1024);
+                        // B = V: MN-major (dims contiguous), tokens 16k.. -> 16 rows of 128 B; dims halves LBO apart
+                        const uint64_t b = desc_sw128(v_addr + k * 16 * 128, HALF, 1024);
+                        mma_ss(tmem + 256, a, b, IDESC_PV, (u > 0 || part_lo > 0 || k > 0) ? 1u : 0u);
+                    }
+                }
+                commit(&bar[B_ODONE]);
+                commit(&bar[B_EMPTY + (u & 1)]);
+                ++issued_pv;
+                return true;
+            };
+            for (int t = 0; t < ntiles && ok; ++t) {
+                const int s = t & 1;
+                ok = mbar_wait_bounded(&bar[B_FULL + s], (t >> 1) & 1, p.err);
+                if (ok && t >= 2) ok = mbar_wait_bounded(&bar[B_SFREE + s], ((t - 2) >> 1) & 1, p.err);
+                if (!ok) break;
+                fence_after();
+                const uint32_t k_addr = smem_u32(smem + KV_OFF + s * STAGE);
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k) {
+                    const uint64_t a = desc_sw128(q_addr + (k >> 2) * HALF + (k & 3) * 32, 16, 1024);
+                    const uint64_t b = desc_sw128(k_addr + (k >> 2) * HALF + (k & 3) * 32, 16, 1024);
+                    mma_ss(tmem + s * 128, a, b, IDESC_S, k > 0 ? 1u : 0u);
+                }
+                commit(&bar[B_SFULL + s]);
+                if (t >= 1) ok = pv(t - 1);
+            }
+            if (ok && ntiles > 0) ok = pv(ntiles - 1);
+            if (!ok) s_abort = 1;
+            // every MMA issued has finished before TMEM is released
+            commit(&bar[B_DRAIN]);
+            mbar_wait_bounded(&bar[B_DRAIN], 0, p.err);
+            (void)issued_pv;
+        }
+    } else {
+        // ---------------- softmax: one query row per thread ----------------
+        const int quarter = warp & 3;                           // TMEM lanes this warp may access
+        const int lr = quarter * 32 + lane;                     // row of the tile = TMEM lane
+        const int r = row_begin + lr;
+        const int qi = r / G, hh = r - qi * G;
+        const int pos = qi < n ? c - n + qi : -1;
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        uint8_t* prow_hi = smem + P_OFF;
+        uint8_t* prow_lo = smem + P_OFF + 2 * HALF;
+        float m_ref = kNegInf, l = 0.f;
+        bool ok = true;
+        for (int t = 0; t < ntiles; ++t) {
+            const int s = t & 1;
+            const bool got = mbar_wait_bounded(&bar[B_SFULL + s], (t >> 1) & 1, p.err);
+            if (__any_sync(0xffffffffu, !got || s_abort != 0)) {
+                ok = false;
+                s_abort = 1;
+                break;
+            }
+            fence_after();
+            float x[TOK];
+#pragma unroll
+            for (int ch = 0; ch < TOK / 32; ++ch) tmem_ld32(lane_base + s * 128 + ch * 32, x + ch * 32);
+            tmem_wait_ld();
+            fence_before();
+            mbar_arrive(&bar[B_SFREE + s]);
+            // V rows past the range (the unwritten tail of the last block, or a stage
+            // row no piece filled) may hold anything, NaN included: P is 0 there, but
+            // 0 * NaN would not be, so those rows are zeroed before the PV product.
+            const int tok_here = min(TOK, ntok - t * TOK);
+            if (lr >= tok_here) {
+                uint8_t* vrow = smem + KV_OFF + s * STAGE + 2 * HALF + lr * 128;
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc)
+                        *reinterpret_cast<uint4*>(vrow + h * HALF + (cc << 4)) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            // masks: past the partition's range, or after the row's position (causal)
+            const int tok0 = kv0 + t * TOK;
+            const int lim = min(pos, kv0 + ntok - 1) - tok0;    // columns 0..lim are visible
+            float mt = kNegInf;
+#pragma unroll
+            for (int j = 0; j < TOK; ++j) {
+                x[j] = j <= lim ? x[j] * p.scale_log2 : kNegInf;
+                mt = fmaxf(mt, x[j]);
+            }
+            const float m_new = fmaxf(m_ref, mt);
+            const bool grow = m_new > m_ref + 8.f;              // also true when m_ref is -inf and the row sees a token
+            if (t > 0) {
+                const bool done = mbar_wait_bounded(&bar[B_ODONE], (t - 1) & 1, p.err);
+                if (__any_sync(0xffffffffu, !done || s_abort != 0)) {
+                    ok = false;
+                    s_abort = 1;
+                    break;
+                }
+                fence_after();
+                if (__any_sync(0xffffffffu, grow && m_ref != kNegInf)) {
+                    const float alpha = (grow && m_ref != kNegInf) ? fast_exp2(m_ref - m_new) : 1.f;
+#pragma unroll
+                    for (int ch = 0; ch < D / 32; ++ch) {
+                        float o[32];
+                        tmem_ld32(lane_base + 256 + ch * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                        tmem_st32(lane_base + 256 + ch * 32, o);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            if (grow) {
+                l = m_ref == kNegInf ? 0.f : l * fast_exp2(m_ref - m_new);
+                m_ref = m_new;
+            }
+            const float ref = m_ref == kNegInf ? 0.f : m_ref;
+            // P = 2^(x - ref) as bf16 high + low parts, row lr of the K-major swizzled operands
+#pragma unroll
+            for (int ch = 0; ch < TOK / 8; ++ch) {
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float p0 = fast_exp2(x[ch * 8 + 2 * e] - ref), p1 = fast_exp2(x[ch * 8 + 2 * e + 1] - ref);
+                    l += p0 + p1;
+                    hi[e] = pack_bf16(p0, p1);
+                    lo[e] = pack_bf16(p0 - bf16lo(hi[e]), p1 - bf16hi(hi[e]));
+                }
+                const int half = ch >> 3, cc = ch & 7;
+                const int off = half * HALF + lr * 128 + ((cc ^ (lr & 7)) << 4);
+                *reinterpret_cast<uint4*>(prow_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4*>(prow_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            fence_before();
+            mbar_arrive(&bar[B_PREADY]);
+        }
+        // the last PV, then this row's output (or the partition's partial)
+        if (ok && ntiles > 0) {
+            const bool done = mbar_wait_bounded(&bar[B_ODONE], (ntiles - 1) & 1, p.err);
+            ok = !__any_sync(0xffffffffu, !done || s_abort != 0);
+        }
+        if (ok) {
+            fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const bool live = qi < n;
+            const int64_t qh = (int64_t)(q0 + (live ? qi : 0)) * p.num_q_heads + kvh * G + hh;
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch) {
+                float o[32];
+                tmem_ld32(lane_base + 256 + ch * 32, o);
+                tmem_wait_ld();
+                if (live) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) mq_store<D>(p, qh, part, direct, ch * 32 + i, o[i] * inv);
+                }
+            }
+            if (live && !direct) {
+                p.ws_ml[(qh * p.num_parts + part) * 2 + 0] = m_ref;
+                p.ws_ml[(qh * p.num_parts + part) * 2 + 1] = l;
+            }
+        }
+    }
+    fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+    }
+}
+
+}  // namespace tc
+}  // namespace attn
+}  // namespace pkv
