@@ -11,8 +11,9 @@
 // issues every tcgen05.mma; warps 2-5 run the softmax, one query row per thread
 // (its TMEM lane), so row max and row sum need no shuffles. The S accumulator
 // is double-buffered, so S of tile t+1 is computed while the softmax of tile t
-// runs. P goes to shared memory as two bf16 parts (high, and the rounding
-// residue) that both multiply V, so the probabilities keep ~16 bits. The online
+// runs. P stays in TMEM as two bf16 parts (high, and the rounding residue) that
+// both multiply V (the A operand read from TMEM), so the probabilities keep ~16
+// bits and shared memory holds only Q and three-stage K and V rings. The online
 // softmax rescales O in TMEM only when a row's running maximum grows by more
 // than 2^8 over the reference it uses (p <= 2^8 stays exact enough in bf16 and
 // fp32), so most tiles skip the O round trip.
@@ -27,18 +28,22 @@ constexpr int TOK = 128;           // KV tokens per tile
 constexpr int D = 128;
 constexpr int THREADS = 192;
 constexpr int HALF = 128 * 128;    // one 64-element-wide half of a 128-row operand, bytes
+constexpr int NST = 3;             // K ring and V ring depth
 constexpr int Q_OFF = 0;
-constexpr int KV_OFF = 2 * HALF;                  // two stages of K (2 halves) + V (2 halves)
-constexpr int STAGE = 4 * HALF;
-constexpr int P_OFF = KV_OFF + 2 * STAGE;         // P high (2 halves), then P low (2 halves)
-constexpr int BAR_OFF = P_OFF + 4 * HALF;
-constexpr int NBAR = 13;
+constexpr int K_OFF = 2 * HALF;                   // NST stages of K (2 halves each)
+constexpr int V_OFF = K_OFF + NST * 2 * HALF;     // NST stages of V
+constexpr int BAR_OFF = V_OFF + NST * 2 * HALF;
+constexpr int NBAR = 20;
 constexpr int SMEM = 1024 + BAR_OFF + NBAR * 8 + 16;
-constexpr int TMEM_COLS = 512;                    // S0 [0,128) S1 [128,256) O [256,384)
+constexpr int TMEM_COLS = 512;     // S0 [0,128) S1 [128,256) O [256,384) P high [384,448) P low [448,512)
+constexpr int T_O = 256, T_PHI = 384, T_PLO = 448;
 static_assert(SMEM <= 232448, "shared memory per CTA");
 
 // Barrier indices.
-enum { B_Q = 0, B_FULL = 1, B_EMPTY = 3, B_SFULL = 5, B_SFREE = 7, B_PREADY = 9, B_ODONE = 10, B_DRAIN = 11 };
+enum {
+    B_Q = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_SFREE = 15, B_PREADY = 17,
+    B_ODONE = 18, B_DRAIN = 19
+};
 
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
@@ -60,6 +65,14 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, 
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
         ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+// A operand from TMEM (lane = row, two bf16 K-elements per 32-bit column).
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
 }
 
 __device__ __forceinline__ void commit(uint64_t* bar) {
@@ -100,6 +113,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
           "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
           "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
           "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+          "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+          "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
         : "memory");
 }
 
@@ -146,9 +170,13 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     if (threadIdx.x == 0) {
         mbar_init(&bar[B_Q], 1);
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(&bar[B_KFULL + s], 1);
+            mbar_init(&bar[B_KEMPTY + s], 1);
+            mbar_init(&bar[B_VFULL + s], 1);
+            mbar_init(&bar[B_VEMPTY + s], 1);
+        }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&bar[B_FULL + s], 1);
-            mbar_init(&bar[B_EMPTY + s], 1);
             mbar_init(&bar[B_SFULL + s], 1);
             mbar_init(&bar[B_SFREE + s], 128);
         }
@@ -158,7 +186,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         s_abort = 0;
         fence_barrier_init();
     }
-    if (warp == 1) {                                            // TMEM: S0, S1, O
+    if (warp == 1) {                                            // TMEM: S0, S1, O, P high, P low
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(TMEM_COLS)
                      : "memory");
@@ -175,47 +203,65 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ---------------- producer: Q once, then K/V tiles ----------------
+        // ---------------- producer: Q once, then K and V tiles into their rings ----------------
+        // The warp loads a tile's block ids with one coalesced load; lane 0 waits
+        // for the stages and issues the copies. K runs ahead of V: K of a tile is
+        // released as soon as S is computed, V only after the PV product.
+        bool ok = true;
+        int issued[2] = {0, 0};                                 // tiles whose K / V copies were issued
         if (lane == 0) {
-            bool ok = true;
-            int issued = 0;
             mbar_arrive_expect_tx(&bar[B_Q], 2 * HALF);
             for (int h = 0; h < 2; ++h)
                 tma_load_3d(smem + Q_OFF + h * HALF, &tm_q, &bar[B_Q], h * 64, kvh * G, q0 + row_begin / G);
-            const uint64_t pol = l2_policy_evict_normal();
-            const int32_t* bt = p.block_tables + (int64_t)seq * p.max_blocks + blk0;
-            for (int t = 0; t < ntiles && ok; ++t) {
-                const int s = t & 1;
-                if (!mbar_wait_bounded(&bar[B_EMPTY + s], ((t >> 1) & 1) ^ 1, p.err)) {
-                    ok = false;
-                    s_abort = 1;
-                    break;
+        }
+        const uint64_t pol = l2_policy_evict_normal();
+        const int32_t* bt = p.block_tables + (int64_t)seq * p.max_blocks + blk0;
+        static_assert(TOK / R <= 32, "one id per lane");
+        for (int t = 0; t < ntiles; ++t) {
+            const int s = t % NST;
+            const uint32_t par = ((t / NST) & 1) ^ 1;
+            const int tok_here = min(TOK, ntok - t * TOK);
+            const int np = (tok_here + R - 1) / R;
+            int id = 0;
+            if (lane < np) {
+                id = __ldg(bt + (t * TOK) / BSZ + lane);
+                if (id < 0 || id >= p.num_blocks) {
+                    flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
+                    id = p.num_blocks;                          // zero-filled tile
                 }
-                const int tok_here = min(TOK, ntok - t * TOK);
-                const int np = (tok_here + R - 1) / R;
-                mbar_arrive_expect_tx(&bar[B_FULL + s], np * 2 * 2 * R * 128);
-                ++issued;
-                uint8_t* kst = smem + KV_OFF + s * STAGE;
-                uint8_t* vst = kst + 2 * HALF;
-                for (int b = 0; b < np; ++b) {
-                    const int j = (t * TOK + b * R) / BSZ;      // block of the partition
-                    const int sub = (t * TOK + b * R) % BSZ;    // first row inside it (0 when R = BSZ)
-                    int id = __ldg(bt + j);
-                    if (id < 0 || id >= p.num_blocks) {
-                        flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
-                        id = p.num_blocks;                      // zero-filled tile
-                    }
+            }
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        tma_load_4d(kst + h * HALF + b * R * 128, &tm_k, &bar[B_FULL + s], h * 64, kvh, sub, id, pol);
-                        tma_load_4d(vst + h * HALF + b * R * 128, &tm_v, &bar[B_FULL + s], h * 64, kvh, sub, id, pol);
+            for (int kv = 0; kv < 2; ++kv) {
+                uint64_t* full = &bar[(kv ? B_VFULL : B_KFULL) + s];
+                if (lane == 0) {
+                    ok = mbar_wait_bounded(&bar[(kv ? B_VEMPTY : B_KEMPTY) + s], par, p.err);
+                    if (ok) {
+                        mbar_arrive_expect_tx(full, np * 2 * R * 128);
+                        ++issued[kv];
+                    } else {
+                        s_abort = 1;
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) break;
+                uint8_t* dst = smem + (kv ? V_OFF : K_OFF) + s * 2 * HALF;
+                const CUtensorMap* map = kv ? &tm_v : &tm_k;
+                for (int b = 0; b < np; ++b) {
+                    const int pb = __shfl_sync(0xffffffffu, id, b);
+                    if (lane == 0) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            tma_load_4d(dst + h * HALF + b * R * 128, map, full, h * 64, kvh, 0, pb, pol);
                     }
                 }
             }
-            if (!ok) {
-                for (int t = max(0, issued - 2); t < issued; ++t)
-                    mbar_wait_bounded(&bar[B_FULL + (t & 1)], (t >> 1) & 1, p.err);
-            }
+            if (!ok) break;
+        }
+        if (lane == 0 && !ok) {
+            // every copy issued has landed before the CTA moves on
+            for (int kv = 0; kv < 2; ++kv)
+                for (int t = max(0, issued[kv] - NST); t < issued[kv]; ++t)
+                    mbar_wait_bounded(&bar[(kv ? B_VFULL : B_KFULL) + t % NST], (t / NST) & 1, p.err);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer (one thread) ----------------
@@ -223,45 +269,42 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             constexpr uint32_t IDESC_S = idesc_bf16(ROWS, TOK, false);
             constexpr uint32_t IDESC_PV = idesc_bf16(ROWS, D, true);
             const uint32_t q_addr = smem_u32(smem + Q_OFF);
-            const uint32_t p_addr = smem_u32(smem + P_OFF);
             bool ok = mbar_wait_bounded(&bar[B_Q], 0, p.err);
-            int issued_pv = 0;
             // PV of tile u: O += P_hi V + P_lo V over the tile's 128 tokens, 8 k-steps of 16
             auto pv = [&](int u) -> bool {
                 if (!mbar_wait_bounded(&bar[B_PREADY], u & 1, p.err)) return false;
+                if (!mbar_wait_bounded(&bar[B_VFULL + u % NST], (u / NST) & 1, p.err)) return false;
                 fence_after();
-                const uint32_t v_addr = smem_u32(smem + KV_OFF + (u & 1) * STAGE + 2 * HALF);
+                const uint32_t v_addr = smem_u32(smem + V_OFF + (u % NST) * 2 * HALF);
 #pragma unroll
                 for (int part_lo = 0; part_lo < 2; ++part_lo) {
 #pragma unroll
                     for (int k = 0; k < TOK / 16; ++k) {
-                        // A = P: K-major rows, tokens 16k..16k+15 -> half k/4, 32 bytes per k-step inside it
-                        const uint64_t a = desc_sw128(p_addr + part_lo * 2 * HALF + (k >> 2) * HALF + (k & 3) * 32,
-                                                      16, 1024);
-                        // B = V: MN-major (dims contiguous), tokens 16k.. -> 16 rows of 128 B; dims halves LBO apart
+                        // B = V: MN-major (dims contiguous); tokens 16k.. -> 16 rows of 128 B; dim halves HALF apart
                         const uint64_t b = desc_sw128(v_addr + k * 16 * 128, HALF, 1024);
-                        mma_ss(tmem + 256, a, b, IDESC_PV, (u > 0 || part_lo > 0 || k > 0) ? 1u : 0u);
+                        mma_ts(tmem + T_O, tmem + (part_lo ? T_PLO : T_PHI) + k * 8, b, IDESC_PV,
+                               (u > 0 || part_lo > 0 || k > 0) ? 1u : 0u);
                     }
                 }
                 commit(&bar[B_ODONE]);
-                commit(&bar[B_EMPTY + (u & 1)]);
-                ++issued_pv;
+                commit(&bar[B_VEMPTY + u % NST]);
                 return true;
             };
             for (int t = 0; t < ntiles && ok; ++t) {
-                const int s = t & 1;
-                ok = mbar_wait_bounded(&bar[B_FULL + s], (t >> 1) & 1, p.err);
-                if (ok && t >= 2) ok = mbar_wait_bounded(&bar[B_SFREE + s], ((t - 2) >> 1) & 1, p.err);
+                const int sb = t & 1, ks = t % NST;
+                ok = mbar_wait_bounded(&bar[B_KFULL + ks], (t / NST) & 1, p.err);
+                if (ok && t >= 2) ok = mbar_wait_bounded(&bar[B_SFREE + sb], ((t - 2) >> 1) & 1, p.err);
                 if (!ok) break;
                 fence_after();
-                const uint32_t k_addr = smem_u32(smem + KV_OFF + s * STAGE);
+                const uint32_t k_addr = smem_u32(smem + K_OFF + ks * 2 * HALF);
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint64_t a = desc_sw128(q_addr + (k >> 2) * HALF + (k & 3) * 32, 16, 1024);
                     const uint64_t b = desc_sw128(k_addr + (k >> 2) * HALF + (k & 3) * 32, 16, 1024);
-                    mma_ss(tmem + s * 128, a, b, IDESC_S, k > 0 ? 1u : 0u);
+                    mma_ss(tmem + sb * 128, a, b, IDESC_S, k > 0 ? 1u : 0u);
                 }
-                commit(&bar[B_SFULL + s]);
+                commit(&bar[B_SFULL + sb]);
+                commit(&bar[B_KEMPTY + ks]);
                 if (t >= 1) ok = pv(t - 1);
             }
             if (ok && ntiles > 0) ok = pv(ntiles - 1);
@@ -269,7 +312,6 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // every MMA issued has finished before TMEM is released
             commit(&bar[B_DRAIN]);
             mbar_wait_bounded(&bar[B_DRAIN], 0, p.err);
-            (void)issued_pv;
         }
     } else {
         // ---------------- softmax: one query row per thread ----------------
@@ -279,8 +321,6 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const int qi = r / G, hh = r - qi * G;
         const int pos = qi < n ? c - n + qi : -1;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-        uint8_t* prow_hi = smem + P_OFF;
-        uint8_t* prow_lo = smem + P_OFF + 2 * HALF;
         float m_ref = kNegInf, l = 0.f;
         bool ok = true;
         for (int t = 0; t < ntiles; ++t) {
@@ -298,29 +338,41 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             tmem_wait_ld();
             fence_before();
             mbar_arrive(&bar[B_SFREE + s]);
+            // masks: past the partition's range, or after the row's position (causal)
+            const int tok0 = kv0 + t * TOK;
+            const int lim = min(pos, kv0 + ntok - 1) - tok0;    // columns 0..lim are visible
+            float mt = kNegInf;
+            if (lim >= TOK - 1) {                               // the whole tile is visible to this row
+#pragma unroll
+                for (int j = 0; j < TOK; ++j) {
+                    x[j] *= p.scale_log2;
+                    mt = fmaxf(mt, x[j]);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < TOK; ++j) {
+                    x[j] = j <= lim ? x[j] * p.scale_log2 : kNegInf;
+                    mt = fmaxf(mt, x[j]);
+                }
+            }
+            const float m_new = fmaxf(m_ref, mt);
+            const bool grow = m_new > m_ref + 8.f;              // also true when m_ref is -inf and the row sees a token
             // V rows past the range (the unwritten tail of the last block, or a stage
             // row no piece filled) may hold anything, NaN included: P is 0 there, but
             // 0 * NaN would not be, so those rows are zeroed before the PV product.
             const int tok_here = min(TOK, ntok - t * TOK);
             if (lr >= tok_here) {
-                uint8_t* vrow = smem + KV_OFF + s * STAGE + 2 * HALF + lr * 128;
+                const bool vin = mbar_wait_bounded(&bar[B_VFULL + t % NST], (t / NST) & 1, p.err);
+                if (vin) {
+                    uint8_t* vrow = smem + V_OFF + (t % NST) * 2 * HALF + lr * 128;
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
+                    for (int h = 0; h < 2; ++h)
 #pragma unroll
-                    for (int cc = 0; cc < 8; ++cc)
-                        *reinterpret_cast<uint4*>(vrow + h * HALF + (cc << 4)) = make_uint4(0u, 0u, 0u, 0u);
+                        for (int cc = 0; cc < 8; ++cc)
+                            *reinterpret_cast<uint4*>(vrow + h * HALF + (cc << 4)) = make_uint4(0u, 0u, 0u, 0u);
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                }
             }
-            // masks: past the partition's range, or after the row's position (causal)
-            const int tok0 = kv0 + t * TOK;
-            const int lim = min(pos, kv0 + ntok - 1) - tok0;    // columns 0..lim are visible
-            float mt = kNegInf;
-#pragma unroll
-            for (int j = 0; j < TOK; ++j) {
-                x[j] = j <= lim ? x[j] * p.scale_log2 : kNegInf;
-                mt = fmaxf(mt, x[j]);
-            }
-            const float m_new = fmaxf(m_ref, mt);
-            const bool grow = m_new > m_ref + 8.f;              // also true when m_ref is -inf and the row sees a token
             if (t > 0) {
                 const bool done = mbar_wait_bounded(&bar[B_ODONE], (t - 1) & 1, p.err);
                 if (__any_sync(0xffffffffu, !done || s_abort != 0)) {
@@ -334,13 +386,12 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
                     for (int ch = 0; ch < D / 32; ++ch) {
                         float o[32];
-                        tmem_ld32(lane_base + 256 + ch * 32, o);
+                        tmem_ld32(lane_base + T_O + ch * 32, o);
                         tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 32; ++i) o[i] *= alpha;
-                        tmem_st32(lane_base + 256 + ch * 32, o);
+                        tmem_st32(lane_base + T_O + ch * 32, o);
                     }
-                    tmem_wait_st();
                 }
             }
             if (grow) {
@@ -348,23 +399,21 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 m_ref = m_new;
             }
             const float ref = m_ref == kNegInf ? 0.f : m_ref;
-            // P = 2^(x - ref) as bf16 high + low parts, row lr of the K-major swizzled operands
+            // P = 2^(x - ref) as bf16 high + low parts into TMEM (64 columns each)
 #pragma unroll
-            for (int ch = 0; ch < TOK / 8; ++ch) {
-                uint32_t hi[4], lo[4];
+            for (int ch = 0; ch < TOK / 64; ++ch) {
+                uint32_t hi[32], lo[32];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float p0 = fast_exp2(x[ch * 8 + 2 * e] - ref), p1 = fast_exp2(x[ch * 8 + 2 * e + 1] - ref);
+                for (int e = 0; e < 32; ++e) {
+                    const float p0 = fast_exp2(x[ch * 64 + 2 * e] - ref), p1 = fast_exp2(x[ch * 64 + 2 * e + 1] - ref);
                     l += p0 + p1;
                     hi[e] = pack_bf16(p0, p1);
                     lo[e] = pack_bf16(p0 - bf16lo(hi[e]), p1 - bf16hi(hi[e]));
                 }
-                const int half = ch >> 3, cc = ch & 7;
-                const int off = half * HALF + lr * 128 + ((cc ^ (lr & 7)) << 4);
-                *reinterpret_cast<uint4*>(prow_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4*>(prow_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                tmem_st32u(lane_base + T_PHI + ch * 32, hi);
+                tmem_st32u(lane_base + T_PLO + ch * 32, lo);
             }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tmem_wait_st();
             fence_before();
             mbar_arrive(&bar[B_PREADY]);
         }
@@ -381,7 +430,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
                 float o[32];
-                tmem_ld32(lane_base + 256 + ch * 32, o);
+                tmem_ld32(lane_base + T_O + ch * 32, o);
                 tmem_wait_ld();
                 if (live) {
 #pragma unroll
