@@ -373,6 +373,19 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 }
             }
+            // P = 2^(x - ref) as bf16 high + low parts, computed while the previous
+            // PV product still runs (only writing P into TMEM has to wait for it)
+            const float ref_new = grow ? m_new : m_ref;
+            const float ref = ref_new == kNegInf ? 0.f : ref_new;
+            uint32_t ph[TOK / 2], pl[TOK / 2];
+            float psum = 0.f;
+#pragma unroll
+            for (int e = 0; e < TOK / 2; ++e) {
+                const float p0 = fast_exp2(x[2 * e] - ref), p1 = fast_exp2(x[2 * e + 1] - ref);
+                psum += p0 + p1;
+                ph[e] = pack_bf16(p0, p1);
+                pl[e] = pack_bf16(p0 - bf16lo(ph[e]), p1 - bf16hi(ph[e]));
+            }
             if (t > 0) {
                 const bool done = mbar_wait_bounded(&bar[B_ODONE], (t - 1) & 1, p.err);
                 if (__any_sync(0xffffffffu, !done || s_abort != 0)) {
@@ -398,20 +411,11 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 l = m_ref == kNegInf ? 0.f : l * fast_exp2(m_ref - m_new);
                 m_ref = m_new;
             }
-            const float ref = m_ref == kNegInf ? 0.f : m_ref;
-            // P = 2^(x - ref) as bf16 high + low parts into TMEM (64 columns each)
+            l += psum;
 #pragma unroll
             for (int ch = 0; ch < TOK / 64; ++ch) {
-                uint32_t hi[32], lo[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float p0 = fast_exp2(x[ch * 64 + 2 * e] - ref), p1 = fast_exp2(x[ch * 64 + 2 * e + 1] - ref);
-                    l += p0 + p1;
-                    hi[e] = pack_bf16(p0, p1);
-                    lo[e] = pack_bf16(p0 - bf16lo(hi[e]), p1 - bf16hi(hi[e]));
-                }
-                tmem_st32u(lane_base + T_PHI + ch * 32, hi);
-                tmem_st32u(lane_base + T_PLO + ch * 32, lo);
+                tmem_st32u(lane_base + T_PHI + ch * 32, ph + ch * 32);
+                tmem_st32u(lane_base + T_PLO + ch * 32, pl + ch * 32);
             }
             tmem_wait_st();
             fence_before();
