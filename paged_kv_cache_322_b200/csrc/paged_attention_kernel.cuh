@@ -126,36 +126,34 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 }
             }
             const int qn = min(32 * K::PPB, npiece - q0);
-            for (int qq = 0; qq < qn; ++qq) {
-                const int pb = __shfl_sync(0xffffffffu, id, qq / K::PPB);
-                if (lane == 0 && ok) {
-                    const int q = q0 + qq, sub = qq % K::PPB;     // piece q is rows [sub*R, sub*R + R) of its block
-                    const int si = q / K::BPS, b = q - si * K::BPS, st = si % STAGES;
-                    if (b == 0) {                                 // first piece of a stage: claim it
-                        if (!mbar_wait_bounded(&empty[st], ((si / STAGES) & 1) ^ 1, p.err)) {
-                            ok = false;
-                            s_abort = 1;
-                        } else {
-                            mbar_arrive_expect_tx(&full[st], min(K::BPS, npiece - q) * 2 * KPC * K::PIECE);
-                            ++issued;
-                        }
-                    }
-                    if (ok) {
-#pragma unroll
-                        for (int hd = 0; hd < KPC; ++hd) {
-                            uint8_t* dst = smem + st * K::STAGE_BYTES + hd * K::REGION;
-                            uint8_t* vdst = dst + KPC * K::REGION;
-#pragma unroll
-                            for (int h = 0; h < (K::kMma ? K::NBOX : 1); ++h) {
-                                const int off = K::piece_offset(b, h);
-                                tma_load_4d(dst + off, &tm_k, &full[st], h * K::BOX, kvh + hd, sub * K::R, pb, pol);
-                                tma_load_4d(vdst + off, &tm_v, &full[st], h * K::BOX, kvh + hd, sub * K::R, pb, pol);
-                            }
-                        }
+            // One stage per iteration (BPS pieces; BPS divides 32 * PPB, so a stage
+            // never straddles two id loads). Lane 0 claims the stage; then lane o
+            // issues copy o of the stage's BPS x KPC x boxes x {K, V} copies, in
+            // parallel instead of one thread issuing them all.
+            constexpr int NB = K::kMma ? K::NBOX : 1;
+            static_assert(K::BPS * KPC * NB * 2 <= 32, "one copy per lane");
+            const int kv = lane & 1, hb = lane >> 1;
+            const int h = hb % NB, hd = (hb / NB) % KPC, b = hb / (NB * KPC);
+            for (int qs = 0; qs < qn; qs += K::BPS) {
+                const int q = q0 + qs, si = q / K::BPS, st = si % STAGES;
+                const int nq = min(K::BPS, npiece - q);               // pieces in this stage
+                if (lane == 0) {
+                    if (!mbar_wait_bounded(&empty[st], ((si / STAGES) & 1) ^ 1, p.err)) {
+                        ok = false;
+                        s_abort = 1;
+                    } else {
+                        mbar_arrive_expect_tx(&full[st], nq * 2 * KPC * K::PIECE);
+                        ++issued;
                     }
                 }
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;    // also orders the expect-tx first
                 if (!ok) break;
+                const int pq = qs + (b < nq ? b : 0);                // this lane's piece, chunk-relative
+                const int pb = __shfl_sync(0xffffffffu, id, pq / K::PPB);
+                if (b < nq) {
+                    uint8_t* dst = smem + st * K::STAGE_BYTES + (kv ? KPC + hd : hd) * K::REGION + K::piece_offset(b, h);
+                    tma_load_4d(dst, kv ? &tm_v : &tm_k, &full[st], h * K::BOX, kvh + hd, (pq % K::PPB) * K::R, pb, pol);
+                }
             }
         }
         if (lane == 0 && !ok) {
