@@ -608,8 +608,12 @@ bool plan_mq(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int 
     // few rows (speculative verify, decode): fewer row groups, the KV range split among their warps
     const int64_t rows = (int64_t)max_query_len * group;
     pl->wpr = rows <= MQ_ROWS_PER_WARP ? 4 : (rows <= 2 * MQ_ROWS_PER_WARP ? 2 : 1);
-    // prefill-sized query tiles go to the tcgen05 kernel (head_dim 128)
-    pl->tc = head_dim == 128 && rows >= tc::ROWS;
+    // From 32 query rows per KV head on (prefill chunks, and speculative verify
+    // on grouped-query heads) the tcgen05 kernel wins even with most of its 128
+    // rows idle (measured, 70B-shaped verify of 5 tokens = 40 rows: 1.7x the
+    // mma.sync kernel); below that, the mma.sync kernel splits the KV range over
+    // its warps (head_dim 128 only on tcgen05).
+    pl->tc = head_dim == 128 && rows >= 32;
     const int tile_rows = pl->tc ? tc::ROWS : mq_rows_per_tile(pl->wpr);
     pl->row_tiles = (int)((rows + tile_rows - 1) / tile_rows);
     int pt = partition_tokens;

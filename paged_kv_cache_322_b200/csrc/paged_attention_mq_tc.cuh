@@ -1,7 +1,7 @@
 // Multi-query paged attention on the 5th-generation tensor cores (tcgen05) for
 // prefill-sized query tiles: bf16 caches, head_dim 128, 128 query rows per CTA.
-// Included by paged_attention_mq.cu, which routes a call here when every
-// sequence brings at least one full 128-row tile's worth of query rows.
+// Included by paged_attention_mq.cu, which routes a call here from 32 query rows
+// (query tokens x group) per KV head on; shorter tiles are padded with idle rows.
 //
 //   S  = Q K^T   M = 128 query rows, N = 128 KV tokens, K = 128 dims  (TMEM, fp32)
 //   O += P V     M = 128 rows, N = 128 dims, K = 128 tokens            (TMEM, fp32)

@@ -200,3 +200,16 @@ def test_full_size_chunk_sampled():
                                                 [op.bm.lens[s]], np.array([0, n]), w.scale, w.block_size)
         rows = rng.choice(n, 24, replace=False)
         assert np.abs(got[s * n + rows] - ref[rows]).max() <= 2e-3
+
+
+@pytest.mark.parametrize("part", [0, 512])
+@pytest.mark.parametrize("bs", [16, 64])
+def test_gqa_verify_rows_padded_into_tensor_memory_tiles(part, bs):
+    """Group 8, five draft tokens: 40 query rows per KV head, run on 128-row
+    tcgen05 tiles whose other 88 rows are idle."""
+    ctxs, ns = [17, 1000, 2049, 4000], [5, 5, 5, 5]
+    dev, ref = _mq_problem(8 + bs, 64, 8, 128, bs, ctxs, ns)
+    out = _run(dev, part=part)
+    torch.cuda.synchronize()
+    assert binding.get_device_error() == 0
+    assert np.abs(out.cpu().numpy().astype(np.float64) - ref).max() <= 2e-3
