@@ -300,15 +300,13 @@ cudaError_t dispatch_partitioned(pkv_dtype kv_dtype, bool use_mma, int head_dim,
                                  const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, dim3 grid,
                                  cudaStream_t st) {
     if (kv_dtype == PKV_FP8_E4M3) {
-        // Two KV heads per CTA where the SIMT path splits by block (groups 1, 2)
-        // or on tensor cores: each token's 256 contiguous bytes of K (and of V)
-        // are fetched in one go instead of two 128-byte halves by different CTAs.
-        const bool pair = num_kv_heads % 2 == 0 && (use_mma || group <= 2);
-        if (use_mma)
-            return pair ? launch_decode<uint8_t, 128, 2, 8, stages_for<uint8_t, 128, 2>(), 2, BSZ>(mk, mv, p, grid, st)
-                        : launch_decode<uint8_t, 128, 2, 8, stages_for<uint8_t, 128>(), 1, BSZ>(mk, mv, p, grid, st);
-        return pair ? dispatch_simt<uint8_t, 128, BSZ, 2>(group, mk, mv, p, grid, st)
-                    : dispatch_simt<uint8_t, 128, BSZ>(group, mk, mv, p, grid, st);
+        // e4m3 always runs on tensor cores (use_mma). Two KV heads per CTA: each
+        // token's 256 contiguous bytes of K (and of V) are fetched in one go
+        // instead of two 128-byte halves by different CTAs.
+        (void)use_mma;
+        return num_kv_heads % 2 == 0
+                   ? launch_decode<uint8_t, 128, 2, 8, stages_for<uint8_t, 128, 2>(), 2, BSZ>(mk, mv, p, grid, st)
+                   : launch_decode<uint8_t, 128, 2, 8, stages_for<uint8_t, 128>(), 1, BSZ>(mk, mv, p, grid, st);
     }
     // bf16 on tensor cores: 8-token blocks make 1 KB copies per head, so two KV
     // heads per CTA (measured on B200, 70B-shaped GQA: +16% at block size 8,
