@@ -275,6 +275,21 @@ def attention_bytes(w: wl.Workload, lens_after: np.ndarray, out_elt: int) -> int
     return kv + q + out + tables + 4 * w.num_seqs
 
 
+def mq_flops(lens_after, n: int, hq: int, d: int) -> int:
+    """Causal multi-query attention flops: every sequence's n queries (positions
+    c - n .. c - 1) against their visible tokens, 2 flops per multiply-add in
+    Q K^T and in P V: 4 * Hq * D per (query, visible token)."""
+    return sum(4 * hq * d * (n * (int(c) - n) + n * (n + 1) // 2) for c in lens_after)
+
+
+def mq_attention_bytes(lens_after, n: int, hq: int, hkv: int, d: int, bs: int) -> int:
+    """Algorithmic bytes of one multi-query attention launch (bf16): K and V of
+    every cached token once, q in, out, the block tables."""
+    T = n * len(lens_after)
+    return (int(np.sum(lens_after)) * hkv * d * 2 * 2 + T * hq * d * 2 * 2 +
+            int(sum(-(-int(c) // bs) for c in lens_after)) * 4)
+
+
 def append_bytes(w: wl.Workload) -> int:
     n = w.num_kv_heads * w.head_dim
     return w.num_seqs * (2 * n * (w.in_bytes + w.elt_bytes) + 8)   # K and V rows read and written, slot ids
@@ -609,11 +624,7 @@ def run_mq(args, ws, rank, local):
         return torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
 
     def flops_and_bytes(lens_after):
-        fl = sum(4 * hq * d * (n * (int(c) - n) + n * (n + 1) // 2) for c in lens_after)
-        # the attention launch: K and V of every cached token once, q in, out, block tables
-        by = (int(lens_after.sum()) * hkv * d * 2 * 2 + T * hq * d * 2 * 2 +
-              int(sum(-(-int(c) // bs) for c in lens_after)) * 4)
-        return fl, by
+        return mq_flops(lens_after, n, hq, d), mq_attention_bytes(lens_after, n, hq, hkv, d, bs)
 
     steps = []
     order = np.repeat(ids, n)

@@ -1,0 +1,48 @@
+"""The bench's byte and flop accounting against brute-force counts on small
+cases (CPU only): the reported GB/s and TFLOP/s rest on these."""
+import argparse
+
+import numpy as np
+import pytest
+
+import bench
+from paged_kv_cache_322_b200 import workloads as wl
+
+
+@pytest.mark.parametrize("n,lens", [(1, [1, 5, 40]), (5, [5, 9, 100]), (16, [16, 17, 300]), (3, [3])])
+def test_mq_flops_counts_every_visible_pair(n, lens):
+    hq, d = 3, 4
+    pairs = 0
+    for c in lens:
+        for i in range(n):
+            pairs += (c - n + i) + 1                 # tokens 0 .. position c - n + i
+    assert bench.mq_flops(np.array(lens), n, hq, d) == 4 * hq * d * pairs
+
+
+def test_mq_bytes_and_decode_bytes_agree_for_one_query():
+    w = wl.WORKLOADS["llama2_7b"]
+    lens = np.array([17, 512, 2049])
+    w3 = bench.dataclasses.replace(w, num_seqs=3)
+    # decode counts a 4-byte length per sequence that the multi-query launch does not
+    assert bench.mq_attention_bytes(lens, 1, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size) == \
+        bench.attention_bytes(w3, lens, 2) - 4 * 3
+
+
+def test_attention_bytes_brute_force():
+    w = bench.dataclasses.replace(wl.WORKLOADS["gqa_70b_fp8"], num_seqs=2)
+    lens = np.array([1, 33])
+    kv = sum(lens) * w.num_kv_heads * w.head_dim * 1 * 2                 # e4m3: one byte per element
+    q = 2 * w.num_q_heads * w.head_dim * 2                                # bf16 queries
+    out = 2 * w.num_q_heads * w.head_dim * 2                              # bf16 output
+    tables = (1 + 3) * 4
+    assert bench.attention_bytes(w, lens, 2) == kv + q + out + tables + 4 * 2
+
+
+def test_block_size_override_keeps_pool_tokens():
+    w = wl.WORKLOADS["llama2_7b"]
+    args = argparse.Namespace(block_size=64, num_seqs=0, num_blocks=0)
+    w2 = bench.override_workload(w, args)
+    assert w2.block_size == 64 and w2.num_blocks * 64 == w.num_blocks * w.block_size
+    args = argparse.Namespace(block_size=0, num_seqs=8, num_blocks=100)
+    w3 = bench.override_workload(w, args)
+    assert (w3.num_seqs, w3.num_blocks, w3.block_size) == (8, 100, 16)
