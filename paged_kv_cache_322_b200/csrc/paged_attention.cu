@@ -44,26 +44,75 @@ namespace pkv {
 namespace attn {
 
 // Log-sum-exp merge of partition results. grid = (Hq, B), block = D threads.
+// The (m, l) pairs are staged in shared memory once (coalesced), the weights
+// w_c = l_c 2^(m_c - M) computed once per row, then each thread sums its
+// dimension over the partitions with independent loads in flight (the first
+// version walked the partitions with one dependent load chain per thread).
+constexpr int kMergeSmemParts = 2048;
 template <int D>
 __global__ void __launch_bounds__(D) merge_partitions_kernel(const Params p) {
+    __shared__ float sw[kMergeSmemParts];
+    __shared__ float s_red[D / 32];
     const int qhead = blockIdx.x, seq = blockIdx.y, d = threadIdx.x;
+    const int lane = d & 31, wid = d >> 5;
     int ctx = p.context_lens[seq];
     ctx = ctx < 0 ? 0 : (ctx > p.ctx_cap ? p.ctx_cap : ctx);
     const int nparts = ((ctx + p.block_size - 1) / p.block_size + p.part_blocks - 1) / p.part_blocks;
     if (nparts <= 1) return;
     const int64_t qh = (int64_t)seq * p.num_q_heads + qhead;
     const float* ml = p.ws_ml + qh * p.num_parts * 2;
-    const float* o = p.ws_o + qh * p.num_parts * D;
-    float M = kNegInf;
-    for (int c = 0; c < nparts; ++c) M = fmaxf(M, ml[2 * c]);
+    const float* o = p.ws_o + qh * p.num_parts * D + d;
     float L = 0.f, O = 0.f;
-    if (M != kNegInf) {
-        for (int c = 0; c < nparts; ++c) {
+    if (nparts <= kMergeSmemParts) {
+        // M = max m_c
+        float mx = kNegInf;
+        for (int c = d; c < nparts; c += D) {
             const float mc = ml[2 * c];
-            if (mc == kNegInf) continue;
-            const float w = ml[2 * c + 1] * fast_exp2(mc - M);
-            L += w;
-            O += w * o[(int64_t)c * D + d];
+            sw[c] = mc;
+            mx = fmaxf(mx, mc);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        if (lane == 0) s_red[wid] = mx;
+        __syncthreads();
+        float M = s_red[0];
+#pragma unroll
+        for (int w = 1; w < D / 32; ++w) M = fmaxf(M, s_red[w]);
+        __syncthreads();
+        if (M != kNegInf) {
+            float ls = 0.f;
+            for (int c = d; c < nparts; c += D) {
+                const float mc = sw[c];
+                const float w = mc == kNegInf ? 0.f : ml[2 * c + 1] * fast_exp2(mc - M);
+                sw[c] = w;
+                ls += w;
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
+            if (lane == 0) s_red[wid] = ls;
+            __syncthreads();
+#pragma unroll
+            for (int w = 0; w < D / 32; ++w) L += s_red[w];
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            int c = 0;
+            for (; c + 4 <= nparts; c += 4) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) acc[u] += sw[c + u] * o[(int64_t)(c + u) * D];
+            }
+            for (; c < nparts; ++c) acc[0] += sw[c] * o[(int64_t)c * D];
+            O = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        }
+    } else {
+        float M = kNegInf;
+        for (int c = 0; c < nparts; ++c) M = fmaxf(M, ml[2 * c]);
+        if (M != kNegInf) {
+            for (int c = 0; c < nparts; ++c) {
+                const float mc = ml[2 * c];
+                if (mc == kNegInf) continue;
+                const float w = ml[2 * c + 1] * fast_exp2(mc - M);
+                L += w;
+                O += w * o[(int64_t)c * D];
+            }
         }
     }
     store_out(p, qh * D + d, L > 0.f ? O / L : 0.f);
