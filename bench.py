@@ -249,17 +249,14 @@ def traffic_record(workload: str):
 
 
 def kernel_source_sha1() -> str:
-    """Hash of the partitioned attention kernel's device code (the shared device
-    headers, the kernel template and paged_attention.cu up to its host-side
-    section)."""
+    """Hash of the decode attention kernel's device code: the shared device
+    headers and the kernel template (the traffic records are ncu captures of
+    paged_decode_kernel alone)."""
     csrc = os.path.join(ROOT, "paged_kv_cache_322_b200", "csrc")
     h = hashlib.sha1()
     for name in ("common.cuh", "attention_common.cuh", "paged_attention_kernel.cuh"):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
-    with open(os.path.join(csrc, "paged_attention.cu"), "rb") as f:
-        src = f.read()
-    h.update(src.split(b"// Host side")[0])
     return h.hexdigest()
 
 
