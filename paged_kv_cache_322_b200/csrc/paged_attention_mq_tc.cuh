@@ -11,9 +11,10 @@
 // issues every tcgen05.mma; warps 2-5 run the softmax, one query row per thread
 // (its TMEM lane), so row max and row sum need no shuffles. The S accumulator
 // is double-buffered, so S of tile t+1 is computed while the softmax of tile t
-// runs. P stays in TMEM as two bf16 parts (high, and the rounding residue) that
-// both multiply V (the A operand read from TMEM), so the probabilities keep ~16
-// bits and shared memory holds only Q and three-stage K and V rings. The online
+// runs. P stays in TMEM, written over its own S buffer, as two bf16 parts (high,
+// and the rounding residue) that both multiply V (the A operand read from TMEM),
+// so the probabilities keep ~16 bits, P is double-buffered with S, and shared
+// memory holds only Q and three-stage K and V rings. The online
 // softmax rescales O in TMEM only when a row's running maximum grows by more
 // than 2^8 over the reference it uses (p <= 2^8 stays exact enough in bf16 and
 // fp32), so most tiles skip the O round trip.
@@ -35,14 +36,17 @@ constexpr int V_OFF = K_OFF + NST * 2 * HALF;     // NST stages of V
 constexpr int BAR_OFF = V_OFF + NST * 2 * HALF;
 constexpr int NBAR = 20;
 constexpr int SMEM = 1024 + BAR_OFF + NBAR * 8 + 16;
-constexpr int TMEM_COLS = 512;     // S0 [0,128) S1 [128,256) O [256,384) P high [384,448) P low [448,512)
-constexpr int T_O = 256, T_PHI = 384, T_PLO = 448;
+constexpr int TMEM_COLS = 512;     // S/P 0 [0,128) S/P 1 [128,256) O [256,384)
+constexpr int T_O = 256;
+// P of tile t is written over S of tile t (high part in the buffer's first 64
+// columns, low part in the next 64): the buffer is free once S is read, and
+// S of tile t + 2 is issued after the PV product that reads P of tile t.
 static_assert(SMEM <= 232448, "shared memory per CTA");
 
 // Barrier indices.
 enum {
-    B_Q = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_SFREE = 15, B_PREADY = 17,
-    B_ODONE = 18, B_DRAIN = 19
+    B_Q = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_PREADY = 17, B_ODONE = 18,
+    B_DRAIN = 19
 };
 
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -176,10 +180,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_init(&bar[B_VFULL + s], 1);
             mbar_init(&bar[B_VEMPTY + s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&bar[B_SFULL + s], 1);
-            mbar_init(&bar[B_SFREE + s], 128);
-        }
+        for (int s = 0; s < 2; ++s) mbar_init(&bar[B_SFULL + s], 1);
         mbar_init(&bar[B_PREADY], 128);
         mbar_init(&bar[B_ODONE], 1);
         mbar_init(&bar[B_DRAIN], 1);
@@ -281,7 +282,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     for (int k = 0; k < TOK / 16; ++k) {
                         // B = V: MN-major (dims contiguous); tokens 16k.. -> 16 rows of 128 B; dim halves HALF apart
                         const uint64_t b = desc_sw128(v_addr + k * 16 * 128, HALF, 1024);
-                        mma_ts(tmem + T_O, tmem + (part_lo ? T_PLO : T_PHI) + k * 8, b, IDESC_PV,
+                        mma_ts(tmem + T_O, tmem + (u & 1) * 128 + part_lo * 64 + k * 8, b, IDESC_PV,
                                (u > 0 || part_lo > 0 || k > 0) ? 1u : 0u);
                     }
                 }
@@ -291,8 +292,9 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             };
             for (int t = 0; t < ntiles && ok; ++t) {
                 const int sb = t & 1, ks = t % NST;
+                // S of tile t goes into the buffer of tile t - 2, whose P the PV product
+                // issued in the previous iteration reads first (MMAs run in issue order)
                 ok = mbar_wait_bounded(&bar[B_KFULL + ks], (t / NST) & 1, p.err);
-                if (ok && t >= 2) ok = mbar_wait_bounded(&bar[B_SFREE + sb], ((t - 2) >> 1) & 1, p.err);
                 if (!ok) break;
                 fence_after();
                 const uint32_t k_addr = smem_u32(smem + K_OFF + ks * 2 * HALF);
@@ -335,8 +337,6 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
             for (int ch = 0; ch < TOK / 32; ++ch) tmem_ld32(lane_base + s * 128 + ch * 32, x + ch * 32);
             tmem_wait_ld();
-            fence_before();
-            mbar_arrive(&bar[B_SFREE + s]);
             // masks: past the partition's range, or after the row's position (causal)
             const int tok0 = kv0 + t * TOK;
             const int lim = min(pos, kv0 + ntok - 1) - tok0;    // columns 0..lim are visible
@@ -385,7 +385,12 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 ph[e] = pack_bf16(p0, p1);
                 pl[e] = pack_bf16(p0 - bf16lo(ph[e]), p1 - bf16hi(ph[e]));
             }
-            if (t > 0) {
+            // O must be rescaled only when a row's maximum grew past its reference;
+            // then the PV product of tile t - 1 has to be complete first. S of this
+            // tile being complete already implies PV of tile t - 2 is (one commit
+            // covers every earlier MMA), so O-done is at most one phase behind and
+            // its parity wait is exact.
+            if (t > 0 && __any_sync(0xffffffffu, grow && m_ref != kNegInf)) {
                 const bool done = mbar_wait_bounded(&bar[B_ODONE], (t - 1) & 1, p.err);
                 if (__any_sync(0xffffffffu, !done || s_abort != 0)) {
                     ok = false;
@@ -393,17 +398,15 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     break;
                 }
                 fence_after();
-                if (__any_sync(0xffffffffu, grow && m_ref != kNegInf)) {
-                    const float alpha = (grow && m_ref != kNegInf) ? fast_exp2(m_ref - m_new) : 1.f;
+                const float alpha = (grow && m_ref != kNegInf) ? fast_exp2(m_ref - m_new) : 1.f;
 #pragma unroll
-                    for (int ch = 0; ch < D / 32; ++ch) {
-                        float o[32];
-                        tmem_ld32(lane_base + T_O + ch * 32, o);
-                        tmem_wait_ld();
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    float o[32];
+                    tmem_ld32(lane_base + T_O + ch * 32, o);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] *= alpha;
-                        tmem_st32(lane_base + T_O + ch * 32, o);
-                    }
+                    for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                    tmem_st32(lane_base + T_O + ch * 32, o);
                 }
             }
             if (grow) {
@@ -413,8 +416,8 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             l += psum;
 #pragma unroll
             for (int ch = 0; ch < TOK / 64; ++ch) {
-                tmem_st32u(lane_base + T_PHI + ch * 32, ph + ch * 32);
-                tmem_st32u(lane_base + T_PLO + ch * 32, pl + ch * 32);
+                tmem_st32u(lane_base + s * 128 + ch * 32, ph + ch * 32);
+                tmem_st32u(lane_base + s * 128 + 64 + ch * 32, pl + ch * 32);
             }
             tmem_wait_st();
             fence_before();
@@ -422,7 +425,10 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         // the last PV, then this row's output (or the partition's partial)
         if (ok && ntiles > 0) {
-            const bool done = mbar_wait_bounded(&bar[B_ODONE], (ntiles - 1) & 1, p.err);
+            // O-done may be two phases behind here, where a parity wait cannot tell
+            // them apart: wait for the single-use drain barrier the MMA thread
+            // commits after its last MMA instead
+            const bool done = mbar_wait_bounded(&bar[B_DRAIN], 0, p.err);
             ok = !__any_sync(0xffffffffu, !done || s_abort != 0);
         }
         if (ok) {
