@@ -6,10 +6,11 @@
 //   S  = Q K^T   M = 128 query rows, N = 128 KV tokens, K = 128 dims  (TMEM, fp32)
 //   O += P V     M = 128 rows, N = 128 dims, K = 128 tokens            (TMEM, fp32)
 //
-// Roles (192 threads): warp 0 streams Q once and K/V tiles (TMA, 128-byte
+// Roles (320 threads): warp 0 streams Q once and K/V tiles (TMA, 128-byte
 // swizzle, two stages); warp 1 owns the TMEM allocation and one of its threads
-// issues every tcgen05.mma; warps 2-5 run the softmax, one query row per thread
-// (its TMEM lane), so row max and row sum need no shuffles. The S accumulator
+// issues every tcgen05.mma; warps 2-9 run the softmax, two threads per query row
+// (its TMEM lane; one thread per half of the columns, the row maximum exchanged
+// through TMEM each tile). The S accumulator
 // is double-buffered, so S of tile t+1 is computed while the softmax of tile t
 // runs. P stays in TMEM, written over its own S buffer, as two bf16 parts (high,
 // and the rounding residue) that both multiply V (the A operand read from TMEM),
@@ -27,7 +28,7 @@ namespace tc {
 constexpr int ROWS = 128;          // query rows per CTA (UMMA M)
 constexpr int TOK = 128;           // KV tokens per tile
 constexpr int D = 128;
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;      // warp 0 TMA, warp 1 MMA, warps 2-9 softmax (two per row)
 constexpr int HALF = 128 * 128;    // one 64-element-wide half of a 128-row operand, bytes
 constexpr int NST = 3;             // K ring and V ring depth
 constexpr int Q_OFF = 0;
@@ -36,7 +37,7 @@ constexpr int V_OFF = K_OFF + NST * 2 * HALF;     // NST stages of V
 constexpr int BAR_OFF = V_OFF + NST * 2 * HALF;
 constexpr int NBAR = 20;
 constexpr int SMEM = 1024 + BAR_OFF + NBAR * 8 + 16;
-constexpr int TMEM_COLS = 512;     // S/P 0 [0,128) S/P 1 [128,256) O [256,384)
+constexpr int TMEM_COLS = 512;     // S/P 0 [0,128) S/P 1 [128,256) O [256,384) exchange [384,390)
 constexpr int T_O = 256;
 // P of tile t is written over S of tile t (high part in the buffer's first 64
 // columns, low part in the next 64): the buffer is free once S is read, and
@@ -45,8 +46,8 @@ static_assert(SMEM <= 232448, "shared memory per CTA");
 
 // Barrier indices.
 enum {
-    B_Q = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_PREADY = 17, B_ODONE = 18,
-    B_DRAIN = 19
+    B_Q = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_MAX = 15, B_FIN = 16,
+    B_PREADY = 17, B_ODONE = 18, B_DRAIN = 19
 };
 
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -181,7 +182,9 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_init(&bar[B_VEMPTY + s], 1);
         }
         for (int s = 0; s < 2; ++s) mbar_init(&bar[B_SFULL + s], 1);
-        mbar_init(&bar[B_PREADY], 128);
+        mbar_init(&bar[B_MAX], 256);
+        mbar_init(&bar[B_FIN], 256);
+        mbar_init(&bar[B_PREADY], 256);
         mbar_init(&bar[B_ODONE], 1);
         mbar_init(&bar[B_DRAIN], 1);
         s_abort = 0;
@@ -315,14 +318,20 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_wait_bounded(&bar[B_DRAIN], 0, p.err);
         }
     } else {
-        // ---------------- softmax: one query row per thread ----------------
+        // ---------------- softmax: two threads per query row ----------------
+        // Warps 2-9: warp w reads TMEM lanes 32 (w % 4) .. (its rows) and column
+        // half h = (w - 2) / 4 of every 128-wide buffer, so two warps per SM
+        // sub-partition hide each other's latencies. The two halves of a row
+        // combine their maxima each tile through two free TMEM columns.
         const int quarter = warp & 3;                           // TMEM lanes this warp may access
+        const int half = (warp - 2) >> 2;                       // columns [64 half, 64 half + 64)
         const int lr = quarter * 32 + lane;                     // row of the tile = TMEM lane
         const int r = row_begin + lr;
         const int qi = r / G, hh = r - qi * G;
         const int pos = qi < n ? c - n + qi : -1;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-        float m_ref = kNegInf, l = 0.f;
+        constexpr int HC = TOK / 2;                             // columns per thread
+        float m_ref = kNegInf, l = 0.f;                         // l: this half's share of the row sum
         bool ok = true;
         for (int t = 0; t < ntiles; ++t) {
             const int s = t & 1;
@@ -333,53 +342,71 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 break;
             }
             fence_after();
-            float x[TOK];
+            float x[HC];
 #pragma unroll
-            for (int ch = 0; ch < TOK / 32; ++ch) tmem_ld32(lane_base + s * 128 + ch * 32, x + ch * 32);
+            for (int ch = 0; ch < HC / 32; ++ch) tmem_ld32(lane_base + s * 128 + half * HC + ch * 32, x + ch * 32);
             tmem_wait_ld();
             // masks: past the partition's range, or after the row's position (causal)
-            const int tok0 = kv0 + t * TOK;
-            const int lim = min(pos, kv0 + ntok - 1) - tok0;    // columns 0..lim are visible
+            const int tok0 = kv0 + t * TOK + half * HC;
+            const int lim = min(pos, kv0 + ntok - 1) - tok0;    // this half's columns 0..lim are visible
             float mt = kNegInf;
-            if (lim >= TOK - 1) {                               // the whole tile is visible to this row
+            if (lim >= HC - 1) {
 #pragma unroll
-                for (int j = 0; j < TOK; ++j) {
+                for (int j = 0; j < HC; ++j) {
                     x[j] *= p.scale_log2;
                     mt = fmaxf(mt, x[j]);
                 }
             } else {
 #pragma unroll
-                for (int j = 0; j < TOK; ++j) {
+                for (int j = 0; j < HC; ++j) {
                     x[j] = j <= lim ? x[j] * p.scale_log2 : kNegInf;
                     mt = fmaxf(mt, x[j]);
                 }
+            }
+            // the row maximum: exchange with the other half through TMEM column
+            // 384 + 2 (t % 2) + half (double-buffered by tile parity)
+            {
+                const uint32_t xc = 384 + 2 * (t & 1);
+                uint32_t v = __float_as_uint(mt);
+                asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(lane_base + xc + half), "r"(v)
+                             : "memory");
+                tmem_wait_st();
+                fence_before();
+                mbar_arrive(&bar[B_MAX]);
+                const bool ex = mbar_wait_bounded(&bar[B_MAX], t & 1, p.err);
+                if (__any_sync(0xffffffffu, !ex || s_abort != 0)) {
+                    ok = false;
+                    s_abort = 1;
+                    break;
+                }
+                fence_after();
+                asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v) : "r"(lane_base + xc + (half ^ 1)));
+                tmem_wait_ld();
+                mt = fmaxf(mt, __uint_as_float(v));
             }
             const float m_new = fmaxf(m_ref, mt);
             const bool grow = m_new > m_ref + 8.f;              // also true when m_ref is -inf and the row sees a token
             // V rows past the range (the unwritten tail of the last block, or a stage
             // row no piece filled) may hold anything, NaN included: P is 0 there, but
-            // 0 * NaN would not be, so those rows are zeroed before the PV product.
+            // 0 * NaN would not be, so those rows are zeroed (this thread: its half of
+            // the dims) before the PV product.
             const int tok_here = min(TOK, ntok - t * TOK);
             if (lr >= tok_here) {
                 const bool vin = mbar_wait_bounded(&bar[B_VFULL + t % NST], (t / NST) & 1, p.err);
                 if (vin) {
-                    uint8_t* vrow = smem + V_OFF + (t % NST) * 2 * HALF + lr * 128;
+                    uint8_t* vrow = smem + V_OFF + (t % NST) * 2 * HALF + half * HALF + lr * 128;
 #pragma unroll
-                    for (int h = 0; h < 2; ++h)
-#pragma unroll
-                        for (int cc = 0; cc < 8; ++cc)
-                            *reinterpret_cast<uint4*>(vrow + h * HALF + (cc << 4)) = make_uint4(0u, 0u, 0u, 0u);
+                    for (int cc = 0; cc < 8; ++cc) *reinterpret_cast<uint4*>(vrow + (cc << 4)) = make_uint4(0u, 0u, 0u, 0u);
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 }
             }
-            // P = 2^(x - ref) as bf16 high + low parts, computed while the previous
-            // PV product still runs (only writing P into TMEM has to wait for it)
+            // P = 2^(x - ref) as bf16 high + low parts
             const float ref_new = grow ? m_new : m_ref;
             const float ref = ref_new == kNegInf ? 0.f : ref_new;
-            uint32_t ph[TOK / 2], pl[TOK / 2];
+            uint32_t ph[HC / 2], pl[HC / 2];
             float psum = 0.f;
 #pragma unroll
-            for (int e = 0; e < TOK / 2; ++e) {
+            for (int e = 0; e < HC / 2; ++e) {
                 const float p0 = fast_exp2(x[2 * e] - ref), p1 = fast_exp2(x[2 * e + 1] - ref);
                 psum += p0 + p1;
                 ph[e] = pack_bf16(p0, p1);
@@ -389,7 +416,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // then the PV product of tile t - 1 has to be complete first. S of this
             // tile being complete already implies PV of tile t - 2 is (one commit
             // covers every earlier MMA), so O-done is at most one phase behind and
-            // its parity wait is exact.
+            // its parity wait is exact. Each half rescales its 64 columns of O.
             if (t > 0 && __any_sync(0xffffffffu, grow && m_ref != kNegInf)) {
                 const bool done = mbar_wait_bounded(&bar[B_ODONE], (t - 1) & 1, p.err);
                 if (__any_sync(0xffffffffu, !done || s_abort != 0)) {
@@ -400,13 +427,13 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 fence_after();
                 const float alpha = (grow && m_ref != kNegInf) ? fast_exp2(m_ref - m_new) : 1.f;
 #pragma unroll
-                for (int ch = 0; ch < D / 32; ++ch) {
+                for (int ch = 0; ch < HC / 32; ++ch) {
                     float o[32];
-                    tmem_ld32(lane_base + T_O + ch * 32, o);
+                    tmem_ld32(lane_base + T_O + half * HC + ch * 32, o);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[i] *= alpha;
-                    tmem_st32(lane_base + T_O + ch * 32, o);
+                    tmem_st32(lane_base + T_O + half * HC + ch * 32, o);
                 }
             }
             if (grow) {
@@ -414,16 +441,15 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 m_ref = m_new;
             }
             l += psum;
-#pragma unroll
-            for (int ch = 0; ch < TOK / 64; ++ch) {
-                tmem_st32u(lane_base + s * 128 + ch * 32, ph + ch * 32);
-                tmem_st32u(lane_base + s * 128 + 64 + ch * 32, pl + ch * 32);
-            }
+            // this half's tokens: P high columns [32 half, +32), P low columns 64 + [32 half, +32)
+            tmem_st32u(lane_base + s * 128 + half * 32, ph);
+            tmem_st32u(lane_base + s * 128 + 64 + half * 32, pl);
             tmem_wait_st();
             fence_before();
             mbar_arrive(&bar[B_PREADY]);
         }
-        // the last PV, then this row's output (or the partition's partial)
+        // the last PV, then the row sum of both halves, then this half of the row's
+        // output (or of the partition's partial)
         if (ok && ntiles > 0) {
             // O-done may be two phases behind here, where a parity wait cannot tell
             // them apart: wait for the single-use drain barrier the MMA thread
@@ -432,36 +458,52 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             ok = !__any_sync(0xffffffffu, !done || s_abort != 0);
         }
         if (ok) {
-            fence_after();
+            uint32_t v = __float_as_uint(l);
+            asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(lane_base + 388 + half), "r"(v)
+                         : "memory");
+            tmem_wait_st();
+            fence_before();
+            mbar_arrive(&bar[B_FIN]);
+            const bool fin = mbar_wait_bounded(&bar[B_FIN], 0, p.err);
+            ok = !__any_sync(0xffffffffu, !fin || s_abort != 0);
+            if (ok) {
+                fence_after();
+                asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v) : "r"(lane_base + 388 + (half ^ 1)));
+                tmem_wait_ld();
+                l += __uint_as_float(v);
+            }
+        }
+        if (ok) {
             const float inv = l > 0.f ? 1.f / l : 0.f;
             const bool live = qi < n;
             const int64_t qh = (int64_t)(q0 + (live ? qi : 0)) * p.num_q_heads + kvh * G + hh;
 #pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
+            for (int ch = 0; ch < HC / 32; ++ch) {
                 float o[32];
-                tmem_ld32(lane_base + T_O + ch * 32, o);
+                const int d0 = half * HC + ch * 32;
+                tmem_ld32(lane_base + T_O + d0, o);
                 tmem_wait_ld();
                 if (live) {
-                    // the thread's row is contiguous: 16-byte stores
+                    // the thread's 32 dims are contiguous: 16-byte stores
                     if (direct && !p.out_f32) {
-                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + qh * D + ch * 32);
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + qh * D + d0);
 #pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            dst[v] = make_uint4(pack_bf16(o[8 * v] * inv, o[8 * v + 1] * inv),
-                                                pack_bf16(o[8 * v + 2] * inv, o[8 * v + 3] * inv),
-                                                pack_bf16(o[8 * v + 4] * inv, o[8 * v + 5] * inv),
-                                                pack_bf16(o[8 * v + 6] * inv, o[8 * v + 7] * inv));
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            dst[v4] = make_uint4(pack_bf16(o[8 * v4] * inv, o[8 * v4 + 1] * inv),
+                                                 pack_bf16(o[8 * v4 + 2] * inv, o[8 * v4 + 3] * inv),
+                                                 pack_bf16(o[8 * v4 + 4] * inv, o[8 * v4 + 5] * inv),
+                                                 pack_bf16(o[8 * v4 + 6] * inv, o[8 * v4 + 7] * inv));
                     } else {
-                        float* dst = direct ? static_cast<float*>(p.out) + qh * D + ch * 32
-                                            : p.ws_o + (qh * p.num_parts + part) * D + ch * 32;
+                        float* dst = direct ? static_cast<float*>(p.out) + qh * D + d0
+                                            : p.ws_o + (qh * p.num_parts + part) * D + d0;
 #pragma unroll
-                        for (int v = 0; v < 8; ++v)
-                            reinterpret_cast<float4*>(dst)[v] =
-                                make_float4(o[4 * v] * inv, o[4 * v + 1] * inv, o[4 * v + 2] * inv, o[4 * v + 3] * inv);
+                        for (int v4 = 0; v4 < 8; ++v4)
+                            reinterpret_cast<float4*>(dst)[v4] = make_float4(o[4 * v4] * inv, o[4 * v4 + 1] * inv,
+                                                                             o[4 * v4 + 2] * inv, o[4 * v4 + 3] * inv);
                     }
                 }
             }
-            if (live && !direct) {
+            if (live && !direct && half == 0) {
                 p.ws_ml[(qh * p.num_parts + part) * 2 + 0] = m_ref;
                 p.ws_ml[(qh * p.num_parts + part) * 2 + 1] = l;
             }
