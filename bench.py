@@ -51,10 +51,12 @@ def parse():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="pkv", choices=["pkv", "reference"])
-    ap.add_argument("--op", default="decode", choices=["decode", "swap", "mq"],
+    ap.add_argument("--op", default="decode", choices=["decode", "swap", "mq", "fork"],
                     help="decode: the decode step (append + attention); swap: preemption by swapping half the "
                          "workload's sequences to a page-locked host pool and back; mq: several causal query "
-                         "tokens per sequence (--query-len: 512 = a chunked-prefill chunk, 5 = speculative verify)")
+                         "tokens per sequence (--query-len: 512 = a chunked-prefill chunk, 5 = speculative verify); "
+                         "fork: copy-on-write block copies when every sequence forks into --samples samples")
+    ap.add_argument("--samples", type=int, default=4, help="samples per sequence (--op fork)")
     ap.add_argument("--query-len", type=int, default=512, help="query tokens per sequence and step (--op mq)")
     ap.add_argument("--workload", default="llama2_7b", choices=list(wl.WORKLOADS))
     ap.add_argument("--partition-tokens", type=int, default=-2,
@@ -581,6 +583,130 @@ def run_swap(args, ws, rank, local):
     }
 
 
+def fork_pairs(bm, B: int, samples: int):
+    """One parallel-sampling fork of every sequence 0..B-1 through the block
+    manager: samples - 1 children per parent, each child appending its first own
+    token (a shared, partly filled last block is copied on that write), then the
+    children freed. Returns the copy lists (src, dst) int64."""
+    kids = np.arange(B, B * samples, dtype=np.int64)
+    for c in kids:
+        bm.fork(int((c - B) // (samples - 1)), int(c))
+    _, src, dst = bm.append_slots(kids)
+    for c in kids:
+        bm.free(int(c))
+    return src.copy(), dst.copy()
+
+
+def run_fork(args, ws, rank, local):
+    """copy_blocks under parallel sampling: every sequence of the workload forks
+    into --samples samples; each child's first divergent token copies the shared
+    last block (copy-on-write). The copy kernel is timed alone on the block
+    manager's copy lists, L2 flushed before each step; the e2e leg runs the fork,
+    the copy lists' H2D, the kernel and the error-word read per step."""
+    import torch
+    from paged_kv_cache_322_b200 import binding
+    from paged_kv_cache_322_b200.engine import PagedKVCache
+
+    dev = torch.device("cuda", local)
+    w = replica_workload(wl.WORKLOADS[args.workload], rank)
+    w = override_workload(w, args)
+    K, W, n = args.steps, args.warmup, args.samples
+    if n < 2:
+        raise SystemExit("--samples must be >= 2")
+    lens = wl.context_lens(w)
+    bs, B = w.block_size, w.num_seqs
+    cdt = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.uint8}[w.kv_dtype]
+    cache = PagedKVCache(w.num_blocks, bs, w.num_kv_heads, w.head_dim, cdt, dev, free_order=wl.free_order(w))
+    for s in range(B):
+        cache.bm.allocate(s, int(lens[s]))
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed)
+    for c in (cache.k_cache, cache.v_cache):           # synthetic pool contents (a copy does not read values)
+        c.view(torch.uint8).copy_(torch.randint(0, 256, c.view(torch.uint8).shape, device=dev, dtype=torch.uint8,
+                                                generator=g))
+    block_bytes = bs * w.num_kv_heads * w.head_dim * w.elt_bytes
+    sets = [fork_pairs(cache.bm, B, n) for _ in range(W + K)]   # the free list rotates: new dst blocks each step
+    npairs = int(sets[0][0].size)
+    assert all(s.size == npairs for s, _ in sets)
+    moved = 2 * npairs * block_bytes * 2                 # K and V, read once and written once
+    dsets = [(torch.from_numpy(s).to(dev), torch.from_numpy(d).to(dev)) for s, d in sets]
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for i in range(W):
+        flush.fill_(i)
+        binding.copy_blocks(cache.k_cache, cache.v_cache, *dsets[i])
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(K):
+            flush.fill_(W + i)
+            ev[i][0].record(stream)
+            binding.copy_blocks(cache.k_cache, cache.v_cache, *dsets[W + i])
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    assert binding.get_device_error() == 0
+    ms = sum(a.elapsed_time(b) for a, b in ev)
+    ms_max, total_gbs, _ = aggregate(ms, float(moved * K), float(npairs * K), ws)
+    copy_ms = ms / K
+    ach = moved / (copy_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    del dsets, flush
+
+    # ---- e2e: fork in the block manager, copy lists H2D, kernel, error word D2H ----
+    e2e = None
+    if not args.no_e2e:
+        hs = torch.empty(npairs, dtype=torch.int64, pin_memory=True)
+        hd = torch.empty(npairs, dtype=torch.int64, pin_memory=True)
+        ds, dd = torch.empty(npairs, dtype=torch.int64, device=dev), torch.empty(npairs, dtype=torch.int64, device=dev)
+
+        def step_host():
+            src, dst = fork_pairs(cache.bm, B, n)
+            hs.numpy()[:] = src
+            hd.numpy()[:] = dst
+            ds.copy_(hs, non_blocking=True)
+            dd.copy_(hd, non_blocking=True)
+            binding.copy_blocks(cache.k_cache, cache.v_cache, ds, dd, stream=stream)
+            if binding.get_device_error() != 0:         # D2H of the error word; synchronises the stream
+                raise RuntimeError("copy_blocks flagged a bad block id")
+
+        for _ in range(W):
+            step_host()
+        barrier(ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            step_host()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(ws)
+        e_ms, e_gbs, _ = aggregate(e0.elapsed_time(e1), float(moved * K), float(npairs * K), ws)
+        e2e = {"value": round(e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": 16 * npairs,
+               "d2h_bytes_per_step": 4, "ms_per_step": round(e_ms / K, 4),
+               "path": "block manager fork + append_slots, H2D of the copy lists, copy_blocks, error word D2H"}
+
+    return {
+        "metric": "copy_blocks: copy-on-write block copies under parallel sampling, GB/s (K and V read + written)",
+        "value": round(total_gbs, 2), "unit": "GB/s", "n_gpus": ws, "steps": K, "warmup": W,
+        "ms_per_step": round(ms_max / K, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.kv_dtype, "data": "synthetic",
+        "config": {"workload": f"parallel sampling, {n} samples per sequence, of: {w.description}",
+                   "samples": n, "copies_per_step": npairs, "block_bytes": block_bytes,
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                   "l2": "L2 flushed (write of 2x L2) before each step, outside the timed events"},
+        "roofline": {"bound": "hbm", "kernel": "block_copy_kernel", "achieved": round(ach, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(ach / peak, 4), "avg_launch_ms": round(copy_ms, 5),
+                     "algorithmic_bytes_per_launch": moved, "peak_source": peak_kind, "traffic": None},
+        "e2e": e2e,
+        "gpu_launches": K,
+        "clocks": clocks.summary(),
+    }
+
+
 def run_mq(args, ws, rank, local):
     """Causal multi-query steps: every sequence appends --query-len tokens (a
     prefill chunk, or draft tokens to verify) and attends with them over its
@@ -725,7 +851,8 @@ def run_mq(args, ws, rank, local):
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
                    "l2": "KV per step larger than L2; no flush", "seed": w.seed},
         "roofline": {"bound": "tensor" if tensor else "hbm",
-                     "kernel": "paged_mq_kernel (+ merge_mq_kernel when partitioned)",
+                     "kernel": ("tc::paged_mq_tc_kernel (tcgen05)" if d == 128 and n * (hq // hkv) >= 32
+                                else "paged_mq_kernel (mma.sync)") + " (+ merge_mq_kernel when partitioned)",
                      "achieved": round(ach, 2), "peak": peak, "unit": "TFLOP/s" if tensor else "GB/s",
                      "frac": round(ach / peak, 4), "avg_launch_ms": round(attn_ms, 5),
                      "flops_per_launch": int(fl), "algorithmic_bytes_per_launch": int(by),
@@ -855,7 +982,7 @@ def main():
         return
     ws, rank, local = dist_init(args)
     try:
-        run = {"swap": run_swap, "mq": run_mq}.get(args.op, run_pkv)
+        run = {"swap": run_swap, "mq": run_mq, "fork": run_fork}.get(args.op, run_pkv)
         r = run(args, ws, rank, local)
         if rank == 0:
             print(json.dumps(r), flush=True)

@@ -46,3 +46,35 @@ def test_block_size_override_keeps_pool_tokens():
     args = argparse.Namespace(block_size=0, num_seqs=8, num_blocks=100)
     w3 = bench.override_workload(w, args)
     assert (w3.num_seqs, w3.num_blocks, w3.block_size) == (8, 100, 16)
+
+
+def test_fork_copy_lists_match_the_oracle_block_manager():
+    """The fork bench's copy lists: one copy per child of every parent whose last
+    block is partly filled (a full last block takes a fresh block instead), the
+    same pairs as the oracle's block manager under the same operations, and the
+    pool back to its size after the children are freed."""
+    from oracle.block_manager import BlockManager as OracleBM
+    from paged_kv_cache_322_b200 import binding
+    lens = [16, 17, 31, 32, 1, 100]
+    nb, bs, samples = 64, 16, 3
+    order = np.random.default_rng(0).permutation(nb).astype(np.int32)
+    bm, obm = binding.BlockManager(nb, bs, order), OracleBM(nb, bs, order)
+    for s, c in enumerate(lens):
+        bm.allocate(s, c)
+        obm.allocate(s, c)
+    free0 = bm.num_free()
+    for _ in range(3):
+        src, dst = bench.fork_pairs(bm, len(lens), samples)
+        want = []
+        kids = list(range(len(lens), len(lens) * samples))
+        for c in kids:
+            obm.fork((c - len(lens)) // (samples - 1), c)
+        for c in kids:
+            _, cp = obm.append_slot(c)
+            if cp is not None:
+                want.append(cp)
+        for c in kids:
+            obm.free_seq(c)
+        assert list(zip(src.tolist(), dst.tolist())) == [tuple(p) for p in want]
+        assert len(want) == (samples - 1) * sum(1 for c in lens if c % bs)
+        assert bm.num_free() == free0
