@@ -628,7 +628,7 @@ def run_fork(args, ws, rank, local):
     sets = [fork_pairs(cache.bm, B, n) for _ in range(W + K)]   # the free list rotates: new dst blocks each step
     npairs = int(sets[0][0].size)
     assert all(s.size == npairs for s, _ in sets)
-    moved = 2 * npairs * block_bytes * 2                 # K and V, read once and written once
+    moved = 2 * npairs * block_bytes * 2 + 16 * npairs   # K and V read once and written once; the two ids
     dsets = [(torch.from_numpy(s).to(dev), torch.from_numpy(d).to(dev)) for s, d in sets]
     # L2 flush: write a buffer of 2x L2, then read another one, so that the timed
     # copy starts from an L2 holding only clean, unrelated lines (a write-only
