@@ -49,10 +49,15 @@ namespace attn {
 // dimension over the partitions with independent loads in flight (the first
 // version walked the partitions with one dependent load chain per thread).
 constexpr int kMergeSmemParts = 2048;
+//
+// Launched as a programmatic dependent of the partition kernel: its CTAs may
+// start in the partition kernel's tail and wait here until that grid has
+// completed and its partials are visible (a no-op for a plain launch).
 template <int D>
 __global__ void __launch_bounds__(D) merge_partitions_kernel(const Params p) {
     __shared__ float sw[kMergeSmemParts];
     __shared__ float s_red[D / 32];
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int qhead = blockIdx.x, seq = blockIdx.y, d = threadIdx.x;
     const int lane = d & 31, wid = d >> 5;
     int ctx = p.context_lens[seq];
@@ -375,10 +380,20 @@ pkv_status decode_impl(void* out, pkv_dtype out_dtype, const void* q, const void
     }
     if (e != cudaSuccess) return PKV_ERR_CUDA;
     if (pl.num_parts > 1) {
-        dim3 g2(num_q_heads, num_seqs);
-        if (head_dim == 128) merge_partitions_kernel<128><<<g2, 128, 0, st>>>(p);
-        else merge_partitions_kernel<64><<<g2, 64, 0, st>>>(p);
-        if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
+        // programmatic dependent launch: the merge grid is scheduled into the
+        // partition kernel's tail instead of after a full kernel boundary
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(num_q_heads, num_seqs);
+        cfg.blockDim = dim3(head_dim);
+        cfg.stream = st;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        e = head_dim == 128 ? cudaLaunchKernelEx(&cfg, merge_partitions_kernel<128>, p)
+                            : cudaLaunchKernelEx(&cfg, merge_partitions_kernel<64>, p);
+        if (e != cudaSuccess) return PKV_ERR_CUDA;
     }
     return PKV_OK;
 }
