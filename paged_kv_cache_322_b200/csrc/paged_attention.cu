@@ -50,9 +50,9 @@ namespace attn {
 // version walked the partitions with one dependent load chain per thread).
 constexpr int kMergeSmemParts = 2048;
 //
-// Launched as a programmatic dependent of the partition kernel: its CTAs may
-// start in the partition kernel's tail and wait here until that grid has
-// completed and its partials are visible (a no-op for a plain launch).
+// Launched as a programmatic dependent of the partition kernel: the launch is
+// staged while that kernel runs, and the CTAs wait here until its grid has
+// completed and the partials are visible (a no-op for a plain launch).
 template <int D>
 __global__ void __launch_bounds__(D) merge_partitions_kernel(const Params p) {
     __shared__ float sw[kMergeSmemParts];
@@ -380,8 +380,8 @@ pkv_status decode_impl(void* out, pkv_dtype out_dtype, const void* q, const void
     }
     if (e != cudaSuccess) return PKV_ERR_CUDA;
     if (pl.num_parts > 1) {
-        // programmatic dependent launch: the merge grid is scheduled into the
-        // partition kernel's tail instead of after a full kernel boundary
+        // programmatic dependent launch: the merge grid's CTAs wait for the
+        // partition grid in-kernel instead of behind a full kernel boundary
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(num_q_heads, num_seqs);
         cfg.blockDim = dim3(head_dim);

@@ -82,10 +82,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     const int nblk_seq = (ctx + BSZ - 1) / BSZ;
     const int nparts = (nblk_seq + p.part_blocks - 1) / p.part_blocks;
     if (part > 0 && part >= nparts) return;                       // beyond this sequence's context
-    // once every CTA of this grid has signalled (or exited), the merge grid, a
-    // programmatic dependent, may be scheduled into this grid's tail; it waits
-    // for this grid's completion before it reads the partials
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int blk0 = part * p.part_blocks;
     const int nblk = max(0, min(p.part_blocks, nblk_seq - blk0));
     const int ntok = max(0, min(p.part_blocks * BSZ, ctx - blk0 * BSZ));   // tokens of this partition
