@@ -17,6 +17,12 @@ per-step inputs already in HBM; `e2e` times the same steps through the public
 API from host buffers (host block manager, pinned H2D copies of the step's
 queries / new K,V / metadata, the kernels, D2H of the output).
 
+Other operations, one JSON line each (`--op`): `swap` (preemption swap-out and
+swap-in over the host link), `mq` (causal multi-query attention: chunked
+prefill with --query-len 512, speculative verify with --query-len 5) and
+`fork` (copy-on-write block copies when every sequence forks into --samples
+samples).
+
 Multi-GPU (torchrun): every rank runs its own replica of the batch (decode
 batches are independent; there is no data exchange), times are the max over
 ranks, and `value` is the sum of all ranks' bytes over that time.
