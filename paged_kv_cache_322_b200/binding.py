@@ -134,11 +134,22 @@ def _stream(t, stream) -> int:
 
 
 def _cuda_contig(*ts):
+    """CUDA, contiguous, all on one device and that the current one: the library
+    launches on the current device, where another GPU's pointer is not valid."""
+    dev = None
     for t in ts:
         if not t.is_cuda:
             raise ValueError("tensors must be CUDA tensors")
         if not t.is_contiguous():
             raise ValueError("tensors must be contiguous")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"tensors must be on one device ({dev} and {t.device})")
+    if dev is not None:
+        cur = _torch().cuda.current_device()
+        if dev.index != cur:
+            raise ValueError(f"tensors are on {dev} but the current device is cuda:{cur} (torch.cuda.set_device)")
 
 
 def workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,

@@ -395,3 +395,28 @@ def test_swap_errors(lib):
     assert lib.pkv_swap_blocks(fake, fake, 0, fake, fake, 4, 1, fake, fake, 1, 16, 8, 128, None) == 1
     assert lib.pkv_swap_blocks(fake, fake, 4, fake, fake, 4, 1, fake, fake, -1, 16, 8, 128, None) == 1
     assert lib.pkv_swap_blocks(fake, fake, 4, fake, fake, 4, 2, fake, fake, 1, 1, 1, 8, None) == 2  # 8-byte block
+
+
+def test_binding_requires_one_current_device(monkeypatch):
+    """The binding refuses tensors that are not CUDA, not contiguous, on two
+    devices, or on a device other than the current one (the library launches on
+    the current device). Stand-in tensor objects: no GPU needed."""
+    import torch
+
+    class T:
+        def __init__(self, idx, cuda=True, contig=True):
+            self.device, self.is_cuda, self._contig = torch.device("cuda", idx), cuda, contig
+
+        def is_contiguous(self):
+            return self._contig
+
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 1)
+    binding._cuda_contig(T(1), T(1), T(1))
+    with pytest.raises(ValueError, match="one device"):
+        binding._cuda_contig(T(1), T(0))
+    with pytest.raises(ValueError, match="current device"):
+        binding._cuda_contig(T(0), T(0))
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        binding._cuda_contig(T(1), T(1, cuda=False))
+    with pytest.raises(ValueError, match="contiguous"):
+        binding._cuda_contig(T(1, contig=False))
