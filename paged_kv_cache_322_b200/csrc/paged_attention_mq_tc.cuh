@@ -7,7 +7,7 @@
 //   O += P V     M = 128 rows, N = 128 dims, K = 128 tokens            (TMEM, fp32)
 //
 // Roles (320 threads): warp 0 streams Q once and K/V tiles (TMA, 128-byte
-// swizzle, two stages); warp 1 owns the TMEM allocation and one of its threads
+// swizzle, three-stage K and V rings); warp 1 owns the TMEM allocation and one of its threads
 // issues every tcgen05.mma; warps 2-9 run the softmax, two threads per query row
 // (its TMEM lane; one thread per half of the columns, the row maximum exchanged
 // through TMEM each tile). The S accumulator
