@@ -266,6 +266,50 @@ def test_kernel_entry_points_reject_bad_arguments_on_host(lib):
     assert lib.pkv_copy_blocks(fake, fake, 1, fake, fake, -1, 16, 8, 128, 64, None) == 1
 
 
+def test_fp8_multi_query_and_noalloc_entry_points_reject_bad_arguments_on_host(lib):
+    """Every refusal below happens in host code before any device call, so it
+    runs without a GPU: status 1 = invalid argument, 2 = not built."""
+    fake = ctypes.c_void_p(1 << 20)
+    nan, inf = float("nan"), float("inf")
+
+    def dec8(ks, vs, d=128, part=0):
+        return lib.pkv_paged_attention_decode_fp8(fake, 0, fake, fake, fake, ks, vs, fake, fake, 1.0, 2, 8, 8, d, 16,
+                                                  4, 64, 0, part, None, 0, None)
+    assert dec8(0.0, 1.0) == 1 and dec8(1.0, -1.0) == 1 and dec8(nan, 1.0) == 1 and dec8(1.0, inf) == 1
+    assert dec8(1.0, 1.0, d=64) == 2                 # e4m3 attention is built for head_dim 128
+    assert dec8(1.0, 1.0, part=-1) == 2              # no persistent schedule over e4m3 caches
+    # the plain decode call takes fp32 / bf16 caches only; e4m3 goes through the fp8 entry point
+    assert lib.pkv_paged_attention_decode(fake, 0, fake, fake, fake, 2, fake, fake, 1.0, 2, 8, 8, 128, 16, 4, 64,
+                                          0, 0, None, 0, None) == 1
+
+    def app8(in_dtype=1, ks=1.0, hkv=8, d=128, t=4):
+        return lib.pkv_reshape_and_cache_fp8(fake, fake, in_dtype, fake, fake, ks, 1.0, fake, t, hkv, d, 16, 64, None)
+    assert app8(in_dtype=2) == 1 and app8(ks=0.0) == 1 and app8(ks=nan) == 1
+    assert app8(hkv=1, d=8) == 2                     # 8-element rows: not a whole 16-byte vector of codes
+    assert lib.pkv_reshape_and_cache_fp8(None, None, 1, None, None, 1.0, 1.0, None, 0, 8, 128, 16, 64, None) == 0
+
+    def mq(kv=1, hq=8, hkv=8, d=128, bs=16, mb=4, nq=4, ctx=64, part=0, seqs=2, tokens=8, ws=None, ws_n=0):
+        return lib.pkv_paged_attention_multi_query(fake, 0, fake, fake, fake, kv, fake, fake, fake, 1.0, seqs, tokens,
+                                                   hq, hkv, d, bs, mb, 64, nq, ctx, part, ws, ws_n, None)
+    assert mq(kv=0) == 2 and mq(kv=2) == 2          # bf16 caches only
+    assert mq(kv=7) == 1
+    assert mq(d=96) == 2 and mq(bs=12) == 2 and mq(hq=12, hkv=4) == 2      # head_dim, block size, group 3
+    assert mq(hq=6, hkv=4) == 1 and mq(part=-1) == 1
+    assert mq(nq=100) == 1                           # more query tokens than the table holds
+    assert mq(part=16) == 1                          # four partitions need a workspace; none given
+    assert mq(seqs=0) == 0 and mq(nq=0) == 0 and mq(tokens=0) == 0
+    assert lib.pkv_paged_attention_multi_query_workspace_bytes(2, 8, 8, 8, 128, 16, 4, 4, 64, 16) > 0
+    assert lib.pkv_paged_attention_multi_query_workspace_bytes(2, 8, 8, 8, 128, 16, 4, 4, 64, 64) == 0
+    assert lib.pkv_paged_attention_multi_query_workspace_bytes(2, 8, 8, 8, 128, 16, 4, 100, 64, 0) == \
+        ctypes.c_size_t(-1).value
+
+    # allocation-free decode: sizes whose split-K scratch exceeds the fixed array, and invalid sizes
+    assert lib.pkv_paged_attention_decode_noalloc(fake, 0, fake, fake, fake, 1, fake, fake, 1.0, 1024, 64, 8, 128,
+                                                  16, 2048, 65536, 32768, 512, None) == 2
+    assert lib.pkv_paged_attention_decode_noalloc(fake, 0, fake, fake, fake, 1, fake, fake, 1.0, 2, 6, 4, 128,
+                                                  16, 4, 64, 0, 0, None) == 1
+
+
 def test_workspace_and_partition_rule(lib):
     # 512-token partitions over a 32768-token cap: 64 partitions of (D + 2) floats per row
     n = binding.workspace_bytes(16, 32, 8, 128, 16, 2048, 32768, 512)
