@@ -310,6 +310,25 @@ def test_fp8_multi_query_and_noalloc_entry_points_reject_bad_arguments_on_host(l
                                                   16, 4, 64, 0, 0, None) == 1
 
 
+def test_native_step_refuses_bad_arguments_on_host(lib):
+    """pkv_step_ctx_create and pkv_decode_step refuse invalid sizes, dtypes and
+    scales before touching the device; destroying a null context is a no-op."""
+    h = ctypes.c_void_p()
+
+    def create(seqs=4, hq=8, hkv=8, d=128, mb=4, bs=16, kv=1, out=0, ks=1.0, vs=1.0):
+        return lib.pkv_step_ctx_create(seqs, hq, hkv, d, mb, bs, kv, out, 0, ks, vs, ctypes.byref(h))
+    assert create(seqs=0) == 1 and create(hq=6, hkv=4) == 1 and create(d=0) == 1 and create(mb=0) == 1
+    assert create(bs=0) == 1 and create(kv=5) == 1 and create(out=2) == 1      # e4m3 is not an output type
+    assert create(kv=2, ks=0.0) == 1 and create(kv=2, vs=-1.0) == 1         # e4m3 caches need positive scales
+    assert lib.pkv_step_ctx_create(4, 8, 8, 128, 4, 16, 1, 0, 0, 1.0, 1.0, None) == 1
+    lib.pkv_step_ctx_destroy(None)
+    bm = binding.BlockManager(8, 16)
+    ids = np.zeros(1, np.int64)
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.pkv_decode_step(None, bm._h, ids.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), 1, fake, fake, fake,
+                               fake, fake, 8, 1.0, 0, fake, None) == 1
+
+
 def test_workspace_and_partition_rule(lib):
     # 512-token partitions over a 32768-token cap: 64 partitions of (D + 2) floats per row
     n = binding.workspace_bytes(16, 32, 8, 128, 16, 2048, 32768, 512)
