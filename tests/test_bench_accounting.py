@@ -78,3 +78,19 @@ def test_fork_copy_lists_match_the_oracle_block_manager():
         assert list(zip(src.tolist(), dst.tolist())) == [tuple(p) for p in want]
         assert len(want) == (samples - 1) * sum(1 for c in lens if c % bs)
         assert bm.num_free() == free0
+
+
+def test_reference_arm_line(monkeypatch):
+    """`bench.py --impl reference` (the CPU oracle) prints the contract's keys,
+    with the workload overrides applied and nothing from the other ranks."""
+    orig = bench.cpu_baseline
+    monkeypatch.setattr(bench, "cpu_baseline", lambda w, target_s: orig(w, 0.2))
+    args = argparse.Namespace(workload="tiny_fp32", steps=2, warmup=1, block_size=0, num_seqs=2, num_blocks=0)
+    assert bench.run_reference(args, 1, 1) is None
+    r = bench.run_reference(args, 1, 0)
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in r, k
+    assert r["impl"] == "reference" and r["value"] > 0 and r["ms_per_step"] > 0 and r["config"]["global_batch"] == 2
+    assert r["cpu_baseline"]["kind"] == "oracle" and r["cpu_baseline"]["cores"] >= 1
+    assert r["e2e"]["h2d_bytes_per_step"] == 0 and r["e2e"]["d2h_bytes_per_step"] == 0
