@@ -49,6 +49,7 @@ sys.path.insert(0, ROOT)
 from paged_kv_cache_322_b200 import workloads as wl  # noqa: E402
 
 L2_BYTES = 126 * 2 ** 20
+SPEC_HBM_GBS = 8000.0          # B200 HBM3e, the spec sheet's 8 TB/s (the measured copy peak is the other denominator)
 
 
 def parse():
@@ -74,6 +75,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     ap.add_argument("--num-seqs", type=int, default=0, help="override the batch size (profiling a small case)")
     ap.add_argument("--num-blocks", type=int, default=0, help="override the pool size (profiling a small case)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="default run only: skip the 70B-shaped GQA sub-result")
     ap.add_argument("--block-size", type=int, default=0,
                     help="tokens per block (8, 16, 32, 64); the pool keeps the workload's token capacity")
     return ap.parse_args()
@@ -328,8 +331,6 @@ def run_pkv(args, ws, rank, local):
         k, v = kvs[s]
         cache.add_sequence(s, torch.from_numpy(k).to(dev, dt), torch.from_numpy(v).to(dev, dt))
     ids = np.arange(w.num_seqs, dtype=np.int64)
-    if w.ctx == "shared_prefix":
-        raise SystemExit("the shared-prefix workload is a parity case; bench the decode workloads")
     torch.cuda.synchronize()
     paging = None
     if not args.no_paging_overhead and part != -1:
@@ -449,6 +450,7 @@ def run_pkv(args, ws, rank, local):
         "ms_per_step": round(ms_max / K, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.kv_dtype, "data": "synthetic",
         "pct_of_peak": round(100 * gbs / ws / peak, 1),
+        "pct_of_peak_spec": round(100 * gbs / ws / SPEC_HBM_GBS, 1),
         "decode_tokens_per_s": round(tokens_s, 1),
         "attention_layer_tokens_per_s_per_32_layers": round(tokens_s / 32, 1),
         "config": {"workload": w.description, "global_batch": w.num_seqs * ws, "seq_len": f"U[{w.lo},{w.hi}]",
@@ -459,7 +461,8 @@ def run_pkv(args, ws, rank, local):
                    "seed": w.seed},
         "roofline": {"bound": "hbm", "kernel": "paged_decode_kernel + merge_partitions_kernel (one attention call)",
                      "achieved": round(achieved, 1), "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "avg_launch_ms": round(attn_avg_ms, 5),
+                     "frac": round(achieved / peak, 4), "frac_of_spec": round(achieved / SPEC_HBM_GBS, 4),
+                     "avg_launch_ms": round(attn_avg_ms, 5),
                      "algorithmic_bytes_per_launch": int(attn_bytes_avg),
                      "traffic": (int(tr["traffic_per_algorithmic_byte"] * attn_bytes_avg) if tr else None),
                      "traffic_source": (tr["captured_on"] if tr else None)},
@@ -470,6 +473,272 @@ def run_pkv(args, ws, rank, local):
         "cpu_baseline": cpu,
     }
     return result
+
+
+def unique_attention_bytes(w: wl.Workload, tables: np.ndarray, lens: np.ndarray, out_elt: int) -> int:
+    """Algorithmic bytes of one attention call counting each distinct physical
+    block once: a block shared by several sequences (a common prompt prefix) is
+    charged the tokens its longest reader uses, once. Plus q, out, the block
+    tables and the lengths, as in attention_bytes."""
+    bs = w.block_size
+    used = {}
+    for s in range(len(lens)):
+        n = int(lens[s])
+        for j in range(-(-n // bs)):
+            b = int(tables[s][j])
+            used[b] = max(used.get(b, 0), min(bs, n - j * bs))
+    kv = sum(used.values()) * w.num_kv_heads * w.head_dim * w.elt_bytes * 2
+    q = len(lens) * w.num_q_heads * w.head_dim * w.in_bytes
+    out = len(lens) * w.num_q_heads * w.head_dim * out_elt
+    nt = int(sum(-(-int(n) // bs) for n in lens)) * 4
+    return kv + q + out + nt + 4 * len(lens)
+
+
+def run_shared_prefix(args, ws, rank, local):
+    """The shared-prefix decode step (parallel sampling: 32 sequences share the
+    64 blocks of a 1024-token prompt, ref count 32, plus private tails).
+
+    One step: copy_blocks forks the last shared block (logical 63) for the 31
+    sequences that diverge (the 32nd keeps the original), reshape_and_cache
+    appends one token per sequence, and decode attention runs over the updated
+    contexts. The fork's copy list comes from the block manager's copy-on-write
+    of logical block 63 before the first step; every step replays it (the source
+    block is full and never written again, so each replay rewrites the same
+    bytes), so every timed step does a fork step's work.
+
+    Bytes: the attention is charged both ways, logical (every sequence's context
+    read once, prefix included 32 times) and unique (each physical block once);
+    `value` and % of peak use unique bytes. Timed twice: as a stream of steps with
+    no flush (the 16 MiB prefix stays in L2 between steps), and with L2 flushed
+    before every step (events around the step only)."""
+    import torch
+    from paged_kv_cache_322_b200 import binding
+    from paged_kv_cache_322_b200.engine import PagedKVCache
+
+    dev = torch.device("cuda", local)
+    w = override_workload(wl.WORKLOADS[args.workload], args)
+    w = replica_workload(w, rank)
+    part = w.partition_tokens if args.partition_tokens == -2 else args.partition_tokens
+    K, W = args.steps, args.warmup
+    B, bs, p = w.num_seqs, w.block_size, w.shared_prefix
+    dt = torch.bfloat16 if w.kv_dtype != "f32" else torch.float32
+    lens0 = wl.context_lens(w)
+    total_steps = 2 * (W + 2 * K) + 2
+    mb = -(-int(lens0.max() + total_steps) // bs)
+    ids = np.arange(B, dtype=np.int64)
+
+    # ---- set-up (untimed): the shared prompt once, forked to every sequence, then the private tails ----
+    cache = PagedKVCache(w.num_blocks, bs, w.num_kv_heads, w.head_dim, dt, dev, free_order=wl.free_order(w),
+                         max_blocks_per_seq=mb)
+
+    def tdev(x):
+        return torch.from_numpy(x).to(dev, dt)
+
+    k0, v0 = wl.prompt_kv(w, 0, int(lens0[0]))
+    cache.add_sequence(-1, tdev(k0[:p]), tdev(v0[:p]))
+    for s in range(B):
+        cache.fork(-1, s)
+    cache.free(-1)
+    for s in range(B):
+        n = int(lens0[s])
+        k, v = wl.prompt_kv(w, s, n)
+        slots = np.concatenate([cache.bm.append_slots([s])[0] for _ in range(n - p)])
+        cache.append(tdev(k[p:]), tdev(v[p:]), torch.from_numpy(slots).to(dev))
+    last = p // bs - 1
+    assert cache.bm.ref_count(int(cache.block_tables([0])[0][0][last])) == B
+    pairs = [x for x in (cache.bm.make_writable(int(s), last) for s in ids) if x is not None]
+    assert len(pairs) == B - 1
+    pa = np.asarray(pairs, dtype=np.int64)
+    src_d, dst_d = torch.from_numpy(pa[:, 0].copy()).to(dev), torch.from_numpy(pa[:, 1].copy()).to(dev)
+    block_bytes = bs * w.num_kv_heads * w.head_dim * w.elt_bytes
+    copy_bytes = 2 * len(pairs) * block_bytes * 2 + 16 * len(pairs)      # K and V blocks read + written, the ids
+    torch.cuda.synchronize()
+
+    def make_steps(n, step0):
+        out = []
+        for i in range(n):
+            slots, src, dst = cache.bm.append_slots(ids)
+            assert src.size == 0
+            tables, lens = cache.block_tables(ids)
+            q = wl.decode_q(w, step0 + i)
+            kn, vn = wl.decode_kv(w, step0 + i)
+            out.append(dict(q=tdev(q), kn=tdev(kn), vn=tdev(vn), slots=torch.from_numpy(slots).to(dev),
+                            tables=torch.from_numpy(tables).to(dev), lens=torch.from_numpy(lens).to(dev),
+                            maxlen=int(lens.max()), logical=attention_bytes(w, lens, 2),
+                            unique=unique_attention_bytes(w, tables, lens, 2)))
+        return out
+
+    steps = make_steps(W + 2 * K, 0)
+    maxctx = max(st["maxlen"] for st in steps) + (W + K + 2)
+    out = torch.empty((B, w.num_q_heads, w.head_dim), dtype=torch.bfloat16, device=dev)
+    ws_bytes = binding.workspace_bytes(B, w.num_q_heads, w.num_kv_heads, w.head_dim, bs, mb, maxctx, part)
+    workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    part_used = binding.partition_tokens(B, w.num_q_heads, w.num_kv_heads, w.head_dim, bs, mb, maxctx, part)
+    stream = torch.cuda.current_stream(dev)
+    flush_w = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+    flush_r = torch.ones(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def step_device(st, e_step=None, e_attn=None):
+        if e_step is not None:
+            e_step[0].record(stream)
+        binding.copy_blocks(cache.k_cache, cache.v_cache, src_d, dst_d, stream=stream)
+        cache.append(st["kn"], st["vn"], st["slots"], stream=stream)
+        e_attn[0].record(stream)
+        cache.attention(out, st["q"], st["tables"], st["lens"], w.scale, max_context_len=maxctx,
+                        partition_tokens=part, workspace=workspace, stream=stream)
+        e_attn[1].record(stream)
+        if e_step is not None:
+            e_step[1].record(stream)
+
+    def evpair():
+        return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    for i in range(W):
+        step_device(steps[i], None, evpair())
+    torch.cuda.synchronize()
+    # (a) a stream of steps, no flush
+    ev_a = [evpair() for _ in range(K)]
+    t0, t1 = evpair()
+    barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t0.record(stream)
+        for i in range(K):
+            step_device(steps[W + i], None, ev_a[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    ms_a = t0.elapsed_time(t1)
+    attn_a = [a.elapsed_time(b) for a, b in ev_a]
+    # (b) L2 flushed before every step (write 2x L2, then read another 2x L2), each step timed alone
+    ev_b = [(evpair(), evpair()) for _ in range(K)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks_b:
+        for i in range(K):
+            flush_w.fill_(i)
+            flush_r.sum()
+            step_device(steps[W + K + i], *ev_b[i])
+        torch.cuda.synchronize()
+    barrier(ws)
+    ms_b = sum(a.elapsed_time(b) for (a, b), _ in ev_b)
+    attn_b = [a.elapsed_time(b) for _, (a, b) in ev_b]
+    assert binding.get_device_error() == 0
+
+    ta, tb = steps[W:W + K], steps[W + K:]
+    step_bytes = lambda st, key: st[key] + copy_bytes + append_bytes(w)        # noqa: E731
+    uniq_a, logi_a = sum(step_bytes(st, "unique") for st in ta), sum(step_bytes(st, "logical") for st in ta)
+    uniq_b, logi_b = sum(step_bytes(st, "unique") for st in tb), sum(step_bytes(st, "logical") for st in tb)
+    ms_max, gbs, tokens_s = aggregate(ms_a, float(uniq_a), float(B * K), ws)
+    _, gbs_logical, _ = aggregate(ms_a, float(logi_a), 0.0, ws)
+    msb_max, gbs_b, _ = aggregate(ms_b, float(uniq_b), 0.0, ws)
+    _, gbs_b_logical, _ = aggregate(ms_b, float(logi_b), 0.0, ws)
+    peak, peak_kind = measured_peaks()
+    au = statistics.mean(st["unique"] for st in ta)
+    al = statistics.mean(st["logical"] for st in ta)
+    aa, ab = statistics.mean(attn_a), statistics.mean(attn_b)
+    ach = au / (aa * 1e-3) / 1e9
+    ach_b = statistics.mean(st["unique"] for st in tb) / (ab * 1e-3) / 1e9
+    del steps
+
+    # ---- e2e: public API calls from pinned host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        hsteps = []
+        for i in range(W + K):
+            q = wl.decode_q(w, 1000 + i)
+            kn, vn = wl.decode_kv(w, 1000 + i)
+            hsteps.append(tuple(torch.from_numpy(x).to(dt).pin_memory() for x in (q, kn, vn)))
+        h_pairs = torch.from_numpy(pa.copy()).pin_memory()
+        h_out = torch.empty((B, w.num_q_heads, w.head_dim), dtype=torch.bfloat16).pin_memory()
+        d_q = torch.empty((B, w.num_q_heads, w.head_dim), dtype=dt, device=dev)
+        d_k = torch.empty((B, w.num_kv_heads, w.head_dim), dtype=dt, device=dev)
+        d_v = torch.empty_like(d_k)
+        d_pairs = torch.empty((len(pairs), 2), dtype=torch.int64, device=dev)
+        h_slots = torch.empty(B, dtype=torch.int64).pin_memory()
+        h_tables = torch.empty((B, mb), dtype=torch.int32).pin_memory()
+        h_lens = torch.empty(B, dtype=torch.int32).pin_memory()
+        d_slots = torch.empty(B, dtype=torch.int64, device=dev)
+        d_tables = torch.empty((B, mb), dtype=torch.int32, device=dev)
+        d_lens = torch.empty(B, dtype=torch.int32, device=dev)
+        e2e_bytes = []
+
+        def step_host(hq, hk, hv):
+            slots, src, dst = cache.bm.append_slots(ids)                  # host block manager
+            tables, lens = cache.block_tables(ids)
+            h_slots.numpy()[:] = slots
+            h_tables.numpy()[:] = tables
+            h_lens.numpy()[:] = lens
+            for d, h in ((d_q, hq), (d_k, hk), (d_v, hv), (d_pairs, h_pairs), (d_slots, h_slots),
+                         (d_tables, h_tables), (d_lens, h_lens)):
+                d.copy_(h, non_blocking=True)
+            binding.copy_blocks(cache.k_cache, cache.v_cache, d_pairs[:, 0], d_pairs[:, 1], stream=stream)
+            cache.append(d_k, d_v, d_slots, stream=stream)
+            cache.attention(out, d_q, d_tables, d_lens, w.scale, max_context_len=maxctx, partition_tokens=part,
+                            workspace=workspace, stream=stream)
+            h_out.copy_(out, non_blocking=True)
+            stream.synchronize()
+            return unique_attention_bytes(w, tables, lens, 2) + copy_bytes + append_bytes(w)
+
+        for i in range(W):
+            step_host(*hsteps[i])
+        barrier(ws)
+        torch.cuda.synchronize()
+        e0, e1 = evpair()
+        e0.record(stream)
+        for i in range(K):
+            e2e_bytes.append(step_host(*hsteps[W + i]))
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(ws)
+        assert binding.get_device_error() == 0
+        e_ms, e_gbs, e_tok = aggregate(e0.elapsed_time(e1), float(sum(e2e_bytes)), float(B * K), ws)
+        eb = w.in_bytes
+        h2d = (B * w.num_q_heads * w.head_dim * eb + 2 * B * w.num_kv_heads * w.head_dim * eb +
+               16 * len(pairs) + B * (8 + mb * 4 + 4))
+        e2e = {"value": round(e_gbs, 1), "unit": "GB/s", "decode_tokens_per_s": round(e_tok, 1),
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(B * w.num_q_heads * w.head_dim * 2),
+               "ms_per_step": round(e_ms / K, 4),
+               "path": "host block manager append, H2D of q / new K,V / copy list / slots / tables / lengths, "
+                       "copy_blocks, reshape_and_cache, paged_attention_decode, D2H of the output, stream sync "
+                       "(unique bytes)"}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_seconds)
+    return {
+        "metric": "paged decode attention achieved HBM GB/s (% of B200 peak); decode tokens/s",
+        "value": round(gbs, 1), "unit": "GB/s", "n_gpus": ws, "steps": K, "warmup": W,
+        "ms_per_step": round(ms_max / K, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.kv_dtype, "data": "synthetic",
+        "bytes_basis": "unique: each physical block's K/V once (the shared prefix once per step)",
+        "pct_of_peak": round(100 * gbs / ws / peak, 1), "pct_of_peak_spec": round(100 * gbs / ws / SPEC_HBM_GBS, 1),
+        "value_logical": round(gbs_logical, 1),
+        "decode_tokens_per_s": round(tokens_s, 1),
+        "bytes_per_step": {"attention_unique": int(au), "attention_logical": int(al), "copy_blocks": copy_bytes,
+                           "append": append_bytes(w), "copies": len(pairs), "block_bytes": block_bytes},
+        "l2_flushed": {"value": round(gbs_b, 1), "value_logical": round(gbs_b_logical, 1),
+                       "ms_per_step": round(msb_max / K, 4), "attention_achieved_unique": round(ach_b, 1),
+                       "attention_frac_unique": round(ach_b / peak, 4), "avg_attention_ms": round(ab, 5),
+                       "clocks": clocks_b.summary()},
+        "config": {"workload": w.description, "global_batch": B * ws, "seq_len": f"{p} shared + U[{w.lo},{w.hi}]",
+                   "block_size": bs, "schedule": f"partitions of {part_used} tokens" if part != -1 else "persistent",
+                   "step": f"copy_blocks of {len(pairs)} copy-on-write pairs (logical block {last}), "
+                           f"reshape_and_cache of {B} tokens, paged decode attention",
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                   "l2": "value: no flush between steps (the 16 MiB prefix stays in L2); l2_flushed: L2 flushed "
+                         "before every step (write of 2x L2 then read of another 2x L2), outside the events",
+                   "seed": w.seed},
+        "roofline": {"bound": "hbm", "kernel": "paged_decode_kernel (one attention call)",
+                     "achieved": round(ach, 1), "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
+                     "frac": round(ach / peak, 4), "frac_of_spec": round(ach / SPEC_HBM_GBS, 4),
+                     "achieved_logical": round(al / (aa * 1e-3) / 1e9, 1), "avg_launch_ms": round(aa, 5),
+                     "algorithmic_bytes_per_launch": int(au), "bytes_basis": "unique", "traffic": None},
+        "e2e": e2e,
+        "gpu_launches": (3 + (1 if (part_used > 0 and maxctx > part_used) else 0)) * K,
+        "clocks": clocks.summary(),
+        "cpu_baseline": cpu,
+    }
 
 
 def run_swap(args, ws, rank, local):
@@ -998,6 +1267,24 @@ def run_reference(args, ws, rank):
             "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def sub_result(workload: str, args) -> dict:
+    """The same decode-step measurement on another workload, run as a child
+    process on the same GPU (its own caches; no e2e, CPU baseline or paging
+    run), reduced to its throughput, roofline and clocks."""
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--workload", workload, "--steps", str(args.steps),
+           "--warmup", str(args.warmup), "--no-e2e", "--no-cpu-baseline", "--no-paging-overhead", "--no-extra"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=900)
+    lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
+    if r.returncode != 0 or not lines:
+        return {"workload": workload, "error": (r.stderr or r.stdout)[-500:]}
+    d = json.loads(lines[-1])
+    keep = ("value", "unit", "ms_per_step", "pct_of_peak", "pct_of_peak_spec", "decode_tokens_per_s", "roofline",
+            "clocks", "gpu_launches")
+    out = {"workload": d["config"]["workload"], "schedule": d["config"]["schedule"]}
+    out.update({k: d[k] for k in keep if k in d})
+    return out
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -1010,7 +1297,12 @@ def main():
     ws, rank, local = dist_init(args)
     try:
         run = {"swap": run_swap, "mq": run_mq, "fork": run_fork}.get(args.op, run_pkv)
+        if args.op == "decode" and wl.WORKLOADS[args.workload].ctx == "shared_prefix":
+            run = run_shared_prefix
         r = run(args, ws, rank, local)
+        if (rank == 0 and ws == 1 and args.op == "decode" and args.workload == "llama2_7b" and not args.no_extra
+                and not (args.num_seqs or args.num_blocks or args.block_size)):
+            r["gqa_70b"] = sub_result("gqa_70b", args)
         if rank == 0:
             print(json.dumps(r), flush=True)
     finally:

@@ -194,9 +194,15 @@ int pkv_paged_attention_partition_tokens(
  * nothing (use larger partition_tokens, fewer sequences per call, or the
  * regular entry point with your own workspace).
  *
- * Every call uses the same array and leaves its contents behind; nothing in it
- * needs to start at zero. Calls whose kernels overlap on the GPU (two streams,
- * two host threads) race on it: serialise them.
+ * Every call uses the same array and leaves its contents behind. The only part
+ * that must start at zero (the persistent schedule's arrival counters) is
+ * cleared by each call on `stream` before its kernel runs, so a previous call's
+ * leftovers do no harm. Calls whose kernels overlap on the GPU (two streams, two
+ * host threads) race on the array: serialise them.
+ *
+ * The device address is looked up once per device and kept for the life of the
+ * process. A device reset (cudaDeviceReset) may move the array, so this entry
+ * point must not be called after a device reset in the same process.
  */
 pkv_status pkv_paged_attention_decode_noalloc(
     void* out, pkv_dtype out_dtype,
@@ -337,6 +343,30 @@ pkv_status pkv_reshape_and_cache_fp8(
  * by a kernel). Synchronises `stream` first. `code` is a host pointer.
  */
 pkv_status pkv_get_device_error(int* code, void* stream);
+
+/*
+ * Test hook for the kernels' bounded waits (no counterpart on the pages; it
+ * exists so that a test can watch a wait give up without faulting the GPU).
+ * Arms a one-shot change of the NEXT launch of one kernel, made from any host
+ * thread:
+ *   kernel 0  the partitioned decode kernel of pkv_paged_attention_decode
+ *             (partition_tokens >= 0): in its first CTA the producer never issues
+ *             the copies of ring stage `index` (16 tokens, 32 for e4m3 caches) nor
+ *             arrives on that stage's barrier;
+ *   kernel 1  the tcgen05 multi-query kernel of pkv_paged_attention_multi_query
+ *             (from 32 query rows per KV head, head_dim 128): in its first CTA
+ *             the producer never issues the K copies of 128-token tile `index`.
+ * Every bounded wait of that launch then gives up after wait_limit_ns
+ * (100 us .. 2 s) instead of 2 s. No copy is left in flight: the withheld one is
+ * never issued and the rest are drained. The launch records
+ * PKV_ERR_DEVICE_TIMEOUT in the device error word (when the withheld stage is
+ * reached, i.e. the first CTA has more than `index` stages or tiles), leaves its
+ * output unspecified and releases everything it holds (shared memory, tensor
+ * memory), so the next call on the stream runs normally.
+ * index -1 disarms. Returns PKV_ERR_INVALID_ARG for another kernel id or a limit
+ * outside the range.
+ */
+pkv_status pkv_test_withhold_copy(int kernel, int index, unsigned long long wait_limit_ns);
 
 /* ------------------------------------------------------------------------- */
 /* One decode step from host buffers ([VP] §3.3 decode, §4.1 copy-on-write)  */

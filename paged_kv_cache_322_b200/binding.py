@@ -53,6 +53,7 @@ _SIGS = {
     "pkv_copy_blocks": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pkv_swap_blocks": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp]),
     "pkv_get_device_error": (_i32, [_c.POINTER(_c.c_int), _vp]),
+    "pkv_test_withhold_copy": (_i32, [_i32, _i32, _c.c_ulonglong]),
     "pkv_step_ctx_create": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _f32,
                                    _c.POINTER(_vp)]),
     "pkv_step_ctx_destroy": (None, [_vp]),
@@ -199,6 +200,7 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
 
 
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+SCHEDULE_PERSISTENT = -1          # partition_tokens value of the persistent schedule
 
 
 def paged_attention_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
@@ -384,6 +386,15 @@ def get_device_error(stream=None) -> int:
 # ---------------------------------------------------------------------------
 # host block manager
 # ---------------------------------------------------------------------------
+WITHHOLD_DECODE, WITHHOLD_MULTI_QUERY_TC = 0, 1
+
+
+def test_withhold_copy(kernel: int, index: int, wait_limit_ns: int):
+    """Test hook: the next launch of `kernel` withholds one copy in its first CTA
+    and gives every bounded wait `wait_limit_ns` (see pkv_test_withhold_copy)."""
+    _check(_lib().pkv_test_withhold_copy(kernel, index, wait_limit_ns), "pkv_test_withhold_copy")
+
+
 class BlockManager:
     """The library's C++ block manager (free list, tables, slots, refcounts, CoW)."""
 

@@ -46,6 +46,9 @@ struct Params {
     unsigned long long* counters;   // [B * Hkv]: (epoch << 24) | pieces arrived
     unsigned long long epoch;       // distinct per call
     int team_size;                  // CTAs per team (one KV head each), divides Hkv and the grid
+    // bounded waits
+    unsigned long long wait_ns;     // limit of every mbarrier wait (2 s unless the test hook shortened it)
+    int withhold;                   // test hook: ring stage whose copies the first CTA never issues (-1: none)
 };
 
 __device__ __forceinline__ void consumers_barrier() {

@@ -23,6 +23,10 @@ __device__ __forceinline__ void flag_error(int* err, int code) {
 
 // Device address of the current device's error word (status.cu).
 int* device_error_word();
+// Test hook state for the next launch of `kernel` (0: partitioned decode
+// kernel, 1: tcgen05 multi-query kernel): the copy to withhold (-1: none) and the
+// wait limit (kDefaultWaitNs unless armed). Clears what it hands out (status.cu).
+void take_wait_hook(int kernel, int* withhold, unsigned long long* wait_ns);
 // Maps a CUDA error to a status, remembering nothing.
 inline pkv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA; }
 
@@ -109,11 +113,16 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
+// Limit of a bounded wait inside a kernel (2 s of wall time).
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+
 // Bounded wait on an mbarrier phase. Gives up after ~`limit_ns` of wall time
-// (checked every 256 polls), records PKV_ERR_DEVICE_TIMEOUT and returns false.
+// (checked every 256 polls; 0 means the default limit), records
+// PKV_ERR_DEVICE_TIMEOUT and returns false.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err,
-                                                  uint64_t limit_ns = 2000000000ull) {
+                                                  uint64_t limit_ns = kDefaultWaitNs) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (limit_ns == 0) limit_ns = kDefaultWaitNs;
     uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;

@@ -11,8 +11,14 @@
 // The array costs PKV_NOALLOC_SCRATCH_BYTES on every GPU that loads this
 // library, for the life of the process. Calls share it: two calls that overlap
 // on the GPU (different streams, or different host threads) race on it.
-// The decode kernels write every scratch entry they later read, so nothing in
-// it has to start at zero and the previous call's contents do no harm.
+// The split-K kernels write every scratch entry they later read; the one part
+// that must start at zero, the persistent schedule's arrival counters, is
+// cleared on the stream by each call before its launch (a memset, which
+// allocates nothing). So the previous call's contents do no harm.
+//
+// The array's device address is looked up once per device and kept. A device
+// reset (cudaDeviceReset) unloads the module and may move the array, so no call
+// of this entry point may follow a device reset in the same process.
 #include <mutex>
 
 #include "common.cuh"

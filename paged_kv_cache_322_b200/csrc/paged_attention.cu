@@ -350,6 +350,9 @@ pkv_status decode_impl(void* out, pkv_dtype out_dtype, const void* q, const void
     p.part_blocks = pl.part_tokens / block_size;
     p.num_parts = pl.num_parts;
     p.num_seqs = num_seqs;
+    p.withhold = -1;
+    p.wait_ns = kDefaultWaitNs;
+    if (!pl.persistent) take_wait_hook(0, &p.withhold, &p.wait_ns);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (pl.persistent) {
         static std::atomic<unsigned long long> epoch{1};
@@ -359,6 +362,12 @@ pkv_status decode_impl(void* out, pkv_dtype out_dtype, const void* q, const void
             ((((size_t)2 * pl.grid * group * (head_dim + 2) * 4) + 255) & ~size_t(255)));
         p.epoch = epoch.fetch_add(1) & ((1ull << 40) - 1);
         p.team_size = pl.team_size;
+        // The arrival counters start at zero on every call. The epoch tag alone
+        // cannot tell a counter from other bytes a previous call (a split-K call
+        // sharing this workspace) left there, so they are cleared on the stream.
+        if (cudaMemsetAsync(p.counters, 0, (size_t)num_seqs * num_kv_heads * sizeof(unsigned long long), st) !=
+            cudaSuccess)
+            return PKV_ERR_CUDA;
         if (launch_persistent(bf16, use_mma, head_dim, group, mk, mv, p, pl.grid, st) != cudaSuccess)
             return PKV_ERR_CUDA;
         return PKV_OK;

@@ -111,8 +111,11 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         // ---------------- producer ----------------
         const uint64_t pol = l2_policy_evict_first();
         const int32_t* bt = p.block_tables + (int64_t)seq * p.max_blocks + blk0;
-        int issued = 0;
+        int issued = 0;                                             // stages claimed (copies issued)
         bool ok = true;
+        // test hook: the first CTA never issues this stage's copies (and never
+        // arrives on its barrier), so its consumer's bounded wait runs out
+        const int withheld = (blockIdx.x | blockIdx.y | blockIdx.z) == 0 ? p.withhold : -1;
         // 32 blocks' ids per coalesced load; each block gives PPB pieces, the
         // pieces past the partition's last token are not loaded.
         for (int q0 = 0; q0 < npiece && ok; q0 += 32 * K::PPB) {
@@ -138,19 +141,19 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 const int q = q0 + qs, si = q / K::BPS, st = si % STAGES;
                 const int nq = min(K::BPS, npiece - q);               // pieces in this stage
                 if (lane == 0) {
-                    if (!mbar_wait_bounded(&empty[st], ((si / STAGES) & 1) ^ 1, p.err)) {
+                    if (!mbar_wait_bounded(&empty[st], ((si / STAGES) & 1) ^ 1, p.err, p.wait_ns)) {
                         ok = false;
                         s_abort = 1;
                     } else {
-                        mbar_arrive_expect_tx(&full[st], nq * 2 * KPC * K::PIECE);
-                        ++issued;
+                        if (si != withheld) mbar_arrive_expect_tx(&full[st], nq * 2 * KPC * K::PIECE);
+                        issued = si + 1;
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;    // also orders the expect-tx first
                 if (!ok) break;
                 const int pq = qs + (b < nq ? b : 0);                // this lane's piece, chunk-relative
                 const int pb = __shfl_sync(0xffffffffu, id, pq / K::PPB);
-                if (b < nq) {
+                if (b < nq && si != withheld) {
                     uint8_t* dst = smem + st * K::STAGE_BYTES + (kv ? KPC + hd : hd) * K::REGION + K::piece_offset(b, h);
                     tma_load_4d(dst, kv ? &tm_v : &tm_k, &full[st], h * K::BOX, kvh + hd, (pq % K::PPB) * K::R, pb, pol);
                 }
@@ -159,7 +162,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         if (lane == 0 && !ok) {
             // Drain: wait (bounded) for every copy still in flight before the CTA exits.
             for (int j = max(0, issued - STAGES); j < issued; ++j)
-                mbar_wait_bounded(&full[j % STAGES], (j / STAGES) & 1, p.err);
+                if (j != withheld) mbar_wait_bounded(&full[j % STAGES], (j / STAGES) & 1, p.err, p.wait_ns);
         }
     } else {
         // ---------------- consumers ----------------
@@ -175,7 +178,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             c.init(reinterpret_cast<const __nv_bfloat16*>(qbase), group, lane);
             for (int j = sub; j < nstage; j += K::WPH) {
                 const int st = j % STAGES;
-                const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err);
+                const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err, p.wait_ns);
                 if (__any_sync(0xffffffffu, !got || s_abort != 0)) {   // warp-uniform exit
                     s_abort = 1;
                     break;
@@ -198,7 +201,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             const int jstart = PATH == 1 ? 0 : sub, jstep = PATH == 1 ? 1 : K::WPH;
             for (int j = jstart; j < nstage; j += jstep) {
                 const int st = j % STAGES;
-                const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err);
+                const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err, p.wait_ns);
                 if (__any_sync(0xffffffffu, !got || s_abort != 0)) {
                     s_abort = 1;
                     break;

@@ -54,6 +54,8 @@ struct MqParams {
     int max_blocks, num_blocks, ctx_cap, max_query_len;
     int block_size, part_blocks, num_parts, row_tiles;
     int wpr;                      // warps per row group: 1, 2 or 4
+    unsigned long long wait_ns;   // limit of every mbarrier wait (2 s unless the test hook shortened it)
+    int withhold;                 // test hook: KV tile whose K copies the first CTA never issues (-1: none)
 };
 
 // One normalised output value of row qh (sequence-level token row x head),
@@ -367,7 +369,7 @@ paged_mq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     const int q = q0p + qq, sub = qq % K::PPB;
                     const int si = q / K::BPS, b = q - si * K::BPS, st = si % STAGES;
                     if (b == 0) {
-                        if (!mbar_wait_bounded(&empty[st], ((si / STAGES) & 1) ^ 1, p.err)) {
+                        if (!mbar_wait_bounded(&empty[st], ((si / STAGES) & 1) ^ 1, p.err, p.wait_ns)) {
                             ok = false;
                             s_abort = 1;
                         } else {
@@ -392,7 +394,7 @@ paged_mq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         if (lane == 0 && !ok) {
             for (int j = max(0, issued - STAGES); j < issued; ++j)
-                mbar_wait_bounded(&full[j % STAGES], (j / STAGES) & 1, p.err);
+                mbar_wait_bounded(&full[j % STAGES], (j / STAGES) & 1, p.err, p.wait_ns);
         }
     } else {
         // ---------------- consumers: row group rg, turn sub of its wpr warps ----------------
@@ -406,7 +408,7 @@ paged_mq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         // warp of each group, so no warp can run a ring phase ahead of the producer.
         for (int j = sub; j < nstage; j += wpr) {
             const int st = j % STAGES;
-            const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err);
+            const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err, p.wait_ns);
             if (__any_sync(0xffffffffu, !got || s_abort != 0)) {
                 s_abort = 1;
                 break;
@@ -731,6 +733,9 @@ pkv_status pkv_paged_attention_multi_query(void* out, pkv_dtype out_dtype, const
     p.num_parts = pl.num_parts;
     p.row_tiles = pl.row_tiles;
     p.wpr = pl.wpr;
+    p.withhold = -1;
+    p.wait_ns = kDefaultWaitNs;
+    if (pl.tc) take_wait_hook(1, &p.withhold, &p.wait_ns);
     if (need > 0) {
         const size_t rows = (size_t)num_tokens * num_q_heads * pl.num_parts;
         p.ws_o = static_cast<float*>(workspace);

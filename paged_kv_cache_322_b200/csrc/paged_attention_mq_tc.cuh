@@ -35,7 +35,7 @@ constexpr int Q_OFF = 0;
 constexpr int K_OFF = 2 * HALF;                   // NST stages of K (2 halves each)
 constexpr int V_OFF = K_OFF + NST * 2 * HALF;     // NST stages of V
 constexpr int BAR_OFF = V_OFF + NST * 2 * HALF;
-constexpr int NBAR = 20;
+constexpr int NBAR = 21;
 constexpr int SMEM = 1024 + BAR_OFF + NBAR * 8 + 16;
 constexpr int TMEM_COLS = 512;     // S/P 0 [0,128) S/P 1 [128,256) O [256,384) exchange [384,390)
 constexpr int T_O = 256;
@@ -44,10 +44,14 @@ constexpr int T_O = 256;
 // S of tile t + 2 is issued after the PV product that reads P of tile t.
 static_assert(SMEM <= 232448, "shared memory per CTA");
 
-// Barrier indices.
+// Barrier indices. P-ready is one barrier per tile parity: S of tile t + 1 is
+// issued before the MMA thread waits for P of tile t, so the softmax may finish
+// tiles t and t + 1 before that wait; on a single barrier that would put the
+// phase two ahead of the waiter, where a parity wait cannot tell it apart.
+// Tile t + 2 cannot arrive before that wait (its S is issued after PV of t).
 enum {
     B_Q = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_MAX = 15, B_FIN = 16,
-    B_PREADY = 17, B_ODONE = 18, B_DRAIN = 19
+    B_PREADY = 17, B_ODONE = 19, B_DRAIN = 20
 };
 
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -184,7 +188,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int s = 0; s < 2; ++s) mbar_init(&bar[B_SFULL + s], 1);
         mbar_init(&bar[B_MAX], 256);
         mbar_init(&bar[B_FIN], 256);
-        mbar_init(&bar[B_PREADY], 256);
+        for (int s = 0; s < 2; ++s) mbar_init(&bar[B_PREADY + s], 256);
         mbar_init(&bar[B_ODONE], 1);
         mbar_init(&bar[B_DRAIN], 1);
         s_abort = 0;
@@ -213,6 +217,9 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // released as soon as S is computed, V only after the PV product.
         bool ok = true;
         int issued[2] = {0, 0};                                 // tiles whose K / V copies were issued
+        // test hook: the first CTA never issues this tile's K copies (nor arrives
+        // on their barrier), so the MMA thread's bounded wait for them runs out
+        const int withheld = (blockIdx.x | blockIdx.y | blockIdx.z) == 0 ? p.withhold : -1;
         if (lane == 0) {
             mbar_arrive_expect_tx(&bar[B_Q], 2 * HALF);
             for (int h = 0; h < 2; ++h)
@@ -237,11 +244,12 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
             for (int kv = 0; kv < 2; ++kv) {
                 uint64_t* full = &bar[(kv ? B_VFULL : B_KFULL) + s];
+                const bool skip = kv == 0 && t == withheld;
                 if (lane == 0) {
-                    ok = mbar_wait_bounded(&bar[(kv ? B_VEMPTY : B_KEMPTY) + s], par, p.err);
+                    ok = mbar_wait_bounded(&bar[(kv ? B_VEMPTY : B_KEMPTY) + s], par, p.err, p.wait_ns);
                     if (ok) {
-                        mbar_arrive_expect_tx(full, np * 2 * R * 128);
-                        ++issued[kv];
+                        if (!skip) mbar_arrive_expect_tx(full, np * 2 * R * 128);
+                        issued[kv] = t + 1;
                     } else {
                         s_abort = 1;
                     }
@@ -252,7 +260,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // was the bound (measured: a tile of 16-token blocks takes 32 copies)
                 uint8_t* dst = smem + (kv ? V_OFF : K_OFF) + s * 2 * HALF;
                 const CUtensorMap* map = kv ? &tm_v : &tm_k;
-                if (lane < np) {
+                if (lane < np && !skip) {
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
                         tma_load_4d(dst + h * HALF + lane * R * 128, map, full, h * 64, kvh, 0, id, pol);
@@ -264,7 +272,8 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // every copy issued has landed before the CTA moves on
             for (int kv = 0; kv < 2; ++kv)
                 for (int t = max(0, issued[kv] - NST); t < issued[kv]; ++t)
-                    mbar_wait_bounded(&bar[(kv ? B_VFULL : B_KFULL) + t % NST], (t / NST) & 1, p.err);
+                    if (kv != 0 || t != withheld)
+                        mbar_wait_bounded(&bar[(kv ? B_VFULL : B_KFULL) + t % NST], (t / NST) & 1, p.err, p.wait_ns);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer (one thread) ----------------
@@ -272,11 +281,11 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             constexpr uint32_t IDESC_S = idesc_bf16(ROWS, TOK, false);
             constexpr uint32_t IDESC_PV = idesc_bf16(ROWS, D, true);
             const uint32_t q_addr = smem_u32(smem + Q_OFF);
-            bool ok = mbar_wait_bounded(&bar[B_Q], 0, p.err);
+            bool ok = mbar_wait_bounded(&bar[B_Q], 0, p.err, p.wait_ns);
             // PV of tile u: O += P_hi V + P_lo V over the tile's 128 tokens, 8 k-steps of 16
             auto pv = [&](int u) -> bool {
-                if (!mbar_wait_bounded(&bar[B_PREADY], u & 1, p.err)) return false;
-                if (!mbar_wait_bounded(&bar[B_VFULL + u % NST], (u / NST) & 1, p.err)) return false;
+                if (!mbar_wait_bounded(&bar[B_PREADY + (u & 1)], (u >> 1) & 1, p.err, p.wait_ns)) return false;
+                if (!mbar_wait_bounded(&bar[B_VFULL + u % NST], (u / NST) & 1, p.err, p.wait_ns)) return false;
                 fence_after();
                 const uint32_t v_addr = smem_u32(smem + V_OFF + (u % NST) * 2 * HALF);
 #pragma unroll
@@ -297,7 +306,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const int sb = t & 1, ks = t % NST;
                 // S of tile t goes into the buffer of tile t - 2, whose P the PV product
                 // issued in the previous iteration reads first (MMAs run in issue order)
-                ok = mbar_wait_bounded(&bar[B_KFULL + ks], (t / NST) & 1, p.err);
+                ok = mbar_wait_bounded(&bar[B_KFULL + ks], (t / NST) & 1, p.err, p.wait_ns);
                 if (!ok) break;
                 fence_after();
                 const uint32_t k_addr = smem_u32(smem + K_OFF + ks * 2 * HALF);
@@ -315,7 +324,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (!ok) s_abort = 1;
             // every MMA issued has finished before TMEM is released
             commit(&bar[B_DRAIN]);
-            mbar_wait_bounded(&bar[B_DRAIN], 0, p.err);
+            mbar_wait_bounded(&bar[B_DRAIN], 0, p.err, p.wait_ns);
         }
     } else {
         // ---------------- softmax: two threads per query row ----------------
@@ -335,7 +344,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         bool ok = true;
         for (int t = 0; t < ntiles; ++t) {
             const int s = t & 1;
-            const bool got = mbar_wait_bounded(&bar[B_SFULL + s], (t >> 1) & 1, p.err);
+            const bool got = mbar_wait_bounded(&bar[B_SFULL + s], (t >> 1) & 1, p.err, p.wait_ns);
             if (__any_sync(0xffffffffu, !got || s_abort != 0)) {
                 ok = false;
                 s_abort = 1;
@@ -373,7 +382,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 tmem_wait_st();
                 fence_before();
                 mbar_arrive(&bar[B_MAX]);
-                const bool ex = mbar_wait_bounded(&bar[B_MAX], t & 1, p.err);
+                const bool ex = mbar_wait_bounded(&bar[B_MAX], t & 1, p.err, p.wait_ns);
                 if (__any_sync(0xffffffffu, !ex || s_abort != 0)) {
                     ok = false;
                     s_abort = 1;
@@ -392,7 +401,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // the dims) before the PV product.
             const int tok_here = min(TOK, ntok - t * TOK);
             if (lr >= tok_here) {
-                const bool vin = mbar_wait_bounded(&bar[B_VFULL + t % NST], (t / NST) & 1, p.err);
+                const bool vin = mbar_wait_bounded(&bar[B_VFULL + t % NST], (t / NST) & 1, p.err, p.wait_ns);
                 if (vin) {
                     uint8_t* vrow = smem + V_OFF + (t % NST) * 2 * HALF + half * HALF + lr * 128;
 #pragma unroll
@@ -418,7 +427,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // covers every earlier MMA), so O-done is at most one phase behind and
             // its parity wait is exact. Each half rescales its 64 columns of O.
             if (t > 0 && __any_sync(0xffffffffu, grow && m_ref != kNegInf)) {
-                const bool done = mbar_wait_bounded(&bar[B_ODONE], (t - 1) & 1, p.err);
+                const bool done = mbar_wait_bounded(&bar[B_ODONE], (t - 1) & 1, p.err, p.wait_ns);
                 if (__any_sync(0xffffffffu, !done || s_abort != 0)) {
                     ok = false;
                     s_abort = 1;
@@ -446,7 +455,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             tmem_st32u(lane_base + s * 128 + 64 + half * 32, pl);
             tmem_wait_st();
             fence_before();
-            mbar_arrive(&bar[B_PREADY]);
+            mbar_arrive(&bar[B_PREADY + s]);
         }
         // the last PV, then the row sum of both halves, then this half of the row's
         // output (or of the partition's partial)
@@ -454,7 +463,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // O-done may be two phases behind here, where a parity wait cannot tell
             // them apart: wait for the single-use drain barrier the MMA thread
             // commits after its last MMA instead
-            const bool done = mbar_wait_bounded(&bar[B_DRAIN], 0, p.err);
+            const bool done = mbar_wait_bounded(&bar[B_DRAIN], 0, p.err, p.wait_ns);
             ok = !__any_sync(0xffffffffu, !done || s_abort != 0);
         }
         if (ok) {
@@ -464,7 +473,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             tmem_wait_st();
             fence_before();
             mbar_arrive(&bar[B_FIN]);
-            const bool fin = mbar_wait_bounded(&bar[B_FIN], 0, p.err);
+            const bool fin = mbar_wait_bounded(&bar[B_FIN], 0, p.err, p.wait_ns);
             ok = !__any_sync(0xffffffffu, !fin || s_abort != 0);
             if (ok) {
                 fence_after();

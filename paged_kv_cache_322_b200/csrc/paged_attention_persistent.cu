@@ -22,8 +22,9 @@
 //     the workspace and bumps the item's counter; the CTA that brings the count
 //     to the number of pieces merges all pieces (log-sum-exp) and writes the
 //     output. No second kernel, no spin-wait on another CTA.
-//   * Counters carry an epoch that is new on every call, so the workspace needs
-//     no zeroing: a stale counter from an older call reads as zero.
+//   * The host clears the counters on the stream before each launch (B * Hkv
+//     words of the workspace), so a counter never starts from bytes an earlier
+//     call left behind; each also carries an epoch that is new on every call.
 #include <atomic>
 
 #include "attention_common.cuh"
@@ -201,7 +202,7 @@ paged_decode_persistent_kernel(const __grid_constant__ CUtensorMap tm_k, const _
         while (wk.next(prefix, ctxs, ts, member, sg)) {
             if (lane == 0 && !s_abort) {
                 const int qs = k % kQStages;
-                if (!mbar_wait_bounded(&qempty[qs], ((k / kQStages) & 1) ^ 1, p.err)) {
+                if (!mbar_wait_bounded(&qempty[qs], ((k / kQStages) & 1) ^ 1, p.err, p.wait_ns)) {
                     s_abort = 1;
                 } else {
                     mbar_arrive_expect_tx(&qfull[qs], qbytes);
@@ -225,7 +226,7 @@ paged_decode_persistent_kernel(const __grid_constant__ CUtensorMap tm_k, const _
                     const int pb = __shfl_sync(0xffffffffu, id, jj);
                     if (lane == 0 && !s_abort) {
                         const int st = (int)(i % STAGES);
-                        if (!mbar_wait_bounded(&empty[st], (uint32_t)((i / STAGES) & 1) ^ 1u, p.err)) {
+                        if (!mbar_wait_bounded(&empty[st], (uint32_t)((i / STAGES) & 1) ^ 1u, p.err, p.wait_ns)) {
                             s_abort = 1;
                         } else {
                             mbar_arrive_expect_tx(&full[st], K::STAGE_BYTES);
@@ -264,7 +265,7 @@ paged_decode_persistent_kernel(const __grid_constant__ CUtensorMap tm_k, const _
         while (wk.next(prefix, ctxs, ts, member, sg)) {
             const int qs = k % kQStages;
             const long long iend = i + (sg.j1 - sg.j0);
-            bool ok = !s_abort && mbar_wait_bounded(&qfull[qs], (uint32_t)((k / kQStages) & 1), p.err);
+            bool ok = !s_abort && mbar_wait_bounded(&qfull[qs], (uint32_t)((k / kQStages) & 1), p.err, p.wait_ns);
             if (__any_sync(0xffffffffu, !ok)) { s_abort = 1; ok = false; }
             const T* qrows = reinterpret_cast<const T*>(qbuf + qs * K::QBYTES);
             const int slot = PATH == 1 ? 0 : cw;
@@ -274,7 +275,7 @@ paged_decode_persistent_kernel(const __grid_constant__ CUtensorMap tm_k, const _
                 const long long first = i + ((cw - (int)(i % NCW)) + NCW) % NCW;
                 for (long long ii = first; ii < iend && ok; ii += NCW) {
                     const int st = (int)(ii % STAGES);
-                    const bool got = !s_abort && mbar_wait_bounded(&full[st], (uint32_t)((ii / STAGES) & 1), p.err);
+                    const bool got = !s_abort && mbar_wait_bounded(&full[st], (uint32_t)((ii / STAGES) & 1), p.err, p.wait_ns);
                     if (__any_sync(0xffffffffu, !got)) { s_abort = 1; ok = false; break; }
                     uint8_t* stage = ring + st * K::STAGE_BYTES;
                     const int j = sg.j0 + (int)(ii - i);
@@ -294,7 +295,7 @@ paged_decode_persistent_kernel(const __grid_constant__ CUtensorMap tm_k, const _
                 const int step = PATH == 1 ? 1 : NCW;
                 for (long long ii = first; ii < iend && ok; ii += step) {
                     const int st = (int)(ii % STAGES);
-                    const bool got = !s_abort && mbar_wait_bounded(&full[st], (uint32_t)((ii / STAGES) & 1), p.err);
+                    const bool got = !s_abort && mbar_wait_bounded(&full[st], (uint32_t)((ii / STAGES) & 1), p.err, p.wait_ns);
                     if (__any_sync(0xffffffffu, !got)) { s_abort = 1; ok = false; break; }
                     const uint8_t* stage = ring + st * K::STAGE_BYTES;
                     const int j = sg.j0 + (int)(ii - i);

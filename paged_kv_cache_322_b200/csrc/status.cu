@@ -38,9 +38,38 @@ int* device_error_word() {
     return p;
 }
 
+// One-shot test hook: the next launch of the named kernel withholds one copy in
+// its first CTA and uses a short wait limit (pkv_test_withhold_copy).
+namespace {
+std::mutex g_hook_mutex;
+int g_hook_index[2] = {-1, -1};
+unsigned long long g_hook_wait_ns[2] = {0, 0};
+}  // namespace
+
+void take_wait_hook(int kernel, int* withhold, unsigned long long* wait_ns) {
+    *withhold = -1;
+    *wait_ns = kDefaultWaitNs;
+    std::lock_guard<std::mutex> lock(g_hook_mutex);
+    if (g_hook_index[kernel] >= 0) {
+        *withhold = g_hook_index[kernel];
+        *wait_ns = g_hook_wait_ns[kernel];
+        g_hook_index[kernel] = -1;
+    }
+}
+
 }  // namespace pkv
 
 extern "C" {
+
+pkv_status pkv_test_withhold_copy(int kernel, int index, unsigned long long wait_limit_ns) {
+    if (kernel != 0 && kernel != 1) return PKV_ERR_INVALID_ARG;
+    if (index < -1 || (index >= 0 && (wait_limit_ns < 100000ull || wait_limit_ns > pkv::kDefaultWaitNs)))
+        return PKV_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(pkv::g_hook_mutex);
+    pkv::g_hook_index[kernel] = index;
+    pkv::g_hook_wait_ns[kernel] = index >= 0 ? wait_limit_ns : 0;
+    return PKV_OK;
+}
 
 const char* pkv_status_string(int status) {
     switch (status) {

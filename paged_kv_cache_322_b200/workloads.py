@@ -74,6 +74,10 @@ WORKLOADS = {
     "llama2_7b": Workload(
         "llama2_7b", 64, 32, 32, 128, 16, 16384, "bf16", "uniform", lo=512, hi=2048, seed=1001,
         description="Llama-2-7B-shaped decode: B=64, 32/32 heads, D=128, bf16, bs=16, ctx U[512,2048], 16384-block pool"),
+    "llama2_13b": Workload(
+        "llama2_13b", 64, 40, 40, 128, 16, 16384, "bf16", "uniform", lo=512, hi=2048, seed=1005,
+        description="Llama-2-13B-shaped decode: B=64, 40/40 heads, D=128, bf16, bs=16, ctx U[512,2048], "
+                    "16384-block pool"),
     "gqa_70b": Workload(
         "gqa_70b", 128, 64, 8, 128, 16, 65536, "bf16", "uniform", lo=1024, hi=4096, seed=1002,
         description="70B-shaped GQA decode: B=128, 64/8 heads, D=128, bf16, bs=16, ctx U[1024,4096], 65536-block pool"),

@@ -483,3 +483,17 @@ def test_binding_requires_one_current_device(monkeypatch):
         binding._cuda_contig(T(1), T(1, cuda=False))
     with pytest.raises(ValueError, match="contiguous"):
         binding._cuda_contig(T(1, contig=False))
+
+
+def test_wait_hook_checks_its_arguments_on_host(lib):
+    """pkv_test_withhold_copy (test hook for the bounded waits): known kernel ids
+    only, a limit in [100 us, 2 s] when arming, -1 disarms without a limit."""
+    f = lib.pkv_test_withhold_copy
+    assert f(2, 0, 5_000_000) == 1
+    assert f(-1, 0, 5_000_000) == 1
+    assert f(0, 3, 10) == 1                      # limit too short
+    assert f(1, 3, 3_000_000_000) == 1           # longer than the default limit
+    assert f(0, -2, 5_000_000) == 1
+    assert f(0, 3, 5_000_000) == 0               # armed ...
+    assert f(0, -1, 0) == 0                      # ... and disarmed
+    assert f(1, -1, 0) == 0

@@ -38,6 +38,7 @@ def check_bf16_out(got_bf16: torch.Tensor, ref: np.ndarray):
 SMALL = {
     "tiny_fp32": wl.WORKLOADS["tiny_fp32"],
     "llama2_7b": dataclasses.replace(wl.WORKLOADS["llama2_7b"], num_seqs=6, num_blocks=2048),
+    "llama2_13b": dataclasses.replace(wl.WORKLOADS["llama2_13b"], num_seqs=4, num_blocks=1024),
     "gqa_70b": dataclasses.replace(wl.WORKLOADS["gqa_70b"], num_seqs=5, num_blocks=4096),
     "long_splitk": dataclasses.replace(wl.WORKLOADS["long_splitk"], num_seqs=6, num_blocks=12288),
 }

@@ -11,7 +11,8 @@ from tests.paged_problem import OracleProblem, gpu_problem, step_inputs, toleran
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("name,part", [("llama2_7b", 0), ("gqa_70b", 0), ("shared_prefix", 0), ("long_splitk", 512),
+@pytest.mark.parametrize("name,part", [("llama2_7b", 0), ("llama2_13b", 0), ("gqa_70b", 0), ("shared_prefix", 0),
+                                       ("long_splitk", 512),
                                        ("long_splitk", -1), ("llama2_7b", -1), ("gqa_70b", -1)])
 def test_full_size_sampled_against_oracle(name, part):
     """part 0: library-chosen partitions; 512: fixed 512-token partitions;

@@ -74,7 +74,7 @@ CASES = {
 
 @pytest.mark.parametrize("case", list(CASES))
 @pytest.mark.parametrize("hq,hkv,d", [(4, 4, 128), (8, 2, 128), (16, 2, 64), (8, 2, 64), (16, 4, 128)])
-@pytest.mark.parametrize("bs", [8, 16, 64])
+@pytest.mark.parametrize("bs", [8, 16, 32, 64])
 @pytest.mark.parametrize("part", [0, 64, 256])
 def test_multi_query_matches_oracle(case, hq, hkv, d, bs, part):
     ctxs, ns = CASES[case]
@@ -203,7 +203,7 @@ def test_full_size_chunk_sampled():
 
 
 @pytest.mark.parametrize("part", [0, 512])
-@pytest.mark.parametrize("bs", [16, 64])
+@pytest.mark.parametrize("bs", [16, 32, 64])
 def test_gqa_verify_rows_padded_into_tensor_memory_tiles(part, bs):
     """Group 8, five draft tokens: 40 query rows per KV head, run on 128-row
     tcgen05 tiles whose other 88 rows are idle."""
@@ -213,3 +213,17 @@ def test_gqa_verify_rows_padded_into_tensor_memory_tiles(part, bs):
     torch.cuda.synchronize()
     assert binding.get_device_error() == 0
     assert np.abs(out.cpu().numpy().astype(np.float64) - ref).max() <= 2e-3
+
+
+@pytest.mark.parametrize("bs", [8, 16, 32, 64])
+def test_both_kernels_at_every_block_size(bs):
+    """The same sequences through the mma.sync kernel (4 query tokens x group 4 =
+    16 rows per KV head) and the tcgen05 kernel (64 tokens x group 4 = 256 rows),
+    at each block size, against the oracle."""
+    ctxs = [129, 1000, 33]
+    for ns in ([4, 4, 4], [64, 64, 33]):
+        dev, ref = _mq_problem(40 + bs + ns[0], 16, 4, 128, bs, ctxs, ns)
+        out = _run(dev)
+        torch.cuda.synchronize()
+        assert binding.get_device_error() == 0
+        assert np.abs(out.cpu().numpy().astype(np.float64) - ref).max() <= 2e-3

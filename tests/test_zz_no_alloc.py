@@ -19,6 +19,8 @@ from paged_kv_cache_322_b200 import binding
 pytestmark = pytest.mark.gpu
 
 TOL = 2e-3      # the bf16-input attention tolerance used by the parity tests
+# Both entry points run the same kernels on the same inputs, so their outputs
+# are compared for bit equality (a tolerance would hide a scratch-reuse bug).
 
 
 def _problem(seed=21, hq=32, hkv=8, d=128, lens=(3000, 4097, 17, 8191, 1, 600)):
@@ -54,7 +56,33 @@ def test_noalloc_matches_regular_entry_point_twice(part):
         torch.cuda.synchronize()
         assert binding.get_device_error() == 0
         assert torch.isfinite(out).all()
-        assert (out - ref).abs().max().item() <= TOL
+        assert torch.equal(out, ref)
+
+
+def test_noalloc_persistent_schedule_after_split_k_leftovers():
+    """The persistent schedule keeps arrival counters in the scratch array. A
+    128-token split-K call first fills the array with partial outputs; the
+    persistent call that follows must not read them as counters. Two persistent
+    calls in a row, each bit-equal to the regular entry point with its own
+    workspace, and within the tolerance of the split-K result."""
+    q, kc, vc, tables, ctx, scale, maxlen = _problem(seed=22)
+    split = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    binding.paged_attention_decode_noalloc(split, q, kc, vc, tables, ctx, scale, max_context_len=maxlen,
+                                           partition_tokens=128)
+    need = binding.workspace_bytes(q.shape[0], q.shape[1], kc.shape[2], q.shape[2], 16, tables.shape[1], maxlen,
+                                   binding.SCHEDULE_PERSISTENT)
+    assert 0 < need <= binding.NOALLOC_SCRATCH_BYTES
+    ref = torch.empty_like(split)
+    binding.paged_attention_decode(ref, q, kc, vc, tables, ctx, scale, max_context_len=maxlen,
+                                   partition_tokens=binding.SCHEDULE_PERSISTENT)
+    for _ in range(2):
+        out = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
+        binding.paged_attention_decode_noalloc(out, q, kc, vc, tables, ctx, scale, max_context_len=maxlen,
+                                               partition_tokens=binding.SCHEDULE_PERSISTENT)
+        torch.cuda.synchronize()
+        assert binding.get_device_error() == 0
+        assert torch.equal(out, ref)
+    assert (ref - split).abs().max().item() <= TOL
 
 
 def test_noalloc_without_split_needs_no_scratch():
@@ -65,7 +93,7 @@ def test_noalloc_without_split_needs_no_scratch():
     binding.paged_attention_decode_noalloc(out, q, kc, vc, tables, ctx, scale, max_context_len=maxlen,
                                            partition_tokens=512)
     torch.cuda.synchronize()
-    assert (out - ref).abs().max().item() <= TOL
+    assert torch.equal(out, ref)
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
