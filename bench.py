@@ -49,6 +49,7 @@ sys.path.insert(0, ROOT)
 from paged_kv_cache_322_b200 import workloads as wl  # noqa: E402
 
 L2_BYTES = 126 * 2 ** 20
+BREAKDOWN_STEPS = 20           # e2e steps run again with the native step's phase timing on
 SPEC_HBM_GBS = 8000.0          # B200 HBM3e, the spec sheet's 8 TB/s (the measured copy peak is the other denominator)
 
 
@@ -317,7 +318,7 @@ def run_pkv(args, ws, rank, local):
     w = replica_workload(w, rank)
     part = w.partition_tokens if args.partition_tokens == -2 else args.partition_tokens
     K, W = args.steps, args.warmup
-    total_steps = 2 * (K + W) + 2
+    total_steps = 2 * (K + W) + 2 + BREAKDOWN_STEPS
     lens0 = wl.context_lens(w)
     dt = torch.float32 if w.kv_dtype == "f32" else torch.bfloat16       # q and the appended K/V
     cdt = torch.uint8 if w.kv_dtype == "fp8" else dt                     # cache storage
@@ -438,6 +439,24 @@ def run_pkv(args, ws, rank, local):
                "decode_tokens_per_s": round(e_tok, 1),
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e_ms / K, 4),
                "path": "pkv_decode_step (C ABI, host buffers): block manager, H2D, kernels, D2H, stream sync"}
+        # where the end-to-end step's time goes: the same steps again with the
+        # context's phase timing on (host clock + events), medians, after the timed loop
+        native.set_timing(True)
+        phases = []
+        for i in range(BREAKDOWN_STEPS):
+            t_w = time.perf_counter()
+            native(ids, *host[i % len(host)], out_host, w.scale, stream=stream)
+            stream.synchronize()
+            ph = native.last_timing()
+            ph["wall"] = (time.perf_counter() - t_w) * 1e3
+            phases.append(ph)
+        native.set_timing(False)
+        bd = {k: round(statistics.median(x[k] for x in phases), 4) for k in phases[0]}
+        bd["other"] = round(bd["wall"] - bd["host_block_manager"] - bd["h2d"] - bd["kernels"] - bd["d2h"], 4)
+        bd["what"] = ("medians over %d steps, ms: host block manager (host clock), H2D, kernels, D2H (events on the "
+                      "stream); wall = the Python call + stream sync; other = wall minus the four (API, launch and "
+                      "sync latency)" % BREAKDOWN_STEPS)
+        e2e["breakdown_ms"] = bd
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -649,12 +668,14 @@ def run_shared_prefix(args, ws, rank, local):
             q = wl.decode_q(w, 1000 + i)
             kn, vn = wl.decode_kv(w, 1000 + i)
             hsteps.append(tuple(torch.from_numpy(x).to(dt).pin_memory() for x in (q, kn, vn)))
-        h_pairs = torch.from_numpy(pa.copy()).pin_memory()
+        h_src = torch.from_numpy(pa[:, 0].copy()).pin_memory()
+        h_dst = torch.from_numpy(pa[:, 1].copy()).pin_memory()
         h_out = torch.empty((B, w.num_q_heads, w.head_dim), dtype=torch.bfloat16).pin_memory()
         d_q = torch.empty((B, w.num_q_heads, w.head_dim), dtype=dt, device=dev)
         d_k = torch.empty((B, w.num_kv_heads, w.head_dim), dtype=dt, device=dev)
         d_v = torch.empty_like(d_k)
-        d_pairs = torch.empty((len(pairs), 2), dtype=torch.int64, device=dev)
+        d_src = torch.empty(len(pairs), dtype=torch.int64, device=dev)
+        d_dst = torch.empty(len(pairs), dtype=torch.int64, device=dev)
         h_slots = torch.empty(B, dtype=torch.int64).pin_memory()
         h_tables = torch.empty((B, mb), dtype=torch.int32).pin_memory()
         h_lens = torch.empty(B, dtype=torch.int32).pin_memory()
@@ -669,10 +690,10 @@ def run_shared_prefix(args, ws, rank, local):
             h_slots.numpy()[:] = slots
             h_tables.numpy()[:] = tables
             h_lens.numpy()[:] = lens
-            for d, h in ((d_q, hq), (d_k, hk), (d_v, hv), (d_pairs, h_pairs), (d_slots, h_slots),
+            for d, h in ((d_q, hq), (d_k, hk), (d_v, hv), (d_src, h_src), (d_dst, h_dst), (d_slots, h_slots),
                          (d_tables, h_tables), (d_lens, h_lens)):
                 d.copy_(h, non_blocking=True)
-            binding.copy_blocks(cache.k_cache, cache.v_cache, d_pairs[:, 0], d_pairs[:, 1], stream=stream)
+            binding.copy_blocks(cache.k_cache, cache.v_cache, d_src, d_dst, stream=stream)
             cache.append(d_k, d_v, d_slots, stream=stream)
             cache.attention(out, d_q, d_tables, d_lens, w.scale, max_context_len=maxctx, partition_tokens=part,
                             workspace=workspace, stream=stream)

@@ -45,7 +45,9 @@
  *   - Supported: head_dim 64 or 128; block_size 8, 16, 32 or 64 ("vLLM
  *     PagedAttention 深度解析" §8.1 names powers of two with 16 the default;
  *     the persistent schedule takes 16 only); num_q_heads a multiple of
- *     num_kv_heads with group size num_q_heads/num_kv_heads in {1, 2, 4, 8};
+ *     num_kv_heads with group size num_q_heads/num_kv_heads in {1, 2, 4, 8, 16}
+ *     (other groups return PKV_ERR_UNSUPPORTED; the persistent schedule takes
+ *     groups up to 8);
  *     kv dtype f32 or bf16 (q has the kv dtype). Query head h reads KV head
  *     h / group (a reading: the pages do not discuss grouped-query attention).
  *   - Errors detected on the host (bad sizes, null pointers, unsupported shapes,
@@ -304,7 +306,7 @@ pkv_status pkv_swap_blocks(
  *   partition_tokens  > 0 fixed KV partitions, 0 chosen from the shapes (no
  *                  persistent schedule); the workspace is sized by
  *                  pkv_paged_attention_multi_query_workspace_bytes.
- * Supported: bf16 caches, head_dim 64 or 128, groups 1, 2, 4, 8, block sizes 8-64
+ * Supported: bf16 caches, head_dim 64 or 128, groups 1, 2, 4, 8, 16, block sizes 8-64
  * (PKV_ERR_UNSUPPORTED otherwise). A sequence whose n_s, c_s or rows break the
  * rules above (n_s > c_s, n_s > max_query_len, c_s above the capacity, rows
  * outside q) is skipped and flagged PKV_ERR_DEVICE_BOUNDS in the device word; its
@@ -410,6 +412,20 @@ pkv_status pkv_decode_step(pkv_step_ctx* ctx, pkv_block_manager* bm, const int64
                            const void* q_host, const void* k_host, const void* v_host,
                            void* k_cache, void* v_cache, int num_blocks, float scale,
                            int partition_tokens, void* out_host, void* stream);
+
+/*
+ * Phase timing of the steps of a context (off by default; a measurement aid,
+ * not part of the method). When enabled, each pkv_decode_step records the host
+ * time of its block-manager work and CUDA events around its H2D copies, its
+ * kernels and its D2H copy on the step's stream; pkv_step_ctx_last_timing waits
+ * for the last timed step's D2H and writes, in milliseconds,
+ *   out[0] host: block-manager append + block tables (host clock),
+ *   out[1] H2D copies (metadata, q, new K and V), out[2] kernels (copy_blocks,
+ *   KV append, attention), out[3] D2H copy of the output (device events).
+ * PKV_ERR_INVALID_ARG if no step ran with timing enabled since it was enabled.
+ */
+pkv_status pkv_step_ctx_set_timing(pkv_step_ctx* ctx, int enable);
+pkv_status pkv_step_ctx_last_timing(pkv_step_ctx* ctx, float* out);
 
 /* ------------------------------------------------------------------------- */
 /* Host block manager ([ENG] §2.3; [VP] §3.3, §4.1, §4.2; [BT])              */

@@ -57,6 +57,8 @@ _SIGS = {
     "pkv_step_ctx_create": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _f32,
                                    _c.POINTER(_vp)]),
     "pkv_step_ctx_destroy": (None, [_vp]),
+    "pkv_step_ctx_set_timing": (_i32, [_vp, _i32]),
+    "pkv_step_ctx_last_timing": (_i32, [_vp, _c.POINTER(_c.c_float)]),
     "pkv_decode_step": (_i32, [_vp, _vp, _pi64, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _f32, _i32, _vp, _vp]),
     "pkv_bm_create": (_i32, [_i32, _i32, _pi32, _c.POINTER(_vp)]),
     "pkv_bm_destroy": (None, [_vp]),
@@ -545,3 +547,14 @@ class DecodeStep:
                                     self.v_cache.data_ptr(), self.num_blocks, float(scale), self.partition_tokens,
                                     out_host.data_ptr(), s.cuda_stream)
         _check(st, "pkv_decode_step")
+
+    def set_timing(self, enable: bool):
+        """Phase timing of the following steps (pkv_step_ctx_set_timing)."""
+        _check(_lib().pkv_step_ctx_set_timing(self._h, 1 if enable else 0), "pkv_step_ctx_set_timing")
+
+    def last_timing(self) -> dict:
+        """Phases of the last timed step in ms: host block manager, H2D, kernels, D2H
+        (waits for that step's D2H)."""
+        out = (ctypes.c_float * 4)()
+        _check(_lib().pkv_step_ctx_last_timing(self._h, out), "pkv_step_ctx_last_timing")
+        return {"host_block_manager": out[0], "h2d": out[1], "kernels": out[2], "d2h": out[3]}

@@ -216,37 +216,42 @@ struct SimtConsumer {
 };
 
 // ---------------------------------------------------------------------------
-// Tensor-core consumer (bf16, up to 8 query heads per KV head).
+// Tensor-core consumer (bf16, up to 8 * NT query heads per KV head: NT 8-wide
+// MMA n-tiles of query heads share every K and V fragment).
 // Stage layout: for K then V, D/64 half-tiles of [16 rows x 128 B], each
 // written by TMA with the 128-byte swizzle (16-byte chunk c of row r lives at
 // chunk c ^ (r & 7)), so ldmatrix reads are bank-conflict free.
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, int NT = 1>
 struct MmaConsumer {
     static constexpr int KS = D / 16;          // k-steps of S^T = K Q^T
     static constexpr int MT = D / 16;          // m-tiles of O^T
     static constexpr int HALF = TILE_ROWS * 128;   // bytes of one 64-wide half tile
 
-    uint32_t qb[KS][2];                        // Q^T as B fragments (N = 8 query heads)
-    float o[MT][4];                            // O^T fragments: dims x heads
-    float m0, m1, l0, l1;                      // heads 2t, 2t+1
+    uint32_t qb[NT][KS][2];                    // Q^T as B fragments (N = 8 query heads per n-tile)
+    float o[NT][MT][4];                        // O^T fragments: dims x heads
+    float m0[NT], m1[NT], l0[NT], l1[NT];      // heads 8 nt + 2t, 8 nt + 2t + 1
 
     __device__ __forceinline__ void init(const __nv_bfloat16* q_rows, int group, int lane) {
         const int g = lane >> 2, t = lane & 3;
-        const uint32_t* row = reinterpret_cast<const uint32_t*>(q_rows + (int64_t)g * D);
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            if (g < group) {
-                qb[ks][0] = row[(ks * 16 + 2 * t) / 2];
-                qb[ks][1] = row[(ks * 16 + 2 * t + 8) / 2];
-            } else {
-                qb[ks][0] = qb[ks][1] = 0u;
+        for (int nt = 0; nt < NT; ++nt) {
+            const int h = 8 * nt + g;
+            const uint32_t* row = reinterpret_cast<const uint32_t*>(q_rows + (int64_t)h * D);
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                if (h < group) {
+                    qb[nt][ks][0] = row[(ks * 16 + 2 * t) / 2];
+                    qb[nt][ks][1] = row[(ks * 16 + 2 * t + 8) / 2];
+                } else {
+                    qb[nt][ks][0] = qb[nt][ks][1] = 0u;
+                }
             }
-        }
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-        m0 = m1 = kNegInf;
-        l0 = l1 = 0.f;
+            for (int mt = 0; mt < MT; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+            m0[nt] = m1[nt] = kNegInf;
+            l0[nt] = l1[nt] = 0.f;
+        }
     }
 
     __device__ __forceinline__ void consume(uint32_t ks_base, uint32_t vs_base, uint8_t* vs_ptr, int nvalid,
@@ -263,59 +268,68 @@ struct MmaConsumer {
             }
             __syncwarp();
         }
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        float s[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
             const int r = lane & 15;
             const int c = ((ks & 3) << 1) + (lane >> 4);
             uint32_t a0, a1, a2, a3;
             ldmatrix_x4(a0, a1, a2, a3, ks_base + (ks >> 2) * HALF + r * 128 + ((c ^ (r & 7)) << 4));
-            mma_bf16_16816(s, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
-        }
-        // s[0]: (token g, head 2t)  s[1]: (g, 2t+1)  s[2]: (g+8, 2t)  s[3]: (g+8, 2t+1)
-        float x0 = g < nvalid ? s[0] * scale_log2 : kNegInf;
-        float x1 = g < nvalid ? s[1] * scale_log2 : kNegInf;
-        float x2 = g + 8 < nvalid ? s[2] * scale_log2 : kNegInf;
-        float x3 = g + 8 < nvalid ? s[3] * scale_log2 : kNegInf;
-        float b0 = fmaxf(x0, x2), b1 = fmaxf(x1, x3);
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-            b0 = fmaxf(b0, __shfl_xor_sync(0xffffffffu, b0, off));
-            b1 = fmaxf(b1, __shfl_xor_sync(0xffffffffu, b1, off));
+            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
         }
-        const float n0 = fmaxf(m0, b0), n1 = fmaxf(m1, b1);
-        const float al0 = fast_exp2(m0 - n0), al1 = fast_exp2(m1 - n1);
-        m0 = n0;
-        m1 = n1;
-        const float p0 = fast_exp2(x0 - n0), p1 = fast_exp2(x1 - n1);
-        const float p2 = fast_exp2(x2 - n0), p3 = fast_exp2(x3 - n1);
-        l0 = l0 * al0 + (p0 + p2);
-        l1 = l1 * al1 + (p1 + p3);
+        uint32_t bh0[NT], bh1[NT], bl0[NT], bl1[NT];
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-            o[mt][0] *= al0; o[mt][1] *= al1; o[mt][2] *= al0; o[mt][3] *= al1;
+        for (int nt = 0; nt < NT; ++nt) {
+            // s[0]: (token g, head 2t)  s[1]: (g, 2t+1)  s[2]: (g+8, 2t)  s[3]: (g+8, 2t+1)
+            const float x0 = g < nvalid ? s[nt][0] * scale_log2 : kNegInf;
+            const float x1 = g < nvalid ? s[nt][1] * scale_log2 : kNegInf;
+            const float x2 = g + 8 < nvalid ? s[nt][2] * scale_log2 : kNegInf;
+            const float x3 = g + 8 < nvalid ? s[nt][3] * scale_log2 : kNegInf;
+            float b0 = fmaxf(x0, x2), b1 = fmaxf(x1, x3);
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                b0 = fmaxf(b0, __shfl_xor_sync(0xffffffffu, b0, off));
+                b1 = fmaxf(b1, __shfl_xor_sync(0xffffffffu, b1, off));
+            }
+            const float n0 = fmaxf(m0[nt], b0), n1 = fmaxf(m1[nt], b1);
+            const float al0 = fast_exp2(m0[nt] - n0), al1 = fast_exp2(m1[nt] - n1);
+            m0[nt] = n0;
+            m1[nt] = n1;
+            const float p0 = fast_exp2(x0 - n0), p1 = fast_exp2(x1 - n1);
+            const float p2 = fast_exp2(x2 - n0), p3 = fast_exp2(x3 - n1);
+            l0[nt] = l0[nt] * al0 + (p0 + p2);
+            l1[nt] = l1[nt] * al1 + (p1 + p3);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                o[nt][mt][0] *= al0; o[nt][mt][1] *= al1; o[nt][mt][2] *= al0; o[nt][mt][3] *= al1;
+            }
+            // P^T as B fragments (k = token, n = head), high and low bf16 parts.
+            const uint32_t h02 = pack_bf16(p0, p2), h13 = pack_bf16(p1, p3);
+            const uint32_t e02 = pack_bf16(p0 - bf16lo(h02), p2 - bf16hi(h02));
+            const uint32_t e13 = pack_bf16(p1 - bf16lo(h13), p3 - bf16hi(h13));
+            const int srcA = (2 * t) * 4 + (g >> 1), srcB = srcA + 4;
+            const bool odd = g & 1;
+            uint32_t ya, yb, za, zb;
+            {
+                const uint32_t u0 = __shfl_sync(0xffffffffu, h02, srcA), u1 = __shfl_sync(0xffffffffu, h13, srcA);
+                const uint32_t v0 = __shfl_sync(0xffffffffu, h02, srcB), v1 = __shfl_sync(0xffffffffu, h13, srcB);
+                ya = odd ? u1 : u0;
+                yb = odd ? v1 : v0;
+            }
+            {
+                const uint32_t u0 = __shfl_sync(0xffffffffu, e02, srcA), u1 = __shfl_sync(0xffffffffu, e13, srcA);
+                const uint32_t v0 = __shfl_sync(0xffffffffu, e02, srcB), v1 = __shfl_sync(0xffffffffu, e13, srcB);
+                za = odd ? u1 : u0;
+                zb = odd ? v1 : v0;
+            }
+            bh0[nt] = __byte_perm(ya, yb, 0x5410);
+            bh1[nt] = __byte_perm(ya, yb, 0x7632);
+            bl0[nt] = __byte_perm(za, zb, 0x5410);
+            bl1[nt] = __byte_perm(za, zb, 0x7632);
         }
-        // P^T as B fragments (k = token, n = head), high and low bf16 parts.
-        const uint32_t h02 = pack_bf16(p0, p2), h13 = pack_bf16(p1, p3);
-        const uint32_t e02 = pack_bf16(p0 - bf16lo(h02), p2 - bf16hi(h02));
-        const uint32_t e13 = pack_bf16(p1 - bf16lo(h13), p3 - bf16hi(h13));
-        const int srcA = (2 * t) * 4 + (g >> 1), srcB = srcA + 4;
-        const bool odd = g & 1;
-        uint32_t ya, yb, za, zb;
-        {
-            const uint32_t u0 = __shfl_sync(0xffffffffu, h02, srcA), u1 = __shfl_sync(0xffffffffu, h13, srcA);
-            const uint32_t v0 = __shfl_sync(0xffffffffu, h02, srcB), v1 = __shfl_sync(0xffffffffu, h13, srcB);
-            ya = odd ? u1 : u0;
-            yb = odd ? v1 : v0;
-        }
-        {
-            const uint32_t u0 = __shfl_sync(0xffffffffu, e02, srcA), u1 = __shfl_sync(0xffffffffu, e13, srcA);
-            const uint32_t v0 = __shfl_sync(0xffffffffu, e02, srcB), v1 = __shfl_sync(0xffffffffu, e13, srcB);
-            za = odd ? u1 : u0;
-            zb = odd ? v1 : v0;
-        }
-        const uint32_t bh0 = __byte_perm(ya, yb, 0x5410), bh1 = __byte_perm(ya, yb, 0x7632);
-        const uint32_t bl0 = __byte_perm(za, zb, 0x5410), bl1 = __byte_perm(za, zb, 0x7632);
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
             const int mi = lane >> 3;
@@ -324,33 +338,40 @@ struct MmaConsumer {
             uint32_t a0, a1, a2, a3;
             ldmatrix_x4_trans(a0, a1, a2, a3,
                               vs_base + ((mt * 16) >> 6) * HALF + tok * 128 + ((c ^ (tok & 7)) << 4));
-            mma_bf16_16816(o[mt], a0, a1, a2, a3, bh0, bh1);
-            mma_bf16_16816(o[mt], a0, a1, a2, a3, bl0, bl1);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                mma_bf16_16816(o[nt][mt], a0, a1, a2, a3, bh0[nt], bh1[nt]);
+                mma_bf16_16816(o[nt][mt], a0, a1, a2, a3, bl0[nt], bl1[nt]);
+            }
         }
     }
 
     __device__ __forceinline__ void finish(float* red_o, float* red_m, float* red_l, int group, int lane) {
         const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-            l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-            l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-        }
-        const int h0 = 2 * t, h1 = 2 * t + 1;
+        for (int nt = 0; nt < NT; ++nt) {
+            float a = l0[nt], b = l1[nt];
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-            if (h0 < group) {
-                red_o[h0 * D + mt * 16 + g] = o[mt][0];
-                red_o[h0 * D + mt * 16 + g + 8] = o[mt][2];
+            for (int off = 4; off < 32; off <<= 1) {
+                a += __shfl_xor_sync(0xffffffffu, a, off);
+                b += __shfl_xor_sync(0xffffffffu, b, off);
             }
-            if (h1 < group) {
-                red_o[h1 * D + mt * 16 + g] = o[mt][1];
-                red_o[h1 * D + mt * 16 + g + 8] = o[mt][3];
+            const int h0 = 8 * nt + 2 * t, h1 = h0 + 1;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                if (h0 < group) {
+                    red_o[h0 * D + mt * 16 + g] = o[nt][mt][0];
+                    red_o[h0 * D + mt * 16 + g + 8] = o[nt][mt][2];
+                }
+                if (h1 < group) {
+                    red_o[h1 * D + mt * 16 + g] = o[nt][mt][1];
+                    red_o[h1 * D + mt * 16 + g + 8] = o[nt][mt][3];
+                }
             }
-        }
-        if (g == 0) {
-            if (h0 < group) { red_m[h0] = m0; red_l[h0] = l0; }
-            if (h1 < group) { red_m[h1] = m1; red_l[h1] = l1; }
+            if (g == 0) {
+                if (h0 < group) { red_m[h0] = m0[nt]; red_l[h0] = a; }
+                if (h1 < group) { red_m[h1] = m1[nt]; red_l[h1] = b; }
+            }
         }
     }
 };
@@ -371,15 +392,15 @@ struct MmaConsumer {
 //   and the odd-dim row (fragment row g + 8), so each 16-dim chunk is one MMA
 //   whose output rows are dims 2g and 2g + 1.
 // ---------------------------------------------------------------------------
-template <int NT>      // 16-token tiles per stage (1 or 2)
+template <int NT, int NH = 1>      // 16-token tiles per stage (1 or 2); 8-wide query-head tiles (1 or 2)
 struct MmaConsumerFp8 {
     static constexpr int D = 128;
     static constexpr int NCHUNK = D / 16;
     static constexpr int TOK = 16 * NT;
 
-    uint32_t qb[NCHUNK][2];
-    float o[NCHUNK][4];
-    float m0, m1, l0, l1;
+    uint32_t qb[NH][NCHUNK][2];
+    float o[NH][NCHUNK][4];
+    float m0[NH], m1[NH], l0[NH], l1[NH];
 
     __device__ __forceinline__ static uint32_t f16pair(float a, float b) {
         return pack_f16(fminf(fmaxf(a, -65504.f), 65504.f), fminf(fmaxf(b, -65504.f), 65504.f));
@@ -388,19 +409,23 @@ struct MmaConsumerFp8 {
     __device__ __forceinline__ void init(const __nv_bfloat16* q_rows, int group, int lane) {
         const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-        for (int ks = 0; ks < NCHUNK; ++ks) {
-            if (g < group) {
-                const uint2 w = *reinterpret_cast<const uint2*>(q_rows + (int64_t)g * D + 16 * ks + 4 * t);
-                qb[ks][0] = f16pair(bf16lo(w.x), bf16hi(w.x));
-                qb[ks][1] = f16pair(bf16lo(w.y), bf16hi(w.y));
-            } else {
-                qb[ks][0] = qb[ks][1] = 0u;
-            }
-        }
+        for (int nh = 0; nh < NH; ++nh) {
+            const int h = 8 * nh + g;
 #pragma unroll
-        for (int c = 0; c < NCHUNK; ++c) o[c][0] = o[c][1] = o[c][2] = o[c][3] = 0.f;
-        m0 = m1 = kNegInf;
-        l0 = l1 = 0.f;
+            for (int ks = 0; ks < NCHUNK; ++ks) {
+                if (h < group) {
+                    const uint2 w = *reinterpret_cast<const uint2*>(q_rows + (int64_t)h * D + 16 * ks + 4 * t);
+                    qb[nh][ks][0] = f16pair(bf16lo(w.x), bf16hi(w.x));
+                    qb[nh][ks][1] = f16pair(bf16lo(w.y), bf16hi(w.y));
+                } else {
+                    qb[nh][ks][0] = qb[nh][ks][1] = 0u;
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < NCHUNK; ++c) o[nh][c][0] = o[nh][c][1] = o[nh][c][2] = o[nh][c][3] = 0.f;
+            m0[nh] = m1[nh] = kNegInf;
+            l0[nh] = l1[nh] = 0.f;
+        }
     }
 
     // P^T of one 16-token tile as f16 B fragments (high and low parts).
@@ -431,14 +456,18 @@ struct MmaConsumerFp8 {
         bl1 = __byte_perm(za, zb, 0x7632);
     }
 
-    // One even/odd-dim MMA pair input from two ldmatrix.trans registers (tokens 0-7, 8-15 of a tile).
-    __device__ __forceinline__ void pv(int c, uint32_t rlo, uint32_t rhi, uint32_t bh0, uint32_t bh1, uint32_t bl0,
-                                       uint32_t bl1) {
+    // One even/odd-dim MMA pair input from two ldmatrix.trans registers (tokens 0-7, 8-15 of a tile),
+    // applied to every head tile.
+    __device__ __forceinline__ void pv(int c, uint32_t rlo, uint32_t rhi, const uint32_t (&bh)[NH][2],
+                                       const uint32_t (&bl)[NH][2]) {
         const uint32_t x = __byte_perm(rlo, 0u, 0x3120), y = __byte_perm(rhi, 0u, 0x3120);
         const uint32_t a0 = e4m3x2_to_f16x2(x & 0xffffu), a1 = e4m3x2_to_f16x2(x >> 16);
         const uint32_t a2 = e4m3x2_to_f16x2(y & 0xffffu), a3 = e4m3x2_to_f16x2(y >> 16);
-        mma_f16_16816(o[c], a0, a1, a2, a3, bh0, bh1);
-        mma_f16_16816(o[c], a0, a1, a2, a3, bl0, bl1);
+#pragma unroll
+        for (int nh = 0; nh < NH; ++nh) {
+            mma_f16_16816(o[nh][c], a0, a1, a2, a3, bh[nh][0], bh[nh][1]);
+            mma_f16_16816(o[nh][c], a0, a1, a2, a3, bl[nh][0], bl[nh][1]);
+        }
     }
 
     __device__ __forceinline__ void consume(uint32_t ks_base, uint32_t vs_base, uint8_t* vs_ptr, int nvalid,
@@ -451,9 +480,11 @@ struct MmaConsumerFp8 {
             }
             __syncwarp();
         }
-        float s[NT][4];
+        float s[NH][NT][4];
 #pragma unroll
-        for (int tt = 0; tt < NT; ++tt) s[tt][0] = s[tt][1] = s[tt][2] = s[tt][3] = 0.f;
+        for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+            for (int tt = 0; tt < NT; ++tt) s[nh][tt][0] = s[nh][tt][1] = s[nh][tt][2] = s[nh][tt][3] = 0.f;
         const int mi = lane >> 3;
         const int row = (lane & 7) + ((mi & 1) << 3);
 #pragma unroll
@@ -464,48 +495,55 @@ struct MmaConsumerFp8 {
                 const int r = tt * 16 + row;
                 uint32_t r0, r1, r2, r3;
                 ldmatrix_x4(r0, r1, r2, r3, ks_base + r * 128 + ((chunk ^ (r & 7)) << 4));
-                mma_f16_16816(s[tt], e4m3x2_to_f16x2(r0 & 0xffffu), e4m3x2_to_f16x2(r1 & 0xffffu),
-                              e4m3x2_to_f16x2(r0 >> 16), e4m3x2_to_f16x2(r1 >> 16), qb[2 * kp][0], qb[2 * kp][1]);
-                mma_f16_16816(s[tt], e4m3x2_to_f16x2(r2 & 0xffffu), e4m3x2_to_f16x2(r3 & 0xffffu),
-                              e4m3x2_to_f16x2(r2 >> 16), e4m3x2_to_f16x2(r3 >> 16), qb[2 * kp + 1][0],
-                              qb[2 * kp + 1][1]);
+                const uint32_t k00 = e4m3x2_to_f16x2(r0 & 0xffffu), k01 = e4m3x2_to_f16x2(r1 & 0xffffu);
+                const uint32_t k02 = e4m3x2_to_f16x2(r0 >> 16), k03 = e4m3x2_to_f16x2(r1 >> 16);
+                const uint32_t k10 = e4m3x2_to_f16x2(r2 & 0xffffu), k11 = e4m3x2_to_f16x2(r3 & 0xffffu);
+                const uint32_t k12 = e4m3x2_to_f16x2(r2 >> 16), k13 = e4m3x2_to_f16x2(r3 >> 16);
+#pragma unroll
+                for (int nh = 0; nh < NH; ++nh) {
+                    mma_f16_16816(s[nh][tt], k00, k01, k02, k03, qb[nh][2 * kp][0], qb[nh][2 * kp][1]);
+                    mma_f16_16816(s[nh][tt], k10, k11, k12, k13, qb[nh][2 * kp + 1][0], qb[nh][2 * kp + 1][1]);
+                }
             }
         }
-        float x[NT][4];
-        float b0 = kNegInf, b1 = kNegInf;
+        uint32_t bh[NT][NH][2], bl[NT][NH][2];
 #pragma unroll
-        for (int tt = 0; tt < NT; ++tt) {
-            x[tt][0] = tt * 16 + g < nvalid ? s[tt][0] * scale_log2 : kNegInf;
-            x[tt][1] = tt * 16 + g < nvalid ? s[tt][1] * scale_log2 : kNegInf;
-            x[tt][2] = tt * 16 + g + 8 < nvalid ? s[tt][2] * scale_log2 : kNegInf;
-            x[tt][3] = tt * 16 + g + 8 < nvalid ? s[tt][3] * scale_log2 : kNegInf;
-            b0 = fmaxf(b0, fmaxf(x[tt][0], x[tt][2]));
-            b1 = fmaxf(b1, fmaxf(x[tt][1], x[tt][3]));
-        }
+        for (int nh = 0; nh < NH; ++nh) {
+            float x[NT][4];
+            float b0 = kNegInf, b1 = kNegInf;
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-            b0 = fmaxf(b0, __shfl_xor_sync(0xffffffffu, b0, off));
-            b1 = fmaxf(b1, __shfl_xor_sync(0xffffffffu, b1, off));
-        }
-        const float n0 = fmaxf(m0, b0), n1 = fmaxf(m1, b1);
-        const float al0 = fast_exp2(m0 - n0), al1 = fast_exp2(m1 - n1);
-        m0 = n0;
-        m1 = n1;
-        float ps0 = 0.f, ps1 = 0.f;
-        uint32_t bh[NT][2], bl[NT][2];
+            for (int tt = 0; tt < NT; ++tt) {
+                x[tt][0] = tt * 16 + g < nvalid ? s[nh][tt][0] * scale_log2 : kNegInf;
+                x[tt][1] = tt * 16 + g < nvalid ? s[nh][tt][1] * scale_log2 : kNegInf;
+                x[tt][2] = tt * 16 + g + 8 < nvalid ? s[nh][tt][2] * scale_log2 : kNegInf;
+                x[tt][3] = tt * 16 + g + 8 < nvalid ? s[nh][tt][3] * scale_log2 : kNegInf;
+                b0 = fmaxf(b0, fmaxf(x[tt][0], x[tt][2]));
+                b1 = fmaxf(b1, fmaxf(x[tt][1], x[tt][3]));
+            }
 #pragma unroll
-        for (int tt = 0; tt < NT; ++tt) {
-            const float p0 = fast_exp2(x[tt][0] - n0), p1 = fast_exp2(x[tt][1] - n1);
-            const float p2 = fast_exp2(x[tt][2] - n0), p3 = fast_exp2(x[tt][3] - n1);
-            ps0 += p0 + p2;
-            ps1 += p1 + p3;
-            p_fragments(p0, p1, p2, p3, lane, bh[tt][0], bh[tt][1], bl[tt][0], bl[tt][1]);
-        }
-        l0 = l0 * al0 + ps0;
-        l1 = l1 * al1 + ps1;
+            for (int off = 4; off < 32; off <<= 1) {
+                b0 = fmaxf(b0, __shfl_xor_sync(0xffffffffu, b0, off));
+                b1 = fmaxf(b1, __shfl_xor_sync(0xffffffffu, b1, off));
+            }
+            const float n0 = fmaxf(m0[nh], b0), n1 = fmaxf(m1[nh], b1);
+            const float al0 = fast_exp2(m0[nh] - n0), al1 = fast_exp2(m1[nh] - n1);
+            m0[nh] = n0;
+            m1[nh] = n1;
+            float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
-        for (int c = 0; c < NCHUNK; ++c) {
-            o[c][0] *= al0; o[c][1] *= al1; o[c][2] *= al0; o[c][3] *= al1;
+            for (int tt = 0; tt < NT; ++tt) {
+                const float p0 = fast_exp2(x[tt][0] - n0), p1 = fast_exp2(x[tt][1] - n1);
+                const float p2 = fast_exp2(x[tt][2] - n0), p3 = fast_exp2(x[tt][3] - n1);
+                ps0 += p0 + p2;
+                ps1 += p1 + p3;
+                p_fragments(p0, p1, p2, p3, lane, bh[tt][nh][0], bh[tt][nh][1], bl[tt][nh][0], bl[tt][nh][1]);
+            }
+            l0[nh] = l0[nh] * al0 + ps0;
+            l1[nh] = l1[nh] * al1 + ps1;
+#pragma unroll
+            for (int c = 0; c < NCHUNK; ++c) {
+                o[nh][c][0] *= al0; o[nh][c][1] *= al1; o[nh][c][2] *= al0; o[nh][c][3] *= al1;
+            }
         }
         if constexpr (NT == 1) {
             const int tok = (lane & 7) + ((mi & 1) << 3);
@@ -515,8 +553,8 @@ struct MmaConsumerFp8 {
                 uint32_t r0, r1, r2, r3;
                 ldmatrix_x4_trans(r0, r1, r2, r3, vs_base + tok * 128 + ((chunk ^ (tok & 7)) << 4));
                 // r0: tokens 0-7 of chunk 2cp, r1: tokens 8-15 of it; r2, r3: chunk 2cp + 1
-                pv(2 * cp, r0, r1, bh[0][0], bh[0][1], bl[0][0], bl[0][1]);
-                pv(2 * cp + 1, r2, r3, bh[0][0], bh[0][1], bl[0][0], bl[0][1]);
+                pv(2 * cp, r0, r1, bh[0], bl[0]);
+                pv(2 * cp + 1, r2, r3, bh[0], bl[0]);
             }
         } else {
             // one ldmatrix.x4.trans per chunk: tokens 0-7, 8-15 (tile 0) and 16-23, 24-31 (tile 1)
@@ -525,8 +563,8 @@ struct MmaConsumerFp8 {
             for (int c = 0; c < NCHUNK; ++c) {
                 uint32_t r0, r1, r2, r3;
                 ldmatrix_x4_trans(r0, r1, r2, r3, vs_base + tok * 128 + ((c ^ (tok & 7)) << 4));
-                pv(c, r0, r1, bh[0][0], bh[0][1], bl[0][0], bl[0][1]);
-                pv(c, r2, r3, bh[1][0], bh[1][1], bl[1][0], bl[1][1]);
+                pv(c, r0, r1, bh[0], bl[0]);
+                pv(c, r2, r3, bh[1], bl[1]);
             }
         }
     }
@@ -534,26 +572,30 @@ struct MmaConsumerFp8 {
     __device__ __forceinline__ void finish(float* red_o, float* red_m, float* red_l, int group, int lane) {
         const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-            l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-            l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-        }
-        const int h0 = 2 * t, h1 = 2 * t + 1;
+        for (int nh = 0; nh < NH; ++nh) {
+            float a = l0[nh], b = l1[nh];
 #pragma unroll
-        for (int c = 0; c < NCHUNK; ++c) {
-            const int de = 16 * c + 2 * g;            // fragment rows g / g + 8 are dims de / de + 1
-            if (h0 < group) {
-                red_o[h0 * D + de] = o[c][0];
-                red_o[h0 * D + de + 1] = o[c][2];
+            for (int off = 4; off < 32; off <<= 1) {
+                a += __shfl_xor_sync(0xffffffffu, a, off);
+                b += __shfl_xor_sync(0xffffffffu, b, off);
             }
-            if (h1 < group) {
-                red_o[h1 * D + de] = o[c][1];
-                red_o[h1 * D + de + 1] = o[c][3];
+            const int h0 = 8 * nh + 2 * t, h1 = h0 + 1;
+#pragma unroll
+            for (int c = 0; c < NCHUNK; ++c) {
+                const int de = 16 * c + 2 * g;            // fragment rows g / g + 8 are dims de / de + 1
+                if (h0 < group) {
+                    red_o[h0 * D + de] = o[nh][c][0];
+                    red_o[h0 * D + de + 1] = o[nh][c][2];
+                }
+                if (h1 < group) {
+                    red_o[h1 * D + de] = o[nh][c][1];
+                    red_o[h1 * D + de + 1] = o[nh][c][3];
+                }
             }
-        }
-        if (g == 0) {
-            if (h0 < group) { red_m[h0] = m0; red_l[h0] = l0; }
-            if (h1 < group) { red_m[h1] = m1; red_l[h1] = l1; }
+            if (g == 0) {
+                if (h0 < group) { red_m[h0] = m0[nh]; red_l[h0] = a; }
+                if (h1 < group) { red_m[h1] = m1[nh]; red_l[h1] = b; }
+            }
         }
     }
 };

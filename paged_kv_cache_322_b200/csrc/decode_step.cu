@@ -15,6 +15,7 @@
 // step's copy is still in flight).
 #include <cuda_runtime.h>
 
+#include <chrono>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -38,6 +39,11 @@ struct pkv_step_ctx {
     cudaEvent_t meta_done[2] = {nullptr, nullptr};
     int slot = 0;
     int device = 0;
+    // optional phase timing of the last step (pkv_step_ctx_set_timing)
+    bool timing = false;
+    cudaEvent_t tev[4] = {nullptr, nullptr, nullptr, nullptr};   // before H2D, after H2D, after kernels, after D2H
+    float host_ms = 0.f;                                          // block manager + tables, host clock
+    bool timed_step = false;
 };
 
 namespace {
@@ -61,6 +67,8 @@ void release(pkv_step_ctx* c) {
         if (c->h_meta[i]) cudaFreeHost(c->h_meta[i]);
         if (c->meta_done[i]) cudaEventDestroy(c->meta_done[i]);
     }
+    for (int i = 0; i < 4; ++i)
+        if (c->tev[i]) cudaEventDestroy(c->tev[i]);
     cudaSetDevice(prev);
     delete c;
 }
@@ -134,6 +142,9 @@ pkv_status pkv_decode_step(pkv_step_ctx* c, pkv_block_manager* bm, const int64_t
     if (n == 0) return PKV_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t S = (size_t)c->max_seqs;
+    const bool timing = c->timing;
+    c->timed_step = false;
+    const auto t_host0 = std::chrono::steady_clock::now();
     // 1. host metadata into a pinned slot whose previous copy has finished
     const int sl = c->slot;
     c->slot ^= 1;
@@ -152,6 +163,10 @@ pkv_status pkv_decode_step(pkv_step_ctx* c, pkv_block_manager* bm, const int64_t
     if (s != PKV_OK) return s;
     int max_len = 0;
     for (int i = 0; i < n; ++i) max_len = lens[i] > max_len ? lens[i] : max_len;
+    if (timing) {
+        c->host_ms = std::chrono::duration<float, std::milli>(std::chrono::steady_clock::now() - t_host0).count();
+        if (cudaEventRecord(c->tev[0], st) != cudaSuccess) return PKV_ERR_CUDA;
+    }
     // 2. copies to the device
     if (cudaMemcpyAsync(c->d_meta, h, c->meta_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaEventRecord(c->meta_done[sl], st) != cudaSuccess)
@@ -162,6 +177,7 @@ pkv_status pkv_decode_step(pkv_step_ctx* c, pkv_block_manager* bm, const int64_t
         cudaMemcpyAsync(c->d_k, k_host, kb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(c->d_v, v_host, kb, cudaMemcpyHostToDevice, st) != cudaSuccess)
         return PKV_ERR_CUDA;
+    if (timing && cudaEventRecord(c->tev[1], st) != cudaSuccess) return PKV_ERR_CUDA;
     const int64_t* d_slots = reinterpret_cast<const int64_t*>(c->d_meta);
     const int64_t* d_src = d_slots + S;
     const int64_t* d_dst = d_src + S;
@@ -190,9 +206,40 @@ pkv_status pkv_decode_step(pkv_step_ctx* c, pkv_block_manager* bm, const int64_t
                                          c->max_blocks, num_blocks, max_len, partition_tokens, c->d_ws, c->ws_bytes,
                                          stream);
     if (s != PKV_OK) return s;
+    if (timing && cudaEventRecord(c->tev[2], st) != cudaSuccess) return PKV_ERR_CUDA;
     // 4. the result back to the host
     const size_t ob = (size_t)n * c->num_q_heads * c->head_dim * elt(c->out_dtype);
     if (cudaMemcpyAsync(out_host, c->d_out, ob, cudaMemcpyDeviceToHost, st) != cudaSuccess) return PKV_ERR_CUDA;
+    if (timing) {
+        if (cudaEventRecord(c->tev[3], st) != cudaSuccess) return PKV_ERR_CUDA;
+        c->timed_step = true;
+    }
+    return PKV_OK;
+}
+
+pkv_status pkv_step_ctx_set_timing(pkv_step_ctx* c, int enable) {
+    if (!c) return PKV_ERR_INVALID_ARG;
+    if (enable && !c->tev[0]) {
+        int prev = 0;
+        cudaGetDevice(&prev);
+        cudaSetDevice(c->device);
+        bool ok = true;
+        for (int i = 0; i < 4 && ok; ++i) ok = cudaEventCreate(&c->tev[i]) == cudaSuccess;
+        cudaSetDevice(prev);
+        if (!ok) return PKV_ERR_CUDA;
+    }
+    c->timing = enable != 0;
+    c->timed_step = false;
+    return PKV_OK;
+}
+
+pkv_status pkv_step_ctx_last_timing(pkv_step_ctx* c, float* out) {
+    if (!c || !out) return PKV_ERR_INVALID_ARG;
+    if (!c->timed_step) return PKV_ERR_INVALID_ARG;
+    if (cudaEventSynchronize(c->tev[3]) != cudaSuccess) return PKV_ERR_CUDA;
+    out[0] = c->host_ms;
+    for (int i = 0; i < 3; ++i)
+        if (cudaEventElapsedTime(&out[1 + i], c->tev[i], c->tev[i + 1]) != cudaSuccess) return PKV_ERR_CUDA;
     return PKV_OK;
 }
 

@@ -43,23 +43,32 @@
 namespace pkv {
 namespace attn {
 
-// Log-sum-exp merge of partition results. grid = (Hq, B), block = D threads.
-// The (m, l) pairs are staged in shared memory once (coalesced), the weights
-// w_c = l_c 2^(m_c - M) computed once per row, then each thread sums its
-// dimension over the partitions with independent loads in flight (the first
-// version walked the partitions with one dependent load chain per thread).
+// Log-sum-exp merge of partition results. grid = (Hq, B), block = GROUPS x D
+// threads. The (m, l) pairs are staged in shared memory once (coalesced), the
+// weights w_c = l_c 2^(m_c - M) computed once per row; then each group of D
+// threads (one thread per dimension) sums over every GROUPS-th partition with
+// eight independent loads in flight, and the groups' sums are added. Calls with
+// many partitions per context take four groups (one group walking 50
+// partitions four loads at a time took 12.5 us of mostly DRAM latency on the
+// long-context workload, four groups with eight loads each 9.0 us, ncu); calls
+// with a few partitions take one group (fewer threads to launch).
 constexpr int kMergeSmemParts = 2048;
+constexpr int kMergeManyParts = 8;      // partitions per context from which four groups are launched
 //
 // Launched as a programmatic dependent of the partition kernel: the launch is
 // staged while that kernel runs, and the CTAs wait here until its grid has
 // completed and the partials are visible (a no-op for a plain launch).
-template <int D>
-__global__ void __launch_bounds__(D) merge_partitions_kernel(const Params p) {
+template <int D, int GROUPS>
+__global__ void __launch_bounds__(GROUPS * D) merge_partitions_kernel(const Params p) {
+    constexpr int NT = GROUPS * D;
+    constexpr int kMergeGroups = GROUPS;
     __shared__ float sw[kMergeSmemParts];
-    __shared__ float s_red[D / 32];
+    __shared__ float s_red[NT / 32];
+    __shared__ float s_o[GROUPS > 1 ? GROUPS - 1 : 1][D];
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int qhead = blockIdx.x, seq = blockIdx.y, d = threadIdx.x;
-    const int lane = d & 31, wid = d >> 5;
+    const int qhead = blockIdx.x, seq = blockIdx.y, tid = threadIdx.x;
+    const int lane = tid & 31, wid = tid >> 5;
+    const int grp = tid / D, d = tid - grp * D;
     int ctx = p.context_lens[seq];
     ctx = ctx < 0 ? 0 : (ctx > p.ctx_cap ? p.ctx_cap : ctx);
     const int nparts = ((ctx + p.block_size - 1) / p.block_size + p.part_blocks - 1) / p.part_blocks;
@@ -71,7 +80,7 @@ __global__ void __launch_bounds__(D) merge_partitions_kernel(const Params p) {
     if (nparts <= kMergeSmemParts) {
         // M = max m_c
         float mx = kNegInf;
-        for (int c = d; c < nparts; c += D) {
+        for (int c = tid; c < nparts; c += NT) {
             const float mc = ml[2 * c];
             sw[c] = mc;
             mx = fmaxf(mx, mc);
@@ -82,11 +91,11 @@ __global__ void __launch_bounds__(D) merge_partitions_kernel(const Params p) {
         __syncthreads();
         float M = s_red[0];
 #pragma unroll
-        for (int w = 1; w < D / 32; ++w) M = fmaxf(M, s_red[w]);
+        for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, s_red[w]);
         __syncthreads();
-        if (M != kNegInf) {
+        if (M != kNegInf) {                                      // uniform over the CTA
             float ls = 0.f;
-            for (int c = d; c < nparts; c += D) {
+            for (int c = tid; c < nparts; c += NT) {
                 const float mc = sw[c];
                 const float w = mc == kNegInf ? 0.f : ml[2 * c + 1] * fast_exp2(mc - M);
                 sw[c] = w;
@@ -97,17 +106,29 @@ __global__ void __launch_bounds__(D) merge_partitions_kernel(const Params p) {
             if (lane == 0) s_red[wid] = ls;
             __syncthreads();
 #pragma unroll
-            for (int w = 0; w < D / 32; ++w) L += s_red[w];
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            int c = 0;
-            for (; c + 4 <= nparts; c += 4) {
+            for (int w = 0; w < NT / 32; ++w) L += s_red[w];
+            // this group's partitions grp, grp + 4, ...: eight loads issued before they are used
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            int c = grp;
+            for (; c + 7 * kMergeGroups < nparts; c += 8 * kMergeGroups) {
+                float v[8];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) acc[u] += sw[c + u] * o[(int64_t)(c + u) * D];
+                for (int u = 0; u < 8; ++u) v[u] = o[(int64_t)(c + u * kMergeGroups) * D];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) acc[u] += sw[c + u * kMergeGroups] * v[u];
             }
-            for (; c < nparts; ++c) acc[0] += sw[c] * o[(int64_t)c * D];
-            O = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            for (; c < nparts; c += kMergeGroups) acc[0] += sw[c] * o[(int64_t)c * D];
+            O = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        }
+        if constexpr (GROUPS > 1) {
+            if (grp > 0) s_o[grp - 1][d] = O;
+            __syncthreads();
+            if (grp > 0) return;
+#pragma unroll
+            for (int g = 0; g < GROUPS - 1; ++g) O += s_o[g][d];
         }
     } else {
+        if (grp > 0) return;
         float M = kNegInf;
         for (int c = 0; c < nparts; ++c) M = fmaxf(M, ml[2 * c]);
         if (M != kNegInf) {
@@ -304,7 +325,8 @@ pkv_status decode_impl(void* out, pkv_dtype out_dtype, const void* q, const void
     if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
     if (fp8 && (head_dim != 128 || partition_tokens == -1)) return PKV_ERR_UNSUPPORTED;
     if (!block_size_built(block_size) || (partition_tokens == -1 && block_size != 16)) return PKV_ERR_UNSUPPORTED;
-    if (group != 1 && group != 2 && group != 4 && group != 8) return PKV_ERR_UNSUPPORTED;
+    if (group != 1 && group != 2 && group != 4 && group != 8 && group != 16) return PKV_ERR_UNSUPPORTED;
+    if (partition_tokens == -1 && group > 8) return PKV_ERR_UNSUPPORTED;   // persistent: one 8-wide head tile
     if (num_seqs == 0) return PKV_OK;
     if (num_seqs > 65535) return PKV_ERR_UNSUPPORTED;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_ERR_INVALID_ARG;
@@ -392,16 +414,21 @@ pkv_status decode_impl(void* out, pkv_dtype out_dtype, const void* q, const void
         // programmatic dependent launch: the merge grid's CTAs wait for the
         // partition grid in-kernel instead of behind a full kernel boundary
         cudaLaunchConfig_t cfg = {};
+        const int groups = pl.num_parts >= kMergeManyParts ? 4 : 1;
         cfg.gridDim = dim3(num_q_heads, num_seqs);
-        cfg.blockDim = dim3(head_dim);
+        cfg.blockDim = dim3(groups * head_dim);
         cfg.stream = st;
         cudaLaunchAttribute at[1];
         at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         at[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = at;
         cfg.numAttrs = 1;
-        e = head_dim == 128 ? cudaLaunchKernelEx(&cfg, merge_partitions_kernel<128>, p)
-                            : cudaLaunchKernelEx(&cfg, merge_partitions_kernel<64>, p);
+        if (groups == 4)
+            e = head_dim == 128 ? cudaLaunchKernelEx(&cfg, merge_partitions_kernel<128, 4>, p)
+                                : cudaLaunchKernelEx(&cfg, merge_partitions_kernel<64, 4>, p);
+        else
+            e = head_dim == 128 ? cudaLaunchKernelEx(&cfg, merge_partitions_kernel<128, 1>, p)
+                                : cudaLaunchKernelEx(&cfg, merge_partitions_kernel<64, 1>, p);
         if (e != cudaSuccess) return PKV_ERR_CUDA;
     }
     return PKV_OK;

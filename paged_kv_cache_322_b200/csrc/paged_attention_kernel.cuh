@@ -18,7 +18,7 @@ namespace attn {
 // The pipelined kernel.
 //   PATH 0: SIMT, block-split (each consumer warp takes whole blocks, HPW = group)
 //   PATH 1: SIMT, head-split (every warp reads every block, HPW = group / NCW)
-//   PATH 2: tensor cores, block-split (group <= 8)
+//   PATH 2: tensor cores, block-split (group <= HPW: 8, or 16 as two 8-wide head tiles)
 // ---------------------------------------------------------------------------
 template <typename T, int D, int PATH, int HPW, int STAGES, int KPC, int BSZ>
 struct Kern {
@@ -49,7 +49,8 @@ struct Kern {
     static_assert(PATH != 1 || KPC == 1, "head-split consumers serve one KV head");
     static constexpr int RING = STAGES * STAGE_BYTES;
     static constexpr int NSLOT = PATH == 1 ? 1 : NCW;                  // partial states to merge
-    static constexpr int MAXG = PATH == 2 ? 8 : (PATH == 1 ? HPW * NCW : HPW);
+    static constexpr int MAXG = PATH == 2 ? HPW : (PATH == 1 ? HPW * NCW : HPW);
+    static_assert(PATH != 2 || HPW == 8 || HPW == 16, "tensor-core consumers take one or two 8-wide head tiles");
     static constexpr int RED = NSLOT * MAXG * (D + 2) * 4;
     static constexpr int BODY = RING > RED ? RING : RED;
     static constexpr int SMEM = 1024 /*align slack*/ + BODY + 2 * STAGES * 8;
@@ -173,7 +174,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         const int nstage = (npiece + K::BPS - 1) / K::BPS;
         const int kofs = hd * K::REGION, vofs = (KPC + hd) * K::REGION;
         if constexpr (PATH == 2) {
-            using Cons = std::conditional_t<sizeof(T) == 1, MmaConsumerFp8<K::TOK / TILE_ROWS>, MmaConsumer<D>>;
+            using Cons = std::conditional_t<sizeof(T) == 1, MmaConsumerFp8<K::TOK / TILE_ROWS, HPW / 8>,
+                                            MmaConsumer<D, HPW / 8>>;
             Cons c;
             c.init(reinterpret_cast<const __nv_bfloat16*>(qbase), group, lane);
             for (int j = sub; j < nstage; j += K::WPH) {
@@ -294,35 +296,42 @@ cudaError_t dispatch_simt(int group, const CUtensorMap& mk, const CUtensorMap& m
                                 : cudaErrorInvalidValue;
         case 8: return KPC == 1 ? launch_decode<T, D, 1, 2, stages_for<T, D>(), 1, BSZ>(mk, mv, p, grid, st)
                                 : cudaErrorInvalidValue;
+        case 16: return KPC == 1 ? launch_decode<T, D, 1, 4, stages_for<T, D>(), 1, BSZ>(mk, mv, p, grid, st)
+                                 : cudaErrorInvalidValue;
         default: return cudaErrorInvalidValue;
     }
+}
+
+// Tensor-core consumers for groups up to HG (8: one 8-wide head tile, 16: two).
+template <int BSZ, int HG>
+cudaError_t dispatch_mma(pkv_dtype kv_dtype, int head_dim, int num_kv_heads, const CUtensorMap& mk,
+                         const CUtensorMap& mv, const Params& p, dim3 grid, cudaStream_t st) {
+    if (kv_dtype == PKV_FP8_E4M3) {
+        // Two KV heads per CTA: each token's 256 contiguous bytes of K (and of V)
+        // are fetched in one go instead of two 128-byte halves by different CTAs.
+        return num_kv_heads % 2 == 0
+                   ? launch_decode<uint8_t, 128, 2, HG, stages_for<uint8_t, 128, 2>(), 2, BSZ>(mk, mv, p, grid, st)
+                   : launch_decode<uint8_t, 128, 2, HG, stages_for<uint8_t, 128>(), 1, BSZ>(mk, mv, p, grid, st);
+    }
+    // bf16: 8-token blocks make 1 KB copies per head, so two KV heads per CTA
+    // (measured on B200, 70B-shaped GQA: +16% at block size 8, within 3% at
+    // 16-64 where halving the CTA count costs long-context, small batches far more).
+    if (HG == 8 && BSZ < 16 && head_dim == 128 && num_kv_heads % 2 == 0)
+        return launch_decode<__nv_bfloat16, 128, 2, HG, stages_for<__nv_bfloat16, 128, 2>(), 2, BSZ>(mk, mv, p, grid,
+                                                                                                   st);
+    return head_dim == 128
+               ? launch_decode<__nv_bfloat16, 128, 2, HG, stages_for<__nv_bfloat16, 128>(), 1, BSZ>(mk, mv, p, grid, st)
+               : launch_decode<__nv_bfloat16, 64, 2, HG, stages_for<__nv_bfloat16, 64>(), 1, BSZ>(mk, mv, p, grid, st);
 }
 
 template <int BSZ>
 cudaError_t dispatch_partitioned(pkv_dtype kv_dtype, bool use_mma, int head_dim, int group, int num_kv_heads,
                                  const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, dim3 grid,
                                  cudaStream_t st) {
-    if (kv_dtype == PKV_FP8_E4M3) {
-        // e4m3 always runs on tensor cores (use_mma). Two KV heads per CTA: each
-        // token's 256 contiguous bytes of K (and of V) are fetched in one go
-        // instead of two 128-byte halves by different CTAs.
-        (void)use_mma;
-        return num_kv_heads % 2 == 0
-                   ? launch_decode<uint8_t, 128, 2, 8, stages_for<uint8_t, 128, 2>(), 2, BSZ>(mk, mv, p, grid, st)
-                   : launch_decode<uint8_t, 128, 2, 8, stages_for<uint8_t, 128>(), 1, BSZ>(mk, mv, p, grid, st);
-    }
-    // bf16 on tensor cores: 8-token blocks make 1 KB copies per head, so two KV
-    // heads per CTA (measured on B200, 70B-shaped GQA: +16% at block size 8,
-    // within 3% at 16-64 where halving the CTA count costs long-context, small
-    // batches far more).
-    if (use_mma && BSZ < 16 && head_dim == 128 && num_kv_heads % 2 == 0)
-        return launch_decode<__nv_bfloat16, 128, 2, 8, stages_for<__nv_bfloat16, 128, 2>(), 2, BSZ>(mk, mv, p, grid, st);
-    if (use_mma)
-        return head_dim == 128
-                   ? launch_decode<__nv_bfloat16, 128, 2, 8, stages_for<__nv_bfloat16, 128>(), 1, BSZ>(mk, mv, p, grid,
-                                                                                                     st)
-                   : launch_decode<__nv_bfloat16, 64, 2, 8, stages_for<__nv_bfloat16, 64>(), 1, BSZ>(mk, mv, p, grid,
-                                                                                                   st);
+    // e4m3 always runs on tensor cores (use_mma is set for it)
+    if (use_mma || kv_dtype == PKV_FP8_E4M3)
+        return group <= 8 ? dispatch_mma<BSZ, 8>(kv_dtype, head_dim, num_kv_heads, mk, mv, p, grid, st)
+                          : dispatch_mma<BSZ, 16>(kv_dtype, head_dim, num_kv_heads, mk, mv, p, grid, st);
     if (kv_dtype == PKV_BF16)
         return head_dim == 128 ? dispatch_simt<__nv_bfloat16, 128, BSZ>(group, mk, mv, p, grid, st)
                                : dispatch_simt<__nv_bfloat16, 64, BSZ>(group, mk, mv, p, grid, st);

@@ -689,7 +689,7 @@ pkv_status pkv_paged_attention_multi_query(void* out, pkv_dtype out_dtype, const
     if (kv_dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
     if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
     if (!block_size_built(block_size)) return PKV_ERR_UNSUPPORTED;
-    if (group != 1 && group != 2 && group != 4 && group != 8) return PKV_ERR_UNSUPPORTED;
+    if (group != 1 && group != 2 && group != 4 && group != 8 && group != 16) return PKV_ERR_UNSUPPORTED;
     if (num_seqs == 0 || num_tokens == 0 || max_query_len == 0) return PKV_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start)
         return PKV_ERR_INVALID_ARG;

@@ -358,20 +358,24 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // masks: past the partition's range, or after the row's position (causal)
             const int tok0 = kv0 + t * TOK + half * HC;
             const int lim = min(pos, kv0 + ntok - 1) - tok0;    // this half's columns 0..lim are visible
-            float mt = kNegInf;
+            // the maximum as eight independent chains joined by a tree (one serial
+            // chain over the 64 values was the softmax's critical path)
+            float e8[8] = {kNegInf, kNegInf, kNegInf, kNegInf, kNegInf, kNegInf, kNegInf, kNegInf};
             if (lim >= HC - 1) {
 #pragma unroll
                 for (int j = 0; j < HC; ++j) {
                     x[j] *= p.scale_log2;
-                    mt = fmaxf(mt, x[j]);
+                    e8[j & 7] = fmaxf(e8[j & 7], x[j]);
                 }
             } else {
 #pragma unroll
                 for (int j = 0; j < HC; ++j) {
                     x[j] = j <= lim ? x[j] * p.scale_log2 : kNegInf;
-                    mt = fmaxf(mt, x[j]);
+                    e8[j & 7] = fmaxf(e8[j & 7], x[j]);
                 }
             }
+            float mt = fmaxf(fmaxf(fmaxf(e8[0], e8[1]), fmaxf(e8[2], e8[3])),
+                             fmaxf(fmaxf(e8[4], e8[5]), fmaxf(e8[6], e8[7])));
             // the row maximum: exchange with the other half through TMEM column
             // 384 + 2 (t % 2) + half (double-buffered by tile parity)
             {
@@ -413,11 +417,11 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const float ref_new = grow ? m_new : m_ref;
             const float ref = ref_new == kNegInf ? 0.f : ref_new;
             uint32_t ph[HC / 2], pl[HC / 2];
-            float psum = 0.f;
+            float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int e = 0; e < HC / 2; ++e) {
                 const float p0 = fast_exp2(x[2 * e] - ref), p1 = fast_exp2(x[2 * e + 1] - ref);
-                psum += p0 + p1;
+                ps8[e & 7] += p0 + p1;
                 ph[e] = pack_bf16(p0, p1);
                 pl[e] = pack_bf16(p0 - bf16lo(ph[e]), p1 - bf16hi(ph[e]));
             }
@@ -449,7 +453,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 l = m_ref == kNegInf ? 0.f : l * fast_exp2(m_ref - m_new);
                 m_ref = m_new;
             }
-            l += psum;
+            l += ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
             // this half's tokens: P high columns [32 half, +32), P low columns 64 + [32 half, +32)
             tmem_st32u(lane_base + s * 128 + half * 32, ph);
             tmem_st32u(lane_base + s * 128 + 64 + half * 32, pl);

@@ -497,3 +497,9 @@ def test_wait_hook_checks_its_arguments_on_host(lib):
     assert f(0, 3, 5_000_000) == 0               # armed ...
     assert f(0, -1, 0) == 0                      # ... and disarmed
     assert f(1, -1, 0) == 0
+
+
+def test_step_timing_checks_its_arguments_on_host(lib):
+    buf = (ctypes.c_float * 4)()
+    assert lib.pkv_step_ctx_set_timing(None, 1) == 1
+    assert lib.pkv_step_ctx_last_timing(None, buf) == 1

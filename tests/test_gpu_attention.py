@@ -148,6 +148,54 @@ def test_edge_contexts(dtype, d, hq, hkv, part):
     assert np.abs(got - ref).max() <= tol
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("bs", [8, 16, 64])
+@pytest.mark.parametrize("part", [0, 16, 64, 512])
+def test_group_16_edge_contexts(dtype, d, bs, part):
+    """Group 16 (32 query heads on 2 KV heads): bf16 runs two 8-wide tensor-core
+    head tiles per KV head, f32 four heads per CUDA-core warp."""
+    dev, ref = _edge_problem(16000 + d + bs, 32, 2, d, dtype, EDGE_LENS, bs=bs)
+    out = _run(dev, partition_tokens=part)
+    torch.cuda.synchronize()
+    assert binding.get_device_error() == 0
+    got = out.cpu().numpy().astype(np.float64)
+    assert np.isfinite(got).all()
+    assert np.array_equal(got[0], np.zeros_like(got[0]))
+    assert np.abs(got - ref).max() <= (1e-5 if dtype == "f32" else 2e-3)
+
+
+def test_group_16_persistent_schedule_is_refused():
+    dev, _ = _edge_problem(17, 32, 2, 128, "bf16", [40, 50])
+    with pytest.raises(binding.PkvError) as e:
+        _run(dev, partition_tokens=-1)
+    assert e.value.status == 2
+
+
+@pytest.mark.parametrize("hq,hkv", [(24, 4), (12, 2), (3, 1)])
+def test_groups_outside_the_built_set_are_refused(hq, hkv):
+    dev, _ = _edge_problem(18, hq, hkv, 128, "bf16", [40, 50])
+    with pytest.raises(binding.PkvError) as e:
+        _run(dev)
+    assert e.value.status == 2
+
+
+@pytest.mark.parametrize("nseq", [256, 300])
+def test_many_short_sequences_partitioned(nseq):
+    """Batches at and above the live-first grid order's sequence limit (256):
+    both grid orders over short, mixed lengths with small partitions."""
+    rng = np.random.default_rng(nseq)
+    lens = [int(x) for x in rng.integers(0, 120, size=nseq)]
+    lens[5] = 0
+    dev, ref = _edge_problem(19 + nseq, 8, 2, 64, "bf16", lens)
+    out = _run(dev, partition_tokens=32)
+    torch.cuda.synchronize()
+    assert binding.get_device_error() == 0
+    got = out.cpu().numpy().astype(np.float64)
+    assert np.array_equal(got[5], np.zeros_like(got[5]))
+    assert np.abs(got - ref).max() <= 2e-3
+
+
 def test_partition_counts_agree():
     dev, ref = _edge_problem(5, 32, 8, 128, "bf16", [3000, 4097, 17, 8191])
     outs = [_run(dev, partition_tokens=p).cpu().numpy() for p in (16, 128, 512, 2048, 8192, 0, -1)]

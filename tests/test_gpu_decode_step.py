@@ -70,3 +70,30 @@ def test_native_step_matches_python_step_and_oracle(hq, hkv, part):
         assert np.abs(out_host.numpy() - ref).max() <= 2e-3
     for a, b in ((caches[0].k_cache, caches[1].k_cache), (caches[0].v_cache, caches[1].v_cache)):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_native_step_phase_timing():
+    """The context's phase timing: every phase measured, the output unchanged."""
+    rng = np.random.default_rng(11)
+    nb, bs, hq, hkv, d, mb = 128, 16, 16, 4, 128, 32
+    c = PagedKVCache(nb, bs, hkv, d, torch.bfloat16, "cuda", free_order=rng.permutation(nb).astype(np.int32),
+                     max_blocks_per_seq=mb)
+    for s, n in enumerate([40, 300, 17]):
+        k = torch.randn((n, hkv, d), device="cuda").bfloat16()
+        c.add_sequence(s, k, k.clone())
+    step = binding.DecodeStep(c.bm, c.k_cache, c.v_cache, max_seqs=4, num_q_heads=hq, max_blocks_per_seq=mb,
+                              out_dtype=torch.float32)
+    ids = np.arange(3, dtype=np.int64)
+    with pytest.raises(binding.PkvError):
+        step.last_timing()                       # nothing timed yet
+    step.set_timing(True)
+    qh = torch.randn((3, hq, d)).bfloat16().pin_memory()
+    kh = torch.randn((3, hkv, d)).bfloat16().pin_memory()
+    out_host = torch.empty((3, hq, d), dtype=torch.float32).pin_memory()
+    step(ids, qh, kh, kh.clone(), out_host, 0.1)
+    t = step.last_timing()
+    assert binding.get_device_error() == 0
+    assert set(t) == {"host_block_manager", "h2d", "kernels", "d2h"}
+    assert all(v >= 0 for v in t.values()) and t["kernels"] > 0
+    assert torch.isfinite(out_host).all()
+    step.set_timing(False)

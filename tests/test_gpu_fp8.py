@@ -72,9 +72,10 @@ def test_fp8_decode_steps_match_oracle(name, part):
 EDGE = [1, 2, 15, 16, 17, 33, 255, 513, 1000]
 
 
-@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 4), (16, 4), (16, 2)])
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 4), (16, 4), (16, 2), (32, 2), (16, 1)])
 @pytest.mark.parametrize("part", [0, 64])
 def test_fp8_edge_contexts(hq, hkv, part):
+    """(32, 2) and (16, 1): group 16, two 8-wide head tiles (two KV heads per CTA, and one)."""
     fp8_edge_case(hq, hkv, part)
 
 

@@ -73,7 +73,8 @@ CASES = {
 
 
 @pytest.mark.parametrize("case", list(CASES))
-@pytest.mark.parametrize("hq,hkv,d", [(4, 4, 128), (8, 2, 128), (16, 2, 64), (8, 2, 64), (16, 4, 128)])
+@pytest.mark.parametrize("hq,hkv,d", [(4, 4, 128), (8, 2, 128), (16, 2, 64), (8, 2, 64), (16, 4, 128), (32, 2, 128),
+                                       (32, 2, 64)])
 @pytest.mark.parametrize("bs", [8, 16, 32, 64])
 @pytest.mark.parametrize("part", [0, 64, 256])
 def test_multi_query_matches_oracle(case, hq, hkv, d, bs, part):
@@ -227,3 +228,16 @@ def test_both_kernels_at_every_block_size(bs):
         torch.cuda.synchronize()
         assert binding.get_device_error() == 0
         assert np.abs(out.cpu().numpy().astype(np.float64) - ref).max() <= 2e-3
+
+
+@pytest.mark.parametrize("ctx", [40, 64, 65, 128, 129, 192, 256, 257, 1000])
+def test_verify_rows_at_kv_tile_boundaries(ctx):
+    """Verify-sized rows (group 8, 4 draft tokens = 32 rows per KV head, the
+    tcgen05 kernel) at contexts on both sides of its 128-token KV tiles; bf16
+    output as well."""
+    dev, ref = _mq_problem(50 + ctx, 64, 8, 128, 16, [ctx, ctx + 7], [4, 4])
+    out = _run(dev)
+    torch.cuda.synchronize()
+    assert binding.get_device_error() == 0
+    assert np.abs(out.cpu().numpy().astype(np.float64) - ref).max() <= 2e-3
+    check_bf16_out(_run(dev, out_dtype=torch.bfloat16), ref)
