@@ -35,7 +35,7 @@ constexpr int Q_OFF = 0;
 constexpr int K_OFF = 2 * HALF;                   // NST stages of K (2 halves each)
 constexpr int V_OFF = K_OFF + NST * 2 * HALF;     // NST stages of V
 constexpr int BAR_OFF = V_OFF + NST * 2 * HALF;
-constexpr int NBAR = 21;
+constexpr int NBAR = 27;
 constexpr int SMEM = 1024 + BAR_OFF + NBAR * 8 + 16;
 constexpr int TMEM_COLS = 512;     // S/P 0 [0,128) S/P 1 [128,256) O [256,384) exchange [384,390)
 constexpr int T_O = 256;
@@ -49,9 +49,13 @@ static_assert(SMEM <= 232448, "shared memory per CTA");
 // tiles t and t + 1 before that wait; on a single barrier that would put the
 // phase two ahead of the waiter, where a parity wait cannot tell it apart.
 // Tile t + 2 cannot arrive before that wait (its S is issued after PV of t).
+// The row-maximum and row-sum exchanges have one barrier per TMEM lane quarter
+// (64 arrivals: the two warps that share those rows), so the eight softmax
+// warps are not lock-stepped every tile (one 256-arrival barrier cost ~700
+// cycles per tile, measured with clock64 stamps).
 enum {
-    B_Q = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_MAX = 15, B_FIN = 16,
-    B_PREADY = 17, B_ODONE = 19, B_DRAIN = 20
+    B_Q = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_MAX = 15, B_FIN = 19,
+    B_PREADY = 23, B_ODONE = 25, B_DRAIN = 26
 };
 
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -186,8 +190,10 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_init(&bar[B_VEMPTY + s], 1);
         }
         for (int s = 0; s < 2; ++s) mbar_init(&bar[B_SFULL + s], 1);
-        mbar_init(&bar[B_MAX], 256);
-        mbar_init(&bar[B_FIN], 256);
+        for (int q = 0; q < 4; ++q) {
+            mbar_init(&bar[B_MAX + q], 64);
+            mbar_init(&bar[B_FIN + q], 64);
+        }
         for (int s = 0; s < 2; ++s) mbar_init(&bar[B_PREADY + s], 256);
         mbar_init(&bar[B_ODONE], 1);
         mbar_init(&bar[B_DRAIN], 1);
@@ -211,12 +217,18 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ---------------- producer: Q once, then K and V tiles into their rings ----------------
-        // The warp loads a tile's block ids with one coalesced load; lane 0 waits
-        // for the stages and issues the copies. K runs ahead of V: K of a tile is
-        // released as soon as S is computed, V only after the PV product.
+        // ---------------- producer: Q once, then the K and V streams ----------------
+        // Lanes 0-15 stream K tiles, lanes 16-31 V tiles, each half-warp waiting
+        // for its own ring: K of a tile is released as soon as S is computed, V
+        // only after the PV product, so a V stage that frees late does not hold
+        // back the next K tile. Each half loads the next tile's block ids while it
+        // waits for this tile's stage (one id per lane), and lane b of a half
+        // issues piece b of the tile (one thread issuing every copy serially was
+        // the bound: a tile of 16-token blocks takes 32 copies).
+        const int kv = lane >> 4, hl = lane & 15;                // stream (0: K, 1: V), lane in the half
+        const unsigned hmask = kv ? 0xffff0000u : 0x0000ffffu;
         bool ok = true;
-        int issued[2] = {0, 0};                                 // tiles whose K / V copies were issued
+        int issued = 0;                                         // tiles whose copies this half issued
         // test hook: the first CTA never issues this tile's K copies (nor arrives
         // on their barrier), so the MMA thread's bounded wait for them runs out
         const int withheld = (blockIdx.x | blockIdx.y | blockIdx.z) == 0 ? p.withhold : -1;
@@ -227,74 +239,82 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         const uint64_t pol = l2_policy_evict_normal();
         const int32_t* bt = p.block_tables + (int64_t)seq * p.max_blocks + blk0;
-        static_assert(TOK / R <= 32, "one id per lane");
-        for (int t = 0; t < ntiles; ++t) {
-            const int s = t % NST;
-            const uint32_t par = ((t / NST) & 1) ^ 1;
-            const int tok_here = min(TOK, ntok - t * TOK);
-            const int np = (tok_here + R - 1) / R;
+        static_assert(TOK / R <= 16, "one piece per lane of a half-warp");
+        auto pieces = [&](int t) { return (min(TOK, ntok - t * TOK) + R - 1) / R; };
+        auto load_id = [&](int t) {
             int id = 0;
-            if (lane < np) {
-                id = __ldg(bt + (t * TOK) / BSZ + lane);
+            if (t < ntiles && hl < pieces(t)) {
+                id = __ldg(bt + (t * TOK) / BSZ + hl);
                 if (id < 0 || id >= p.num_blocks) {
                     flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
                     id = p.num_blocks;                          // zero-filled tile
                 }
             }
-#pragma unroll
-            for (int kv = 0; kv < 2; ++kv) {
-                uint64_t* full = &bar[(kv ? B_VFULL : B_KFULL) + s];
-                const bool skip = kv == 0 && t == withheld;
-                if (lane == 0) {
-                    ok = mbar_wait_bounded(&bar[(kv ? B_VEMPTY : B_KEMPTY) + s], par, p.err, p.wait_ns);
-                    if (ok) {
-                        if (!skip) mbar_arrive_expect_tx(full, np * 2 * R * 128);
-                        issued[kv] = t + 1;
-                    } else {
-                        s_abort = 1;
-                    }
-                }
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;    // also orders the expect-tx before the copies
-                if (!ok) break;
-                // lane b issues piece b: one thread issuing every copy of a tile serially
-                // was the bound (measured: a tile of 16-token blocks takes 32 copies)
-                uint8_t* dst = smem + (kv ? V_OFF : K_OFF) + s * 2 * HALF;
-                const CUtensorMap* map = kv ? &tm_v : &tm_k;
-                if (lane < np && !skip) {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        tma_load_4d(dst + h * HALF + lane * R * 128, map, full, h * 64, kvh, 0, id, pol);
+            return id;
+        };
+        int id = load_id(0);
+        uint8_t* const ring = smem + (kv ? V_OFF : K_OFF);
+        const CUtensorMap* map = kv ? &tm_v : &tm_k;
+        for (int t = 0; t < ntiles; ++t) {
+            const int s = t % NST;
+            const int np = pieces(t);
+            const int id_next = load_id(t + 1);
+            uint64_t* full = &bar[(kv ? B_VFULL : B_KFULL) + s];
+            const bool skip = kv == 0 && t == withheld;
+            if (hl == 0) {
+                ok = mbar_wait_bounded(&bar[(kv ? B_VEMPTY : B_KEMPTY) + s], ((t / NST) & 1) ^ 1, p.err, p.wait_ns);
+                if (ok) {
+                    if (!skip) mbar_arrive_expect_tx(full, np * 2 * R * 128);
+                    issued = t + 1;
+                } else {
+                    s_abort = 1;
                 }
             }
+            ok = __shfl_sync(hmask, ok ? 1 : 0, kv << 4) != 0;    // also orders the expect-tx before the copies
             if (!ok) break;
+            if (hl < np && !skip) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    tma_load_4d(ring + s * 2 * HALF + h * HALF + hl * R * 128, map, full, h * 64, kvh, 0, id, pol);
+            }
+            id = id_next;
         }
-        if (lane == 0 && !ok) {
-            // every copy issued has landed before the CTA moves on
-            for (int kv = 0; kv < 2; ++kv)
-                for (int t = max(0, issued[kv] - NST); t < issued[kv]; ++t)
-                    if (kv != 0 || t != withheld)
-                        mbar_wait_bounded(&bar[(kv ? B_VFULL : B_KFULL) + t % NST], (t / NST) & 1, p.err, p.wait_ns);
+        if (hl == 0) {
+            // every copy this half issued has landed before the CTA moves on (on
+            // the normal path the MMA thread waited for each of them already; after
+            // an abort some may still be in flight)
+            for (int t = max(0, issued - NST); t < issued; ++t)
+                if (kv != 0 || t != withheld)
+                    mbar_wait_bounded(&bar[(kv ? B_VFULL : B_KFULL) + t % NST], (t / NST) & 1, p.err, p.wait_ns);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer (one thread) ----------------
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16(ROWS, TOK, false);
             constexpr uint32_t IDESC_PV = idesc_bf16(ROWS, D, true);
-            const uint32_t q_addr = smem_u32(smem + Q_OFF);
+            // Descriptors of Q, and of K and V at ring stage 0, built once: a
+            // descriptor's start-address field holds (address >> 4), so moving it by
+            // d bytes adds d >> 4 (shared addresses stay below 256 KB, no carry).
+            // Building two descriptors per MMA in the loop made one thread's MMA
+            // issue about as slow as the MMAs themselves (clock64 stamps: ~90 cycles
+            // per tcgen05.mma, 24 per tile).
+            const uint64_t qd = desc_sw128(smem_u32(smem + Q_OFF), 16, 1024);
+            const uint64_t kd = desc_sw128(smem_u32(smem + K_OFF), 16, 1024);
+            const uint64_t vd = desc_sw128(smem_u32(smem + V_OFF), HALF, 1024);
             bool ok = mbar_wait_bounded(&bar[B_Q], 0, p.err, p.wait_ns);
             // PV of tile u: O += P_hi V + P_lo V over the tile's 128 tokens, 8 k-steps of 16
             auto pv = [&](int u) -> bool {
                 if (!mbar_wait_bounded(&bar[B_PREADY + (u & 1)], (u >> 1) & 1, p.err, p.wait_ns)) return false;
                 if (!mbar_wait_bounded(&bar[B_VFULL + u % NST], (u / NST) & 1, p.err, p.wait_ns)) return false;
                 fence_after();
-                const uint32_t v_addr = smem_u32(smem + V_OFF + (u % NST) * 2 * HALF);
+                const uint64_t vs = vd + (uint64_t)(((u % NST) * 2 * HALF) >> 4);
+                const uint32_t pa = tmem + (u & 1) * 128;
 #pragma unroll
                 for (int part_lo = 0; part_lo < 2; ++part_lo) {
 #pragma unroll
                     for (int k = 0; k < TOK / 16; ++k) {
                         // B = V: MN-major (dims contiguous); tokens 16k.. -> 16 rows of 128 B; dim halves HALF apart
-                        const uint64_t b = desc_sw128(v_addr + k * 16 * 128, HALF, 1024);
-                        mma_ts(tmem + T_O, tmem + (u & 1) * 128 + part_lo * 64 + k * 8, b, IDESC_PV,
+                        mma_ts(tmem + T_O, pa + part_lo * 64 + k * 8, vs + (uint64_t)((k * 16 * 128) >> 4), IDESC_PV,
                                (u > 0 || part_lo > 0 || k > 0) ? 1u : 0u);
                     }
                 }
@@ -309,12 +329,11 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 ok = mbar_wait_bounded(&bar[B_KFULL + ks], (t / NST) & 1, p.err, p.wait_ns);
                 if (!ok) break;
                 fence_after();
-                const uint32_t k_addr = smem_u32(smem + K_OFF + ks * 2 * HALF);
+                const uint64_t ksd = kd + (uint64_t)((ks * 2 * HALF) >> 4);
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
-                    const uint64_t a = desc_sw128(q_addr + (k >> 2) * HALF + (k & 3) * 32, 16, 1024);
-                    const uint64_t b = desc_sw128(k_addr + (k >> 2) * HALF + (k & 3) * 32, 16, 1024);
-                    mma_ss(tmem + sb * 128, a, b, IDESC_S, k > 0 ? 1u : 0u);
+                    const uint64_t off = (uint64_t)(((k >> 2) * HALF + (k & 3) * 32) >> 4);
+                    mma_ss(tmem + sb * 128, qd + off, ksd + off, IDESC_S, k > 0 ? 1u : 0u);
                 }
                 commit(&bar[B_SFULL + sb]);
                 commit(&bar[B_KEMPTY + ks]);
@@ -358,24 +377,23 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // masks: past the partition's range, or after the row's position (causal)
             const int tok0 = kv0 + t * TOK + half * HC;
             const int lim = min(pos, kv0 + ntok - 1) - tok0;    // this half's columns 0..lim are visible
-            // the maximum as eight independent chains joined by a tree (one serial
+            // the maximum as four independent chains joined by a tree (one serial
             // chain over the 64 values was the softmax's critical path)
-            float e8[8] = {kNegInf, kNegInf, kNegInf, kNegInf, kNegInf, kNegInf, kNegInf, kNegInf};
+            float e4[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
             if (lim >= HC - 1) {
 #pragma unroll
                 for (int j = 0; j < HC; ++j) {
                     x[j] *= p.scale_log2;
-                    e8[j & 7] = fmaxf(e8[j & 7], x[j]);
+                    e4[j & 3] = fmaxf(e4[j & 3], x[j]);
                 }
             } else {
 #pragma unroll
                 for (int j = 0; j < HC; ++j) {
                     x[j] = j <= lim ? x[j] * p.scale_log2 : kNegInf;
-                    e8[j & 7] = fmaxf(e8[j & 7], x[j]);
+                    e4[j & 3] = fmaxf(e4[j & 3], x[j]);
                 }
             }
-            float mt = fmaxf(fmaxf(fmaxf(e8[0], e8[1]), fmaxf(e8[2], e8[3])),
-                             fmaxf(fmaxf(e8[4], e8[5]), fmaxf(e8[6], e8[7])));
+            float mt = fmaxf(fmaxf(e4[0], e4[1]), fmaxf(e4[2], e4[3]));
             // the row maximum: exchange with the other half through TMEM column
             // 384 + 2 (t % 2) + half (double-buffered by tile parity)
             {
@@ -385,8 +403,8 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                              : "memory");
                 tmem_wait_st();
                 fence_before();
-                mbar_arrive(&bar[B_MAX]);
-                const bool ex = mbar_wait_bounded(&bar[B_MAX], t & 1, p.err, p.wait_ns);
+                mbar_arrive(&bar[B_MAX + quarter]);
+                const bool ex = mbar_wait_bounded(&bar[B_MAX + quarter], t & 1, p.err, p.wait_ns);
                 if (__any_sync(0xffffffffu, !ex || s_abort != 0)) {
                     ok = false;
                     s_abort = 1;
@@ -417,11 +435,11 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const float ref_new = grow ? m_new : m_ref;
             const float ref = ref_new == kNegInf ? 0.f : ref_new;
             uint32_t ph[HC / 2], pl[HC / 2];
-            float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            float ps4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int e = 0; e < HC / 2; ++e) {
                 const float p0 = fast_exp2(x[2 * e] - ref), p1 = fast_exp2(x[2 * e + 1] - ref);
-                ps8[e & 7] += p0 + p1;
+                ps4[e & 3] += p0 + p1;
                 ph[e] = pack_bf16(p0, p1);
                 pl[e] = pack_bf16(p0 - bf16lo(ph[e]), p1 - bf16hi(ph[e]));
             }
@@ -453,7 +471,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 l = m_ref == kNegInf ? 0.f : l * fast_exp2(m_ref - m_new);
                 m_ref = m_new;
             }
-            l += ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
+            l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
             // this half's tokens: P high columns [32 half, +32), P low columns 64 + [32 half, +32)
             tmem_st32u(lane_base + s * 128 + half * 32, ph);
             tmem_st32u(lane_base + s * 128 + 64 + half * 32, pl);
@@ -476,8 +494,8 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                          : "memory");
             tmem_wait_st();
             fence_before();
-            mbar_arrive(&bar[B_FIN]);
-            const bool fin = mbar_wait_bounded(&bar[B_FIN], 0, p.err, p.wait_ns);
+            mbar_arrive(&bar[B_FIN + quarter]);
+            const bool fin = mbar_wait_bounded(&bar[B_FIN + quarter], 0, p.err, p.wait_ns);
             ok = !__any_sync(0xffffffffu, !fin || s_abort != 0);
             if (ok) {
                 fence_after();
