@@ -112,7 +112,12 @@ const char* pkv_status_string(int status);
  *        share of the batch's (sequence, block) tiles, with split sequences
  *        merged inside the kernel (at most 2048 sequences; block_size 16,
  *        f32 / bf16 caches).
- * Partial results live in `workspace` (device memory, at least
+ * With partition_tokens >= 0 and more than one sequence, a small planning
+ * kernel first lists the live (sequence, partition) units longest first (full
+ * partitions, then each sequence's last partition by decreasing size) and the
+ * partition kernel takes them in that order, so long units start first and no
+ * CTA is launched for a partition past a sequence's end before those with work.
+ * The list and the partial results live in `workspace` (device memory, at least
  * pkv_paged_attention_workspace_bytes(...) bytes, 256-byte aligned; it may be
  * NULL when that size is 0). Its contents need no initialisation and are
  * scratch between calls; two calls in flight at once need two workspaces.
@@ -374,12 +379,13 @@ pkv_status pkv_test_withhold_copy(int kernel, int index, unsigned long long wait
 /* One decode step from host buffers ([VP] §3.3 decode, §4.1 copy-on-write)  */
 /* ------------------------------------------------------------------------- */
 /*
- * A step context owns the device buffers one decode step needs for up to
- * max_seqs sequences (the step's q / new K,V / metadata / output / split-K
- * workspace) and two pinned staging slots. Creating it allocates (once);
- * pkv_decode_step allocates nothing. partition_tokens is the schedule the steps
- * will use (same meaning as in pkv_paged_attention_decode). One context serves
- * one stream at a time.
+ * A step context owns what one decode step needs for up to max_seqs sequences:
+ * two slots of device buffers (the step's q / new K,V / metadata / output), the
+ * split-K workspace, two pinned metadata staging slots, and three streams (host
+ * to device copies, kernels, device to host copies) with the events that order
+ * them. Creating it allocates (once); pkv_decode_step allocates nothing.
+ * partition_tokens is the schedule the steps will use (same meaning as in
+ * pkv_paged_attention_decode). One context serves one caller stream at a time.
  */
 typedef struct pkv_step_ctx pkv_step_ctx;
 typedef struct pkv_block_manager pkv_block_manager;
@@ -403,10 +409,20 @@ void pkv_step_ctx_destroy(pkv_step_ctx* ctx);
  *      asynchronous);
  *   3. pkv_copy_blocks for the copy-on-write pairs, pkv_reshape_and_cache for
  *      the new tokens, pkv_paged_attention_decode over the updated contexts;
- *   4. the output [n, Hq, D] (out_dtype of the context) is copied to out_host.
- * k_cache / v_cache are the device caches (the context's block_size). Everything is
- * enqueued on `stream`; synchronise it before reading out_host. A block manager
- * error (PKV_ERR_OUT_OF_BLOCKS) is returned before anything is enqueued.
+ *   4. the output [n, Hq, D] (out_dtype of the context) reaches out_host: a
+ *      page-locked out_host is written directly by the attention kernels through
+ *      its device mapping (no copy after them); pageable memory gets a copy.
+ * k_cache / v_cache are the device caches (the context's block_size).
+ * Ordering: the step's device work starts after everything enqueued on `stream`
+ * before the call, runs on the context's own streams, and `stream` passes the
+ * step only once its output is in out_host: synchronise `stream` (or an event
+ * recorded on it after the call) before reading out_host. Consecutive steps of
+ * one context overlap on the device (step i + 1's host-to-device copies, and a
+ * device-to-host copy if there is one, run while step i's kernels run), so a caller that
+ * waits for step i - 1 after issuing step i keeps the copies off the critical
+ * path; the host buffers of a step must stay untouched until `stream` has passed
+ * it. A block manager error (PKV_ERR_OUT_OF_BLOCKS) is returned before anything
+ * is enqueued.
  */
 pkv_status pkv_decode_step(pkv_step_ctx* ctx, pkv_block_manager* bm, const int64_t* seq_ids, int n,
                            const void* q_host, const void* k_host, const void* v_host,

@@ -21,6 +21,7 @@ constexpr bool block_size_built(int bs) { return bs == 8 || bs == 16 || bs == 32
 constexpr int stage_tokens(int elt_bytes) { return elt_bytes == 1 ? 32 : 16; }
 constexpr int piece_rows(int bs, int elt_bytes) { return bs < stage_tokens(elt_bytes) ? bs : stage_tokens(elt_bytes); }
 constexpr int NTHREADS = 32 * (NCW + 1);
+constexpr int kPlanMaxBins = 4096;   // longest-first schedule: partitions of at most this many blocks
 constexpr float kNegInf = -INFINITY;
 
 struct Params {
@@ -46,6 +47,9 @@ struct Params {
     unsigned long long* counters;   // [B * Hkv]: (epoch << 24) | pieces arrived
     unsigned long long epoch;       // distinct per call
     int team_size;                  // CTAs per team (one KV head each), divides Hkv and the grid
+    // longest-first schedule of the partitioned kernel (plan_units_kernel)
+    uint2* units;                   // [B * C]: {seq << 16 | partition, clamped context length}; NULL: grid order
+    int* unit_count;                // live units listed
     // bounded waits
     unsigned long long wait_ns;     // limit of every mbarrier wait (2 s unless the test hook shortened it)
     int withhold;                   // test hook: ring stage whose copies the first CTA never issues (-1: none)

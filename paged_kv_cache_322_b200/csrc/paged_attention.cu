@@ -145,6 +145,111 @@ __global__ void __launch_bounds__(GROUPS * D) merge_partitions_kernel(const Para
 }
 
 // ---------------------------------------------------------------------------
+// Longest-first schedule of the partitioned kernel (one CTA).
+//
+// A grid sized for the longest context leaves most rows without work when
+// lengths are mixed, and CTAs taken in grid order start long partitions late:
+// measured with per-CTA timestamps, a 7B-shaped batch streamed ~7.5 TB/s while
+// all 444 CTA slots were busy, then spent its last 35 of 210 us finishing late
+// long sequences, and the long-context grid had 5528 empty CTAs among 872 with
+// work. This kernel lists the live (sequence, partition) units: every full
+// partition first, then each sequence's last partition by decreasing size (a
+// sequence of length 0 last: its CTA writes the zero output). Row y of the
+// partition grid takes unit y; rows past the list exit at the end of dispatch.
+// It flags lengths outside [0, ctx_cap] and lists them clamped.
+// ---------------------------------------------------------------------------
+constexpr int kPlanThreads = 256;
+
+// Exclusive scan of one value per thread over the CTA; *total gets the sum.
+__device__ __forceinline__ int cta_exclusive_scan(int v, int* s_warp, int* total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += t;
+    }
+    if (lane == 31) s_warp[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+        int w = lane < kPlanThreads / 32 ? s_warp[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, wi, off);
+            if (lane >= off) wi += t;
+        }
+        if (lane < kPlanThreads / 32) s_warp[lane] = wi - w;
+        if (lane == 31) s_warp[kPlanThreads / 32] = wi;
+    }
+    __syncthreads();
+    const int r = s_warp[wid] + incl - v;
+    *total = s_warp[kPlanThreads / 32];
+    __syncthreads();                                            // s_warp is reused by the next scan
+    return r;
+}
+
+__global__ void __launch_bounds__(kPlanThreads) plan_units_kernel(const Params p) {
+    // the partition kernel may start its CTAs now; they wait for the list in-kernel
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    __shared__ int hist[kPlanMaxBins];                          // tails per size (blocks), then their offsets
+    __shared__ int s_warp[kPlanThreads / 32 + 1];
+    const int B = p.num_seqs, pb = p.part_blocks, bsz = p.block_size, tid = threadIdx.x;
+    for (int b = tid; b < pb; b += kPlanThreads) hist[b] = 0;
+    __syncthreads();
+    // full partitions, listed sequence-major; the tails counted by size
+    int nfull = 0;
+    int ctx_keep = 0;                                           // this thread's length when B fits one pass
+    for (int s0 = 0; s0 < B; s0 += kPlanThreads) {
+        const int sq = s0 + tid;
+        int full = 0, ctx = 0;
+        if (sq < B) {
+            ctx = p.context_lens[sq];
+            if (ctx < 0 || ctx > p.ctx_cap) {
+                flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
+                ctx = ctx < 0 ? 0 : p.ctx_cap;
+            }
+            const int nb = (ctx + bsz - 1) / bsz;
+            full = nb / pb;
+            if (nb % pb != 0 || nb == 0) atomicAdd(&hist[nb % pb], 1);
+        }
+        ctx_keep = ctx;
+        int chunk = 0;
+        const int off = nfull + cta_exclusive_scan(full, s_warp, &chunk);
+        for (int k = 0; k < full; ++k) p.units[off + k] = make_uint2(((unsigned)sq << 16) | (unsigned)k, (unsigned)ctx);
+        nfull += chunk;
+    }
+    // tail offsets in decreasing size: offset(size b) = tails longer than b
+    int ntail = 0;
+    for (int b0 = 0; b0 < pb; b0 += kPlanThreads) {
+        const int b = pb - 1 - (b0 + tid);                        // sizes from the largest down
+        const int h = b >= 0 ? hist[b] : 0;
+        int chunk = 0;
+        const int off = ntail + cta_exclusive_scan(h, s_warp, &chunk);
+        if (b >= 0) hist[b] = nfull + off;
+        ntail += chunk;
+        __syncthreads();
+    }
+    // the tails, each at the next free place of its size
+    for (int s0 = 0; s0 < B; s0 += kPlanThreads) {
+        const int sq = s0 + tid;
+        if (sq < B) {
+            int ctx = ctx_keep;
+            if (B > kPlanThreads) {
+                ctx = p.context_lens[sq];
+                ctx = ctx < 0 ? 0 : (ctx > p.ctx_cap ? p.ctx_cap : ctx);
+            }
+            const int nb = (ctx + bsz - 1) / bsz;
+            if (nb % pb != 0 || nb == 0) {
+                const int at = atomicAdd(&hist[nb % pb], 1);
+                p.units[at] = make_uint2(((unsigned)sq << 16) | (unsigned)(nb / pb), (unsigned)ctx);
+            }
+        }
+    }
+    if (tid == 0) *p.unit_count = nfull + ntail;
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -199,7 +304,14 @@ struct Plan {
     bool persistent;
     int grid;           // CTAs of the persistent schedule
     int team_size;      // CTAs per team (one KV head each)
+    bool longest_first; // partitioned: the plan kernel lists the units (plan_units_kernel)
 };
+
+// Bytes of the unit list at the front of the workspace (longest-first schedule).
+size_t units_bytes(int num_seqs, const Plan& pl) {
+    if (!pl.longest_first) return 0;
+    return (((size_t)num_seqs * pl.num_parts * sizeof(uint2) + sizeof(int)) + 255) & ~size_t(255);
+}
 
 // Schedule for one call.
 //   partition_tokens > 0  : fixed partitions of that many tokens (+ merge kernel).
@@ -225,6 +337,7 @@ bool plan(int num_seqs, int num_kv_heads, int block_size, int max_blocks, int ma
     pl->persistent = false;
     pl->grid = 0;
     pl->team_size = 0;
+    pl->longest_first = false;
     if (partition_tokens == -1) {
         const int64_t max_tiles = (int64_t)num_seqs * num_kv_heads * ((cap + BS - 1) / BS);
         if (num_seqs > persistent_max_seqs() || max_tiles >= INT32_MAX) return false;
@@ -259,6 +372,9 @@ bool plan(int num_seqs, int num_kv_heads, int block_size, int max_blocks, int ma
     if (parts > 65535) return false;
     pl->part_tokens = pt;
     pl->num_parts = parts;
+    // Longest-first order whenever there is more than one sequence to order and
+    // the unit list fits a grid dimension (65535 rows).
+    pl->longest_first = num_seqs >= 2 && (int64_t)num_seqs * parts <= 65535 && pt / BS <= kPlanMaxBins;
     return true;
 }
 
@@ -268,10 +384,11 @@ size_t ws_bytes_for(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
         const size_t parts = (((size_t)2 * pl.grid * group * (head_dim + 2) * 4) + 255) & ~size_t(255);
         return parts + (size_t)num_seqs * num_kv_heads * 8;
     }
-    if (pl.num_parts <= 1) return 0;
+    const size_t ub = units_bytes(num_seqs, pl);
+    if (pl.num_parts <= 1) return ub;
     const size_t rows = (size_t)num_seqs * num_q_heads * pl.num_parts;
     const size_t o_bytes = ((rows * head_dim * 4) + 255) & ~size_t(255);
-    return o_bytes + rows * 2 * 4;
+    return ub + o_bytes + rows * 2 * 4;
 }
 
 }  // namespace attn
@@ -394,15 +511,22 @@ pkv_status decode_impl(void* out, pkv_dtype out_dtype, const void* q, const void
             return PKV_ERR_CUDA;
         return PKV_OK;
     }
-    if (need > 0) {
+    const size_t ub = units_bytes(num_seqs, pl);
+    if (pl.num_parts > 1) {
         const size_t rows = (size_t)num_seqs * num_q_heads * pl.num_parts;
-        p.ws_o = static_cast<float*>(workspace);
-        p.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+        p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ub);
+        p.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ub +
                                            (((rows * head_dim * 4) + 255) & ~size_t(255)));
     }
-
     dim3 grid(num_kv_heads, pl.num_parts, num_seqs);
     cudaError_t e;
+    if (pl.longest_first) {
+        p.units = static_cast<uint2*>(workspace);
+        p.unit_count = reinterpret_cast<int*>(p.units + (size_t)num_seqs * pl.num_parts);
+        plan_units_kernel<<<1, kPlanThreads, 0, st>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return PKV_ERR_CUDA;
+        grid = dim3(num_kv_heads, num_seqs * pl.num_parts, 1);
+    }
     switch (block_size) {
         case 8: e = dispatch_partitioned<8>(kv_dtype, use_mma, head_dim, group, num_kv_heads, mk, mv, p, grid, st); break;
         case 16: e = dispatch_partitioned<16>(kv_dtype, use_mma, head_dim, group, num_kv_heads, mk, mv, p, grid, st); break;

@@ -72,13 +72,27 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     uint64_t* empty = full + STAGES;
     __shared__ volatile int s_abort;
 
-    const int kvh = blockIdx.x * KPC, part = blockIdx.y, seq = blockIdx.z;   // first KV head of this CTA
+    const int kvh = blockIdx.x * KPC;                             // first KV head of this CTA
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    int ctx = p.context_lens[seq];
-    if (ctx < 0 || ctx > p.ctx_cap) {
-        if (threadIdx.x == 0 && part == 0 && kvh == 0) flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
-        ctx = ctx < 0 ? 0 : p.ctx_cap;
+    int part, seq, ctx;
+    if (p.units) {
+        // longest-first schedule: row y of the grid takes the y-th listed unit
+        // (the plan kernel, this launch's programmatic predecessor, wrote the list)
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        const int count = *p.unit_count;
+        const uint2 u = p.units[blockIdx.y];
+        if ((int)blockIdx.y >= count) return;                     // no unit left for this row (uniform)
+        seq = (int)(u.x >> 16);
+        part = (int)(u.x & 0xffffu);
+        ctx = (int)u.y;                                           // clamped (and flagged) by the plan kernel
+    } else {
+        part = blockIdx.y;
+        seq = blockIdx.z;
+        ctx = p.context_lens[seq];
+        if (ctx < 0 || ctx > p.ctx_cap) {
+            if (threadIdx.x == 0 && part == 0 && kvh == 0) flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
+            ctx = ctx < 0 ? 0 : p.ctx_cap;
+        }
     }
     const int nblk_seq = (ctx + BSZ - 1) / BSZ;
     const int nparts = (nblk_seq + p.part_blocks - 1) / p.part_blocks;
@@ -272,6 +286,21 @@ cudaError_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const Pa
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
         if (e != cudaSuccess) return e;
         done_mask.fetch_or(bit);
+    }
+    if (p.units) {
+        // a programmatic dependent of the plan kernel: launched while it runs, the
+        // CTAs wait for its list in-kernel (griddepcontrol.wait)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(NTHREADS);
+        cfg.dynamicSmemBytes = K::SMEM;
+        cfg.stream = stream;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, kern, mk, mv, p);
     }
     kern<<<grid, NTHREADS, K::SMEM, stream>>>(mk, mv, p);
     return cudaGetLastError();

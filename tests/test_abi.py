@@ -334,7 +334,9 @@ def test_workspace_and_partition_rule(lib):
     n = binding.workspace_bytes(16, 32, 8, 128, 16, 2048, 32768, 512)
     rows = 16 * 32 * 64
     assert n >= rows * 128 * 4 + rows * 2 * 4
-    assert binding.workspace_bytes(4, 8, 8, 64, 16, 16, 256, 512) == 0      # one partition
+    # one partition: only the longest-first unit list (B units of 8 bytes + a count, 256-byte rounded)
+    assert binding.workspace_bytes(4, 8, 8, 64, 16, 16, 256, 512) == 256
+    assert binding.workspace_bytes(1, 8, 8, 64, 16, 16, 256, 512) == 0      # one sequence: nothing to order
     assert binding.partition_tokens(16, 32, 8, 128, 16, 2048, 32768, 500) == 512
     # -1 = the persistent, evenly split schedule: per-CTA pieces + one counter per (sequence, KV head)
     assert binding.partition_tokens(64, 32, 32, 128, 16, 128, 2048, -1) == 0
@@ -345,7 +347,7 @@ def test_workspace_and_partition_rule(lib):
     # 0 = library-chosen partitions: long ones while the batch fills the GPU, shorter for small batches
     p7 = binding.partition_tokens(64, 32, 32, 128, 16, 256, 2158, 0)                # 7B-shaped batch
     assert p7 >= 2158 and p7 % 16 == 0                                                # one partition, no merge
-    assert binding.workspace_bytes(64, 32, 32, 128, 16, 256, 2158, 0) == 0
+    assert binding.workspace_bytes(64, 32, 32, 128, 16, 256, 2158, 0) == 768    # the unit list only
     p70 = binding.partition_tokens(128, 64, 8, 128, 16, 512, 4100, 0)               # 70B-shaped batch
     assert -(-4100 // p70) == 2 and p70 <= 2560                                       # two partitions
     assert binding.partition_tokens(1, 32, 8, 128, 16, 2048, 32768, 0) == 256       # one long sequence

@@ -13,8 +13,11 @@ from paged_kv_cache_322_b200.engine import PagedKVCache
 pytestmark = pytest.mark.gpu
 
 
+@pytest.mark.parametrize("pinned_out", [True, False])
 @pytest.mark.parametrize("hq,hkv,part", [(32, 8, 0), (16, 16, -1), (8, 2, 64)])
-def test_native_step_matches_python_step_and_oracle(hq, hkv, part):
+def test_native_step_matches_python_step_and_oracle(hq, hkv, part, pinned_out):
+    """pinned_out: the output buffer is page-locked (the kernels write it through
+    its device mapping) or pageable (a copy after the kernels)."""
     rng = np.random.default_rng(hq + hkv)
     nb, bs, d, mb = 256, 16, 128, 64
     order = rng.permutation(nb).astype(np.int32)
@@ -50,7 +53,9 @@ def test_native_step_matches_python_step_and_oracle(hq, hkv, part):
         kh = torch.from_numpy(kn).bfloat16().pin_memory()
         vh = torch.from_numpy(vn).bfloat16().pin_memory()
         out_py = caches[0].decode_step(ids, qh.cuda(), kh.cuda(), vh.cuda(), scale, partition_tokens=part)
-        out_host = torch.empty((len(ids), hq, d), dtype=torch.float32).pin_memory()
+        out_host = torch.empty((len(ids), hq, d), dtype=torch.float32)
+        if pinned_out:
+            out_host = out_host.pin_memory()
         step(ids, qh, kh, vh, out_host, scale)
         torch.cuda.synchronize()
         assert binding.get_device_error() == 0
@@ -97,3 +102,45 @@ def test_native_step_phase_timing():
     assert all(v >= 0 for v in t.values()) and t["kernels"] > 0
     assert torch.isfinite(out_host).all()
     step.set_timing(False)
+
+
+def test_native_steps_in_flight_together():
+    """Steps issued back to back, each result read only after the next step was
+    issued (the pipelined use): every output equals the one of the same steps run
+    one at a time on a twin cache."""
+    rng = np.random.default_rng(12)
+    nb, bs, hq, hkv, d, mb = 256, 16, 16, 4, 128, 64
+    order = rng.permutation(nb).astype(np.int32)
+    lens = [100, 33, 500, 7]
+    prompts = [(torch.randn((n, hkv, d), device="cuda").bfloat16(), torch.randn((n, hkv, d), device="cuda").bfloat16())
+               for n in lens]
+    caches, steps = [], []
+    for _ in range(2):
+        c = PagedKVCache(nb, bs, hkv, d, torch.bfloat16, "cuda", free_order=order, max_blocks_per_seq=mb)
+        for s_, (k, v) in enumerate(prompts):
+            c.add_sequence(s_, k, v)
+        caches.append(c)
+        steps.append(binding.DecodeStep(c.bm, c.k_cache, c.v_cache, max_seqs=4, num_q_heads=hq, max_blocks_per_seq=mb,
+                                        out_dtype=torch.float32))
+    ids = np.arange(4, dtype=np.int64)
+    inputs = [tuple(torch.randn(shape).bfloat16().pin_memory() for shape in ((4, hq, d), (4, hkv, d), (4, hkv, d)))
+              for _ in range(6)]
+    serial = []
+    for q, k, v in inputs:
+        o = torch.empty((4, hq, d), dtype=torch.float32).pin_memory()
+        steps[0](ids, q, k, v, o, 0.1)
+        torch.cuda.current_stream().synchronize()
+        serial.append(o.clone())
+    outs = [torch.empty((4, hq, d), dtype=torch.float32).pin_memory() for _ in inputs]
+    evs = []
+    for j, (q, k, v) in enumerate(inputs):
+        steps[1](ids, q, k, v, outs[j], 0.1)
+        e = torch.cuda.Event()
+        e.record()
+        evs.append(e)
+        if j >= 1:
+            evs[j - 1].synchronize()
+            assert torch.equal(outs[j - 1], serial[j - 1])
+    evs[-1].synchronize()
+    assert torch.equal(outs[-1], serial[-1])
+    assert binding.get_device_error() == 0

@@ -85,7 +85,9 @@ def test_noalloc_persistent_schedule_after_split_k_leftovers():
     assert (ref - split).abs().max().item() <= TOL
 
 
-def test_noalloc_without_split_needs_no_scratch():
+def test_noalloc_with_one_partition():
+    """Contexts within one partition: no split-K partials, only the schedule's
+    unit list in the array."""
     q, kc, vc, tables, ctx, scale, maxlen = _problem(lens=(5, 40, 300))
     ref = torch.empty(q.shape, dtype=torch.float32, device="cuda")
     binding.paged_attention_decode(ref, q, kc, vc, tables, ctx, scale, max_context_len=maxlen, partition_tokens=512)
