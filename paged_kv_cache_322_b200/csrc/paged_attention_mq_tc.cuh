@@ -6,8 +6,8 @@
 //   S  = Q K^T   M = 128 query rows, N = 128 KV tokens, K = 128 dims  (TMEM, fp32)
 //   O += P V     M = 128 rows, N = 128 dims, K = 128 tokens            (TMEM, fp32)
 //
-// Roles (320 threads): warp 0 streams Q once and K/V tiles (TMA, 128-byte
-// swizzle, three-stage K and V rings); warp 1 owns the TMEM allocation and one of its threads
+// Roles (352 threads): warp 0 loads Q once and streams K tiles, warp 10 streams
+// V tiles (TMA, 128-byte swizzle, three-stage K and V rings); warp 1 owns the TMEM allocation and one of its threads
 // issues every tcgen05.mma; warps 2-9 run the softmax, two threads per query row
 // (its TMEM lane; one thread per half of the columns, the row maximum exchanged
 // through TMEM each tile). The S accumulator
@@ -28,7 +28,7 @@ namespace tc {
 constexpr int ROWS = 128;          // query rows per CTA (UMMA M)
 constexpr int TOK = 128;           // KV tokens per tile
 constexpr int D = 128;
-constexpr int THREADS = 320;      // warp 0 TMA, warp 1 MMA, warps 2-9 softmax (two per row)
+constexpr int THREADS = 352;      // warps 0 / 10 K / V loads, warp 1 MMA, warps 2-9 softmax (two per row)
 constexpr int HALF = 128 * 128;    // one 64-element-wide half of a 128-row operand, bytes
 constexpr int NST = 3;             // K ring and V ring depth
 constexpr int Q_OFF = 0;
@@ -216,52 +216,54 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
-        // ---------------- producer: Q once, then the K and V streams ----------------
-        // Lanes 0-15 stream K tiles, lanes 16-31 V tiles, each half-warp waiting
-        // for its own ring: K of a tile is released as soon as S is computed, V
-        // only after the PV product, so a V stage that frees late does not hold
-        // back the next K tile. Each half loads the next tile's block ids while it
-        // waits for this tile's stage (one id per lane), and lane b of a half
-        // issues piece b of the tile (one thread issuing every copy serially was
-        // the bound: a tile of 16-token blocks takes 32 copies).
-        const int kv = lane >> 4, hl = lane & 15;                // stream (0: K, 1: V), lane in the half
-        const unsigned hmask = kv ? 0xffff0000u : 0x0000ffffu;
+    if (warp == 0 || warp == 10) {
+        // ---------------- producers: Q once, then the K stream (warp 0) and the V stream (warp 10) ----------------
+        // One warp per stream: K of a tile is released as soon as S is computed,
+        // V only after the PV product, so a V stage that frees late does not hold
+        // back the next K tile (two half-warps of one warp could not do this:
+        // their spin loops progressed in lockstep, clock64 stamps showed). Block
+        // ids come 32 at a time, one batch ahead of use, and are checked when
+        // used: loading and checking each tile's ids just before its copies put a
+        // dependent global load (~2,700 cycles) on every tile's critical path.
+        // Lane b issues piece b of a tile.
+        const int kv = warp == 10;                              // stream: 0 K, 1 V
         bool ok = true;
-        int issued = 0;                                         // tiles whose copies this half issued
+        int issued = 0;                                         // tiles whose copies this stream issued
         // test hook: the first CTA never issues this tile's K copies (nor arrives
         // on their barrier), so the MMA thread's bounded wait for them runs out
         const int withheld = (blockIdx.x | blockIdx.y | blockIdx.z) == 0 ? p.withhold : -1;
-        if (lane == 0) {
+        if (warp == 0 && lane == 0) {
             mbar_arrive_expect_tx(&bar[B_Q], 2 * HALF);
             for (int h = 0; h < 2; ++h)
                 tma_load_3d(smem + Q_OFF + h * HALF, &tm_q, &bar[B_Q], h * 64, kvh * G, q0 + row_begin / G);
         }
         const uint64_t pol = l2_policy_evict_normal();
         const int32_t* bt = p.block_tables + (int64_t)seq * p.max_blocks + blk0;
-        static_assert(TOK / R <= 16, "one piece per lane of a half-warp");
-        auto pieces = [&](int t) { return (min(TOK, ntok - t * TOK) + R - 1) / R; };
-        auto load_id = [&](int t) {
-            int id = 0;
-            if (t < ntiles && hl < pieces(t)) {
-                id = __ldg(bt + (t * TOK) / BSZ + hl);
-                if (id < 0 || id >= p.num_blocks) {
-                    flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
-                    id = p.num_blocks;                          // zero-filled tile
-                }
-            }
-            return id;
-        };
-        int id = load_id(0);
+        constexpr int PPT = TOK / R;                            // pieces (blocks) per tile, divides 32
+        static_assert(PPT <= 32 && 32 % PPT == 0, "a tile's block ids sit in one batch of 32");
+        const int nblk = (ntok + BSZ - 1) / BSZ;                // blocks of this CTA's KV range
+        auto load_batch = [&](int b) { return 32 * b + lane < nblk ? __ldg(bt + 32 * b + lane) : 0; };
+        int batch = 0;
+        int ids = load_batch(0), ids_next = load_batch(1);
         uint8_t* const ring = smem + (kv ? V_OFF : K_OFF);
         const CUtensorMap* map = kv ? &tm_v : &tm_k;
         for (int t = 0; t < ntiles; ++t) {
             const int s = t % NST;
-            const int np = pieces(t);
-            const int id_next = load_id(t + 1);
+            const int np = (min(TOK, ntok - t * TOK) + R - 1) / R;
+            const int j0 = t * PPT;                             // first block of the tile
+            if (j0 / 32 != batch) {
+                batch = j0 / 32;
+                ids = ids_next;
+                ids_next = load_batch(batch + 1);
+            }
+            int id = __shfl_sync(0xffffffffu, ids, (j0 & 31) + (lane < PPT ? lane : 0));
+            if (lane < np && (id < 0 || id >= p.num_blocks)) {
+                flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
+                id = p.num_blocks;                              // zero-filled tile
+            }
             uint64_t* full = &bar[(kv ? B_VFULL : B_KFULL) + s];
             const bool skip = kv == 0 && t == withheld;
-            if (hl == 0) {
+            if (lane == 0) {
                 ok = mbar_wait_bounded(&bar[(kv ? B_VEMPTY : B_KEMPTY) + s], ((t / NST) & 1) ^ 1, p.err, p.wait_ns);
                 if (ok) {
                     if (!skip) mbar_arrive_expect_tx(full, np * 2 * R * 128);
@@ -270,17 +272,16 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     s_abort = 1;
                 }
             }
-            ok = __shfl_sync(hmask, ok ? 1 : 0, kv << 4) != 0;    // also orders the expect-tx before the copies
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;    // also orders the expect-tx before the copies
             if (!ok) break;
-            if (hl < np && !skip) {
+            if (lane < np && !skip) {
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
-                    tma_load_4d(ring + s * 2 * HALF + h * HALF + hl * R * 128, map, full, h * 64, kvh, 0, id, pol);
+                    tma_load_4d(ring + s * 2 * HALF + h * HALF + lane * R * 128, map, full, h * 64, kvh, 0, id, pol);
             }
-            id = id_next;
         }
-        if (hl == 0) {
-            // every copy this half issued has landed before the CTA moves on (on
+        if (lane == 0) {
+            // every copy this stream issued has landed before the CTA moves on (on
             // the normal path the MMA thread waited for each of them already; after
             // an abort some may still be in flight)
             for (int t = max(0, issued - NST); t < issued; ++t)
