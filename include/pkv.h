@@ -106,8 +106,10 @@ const char* pkv_status_string(int status);
  *   > 0  contexts are cut into partitions of that many tokens (rounded up to a
  *        multiple of block_size), processed in parallel and merged exactly with
  *        a log-sum-exp reduction;
- *   0    the same, with the partition length picked from the shapes (long
- *        partitions whenever the batch still fills the GPU);
+ *   0    the same, with the partition length picked from the shapes: the
+ *        fewest partitions (of at least 256 tokens) whose units fill about
+ *        one wave of the GPU, each sequence's count estimated from
+ *        max_context_len with lengths spread over its upper half;
  *   -1   PKV_SCHEDULE_PERSISTENT: two CTAs per SM, each streaming an equal
  *        share of the batch's (sequence, block) tiles, with split sequences
  *        merged inside the kernel (at most 2048 sequences; block_size 16,

@@ -344,13 +344,21 @@ def test_workspace_and_partition_rule(lib):
     assert n >= 64 * 32 * 8 and n < 32 * 2 ** 20
     with pytest.raises(binding.PkvError):
         binding.workspace_bytes(4096, 32, 8, 128, 16, 64, 1024, -1)   # more than 2048 sequences
-    # 0 = library-chosen partitions: long ones while the batch fills the GPU, shorter for small batches
+    # 0 = library-chosen partitions: the fewest that fill about one wave (3 CTAs x 148 SMs = 444
+    # units), a sequence's partitions estimated at 16 lengths spread over [cap / 2, cap]
     p7 = binding.partition_tokens(64, 32, 32, 128, 16, 256, 2158, 0)                # 7B-shaped batch
     assert p7 >= 2158 and p7 % 16 == 0                                                # one partition, no merge
     assert binding.workspace_bytes(64, 32, 32, 128, 16, 256, 2158, 0) == 768    # the unit list only
-    p70 = binding.partition_tokens(128, 64, 8, 128, 16, 512, 4100, 0)               # 70B-shaped batch
-    assert -(-4100 // p70) == 2 and p70 <= 2560                                       # two partitions
-    assert binding.partition_tokens(1, 32, 8, 128, 16, 2048, 32768, 0) == 256       # one long sequence
+    p70 = binding.partition_tokens(128, 64, 8, 128, 16, 512, 4100, 0)               # 70B-shaped batch: 1024 units
+    assert p70 >= 4100
+    assert binding.workspace_bytes(128, 64, 8, 128, 16, 512, 4100, 0) == 1280   # 128 units + count
+    p32 = binding.partition_tokens(32, 64, 8, 128, 16, 512, 4100, 0)                # 256 units per partition
+    assert -(-4100 // p32) == 2 and p32 == 2064                                       # two: 512 units
+    # one sequence at its full length: 8 heads x 56 partitions = 448 units >= 444 (55 give 440)
+    assert binding.partition_tokens(1, 32, 8, 128, 16, 2048, 32768, 0) == 592
+    assert binding.partition_tokens(1, 32, 8, 128, 16, 2048, 300, 0) == 304        # short: one partition
+    assert binding.partition_tokens(1, 32, 8, 128, 16, 2048, 600, 0) == 304        # two even ones, not 256+256+88
+    assert binding.partition_tokens(1, 32, 8, 128, 16, 2048, 100, 0) == 256        # below the floor: one
 
 
 @pytest.mark.parametrize("seed", range(12))
