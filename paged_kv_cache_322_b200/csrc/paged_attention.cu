@@ -213,6 +213,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_units_kernel(const Params p
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __shared__ int hist[kPlanMaxBins];                          // tails per size (blocks), then their offsets
     __shared__ int s_warp[kPlanThreads / 32 + 1];
+    __shared__ int s_first[kPlanThreads];                       // a pass's first full unit per sequence
+    __shared__ int s_ctx[kPlanThreads];
     const int B = p.num_seqs, pb = p.part_blocks, bsz = p.block_size, tid = threadIdx.x;
     for (int b = tid; b < pb; b += kPlanThreads) hist[b] = 0;
     __syncthreads();
@@ -234,9 +236,23 @@ __global__ void __launch_bounds__(kPlanThreads) plan_units_kernel(const Params p
         }
         ctx_keep = ctx;
         int chunk = 0;
-        const int off = nfull + cta_exclusive_scan(full, s_warp, &chunk);
-        for (int k = 0; k < full; ++k) p.units[off + k] = make_uint2(((unsigned)sq << 16) | (unsigned)k, (unsigned)ctx);
+        const int off = cta_exclusive_scan(full, s_warp, &chunk);
+        s_first[tid] = off;
+        s_ctx[tid] = ctx;
+        __syncthreads();
+        // the pass's full units, spread over the threads: unit u belongs to the
+        // last sequence whose first unit is <= u (binary search)
+        for (int u = tid; u < chunk; u += kPlanThreads) {
+            int lo = 0, hi = kPlanThreads - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (s_first[mid] <= u) lo = mid; else hi = mid - 1;
+            }
+            p.units[nfull + u] = make_uint2(((unsigned)(s0 + lo) << 16) | (unsigned)(u - s_first[lo]),
+                                            (unsigned)s_ctx[lo]);
+        }
         nfull += chunk;
+        __syncthreads();                                        // s_first / s_ctx are reused by the next pass
     }
     // tail offsets in decreasing size: offset(size b) = tails longer than b
     int ntail = 0;

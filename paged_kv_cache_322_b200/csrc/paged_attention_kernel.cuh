@@ -74,6 +74,20 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
     const int kvh = blockIdx.x * KPC;                             // first KV head of this CTA
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // Barriers and tensor-map prefetch first: under the longest-first schedule
+    // this overlaps the plan kernel, which the unit read below waits for.
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], PATH == 1 ? NCW : KPC);
+        }
+        s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
     int part, seq, ctx;
     if (p.units) {
         // longest-first schedule: row y of the grid takes the y-th listed unit
@@ -104,18 +118,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     const int group = p.group;
     const int64_t qh0 = (int64_t)kvh * group;                     // first query head of this KV head
 
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < STAGES; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], PATH == 1 ? NCW : KPC);
-        }
-        s_abort = 0;
-        fence_barrier_init();
-    }
-    if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_v);
-    }
     __syncthreads();
 
     float* red_o = reinterpret_cast<float*>(smem);

@@ -9,8 +9,11 @@
 // Roles (352 threads): warp 0 loads Q once and streams K tiles, warp 10 streams
 // V tiles (TMA, 128-byte swizzle, three-stage K and V rings); warp 1 owns the TMEM allocation and one of its threads
 // issues every tcgen05.mma; warps 2-9 run the softmax, two threads per query row
-// (its TMEM lane; one thread per half of the columns, the row maximum exchanged
-// through TMEM each tile). The S accumulator
+// (its TMEM lane). Each of the two runs an online softmax of its own over one
+// half of every tile's tokens (0-63 or 64-127) with its own O accumulator, so
+// the two never wait for each other inside the loop; they combine their (m, l)
+// and O once, at the end (exchanging the row maximum every tile instead cost
+// each tile's softmax ~640 cycles of waiting, clock64 stamps). The S accumulator
 // is double-buffered, so S of tile t+1 is computed while the softmax of tile t
 // runs. P stays in TMEM, written over its own S buffer, as two bf16 parts (high,
 // and the rounding residue) that both multiply V (the A operand read from TMEM),
@@ -35,10 +38,10 @@ constexpr int Q_OFF = 0;
 constexpr int K_OFF = 2 * HALF;                   // NST stages of K (2 halves each)
 constexpr int V_OFF = K_OFF + NST * 2 * HALF;     // NST stages of V
 constexpr int BAR_OFF = V_OFF + NST * 2 * HALF;
-constexpr int NBAR = 27;
+constexpr int NBAR = 23;
 constexpr int SMEM = 1024 + BAR_OFF + NBAR * 8 + 16;
-constexpr int TMEM_COLS = 512;     // S/P 0 [0,128) S/P 1 [128,256) O [256,384) exchange [384,390)
-constexpr int T_O = 256;
+constexpr int TMEM_COLS = 512;     // S/P 0 [0,128) S/P 1 [128,256) O of token half 0 [256,384), of half 1 [384,512)
+constexpr int T_O = 256;           // O of token half h at T_O + 128 h
 // P of tile t is written over S of tile t (high part in the buffer's first 64
 // columns, low part in the next 64): the buffer is free once S is read, and
 // S of tile t + 2 is issued after the PV product that reads P of tile t.
@@ -49,13 +52,11 @@ static_assert(SMEM <= 232448, "shared memory per CTA");
 // tiles t and t + 1 before that wait; on a single barrier that would put the
 // phase two ahead of the waiter, where a parity wait cannot tell it apart.
 // Tile t + 2 cannot arrive before that wait (its S is issued after PV of t).
-// The row-maximum and row-sum exchanges have one barrier per TMEM lane quarter
-// (64 arrivals: the two warps that share those rows), so the eight softmax
-// warps are not lock-stepped every tile (one 256-arrival barrier cost ~700
-// cycles per tile, measured with clock64 stamps).
+// The final (m, l) exchange of a row's two threads has one barrier per TMEM
+// lane quarter (64 arrivals: the two warps that share those rows).
 enum {
-    B_Q = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_MAX = 15, B_FIN = 19,
-    B_PREADY = 23, B_ODONE = 25, B_DRAIN = 26
+    B_Q = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_FIN = 15,
+    B_PREADY = 19, B_ODONE = 21, B_DRAIN = 22
 };
 
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -190,10 +191,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_init(&bar[B_VEMPTY + s], 1);
         }
         for (int s = 0; s < 2; ++s) mbar_init(&bar[B_SFULL + s], 1);
-        for (int q = 0; q < 4; ++q) {
-            mbar_init(&bar[B_MAX + q], 64);
-            mbar_init(&bar[B_FIN + q], 64);
-        }
+        for (int q = 0; q < 4; ++q) mbar_init(&bar[B_FIN + q], 64);
         for (int s = 0; s < 2; ++s) mbar_init(&bar[B_PREADY + s], 256);
         mbar_init(&bar[B_ODONE], 1);
         mbar_init(&bar[B_DRAIN], 1);
@@ -303,7 +301,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const uint64_t kd = desc_sw128(smem_u32(smem + K_OFF), 16, 1024);
             const uint64_t vd = desc_sw128(smem_u32(smem + V_OFF), HALF, 1024);
             bool ok = mbar_wait_bounded(&bar[B_Q], 0, p.err, p.wait_ns);
-            // PV of tile u: O += P_hi V + P_lo V over the tile's 128 tokens, 8 k-steps of 16
+            // PV of tile u: O_h += P_hi V + P_lo V over token half h (64 tokens, 4 k-steps of 16)
             auto pv = [&](int u) -> bool {
                 if (!mbar_wait_bounded(&bar[B_PREADY + (u & 1)], (u >> 1) & 1, p.err, p.wait_ns)) return false;
                 if (!mbar_wait_bounded(&bar[B_VFULL + u % NST], (u / NST) & 1, p.err, p.wait_ns)) return false;
@@ -311,14 +309,16 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const uint64_t vs = vd + (uint64_t)(((u % NST) * 2 * HALF) >> 4);
                 const uint32_t pa = tmem + (u & 1) * 128;
 #pragma unroll
-                for (int part_lo = 0; part_lo < 2; ++part_lo) {
+                for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
-                    for (int k = 0; k < TOK / 16; ++k) {
-                        // B = V: MN-major (dims contiguous); tokens 16k.. -> 16 rows of 128 B; dim halves HALF apart
-                        mma_ts(tmem + T_O, pa + part_lo * 64 + k * 8, vs + (uint64_t)((k * 16 * 128) >> 4), IDESC_PV,
-                               (u > 0 || part_lo > 0 || k > 0) ? 1u : 0u);
-                    }
-                }
+                    for (int part_lo = 0; part_lo < 2; ++part_lo)
+#pragma unroll
+                        for (int k = 0; k < TOK / 32; ++k)
+                            // A = P: tokens 64 hf + 16 k .. in columns 32 hf + 8 k .. (+64: the low part);
+                            // B = V: MN-major (dims contiguous), those tokens' rows; dim halves HALF apart
+                            mma_ts(tmem + T_O + hf * 128, pa + part_lo * 64 + hf * 32 + k * 8,
+                                   vs + (uint64_t)(((hf * 64 + k * 16) * 128) >> 4), IDESC_PV,
+                                   (u > 0 || part_lo > 0 || k > 0) ? 1u : 0u);
                 commit(&bar[B_ODONE]);
                 commit(&bar[B_VEMPTY + u % NST]);
                 return true;
@@ -349,9 +349,9 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     } else {
         // ---------------- softmax: two threads per query row ----------------
         // Warps 2-9: warp w reads TMEM lanes 32 (w % 4) .. (its rows) and column
-        // half h = (w - 2) / 4 of every 128-wide buffer, so two warps per SM
-        // sub-partition hide each other's latencies. The two halves of a row
-        // combine their maxima each tile through two free TMEM columns.
+        // half h = (w - 2) / 4 of every 128-wide S buffer (tokens 64 h .. 64 h + 63
+        // of the tile), so two warps per SM sub-partition hide each other's
+        // latencies. Each thread's (m, l) and O_h cover its half's tokens only.
         const int quarter = warp & 3;                           // TMEM lanes this warp may access
         const int half = (warp - 2) >> 2;                       // columns [64 half, 64 half + 64)
         const int lr = quarter * 32 + lane;                     // row of the tile = TMEM lane
@@ -360,7 +360,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const int pos = qi < n ? c - n + qi : -1;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         constexpr int HC = TOK / 2;                             // columns per thread
-        float m_ref = kNegInf, l = 0.f;                         // l: this half's share of the row sum
+        float m_ref = kNegInf, l = 0.f;                         // this half's running reference and sum
         bool ok = true;
         for (int t = 0; t < ntiles; ++t) {
             const int s = t & 1;
@@ -394,28 +394,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     e4[j & 3] = fmaxf(e4[j & 3], x[j]);
                 }
             }
-            float mt = fmaxf(fmaxf(e4[0], e4[1]), fmaxf(e4[2], e4[3]));
-            // the row maximum: exchange with the other half through TMEM column
-            // 384 + 2 (t % 2) + half (double-buffered by tile parity)
-            {
-                const uint32_t xc = 384 + 2 * (t & 1);
-                uint32_t v = __float_as_uint(mt);
-                asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(lane_base + xc + half), "r"(v)
-                             : "memory");
-                tmem_wait_st();
-                fence_before();
-                mbar_arrive(&bar[B_MAX + quarter]);
-                const bool ex = mbar_wait_bounded(&bar[B_MAX + quarter], t & 1, p.err, p.wait_ns);
-                if (__any_sync(0xffffffffu, !ex || s_abort != 0)) {
-                    ok = false;
-                    s_abort = 1;
-                    break;
-                }
-                fence_after();
-                asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v) : "r"(lane_base + xc + (half ^ 1)));
-                tmem_wait_ld();
-                mt = fmaxf(mt, __uint_as_float(v));
-            }
+            const float mt = fmaxf(fmaxf(e4[0], e4[1]), fmaxf(e4[2], e4[3]));
             const float m_new = fmaxf(m_ref, mt);
             const bool grow = m_new > m_ref + 8.f;              // also true when m_ref is -inf and the row sees a token
             // V rows past the range (the unwritten tail of the last block, or a stage
@@ -444,11 +423,11 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 ph[e] = pack_bf16(p0, p1);
                 pl[e] = pack_bf16(p0 - bf16lo(ph[e]), p1 - bf16hi(ph[e]));
             }
-            // O must be rescaled only when a row's maximum grew past its reference;
-            // then the PV product of tile t - 1 has to be complete first. S of this
-            // tile being complete already implies PV of tile t - 2 is (one commit
-            // covers every earlier MMA), so O-done is at most one phase behind and
-            // its parity wait is exact. Each half rescales its 64 columns of O.
+            // O_h must be rescaled only when this half's maximum grew past its
+            // reference; then the PV product of tile t - 1 has to be complete first.
+            // S of this tile being complete already implies PV of tile t - 2 is (one
+            // commit covers every earlier MMA), and PV of tile t needs this thread's
+            // P, so O-done is at most one phase behind and its parity wait is exact.
             if (t > 0 && __any_sync(0xffffffffu, grow && m_ref != kNegInf)) {
                 const bool done = mbar_wait_bounded(&bar[B_ODONE], (t - 1) & 1, p.err, p.wait_ns);
                 if (__any_sync(0xffffffffu, !done || s_abort != 0)) {
@@ -459,13 +438,13 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 fence_after();
                 const float alpha = (grow && m_ref != kNegInf) ? fast_exp2(m_ref - m_new) : 1.f;
 #pragma unroll
-                for (int ch = 0; ch < HC / 32; ++ch) {
+                for (int ch = 0; ch < D / 32; ++ch) {
                     float o[32];
-                    tmem_ld32(lane_base + T_O + half * HC + ch * 32, o);
+                    tmem_ld32(lane_base + T_O + half * 128 + ch * 32, o);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[i] *= alpha;
-                    tmem_st32(lane_base + T_O + half * HC + ch * 32, o);
+                    tmem_st32(lane_base + T_O + half * 128 + ch * 32, o);
                 }
             }
             if (grow) {
@@ -480,8 +459,8 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             fence_before();
             mbar_arrive(&bar[B_PREADY + s]);
         }
-        // the last PV, then the row sum of both halves, then this half of the row's
-        // output (or of the partition's partial)
+        // the last PV, then the two halves' (m, l) combined, then this thread's 64
+        // dims of the row's output (or of the partition's partial) from O_0 and O_1
         if (ok && ntiles > 0) {
             // O-done may be two phases behind here, where a parity wait cannot tell
             // them apart: wait for the single-use drain barrier the MMA thread
@@ -489,9 +468,13 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const bool done = mbar_wait_bounded(&bar[B_DRAIN], 0, p.err, p.wait_ns);
             ok = !__any_sync(0xffffffffu, !done || s_abort != 0);
         }
+        float m_oth = kNegInf, l_oth = 0.f;
         if (ok) {
-            uint32_t v = __float_as_uint(l);
-            asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(lane_base + 388 + half), "r"(v)
+            // every MMA is complete, so the S columns are free: (m, l) of half h in
+            // columns 2 h, 2 h + 1 of this row's lane
+            uint32_t v2[2] = {__float_as_uint(m_ref), __float_as_uint(l)};
+            asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(lane_base + 2 * half),
+                         "r"(v2[0]), "r"(v2[1])
                          : "memory");
             tmem_wait_st();
             fence_before();
@@ -500,44 +483,54 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             ok = !__any_sync(0xffffffffu, !fin || s_abort != 0);
             if (ok) {
                 fence_after();
-                asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v) : "r"(lane_base + 388 + (half ^ 1)));
+                asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];"
+                             : "=r"(v2[0]), "=r"(v2[1])
+                             : "r"(lane_base + 2 * (half ^ 1)));
                 tmem_wait_ld();
-                l += __uint_as_float(v);
+                m_oth = __uint_as_float(v2[0]);
+                l_oth = __uint_as_float(v2[1]);
             }
         }
         if (ok) {
-            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const float M = fmaxf(m_ref, m_oth);
+            const float w_me = m_ref == kNegInf ? 0.f : fast_exp2(m_ref - M);
+            const float w_oth = m_oth == kNegInf ? 0.f : fast_exp2(m_oth - M);
+            const float L = l * w_me + l_oth * w_oth;
+            const float inv = L > 0.f ? 1.f / L : 0.f;
+            const float w0 = (half == 0 ? w_me : w_oth) * inv, w1 = (half == 0 ? w_oth : w_me) * inv;
             const bool live = qi < n;
             const int64_t qh = (int64_t)(q0 + (live ? qi : 0)) * p.num_q_heads + kvh * G + hh;
 #pragma unroll
             for (int ch = 0; ch < HC / 32; ++ch) {
-                float o[32];
+                float o[32], o1[32];
                 const int d0 = half * HC + ch * 32;
                 tmem_ld32(lane_base + T_O + d0, o);
+                tmem_ld32(lane_base + T_O + 128 + d0, o1);
                 tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[i] = o[i] * w0 + o1[i] * w1;
                 if (live) {
                     // the thread's 32 dims are contiguous: 16-byte stores
                     if (direct && !p.out_f32) {
                         uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + qh * D + d0);
 #pragma unroll
                         for (int v4 = 0; v4 < 4; ++v4)
-                            dst[v4] = make_uint4(pack_bf16(o[8 * v4] * inv, o[8 * v4 + 1] * inv),
-                                                 pack_bf16(o[8 * v4 + 2] * inv, o[8 * v4 + 3] * inv),
-                                                 pack_bf16(o[8 * v4 + 4] * inv, o[8 * v4 + 5] * inv),
-                                                 pack_bf16(o[8 * v4 + 6] * inv, o[8 * v4 + 7] * inv));
+                            dst[v4] = make_uint4(pack_bf16(o[8 * v4], o[8 * v4 + 1]), pack_bf16(o[8 * v4 + 2], o[8 * v4 + 3]),
+                                                 pack_bf16(o[8 * v4 + 4], o[8 * v4 + 5]),
+                                                 pack_bf16(o[8 * v4 + 6], o[8 * v4 + 7]));
                     } else {
                         float* dst = direct ? static_cast<float*>(p.out) + qh * D + d0
                                             : p.ws_o + (qh * p.num_parts + part) * D + d0;
 #pragma unroll
                         for (int v4 = 0; v4 < 8; ++v4)
-                            reinterpret_cast<float4*>(dst)[v4] = make_float4(o[4 * v4] * inv, o[4 * v4 + 1] * inv,
-                                                                             o[4 * v4 + 2] * inv, o[4 * v4 + 3] * inv);
+                            reinterpret_cast<float4*>(dst)[v4] =
+                                make_float4(o[4 * v4], o[4 * v4 + 1], o[4 * v4 + 2], o[4 * v4 + 3]);
                     }
                 }
             }
             if (live && !direct && half == 0) {
-                p.ws_ml[(qh * p.num_parts + part) * 2 + 0] = m_ref;
-                p.ws_ml[(qh * p.num_parts + part) * 2 + 1] = l;
+                p.ws_ml[(qh * p.num_parts + part) * 2 + 0] = M;
+                p.ws_ml[(qh * p.num_parts + part) * 2 + 1] = L;
             }
         }
     }
