@@ -22,6 +22,9 @@ constexpr int stage_tokens(int elt_bytes) { return elt_bytes == 1 ? 32 : 16; }
 constexpr int piece_rows(int bs, int elt_bytes) { return bs < stage_tokens(elt_bytes) ? bs : stage_tokens(elt_bytes); }
 constexpr int NTHREADS = 32 * (NCW + 1);
 constexpr int kPlanMaxBins = 4096;   // longest-first schedule: partitions of at most this many blocks
+// Partitions per context from which the decode grid works through the unit list
+// in about one wave (paged_attention_kernel.cuh, launch_decode).
+constexpr int kLoopParts = 8;
 constexpr float kNegInf = -INFINITY;
 
 struct Params {
@@ -623,6 +626,8 @@ cudaError_t launch_persistent(bool bf16, bool use_mma, int head_dim, int group, 
                               const CUtensorMap& mv, const Params& p, int grid, cudaStream_t st);
 int persistent_ctas_per_sm();
 int persistent_max_seqs();
+// SMs of the current device (paged_attention.cu).
+int num_sms();
 
 }  // namespace attn
 }  // namespace pkv

@@ -61,7 +61,9 @@ struct Kern {
     static_assert(PATH == 1 || STAGES % WPH == 0, "ring depth must be a multiple of the warps per head");
 };
 
-template <typename T, int D, int PATH, int HPW, int STAGES, int KPC, int BSZ>
+// LOOP: the CTA works through the unit list (a grid of about one wave; see below);
+// without it every CTA takes one unit (row) and the kernel has no loop at all.
+template <typename T, int D, int PATH, int HPW, int STAGES, int KPC, int BSZ, bool LOOP>
 __global__ void __launch_bounds__(NTHREADS, 3)
 paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const Params p) {
@@ -88,14 +90,27 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
     }
+    // Longest-first schedule: the plan kernel, this launch's programmatic
+    // predecessor, listed the units, and row y of the grid takes listed row y.
+    // With LOOP (contexts spanning many partitions, where most of the B x C
+    // rows would find no unit: ~7000 such CTAs kept a long-context launch busy
+    // ~6 us past its last unit) the grid is about one wave and row y also takes
+    // listed rows y + gridDim.y, y + 2 gridDim.y, ... The ring's barriers carry
+    // over from unit to unit: `base` counts the stages this CTA streamed before
+    // the current unit, and every unit ends with a CTA barrier (the reduction
+    // scratch aliases the ring), so a unit's first stages never meet an
+    // unconsumed stage of the one before.
+    int count = 1;
+    if (p.units) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        count = *p.unit_count;
+    }
+    uint32_t base = 0;
+    for (int row = blockIdx.y;;) {
     int part, seq, ctx;
     if (p.units) {
-        // longest-first schedule: row y of the grid takes the y-th listed unit
-        // (the plan kernel, this launch's programmatic predecessor, wrote the list)
-        asm volatile("griddepcontrol.wait;" ::: "memory");
-        const int count = *p.unit_count;
-        const uint2 u = p.units[blockIdx.y];
-        if ((int)blockIdx.y >= count) return;                     // no unit left for this row (uniform)
+        if (row >= count) return;                                 // no unit left for this row (uniform)
+        const uint2 u = p.units[row];
         seq = (int)(u.x >> 16);
         part = (int)(u.x & 0xffffu);
         ctx = (int)u.y;                                           // clamped (and flagged) by the plan kernel
@@ -115,10 +130,11 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     const int nblk = max(0, min(p.part_blocks, nblk_seq - blk0));
     const int ntok = max(0, min(p.part_blocks * BSZ, ctx - blk0 * BSZ));   // tokens of this partition
     const int npiece = (ntok + K::R - 1) / K::R;
+    const int nstage = (npiece + K::BPS - 1) / K::BPS;
     const int group = p.group;
     const int64_t qh0 = (int64_t)kvh * group;                     // first query head of this KV head
 
-    __syncthreads();
+    __syncthreads();   // the barriers are initialised; the previous unit is done with the ring
 
     float* red_o = reinterpret_cast<float*>(smem);
     float* red_m = red_o + K::NSLOT * K::MAXG * D;
@@ -135,7 +151,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         const int withheld = (blockIdx.x | blockIdx.y | blockIdx.z) == 0 ? p.withhold : -1;
         // 32 blocks' ids per coalesced load; each block gives PPB pieces, the
         // pieces past the partition's last token are not loaded.
-        for (int q0 = 0; q0 < npiece && ok; q0 += 32 * K::PPB) {
+        for (int q0 = 0; q0 < npiece && ok; q0 += 32 * K::PPB) {   // (stage g = base + local stage)
             const int j0 = q0 / K::PPB;
             int id = 0;
             if (j0 + lane < nblk) {
@@ -155,7 +171,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             const int kv = lane & 1, hb = lane >> 1;
             const int h = hb % NB, hd = (hb / NB) % KPC, b = hb / (NB * KPC);
             for (int qs = 0; qs < qn; qs += K::BPS) {
-                const int q = q0 + qs, si = q / K::BPS, st = si % STAGES;
+                const int q = q0 + qs, si = (int)base + q / K::BPS, st = si % STAGES;
                 const int nq = min(K::BPS, npiece - q);               // pieces in this stage
                 if (lane == 0) {
                     if (!mbar_wait_bounded(&empty[st], ((si / STAGES) & 1) ^ 1, p.err, p.wait_ns)) {
@@ -187,7 +203,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         const int hd = cw / K::WPH, sub = cw - hd * K::WPH;               // this warp's KV head, and its turn
         using TQ = std::conditional_t<sizeof(T) == 1, __nv_bfloat16, T>;   // an fp8 cache takes bf16 queries
         const TQ* qbase = static_cast<const TQ*>(p.q) + ((int64_t)seq * p.num_q_heads + qh0 + hd * group) * D;
-        const int nstage = (npiece + K::BPS - 1) / K::BPS;
         const int kofs = hd * K::REGION, vofs = (KPC + hd) * K::REGION;
         if constexpr (PATH == 2) {
             using Cons = std::conditional_t<sizeof(T) == 1, MmaConsumerFp8<K::TOK / TILE_ROWS, HPW / 8>,
@@ -195,8 +210,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             Cons c;
             c.init(reinterpret_cast<const __nv_bfloat16*>(qbase), group, lane);
             for (int j = sub; j < nstage; j += K::WPH) {
-                const int st = j % STAGES;
-                const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err, p.wait_ns);
+                const int g = (int)base + j, st = g % STAGES;
+                const bool got = mbar_wait_bounded(&full[st], (g / STAGES) & 1, p.err, p.wait_ns);
                 if (__any_sync(0xffffffffu, !got || s_abort != 0)) {   // warp-uniform exit
                     s_abort = 1;
                     break;
@@ -218,8 +233,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             c.init(qbase + (int64_t)hbase * D, p.scale_log2, lane);
             const int jstart = PATH == 1 ? 0 : sub, jstep = PATH == 1 ? 1 : K::WPH;
             for (int j = jstart; j < nstage; j += jstep) {
-                const int st = j % STAGES;
-                const bool got = mbar_wait_bounded(&full[st], (j / STAGES) & 1, p.err, p.wait_ns);
+                const int g = (int)base + j, st = g % STAGES;
+                const bool got = mbar_wait_bounded(&full[st], (g / STAGES) & 1, p.err, p.wait_ns);
                 if (__any_sync(0xffffffffu, !got || s_abort != 0)) {
                     s_abort = 1;
                     break;
@@ -271,13 +286,20 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
         }
     }
+    if constexpr (!LOOP) {
+        return;                                                   // one unit per CTA
+    } else {
+        base += (uint32_t)nstage;
+        row += gridDim.y;
+    }
+    }
 }
 
-template <typename T, int D, int PATH, int HPW, int STAGES, int KPC, int BSZ>
-cudaError_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, dim3 grid,
-                          cudaStream_t stream) {
+template <typename T, int D, int PATH, int HPW, int STAGES, int KPC, int BSZ, bool LOOP>
+cudaError_t launch_decode_as(const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, dim3 grid,
+                             cudaStream_t stream) {
     using K = Kern<T, D, PATH, HPW, STAGES, KPC, BSZ>;
-    auto kern = paged_decode_kernel<T, D, PATH, HPW, STAGES, KPC, BSZ>;
+    auto kern = paged_decode_kernel<T, D, PATH, HPW, STAGES, KPC, BSZ, LOOP>;
     grid.x /= KPC;
     // Opt in to >48 KB dynamic shared memory once per device.
     static std::atomic<uint64_t> done_mask{0};
@@ -290,6 +312,8 @@ cudaError_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const Pa
         done_mask.fetch_or(bit);
     }
     if (p.units) {
+        // LOOP: about one wave of CTAs (three per SM) works through the unit list
+        if (LOOP) grid.y = std::min<unsigned>(grid.y, (unsigned)std::max(1, 3 * num_sms() / (int)grid.x));
         // a programmatic dependent of the plan kernel: launched while it runs, the
         // CTAs wait for its list in-kernel (griddepcontrol.wait)
         cudaLaunchConfig_t cfg = {};
@@ -306,6 +330,24 @@ cudaError_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const Pa
     }
     kern<<<grid, NTHREADS, K::SMEM, stream>>>(mk, mv, p);
     return cudaGetLastError();
+}
+
+// The unit-list loop is built for 16-token blocks (the shape of the long-context
+// workload) and used when a context can span kLoopParts or more partitions, where
+// the list can be much shorter than B x partitions; elsewhere every CTA takes one
+// unit. Same-box A/B: long-context 512-token partitions 52.3 -> 48.3 us; with two
+// partitions (70B shape, 32 sequences) one unit per CTA is faster (68.7 vs 74.8
+// us: a fixed stride left some CTAs two long units, and claiming rows from a
+// counter as units finish still cost 3 %); compiled into the one-unit kernel, the
+// loop alone cost ~1 % on single-partition calls.
+template <typename T, int D, int PATH, int HPW, int STAGES, int KPC, int BSZ>
+cudaError_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, dim3 grid,
+                          cudaStream_t stream) {
+    if constexpr (BSZ == 16) {
+        if (p.units && p.num_parts >= kLoopParts)
+            return launch_decode_as<T, D, PATH, HPW, STAGES, KPC, BSZ, true>(mk, mv, p, grid, stream);
+    }
+    return launch_decode_as<T, D, PATH, HPW, STAGES, KPC, BSZ, false>(mk, mv, p, grid, stream);
 }
 
 // Ring depth: about 64 KB of stages per CTA (8 KB per stage for bf16 D=128),
