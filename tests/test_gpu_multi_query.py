@@ -241,3 +241,27 @@ def test_verify_rows_at_kv_tile_boundaries(ctx):
     assert binding.get_device_error() == 0
     assert np.abs(out.cpu().numpy().astype(np.float64) - ref).max() <= 2e-3
     check_bf16_out(_run(dev, out_dtype=torch.bfloat16), ref)
+
+
+@pytest.mark.parametrize("hq,hkv,ns", [
+    (64, 8, [5, 3, 5]),        # 40 rows per KV head (5 draft tokens x group 8)
+    (64, 8, [8, 1, 6]),        # 64 rows
+    (32, 8, [9, 2, 9]),        # 36 rows, group 4
+    (8, 8, [33, 1, 20]),       # 33 rows, group 1
+    (64, 8, [8, 8, 9]),        # 72 rows
+])
+@pytest.mark.parametrize("bs", [8, 16, 32, 64])
+@pytest.mark.parametrize("part", [0, 256])
+def test_verify_sized_rows_on_tcgen05(hq, hkv, ns, bs, part):
+    """33-72 rows per KV head (verify-sized: draft tokens x group) on the tcgen05
+    kernel, its 128-row tile mostly padding; contexts around its 128-token KV tiles
+    and block boundaries, with and without partitions; bf16 output as well."""
+    ctxs = [n + c for n, c in zip(ns, [300, 127, 1000])]
+    dev, ref = _mq_problem(zlib.crc32(repr((hq, hkv, ns, bs)).encode()), hq, hkv, 128, bs, ctxs, ns)
+    out = _run(dev, part=part)
+    torch.cuda.synchronize()
+    assert binding.get_device_error() == 0
+    got = out.cpu().numpy().astype(np.float64)
+    assert np.isfinite(got).all()
+    assert np.abs(got - ref).max() <= 2e-3
+    check_bf16_out(_run(dev, out_dtype=torch.bfloat16, part=part), ref)
