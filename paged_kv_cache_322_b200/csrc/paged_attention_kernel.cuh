@@ -312,8 +312,9 @@ cudaError_t launch_decode_as(const CUtensorMap& mk, const CUtensorMap& mv, const
         done_mask.fetch_or(bit);
     }
     if (p.units) {
-        // LOOP: about one wave of CTAs (three per SM) works through the unit list
-        if (LOOP) grid.y = std::min<unsigned>(grid.y, (unsigned)std::max(1, 3 * num_sms() / (int)grid.x));
+        // LOOP with many partitions: about one wave of CTAs (three per SM) works through the unit list
+        if (LOOP && p.num_parts >= kLoopParts)
+            grid.y = std::min<unsigned>(grid.y, (unsigned)std::max(1, 3 * num_sms() / (int)grid.x));
         // a programmatic dependent of the plan kernel: launched while it runs, the
         // CTAs wait for its list in-kernel (griddepcontrol.wait)
         cudaLaunchConfig_t cfg = {};
@@ -344,7 +345,10 @@ template <typename T, int D, int PATH, int HPW, int STAGES, int KPC, int BSZ>
 cudaError_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, dim3 grid,
                           cudaStream_t stream) {
     if constexpr (BSZ == 16) {
-        if (p.units && p.num_parts >= kLoopParts)
+        // e4m3 caches take the loop build for every listed schedule: compiled with the
+        // loop, its fragments fit the 128 registers (no spill; 48-52 bytes without),
+        // and with a grid of one row per unit the loop runs once
+        if (p.units && (p.num_parts >= kLoopParts || sizeof(T) == 1))
             return launch_decode_as<T, D, PATH, HPW, STAGES, KPC, BSZ, true>(mk, mv, p, grid, stream);
     }
     return launch_decode_as<T, D, PATH, HPW, STAGES, KPC, BSZ, false>(mk, mv, p, grid, stream);
