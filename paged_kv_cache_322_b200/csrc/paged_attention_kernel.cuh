@@ -140,15 +140,15 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     float* red_m = red_o + K::NSLOT * K::MAXG * D;
     float* red_l = red_m + K::NSLOT * K::MAXG;
 
+    int issued = (int)base;                                       // ring stages claimed so far (producer lane 0)
+    // test hook: the first CTA never issues this stage's copies (and never
+    // arrives on its barrier), so its consumer's bounded wait runs out
+    const int withheld = (blockIdx.x | blockIdx.y | blockIdx.z) == 0 ? p.withhold : -1;
     if (warp == 0) {
         // ---------------- producer ----------------
         const uint64_t pol = l2_policy_evict_first();
         const int32_t* bt = p.block_tables + (int64_t)seq * p.max_blocks + blk0;
-        int issued = 0;                                             // stages claimed (copies issued)
         bool ok = true;
-        // test hook: the first CTA never issues this stage's copies (and never
-        // arrives on its barrier), so its consumer's bounded wait runs out
-        const int withheld = (blockIdx.x | blockIdx.y | blockIdx.z) == 0 ? p.withhold : -1;
         // 32 blocks' ids per coalesced load; each block gives PPB pieces, the
         // pieces past the partition's last token are not loaded.
         for (int q0 = 0; q0 < npiece && ok; q0 += 32 * K::PPB) {   // (stage g = base + local stage)
@@ -191,11 +191,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     tma_load_4d(dst, kv ? &tm_v : &tm_k, &full[st], h * K::BOX, kvh + hd, (pq % K::PPB) * K::R, pb, pol);
                 }
             }
-        }
-        if (lane == 0 && !ok) {
-            // Drain: wait (bounded) for every copy still in flight before the CTA exits.
-            for (int j = max(0, issued - STAGES); j < issued; ++j)
-                if (j != withheld) mbar_wait_bounded(&full[j % STAGES], (j / STAGES) & 1, p.err, p.wait_ns);
         }
     } else {
         // ---------------- consumers ----------------
@@ -251,7 +246,15 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         }
     }
     __syncthreads();
-    if (s_abort) return;
+    if (s_abort) {
+        // A wait gave up (here or in a consumer). Every copy this CTA issued lands
+        // before it exits: the producer may have issued all of them and left its
+        // loop before a consumer gave up. (Bounded; stages already consumed pass at once.)
+        if (warp == 0 && lane == 0)
+            for (int j = max((int)base, issued - STAGES); j < issued; ++j)
+                if (j != withheld) mbar_wait_bounded(&full[j % STAGES], (j / STAGES) & 1, p.err, p.wait_ns);
+        return;
+    }
 
     // ---------------- merge consumer states, write output or partial ----------------
     // KV head hd of this CTA: its states are in warp slots [hd * NSLOT / KPC, (hd + 1) * NSLOT / KPC).

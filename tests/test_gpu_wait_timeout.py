@@ -55,6 +55,30 @@ def test_decode_wait_runs_out_then_next_call_is_exact(hq, hkv, d):
     assert torch.equal(again, good)
 
 
+def test_decode_unit_loop_wait_runs_out_then_next_call_is_exact():
+    """64-token partitions over contexts up to 900 tokens: 8 or more partitions per
+    context, so the partition kernel's unit-loop build runs (about one wave of
+    CTAs, each taking several listed units with the ring's phases carried between
+    them). The first CTA's first unit never gets ring stage 2: its consumer gives
+    up, the CTA drains and leaves its loop, and the next call is exact."""
+    ctxs = [600, 900, 500, 130]
+    dev, ref = _mq_problem(33, 32, 4, 128, 16, ctxs, [1, 1, 1, 1])
+    good = _decode(dev, part=64)
+    torch.cuda.synchronize()
+    assert binding.get_device_error() == 0
+    assert np.abs(good.cpu().numpy().astype(np.float64) - ref).max() <= 2e-3
+
+    binding.test_withhold_copy(binding.WITHHOLD_DECODE, 2, LIMIT_NS)
+    _decode(dev, part=64)
+    torch.cuda.synchronize()
+    assert binding.get_device_error() == TIMEOUT
+
+    again = _decode(dev, part=64)
+    torch.cuda.synchronize()
+    assert binding.get_device_error() == 0
+    assert torch.equal(again, good)
+
+
 def test_tcgen05_wait_runs_out_then_tensor_memory_is_free():
     """Group 8, 64 query tokens on a 600-token context: the first CTA's query
     tile sees 552 tokens (5 KV tiles of 128); its producer never issues K of
