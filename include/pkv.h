@@ -333,6 +333,44 @@ pkv_status pkv_paged_attention_multi_query(
     size_t workspace_bytes, void* stream);
 
 /*
+ * Decode attention over a batch whose sequences share a prefix (parallel
+ * sampling after a copy-on-write fork: "为什么PagedAttention能让大模型推理吞吐量
+ * 提升数倍", Memory Sharing). The result is pkv_paged_attention_decode's
+ * (softmax over each sequence's whole context), computed as a cascade that
+ * reads the shared blocks once instead of once per sequence: the B queries
+ * attend to the prefix as one block of B x group rows per KV head, each query
+ * to its own tail, and the partial softmaxes merge exactly. The prefix is cut
+ * into partitions of whole 128-token tiles, about two waves of its call's CTAs
+ * (KV heads x 128-row tiles x partitions), each writing its own partial. The
+ * cascade is not a step of the pages' method (their kernel walks each sequence's
+ * table).
+ *
+ *   prefix_tokens  host; the first prefix_tokens / block_size entries of every
+ *                  row of block_tables are the same blocks (the caller's
+ *                  contract; row 0's are read); a multiple of block_size,
+ *                  below max_context_len.
+ *   context_lens   device int32 [num_seqs], each in (prefix_tokens,
+ *                  max_context_len]; a length outside is flagged
+ *                  PKV_ERR_DEVICE_BOUNDS and read as the nearest valid one.
+ *   workspace      device, >= pkv_paged_attention_shared_prefix_workspace_bytes
+ *                  bytes (for the same batch, heads and prefix_tokens), 256-byte
+ *                  aligned; scratch between calls. The size function returns
+ *                  (size_t)-1 for arguments it cannot size.
+ * Other arguments as pkv_paged_attention_decode. Supported: bf16 caches, head_dim
+ * 128, groups 1, 2, 4, 8, 16, block sizes 8-64, num_seqs x group >= 32 (the
+ * prefix runs on the tcgen05 multi-query kernel); PKV_ERR_UNSUPPORTED otherwise.
+ */
+size_t pkv_paged_attention_shared_prefix_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads,
+                                                        int head_dim, int prefix_tokens);
+
+pkv_status pkv_paged_attention_decode_shared_prefix(
+    void* out, pkv_dtype out_dtype, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, int prefix_tokens, float scale,
+    int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+    int max_blocks_per_seq, int num_blocks, int max_context_len, void* workspace,
+    size_t workspace_bytes, void* stream);
+
+/*
  * FP8 KV append ("vLLM PagedAttention 深度解析" §7.4: K/V stored as FP8 so a block
  * holds twice the tokens). Same addressing as pkv_reshape_and_cache; the caches
  * hold e4m3 codes (1 byte per element) and the stored code of an element x is

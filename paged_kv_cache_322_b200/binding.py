@@ -49,6 +49,9 @@ _SIGS = {
     "pkv_paged_attention_multi_query": (_i32, [_vp, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _f32, _i32, _i32, _i32,
                                                _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp]),
     "pkv_paged_attention_partition_tokens": (_i32, [_i32] * 8),
+    "pkv_paged_attention_shared_prefix_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32]),
+    "pkv_paged_attention_decode_shared_prefix": (_i32, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _f32, _i32, _i32,
+                                                        _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp]),
     "pkv_reshape_and_cache": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pkv_copy_blocks": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pkv_swap_blocks": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp]),
@@ -347,6 +350,42 @@ def paged_attention_multi_query(out, q, k_cache, v_cache, block_tables, context_
         block_tables.data_ptr(), context_lens.data_ptr(), query_start.data_ptr(), float(scale), B, T, hq, hkv, d, bs,
         mb, nb, int(max_query_len), int(max_context_len), int(partition_tokens), ws_ptr, ws_n, _stream(q, stream))
     _check(st, "pkv_paged_attention_multi_query")
+    return out
+
+
+def shared_prefix_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, prefix_tokens) -> int:
+    n = _lib().pkv_paged_attention_shared_prefix_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                                                 prefix_tokens)
+    if n == ctypes.c_size_t(-1).value:
+        raise PkvError(1, "pkv_paged_attention_shared_prefix_workspace_bytes")
+    return n
+
+
+def paged_attention_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, context_lens, prefix_tokens: int,
+                                         scale: float, max_context_len: int, workspace=None, stream=None):
+    """Decode attention (the result of paged_attention_decode) for a batch whose
+    block tables share their first prefix_tokens / block_size entries: the shared
+    blocks are read once for the whole batch (a cascade: prefix, tails, exact
+    merge). out, q [B, Hq, D]; bf16 caches [NB, bs, Hkv, D], head_dim 128."""
+    torch = _torch()
+    _cuda_contig(out, q, k_cache, v_cache, block_tables, context_lens)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    B, hq, d = q.shape
+    nb, bs, hkv, d2 = k_cache.shape
+    if d2 != d or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != (B, hq, d):
+        raise ValueError("shape mismatch")
+    if q.dtype != torch.bfloat16 or k_cache.dtype != torch.bfloat16 or v_cache.dtype != torch.bfloat16:
+        raise TypeError("q and the caches must be bfloat16")
+    need = shared_prefix_workspace_bytes(B, hq, hkv, d, int(prefix_tokens))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = _lib().pkv_paged_attention_decode_shared_prefix(
+        out.data_ptr(), _dtype_code(out), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+        block_tables.data_ptr(), context_lens.data_ptr(), int(prefix_tokens), float(scale), B, hq, hkv, d, bs,
+        block_tables.shape[1], nb, int(max_context_len), workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _stream(q, stream))
+    _check(st, "pkv_paged_attention_decode_shared_prefix")
     return out
 
 

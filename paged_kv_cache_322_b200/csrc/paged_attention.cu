@@ -470,6 +470,60 @@ namespace attn {
 // One decode call. kv_dtype: the cache storage (f32, bf16 or fp8 e4m3); q is
 // kv_dtype for f32 / bf16 caches and bf16 for an fp8 cache, whose K and V
 // scales fold into the logit scale and the output.
+pkv_status decode_to_partial(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                             const int32_t* context_lens, float scale, int num_seqs, int num_q_heads,
+                             int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
+                             int ctx_cap, float* ws_o, float* ws_ml, uint2* units, cudaStream_t st) {
+    const int group = num_q_heads / num_kv_heads;
+    int* err = device_error_word();
+    if (!err) return PKV_ERR_CUDA;
+    const bool use_mma = group >= 2;
+    CUtensorMap mk, mv;
+    if (!make_cache_map(&mk, k_cache, PKV_BF16, num_blocks, block_size, num_kv_heads, head_dim, use_mma) ||
+        !make_cache_map(&mv, v_cache, PKV_BF16, num_blocks, block_size, num_kv_heads, head_dim, use_mma))
+        return PKV_ERR_CUDA;
+    Params p{};
+    p.q = q;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.err = err;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.out_scale = 1.0f;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.group = group;
+    p.max_blocks = max_blocks_per_seq;
+    p.num_blocks = num_blocks;
+    p.ctx_cap = ctx_cap;
+    p.block_size = block_size;
+    p.part_blocks = std::max(1, (ctx_cap + block_size - 1) / block_size);   // one partition per sequence
+    p.num_parts = 1;
+    p.num_seqs = num_seqs;
+    p.ws_o = ws_o;
+    p.ws_ml = ws_ml;
+    p.partials_only = 1;
+    p.withhold = -1;
+    p.wait_ns = kDefaultWaitNs;
+    dim3 grid(num_kv_heads, 1, num_seqs);
+    if (units && num_seqs >= 2 && p.part_blocks <= kPlanMaxBins) {
+        // longest first: the plan kernel sorts the sequences by length, the
+        // decode grid (a programmatic dependent) takes them in that order
+        p.units = units;
+        p.unit_count = reinterpret_cast<int*>(units + num_seqs);
+        plan_units_kernel<<<1, kPlanThreads, 0, st>>>(p);
+        if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
+        grid = dim3(num_kv_heads, num_seqs, 1);
+    }
+    cudaError_t e;
+    switch (block_size) {
+        case 8: e = dispatch_partitioned<8>(PKV_BF16, use_mma, head_dim, group, num_kv_heads, mk, mv, p, grid, st); break;
+        case 16: e = dispatch_partitioned<16>(PKV_BF16, use_mma, head_dim, group, num_kv_heads, mk, mv, p, grid, st); break;
+        case 32: e = dispatch_partitioned<32>(PKV_BF16, use_mma, head_dim, group, num_kv_heads, mk, mv, p, grid, st); break;
+        default: e = dispatch_partitioned<64>(PKV_BF16, use_mma, head_dim, group, num_kv_heads, mk, mv, p, grid, st); break;
+    }
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
 pkv_status decode_impl(void* out, pkv_dtype out_dtype, const void* q, const void* k_cache, const void* v_cache,
                        pkv_dtype kv_dtype, float k_scale, float v_scale, const int32_t* block_tables,
                        const int32_t* context_lens, float scale, int num_seqs, int num_q_heads, int num_kv_heads,

@@ -279,7 +279,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         }
         const float val = L > 0.f ? O / L : 0.f;
         const int64_t qh = (int64_t)seq * p.num_q_heads + qh0 + hd * group + h;
-        if (nparts <= 1) {
+        if (nparts <= 1 && !p.partials_only) {
             store_out(p, qh * D + d, val);
         } else {
             p.ws_o[(qh * C + part) * D + d] = val;

@@ -54,6 +54,9 @@ struct MqParams {
     int max_blocks, num_blocks, ctx_cap, max_query_len;
     int block_size, part_blocks, num_parts, row_tiles;
     int wpr;                      // warps per row group: 1, 2 or 4
+    int causal;                   // 1: query i sees positions <= c - n + i; 0: every query sees the whole context
+    int slot;                     // >= 0: write only normalised partials (o / l, m, l), partition k at index
+                                  // slot + k of num_parts (the shared-prefix cascade); -1: output or partitions
     unsigned long long wait_ns;   // limit of every mbarrier wait (2 s unless the test hook shortened it)
     int withhold;                 // test hook: KV tile whose K copies the first CTA never issues (-1: none)
 };
@@ -80,15 +83,16 @@ __device__ __forceinline__ uint64_t l2_policy_evict_normal() {
     return pol;
 }
 
-// Sequence s's query count n and context c, both checked: 0 <= n <= c <= cap and
-// the queries inside [0, T). A bad entry flags PKV_ERR_DEVICE_BOUNDS and the
-// sequence is skipped (n = 0).
+// Sequence s's query count n and context c, both checked: 0 <= n <= c <= cap (with
+// the causal mask off, 0 < c <= cap) and the queries inside [0, T). A bad entry
+// flags PKV_ERR_DEVICE_BOUNDS and the sequence is skipped (n = 0).
 __device__ __forceinline__ void mq_sequence(const MqParams& p, int s, int& q0, int& n, int& c) {
     q0 = p.query_start[s];
     const int q1 = p.query_start[s + 1];
     c = p.context_lens[s];
     n = q1 - q0;
-    if (q0 < 0 || n < 0 || q1 > p.num_tokens || n > p.max_query_len || c < n || c > p.ctx_cap) {
+    if (q0 < 0 || n < 0 || q1 > p.num_tokens || n > p.max_query_len || (p.causal && c < n) || c > p.ctx_cap ||
+        (!p.causal && c <= 0)) {
         if (threadIdx.x == 0) flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
         n = 0;
         c = 0;
@@ -128,7 +132,7 @@ struct MqConsumer {
             for (int cc = 0; cc < 2; ++cc) {
                 const int rc = row0 + nt * 8 + 2 * t + cc;      // the row of fragment column 2t + cc
                 const int ic = rc / G;
-                pos[nt][cc] = ic < n ? c - n + ic : -1;
+                pos[nt][cc] = ic < n ? (p.causal ? c - n + ic : c - 1) : -1;
                 m[nt][cc] = kNegInf;
                 l[nt][cc] = 0.f;
             }
@@ -322,7 +326,7 @@ paged_mq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     if (row_begin >= n * p.group) return;                          // no live rows in this tile
     // last visible position of the tile's rows, and this partition's KV range
     const int last_tok = min(n - 1, (row_begin + rows_per_tile - 1) / p.group);
-    const int kv_end = c - n + last_tok + 1;                       // tokens [0, kv_end) are visible to some row
+    const int kv_end = p.causal ? c - n + last_tok + 1 : c;        // tokens [0, kv_end) are visible to some row
     const int pt = p.part_blocks * BSZ;
     const int kv0 = part * pt;
     if (kv0 >= kv_end) return;                                     // no row of the tile sees this partition
@@ -330,7 +334,8 @@ paged_mq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int npiece = (ntok + K::R - 1) / K::R;
     const int nblk = (ntok + BSZ - 1) / BSZ;
     const int blk0 = part * p.part_blocks;
-    const bool direct = (c + pt - 1) / pt <= 1;                    // the whole context is one partition
+    const bool direct = p.slot < 0 && (c + pt - 1) / pt <= 1;      // the whole context is one partition
+    const int opart = p.slot >= 0 ? p.slot + part : part;          // the partial's index in the workspace
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
@@ -420,7 +425,7 @@ paged_mq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (lane == 0) mbar_arrive(&empty[st]);
         }
         if (wpr == 1) {
-            if (!s_abort) cons.finish(p, row0, kvh, q0, n, part, direct, lane);
+            if (!s_abort) cons.finish(p, row0, kvh, q0, n, opart, direct, lane);
         } else {
             // merge the wpr partial states of each row group through shared memory
             // (the ring is free once every consumer is past its last stage)
@@ -452,10 +457,10 @@ paged_mq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         }
                     }
                     const int64_t qh = (int64_t)(q0 + i) * p.num_q_heads + kvh * G + h;
-                    mq_store<D>(p, qh, part, direct, d, L > 0.f ? O / L : 0.f);
+                    mq_store<D>(p, qh, opart, direct, d, L > 0.f ? O / L : 0.f);
                     if (!direct && d == 0) {
-                        p.ws_ml[(qh * p.num_parts + part) * 2 + 0] = M;
-                        p.ws_ml[(qh * p.num_parts + part) * 2 + 1] = L;
+                        p.ws_ml[(qh * p.num_parts + opart) * 2 + 0] = M;
+                        p.ws_ml[(qh * p.num_parts + opart) * 2 + 1] = L;
                     }
                 }
             }
@@ -733,6 +738,8 @@ pkv_status pkv_paged_attention_multi_query(void* out, pkv_dtype out_dtype, const
     p.num_parts = pl.num_parts;
     p.row_tiles = pl.row_tiles;
     p.wpr = pl.wpr;
+    p.causal = 1;
+    p.slot = -1;
     p.withhold = -1;
     p.wait_ns = kDefaultWaitNs;
     if (pl.tc) take_wait_hook(1, &p.withhold, &p.wait_ns);
@@ -754,6 +761,241 @@ pkv_status pkv_paged_attention_multi_query(void* out, pkv_dtype out_dtype, const
         else merge_mq_kernel<64><<<g2, 64, 0, st>>>(p);
         if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
     }
+    return PKV_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Shared-prefix decode (a cascade): a batch whose sequences all map the same
+// first `prefix` cache tokens (parallel sampling after a copy-on-write fork,
+// "为什么PagedAttention能让大模型推理吞吐量提升数倍", Memory Sharing) reads those
+// blocks once. The batch's B decode queries attend to the prefix as B query
+// tokens of one sequence with the causal mask off (the tcgen05 kernel: every
+// KV head's prefix tiles are loaded once for all B x G rows; the prefix is cut
+// into partitions so the call fills the GPU), each sequence's query attends to
+// its own tail (the decode kernel, tokens prefix .. ctx - 1 through the table
+// entries past the prefix's blocks); all write normalised partials (o / l, m, l)
+// into slots (the prefix's partitions, then the tail), and an exact log-sum-exp
+// merge of the slots gives softmax over the whole context. Not a step of the
+// pages' method, which reads a shared block once per sequence that maps it.
+// ---------------------------------------------------------------------------
+namespace pkv {
+namespace attn {
+namespace {
+
+struct CascadeWs {
+    float* pre_o;    // [B, Hq, prefix partitions, D]
+    float* pre_ml;   // [B, Hq, prefix partitions, 2]
+    float* tail_o;   // [B, Hq, D]
+    float* tail_ml;  // [B, Hq, 2]
+    uint2* units;    // the tails' longest-first list: B entries and their count
+    int32_t* ints;   // tail lengths [B], prefix length [1], prefix query starts [2]
+};
+
+// Prefix partitions: about two waves of the prefix call's CTAs (KV heads x row
+// tiles x partitions), whole 128-token KV tiles, at most one per tile of prefix.
+int cascade_prefix_parts(int num_seqs, int group, int num_kv_heads, int prefix) {
+    const int row_tiles = (int)(((int64_t)num_seqs * group + tc::ROWS - 1) / tc::ROWS);
+    const int want = std::max(1, 2 * num_sms() / std::max(1, num_kv_heads * row_tiles));
+    return std::max(1, std::min(want, (prefix + tc::TOK - 1) / tc::TOK));
+}
+
+int cascade_prefix_part_tokens(int prefix, int parts) {
+    const int pt = (prefix + parts - 1) / parts;
+    return (pt + tc::TOK - 1) / tc::TOK * tc::TOK;             // whole KV tiles (a multiple of every block size)
+}
+
+// The workspace's regions in order, each 256-byte aligned.
+size_t cascade_region(int i, int num_seqs, int num_q_heads, int head_dim, int pre_parts) {
+    const size_t rows_t = (size_t)num_seqs * num_q_heads, rows_p = rows_t * pre_parts;
+    const size_t sz[6] = {rows_p * head_dim * 4, rows_p * 2 * 4, rows_t * head_dim * 4, rows_t * 2 * 4,
+                          (size_t)num_seqs * sizeof(uint2) + sizeof(int), ((size_t)num_seqs + 3) * 4};
+    size_t off = 0;
+    for (int k = 0; k < i; ++k) off += (sz[k] + 255) & ~size_t(255);
+    return off;
+}
+
+size_t cascade_ws_bytes(int num_seqs, int num_q_heads, int head_dim, int pre_parts) {
+    return cascade_region(6, num_seqs, num_q_heads, head_dim, pre_parts);
+}
+
+CascadeWs cascade_ws(void* workspace, int num_seqs, int num_q_heads, int head_dim, int pre_parts) {
+    uint8_t* b = static_cast<uint8_t*>(workspace);
+    auto at = [&](int i) { return b + cascade_region(i, num_seqs, num_q_heads, head_dim, pre_parts); };
+    CascadeWs w;
+    w.pre_o = reinterpret_cast<float*>(at(0));
+    w.pre_ml = reinterpret_cast<float*>(at(1));
+    w.tail_o = reinterpret_cast<float*>(at(2));
+    w.tail_ml = reinterpret_cast<float*>(at(3));
+    w.units = reinterpret_cast<uint2*>(at(4));
+    w.ints = reinterpret_cast<int32_t*>(at(5));
+    return w;
+}
+
+// The calls' lengths: sequence s's tail is ctx_s - prefix tokens (at least 1:
+// its own new token; a shorter context is flagged and read as prefix + 1, a
+// longer one than the cap as the cap); the prefix call has one sequence of B
+// queries.
+__global__ void cascade_prep_kernel(const int32_t* context_lens, int32_t* ints, int num_seqs, int prefix, int cap,
+                                    int* err) {
+    int32_t* tail_len = ints;
+    int32_t* pre_len = ints + num_seqs;
+    int32_t* pre_qs = pre_len + 1;
+    for (int s = threadIdx.x; s < num_seqs; s += blockDim.x) {
+        int c = context_lens[s];
+        if (c <= prefix || c > cap) {
+            flag_error(err, PKV_ERR_DEVICE_BOUNDS);
+            c = c <= prefix ? prefix + 1 : cap;
+        }
+        tail_len[s] = c - prefix;
+    }
+    if (threadIdx.x == 0) {
+        pre_len[0] = prefix;
+        pre_qs[0] = 0;
+        pre_qs[1] = num_seqs;
+    }
+}
+
+// out[s, h] from the prefix's partials and the tail's: M = max m_i,
+// w_i = l_i 2^(m_i - M), out = sum w_i o_i / sum w_i. grid (Hq, B), D threads.
+template <int D>
+__global__ void __launch_bounds__(D) cascade_merge_kernel(void* out, int out_f32, CascadeWs ws, int num_q_heads,
+                                                          int pre_parts) {
+    const int64_t qh = (int64_t)blockIdx.y * num_q_heads + blockIdx.x;
+    const int d = threadIdx.x;
+    const float* ml = ws.pre_ml + qh * pre_parts * 2;
+    const float* o = ws.pre_o + qh * pre_parts * D + d;
+    const float mt = ws.tail_ml[qh * 2], lt = ws.tail_ml[qh * 2 + 1];
+    float M = mt;
+    for (int i = 0; i < pre_parts; ++i) M = fmaxf(M, ml[2 * i]);
+    float L = 0.f, acc = 0.f;
+    if (M != kNegInf) {
+        for (int i = 0; i < pre_parts; ++i) {
+            const float mi = ml[2 * i];
+            if (mi == kNegInf) continue;
+            const float w = ml[2 * i + 1] * fast_exp2(mi - M);
+            L += w;
+            acc += w * o[(int64_t)i * D];
+        }
+        if (mt != kNegInf) {
+            const float w = lt * fast_exp2(mt - M);
+            L += w;
+            acc += w * ws.tail_o[qh * D + d];
+        }
+    }
+    const float v = L > 0.f ? acc / L : 0.f;
+    if (out_f32) static_cast<float*>(out)[qh * D + d] = v;
+    else static_cast<__nv_bfloat16*>(out)[qh * D + d] = __float2bfloat16_rn(v);
+}
+
+}  // namespace
+}  // namespace attn
+}  // namespace pkv
+
+extern "C" {
+
+size_t pkv_paged_attention_shared_prefix_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads,
+                                                        int head_dim, int prefix_tokens) {
+    if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
+        head_dim <= 0 || prefix_tokens <= 0)
+        return (size_t)-1;
+    const int parts = pkv::attn::cascade_prefix_parts(num_seqs, num_q_heads / num_kv_heads, num_kv_heads,
+                                                      prefix_tokens);
+    return pkv::attn::cascade_ws_bytes(num_seqs, num_q_heads, head_dim, parts);
+}
+
+pkv_status pkv_paged_attention_decode_shared_prefix(void* out, pkv_dtype out_dtype, const void* q, const void* k_cache,
+                                                    const void* v_cache, const int32_t* block_tables,
+                                                    const int32_t* context_lens, int prefix_tokens, float scale,
+                                                    int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                                    int block_size, int max_blocks_per_seq, int num_blocks,
+                                                    int max_context_len, void* workspace, size_t workspace_bytes,
+                                                    void* stream) {
+    using namespace pkv;
+    using namespace pkv::attn;
+    if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
+        max_blocks_per_seq <= 0 || num_blocks <= 0 || !std::isfinite(scale) || max_context_len <= 0)
+        return PKV_ERR_INVALID_ARG;
+    if (out_dtype != PKV_F32 && out_dtype != PKV_BF16) return PKV_ERR_INVALID_ARG;
+    const int group = num_q_heads / num_kv_heads;
+    if (head_dim != 128 || !block_size_built(block_size)) return PKV_ERR_UNSUPPORTED;
+    if (group != 1 && group != 2 && group != 4 && group != 8 && group != 16) return PKV_ERR_UNSUPPORTED;
+    // the prefix call runs on the tcgen05 kernel: at least 32 query rows per KV head
+    if ((int64_t)num_seqs * group < 32 || num_seqs > 65535) return PKV_ERR_UNSUPPORTED;
+    if (prefix_tokens <= 0 || prefix_tokens % block_size != 0 || prefix_tokens >= max_context_len ||
+        (int64_t)max_blocks_per_seq * block_size < max_context_len)
+        return PKV_ERR_INVALID_ARG;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_ERR_INVALID_ARG;
+    auto al = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) == 0; };
+    if (!al(out) || !al(q) || !al(k_cache) || !al(v_cache)) return PKV_ERR_INVALID_ARG;
+    const int pre_parts = cascade_prefix_parts(num_seqs, group, num_kv_heads, prefix_tokens);
+    const int pre_pt = cascade_prefix_part_tokens(prefix_tokens, pre_parts);
+    const int npre = (prefix_tokens + pre_pt - 1) / pre_pt;       // the prefix's partitions (<= pre_parts)
+    if (!workspace || workspace_bytes < cascade_ws_bytes(num_seqs, num_q_heads, head_dim, pre_parts) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return PKV_ERR_INVALID_ARG;
+    int* err = device_error_word();
+    if (!err) return PKV_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const CascadeWs ws = cascade_ws(workspace, num_seqs, num_q_heads, head_dim, npre);
+    const int tail_cap = max_context_len - prefix_tokens;
+    cascade_prep_kernel<<<1, 256, 0, st>>>(context_lens, ws.ints, num_seqs, prefix_tokens, max_context_len, err);
+    if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
+
+    MqParams p{};
+    p.out = nullptr;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.ws_o = ws.pre_o;
+    p.ws_ml = ws.pre_ml;
+    p.err = err;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.group = group;
+    p.num_blocks = num_blocks;
+    p.block_size = block_size;
+    p.num_parts = npre;           // the prefix partials of each row
+    p.withhold = -1;
+    p.wait_ns = kDefaultWaitNs;
+
+    // 1. the prefix, once: B queries of one sequence, no causal mask, one partial per partition (tcgen05)
+    {
+        CUtensorMap mk, mv, mqm;
+        const int box_rows = std::min(block_size, tc::TOK);
+        if (!make_cache_map(&mk, k_cache, PKV_BF16, num_blocks, block_size, num_kv_heads, head_dim, true, box_rows) ||
+            !make_cache_map(&mv, v_cache, PKV_BF16, num_blocks, block_size, num_kv_heads, head_dim, true, box_rows) ||
+            !make_q_map(&mqm, q, num_seqs, num_q_heads, head_dim, group))
+            return PKV_ERR_CUDA;
+        MqParams pp = p;
+        pp.block_tables = block_tables;                         // row 0: its first prefix / bs entries
+        pp.context_lens = ws.ints + num_seqs;
+        pp.query_start = ws.ints + num_seqs + 1;
+        pp.num_seqs = 1;
+        pp.num_tokens = num_seqs;
+        pp.max_blocks = max_blocks_per_seq;
+        pp.ctx_cap = prefix_tokens;
+        pp.max_query_len = num_seqs;
+        pp.part_blocks = pre_pt / block_size;
+        pp.row_tiles = (int)(((int64_t)num_seqs * group + tc::ROWS - 1) / tc::ROWS);
+        pp.wpr = 1;
+        pp.causal = 0;
+        pp.slot = 0;
+        dim3 grid(num_kv_heads, npre, pp.row_tiles);
+        if (launch_mq_tc_bs(block_size, mqm, mk, mv, pp, grid, st) != cudaSuccess) return PKV_ERR_CUDA;
+    }
+    // 2. each sequence's tail: its query over tokens prefix .. ctx - 1 (the decode kernel, longest tail first)
+    {
+        const pkv_status ts = decode_to_partial(q, k_cache, v_cache, block_tables + prefix_tokens / block_size,
+                                                ws.ints, scale, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                                block_size, max_blocks_per_seq, num_blocks, tail_cap, ws.tail_o,
+                                                ws.tail_ml, ws.units, st);
+        if (ts != PKV_OK) return ts;
+    }
+    // 3. the exact merge of the partials
+    cascade_merge_kernel<128><<<dim3(num_q_heads, num_seqs), 128, 0, st>>>(out, out_dtype == PKV_F32, ws, num_q_heads,
+                                                                           npre);
+    if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
     return PKV_OK;
 }
 

@@ -173,14 +173,15 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int row_begin = tile * ROWS;
     if (row_begin >= n * G) return;                             // no live rows (uniform over the CTA)
     const int last_tok = min(n - 1, (row_begin + ROWS - 1) / G);
-    const int kv_end = c - n + last_tok + 1;
+    const int kv_end = p.causal ? c - n + last_tok + 1 : c;
     const int pt = p.part_blocks * BSZ;
     const int kv0 = part * pt;
     if (kv0 >= kv_end) return;
     const int ntok = min(pt, kv_end - kv0);
     const int ntiles = (ntok + TOK - 1) / TOK;
     const int blk0 = part * p.part_blocks;
-    const bool direct = (c + pt - 1) / pt <= 1;
+    const bool direct = p.slot < 0 && (c + pt - 1) / pt <= 1;
+    const int opart = p.slot >= 0 ? p.slot + part : part;        // the partial's index in the workspace
 
     if (threadIdx.x == 0) {
         mbar_init(&bar[B_Q], 1);
@@ -357,7 +358,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const int lr = quarter * 32 + lane;                     // row of the tile = TMEM lane
         const int r = row_begin + lr;
         const int qi = r / G, hh = r - qi * G;
-        const int pos = qi < n ? c - n + qi : -1;
+        const int pos = qi < n ? (p.causal ? c - n + qi : c - 1) : -1;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         constexpr int HC = TOK / 2;                             // columns per thread
         float m_ref = kNegInf, l = 0.f;                         // this half's running reference and sum
@@ -520,7 +521,7 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                                  pack_bf16(o[8 * v4 + 6], o[8 * v4 + 7]));
                     } else {
                         float* dst = direct ? static_cast<float*>(p.out) + qh * D + d0
-                                            : p.ws_o + (qh * p.num_parts + part) * D + d0;
+                                            : p.ws_o + (qh * p.num_parts + opart) * D + d0;
 #pragma unroll
                         for (int v4 = 0; v4 < 8; ++v4)
                             reinterpret_cast<float4*>(dst)[v4] =
@@ -529,8 +530,8 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
             }
             if (live && !direct && half == 0) {
-                p.ws_ml[(qh * p.num_parts + part) * 2 + 0] = M;
-                p.ws_ml[(qh * p.num_parts + part) * 2 + 1] = L;
+                p.ws_ml[(qh * p.num_parts + opart) * 2 + 0] = M;
+                p.ws_ml[(qh * p.num_parts + opart) * 2 + 1] = L;
             }
         }
     }

@@ -513,3 +513,32 @@ def test_step_timing_checks_its_arguments_on_host(lib):
     buf = (ctypes.c_float * 4)()
     assert lib.pkv_step_ctx_set_timing(None, 1) == 1
     assert lib.pkv_step_ctx_last_timing(None, buf) == 1
+
+
+def test_shared_prefix_host_refusals(lib):
+    """The shared-prefix decode refuses, before any launch: shapes it does not
+    build (head_dim 64; fewer than 32 query rows per KV head for its tcgen05 prefix
+    call), a prefix that is not whole blocks or reaches the longest context, and
+    a workspace below its size."""
+    fake = ctypes.c_void_p(1 << 20)
+    ws_need = lib.pkv_paged_attention_shared_prefix_workspace_bytes(32, 32, 32, 128, 1008)
+    rows = 32 * 32 * 2                             # at least one prefix partial and the tail's per row
+    assert ws_need >= rows * (128 * 4 + 2 * 4) + 32 * 8 + 4 + (32 + 3) * 4
+    # at most one prefix partial per 128-token tile: 1008 tokens -> 8 tiles; six 256-byte aligned regions
+    assert ws_need <= 32 * 32 * 9 * (128 * 4 + 2 * 4) + 32 * 8 + 4 + (32 + 3) * 4 + 6 * 256
+    bad = ctypes.c_size_t(-1).value
+    assert lib.pkv_paged_attention_shared_prefix_workspace_bytes(0, 32, 32, 128, 1008) == bad
+    assert lib.pkv_paged_attention_shared_prefix_workspace_bytes(32, 32, 5, 128, 1008) == bad
+    assert lib.pkv_paged_attention_shared_prefix_workspace_bytes(32, 32, 32, 128, 0) == bad
+
+    def call(B=32, hq=32, hkv=32, d=128, bs=16, prefix=1008, maxlen=1500, ws_n=None):
+        return lib.pkv_paged_attention_decode_shared_prefix(
+            fake, 1, fake, fake, fake, fake, fake, prefix, 0.088, B, hq, hkv, d, bs, 128, 4096, maxlen, fake,
+            ws_need if ws_n is None else ws_n, None)
+
+    assert call(d=64) == 2                         # PKV_ERR_UNSUPPORTED
+    assert call(B=16) == 2                         # 16 rows per KV head
+    assert call(B=8, hq=64, hkv=8, ws_n=0) == 1    # 64 rows per KV head: past the shape checks
+    assert call(prefix=1000) == 1                  # PKV_ERR_INVALID_ARG: not whole blocks
+    assert call(prefix=1504, maxlen=1500) == 1     # the prefix reaches the longest context
+    assert call(ws_n=ws_need - 1) == 1             # workspace too small
