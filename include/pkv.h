@@ -340,7 +340,7 @@ pkv_status pkv_paged_attention_multi_query(
  * reads the shared blocks once instead of once per sequence: the B queries
  * attend to the prefix as one block of B x group rows per KV head, each query
  * to its own tail, and the partial softmaxes merge exactly. The prefix is cut
- * into partitions of whole 128-token tiles, about two waves of its call's CTAs
+ * into partitions of whole 128-token tiles, at most one wave of its call's CTAs
  * (KV heads x 128-row tiles x partitions), each writing its own partial. The
  * cascade is not a step of the pages' method (their kernel walks each sequence's
  * table).

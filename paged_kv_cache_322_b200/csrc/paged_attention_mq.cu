@@ -793,11 +793,14 @@ struct CascadeWs {
     int32_t* ints;   // tail lengths [B], prefix length [1], prefix query starts [2]
 };
 
-// Prefix partitions: about two waves of the prefix call's CTAs (KV heads x row
-// tiles x partitions), whole 128-token KV tiles, at most one per tile of prefix.
+// Prefix partitions: at most one wave of the prefix call's CTAs (KV heads x row
+// tiles x partitions; one CTA per SM), whole 128-token KV tiles, at most one per
+// tile of prefix. Measured on the shared-prefix workload's shape (32 KV heads, a
+// 1008-token prefix): 4 partitions (128 CTAs) 69 us a call, 8 (256 CTAs, two
+// rounds) 76 us, 1 (32 CTAs) 78 us.
 int cascade_prefix_parts(int num_seqs, int group, int num_kv_heads, int prefix) {
     const int row_tiles = (int)(((int64_t)num_seqs * group + tc::ROWS - 1) / tc::ROWS);
-    const int want = std::max(1, 2 * num_sms() / std::max(1, num_kv_heads * row_tiles));
+    const int want = std::max(1, num_sms() / std::max(1, num_kv_heads * row_tiles));
     return std::max(1, std::min(want, (prefix + tc::TOK - 1) / tc::TOK));
 }
 
@@ -858,12 +861,15 @@ __global__ void cascade_prep_kernel(const int32_t* context_lens, int32_t* ints, 
 }
 
 // out[s, h] from the prefix's partials and the tail's: M = max m_i,
-// w_i = l_i 2^(m_i - M), out = sum w_i o_i / sum w_i. grid (Hq, B), D threads.
+// w_i = l_i 2^(m_i - M), out = sum w_i o_i / sum w_i. grid (Hq, B), D threads;
+// a programmatic dependent of the tails' decode grid: it waits for that grid
+// (and so for everything before it on the stream) in-kernel.
 template <int D>
 __global__ void __launch_bounds__(D) cascade_merge_kernel(void* out, int out_f32, CascadeWs ws, int num_q_heads,
                                                           int pre_parts) {
     const int64_t qh = (int64_t)blockIdx.y * num_q_heads + blockIdx.x;
     const int d = threadIdx.x;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const float* ml = ws.pre_ml + qh * pre_parts * 2;
     const float* o = ws.pre_o + qh * pre_parts * D + d;
     const float mt = ws.tail_ml[qh * 2], lt = ws.tail_ml[qh * 2 + 1];
@@ -993,9 +999,20 @@ pkv_status pkv_paged_attention_decode_shared_prefix(void* out, pkv_dtype out_dty
         if (ts != PKV_OK) return ts;
     }
     // 3. the exact merge of the partials
-    cascade_merge_kernel<128><<<dim3(num_q_heads, num_seqs), 128, 0, st>>>(out, out_dtype == PKV_F32, ws, num_q_heads,
-                                                                           npre);
-    if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(num_q_heads, num_seqs);
+        cfg.blockDim = dim3(128);
+        cfg.stream = st;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, cascade_merge_kernel<128>, out, (int)(out_dtype == PKV_F32), ws, num_q_heads,
+                               npre) != cudaSuccess)
+            return PKV_ERR_CUDA;
+    }
     return PKV_OK;
 }
 

@@ -123,8 +123,9 @@ def test_shared_prefix_refusals():
 
 
 def test_shared_prefix_long_prefix_fewer_partitions_than_sized():
-    """A 4000-token prefix over 16 KV heads: the workspace is sized for 18 prefix
-    partitions, whole 256-token ones give 16 (the last one ragged)."""
+    """A 4000-token prefix over 16 KV heads: the workspace is sized for 9 prefix
+    partitions (one wave of 148 CTAs), whole 512-token ones give 8 (the last one
+    ragged)."""
     rng = np.random.default_rng(77)
     tails = rng.integers(1, 200, size=16).tolist()
     dev, ref = _problem(77, 16, 32, 16, 16, 250, tails)
