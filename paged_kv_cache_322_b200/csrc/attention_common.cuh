@@ -53,10 +53,13 @@ struct Params {
     // longest-first schedule of the partitioned kernel (plan_units_kernel)
     uint2* units;                   // [B * C]: {seq << 16 | partition, clamped context length}; NULL: grid order
     int* unit_count;                // live units listed
-    // 1: every partition writes its normalised partial (o / l, m, l) to ws_o /
-    // ws_ml, a single one too, never the output (the tails of the shared-prefix
-    // cascade); 0: a context of one partition writes the output directly
-    int partials_only;
+    // pre_parts > 0 (the tails of the shared-prefix cascade, one partition per
+    // sequence): each (sequence, query head) merges the prefix's normalised
+    // partials (pre_o [B, Hq, pre_parts, D], pre_ml [B, Hq, pre_parts, 2]: m in
+    // log2 units, l) with its own result before writing the output
+    const float* pre_o;
+    const float* pre_ml;
+    int pre_parts;
     // bounded waits
     unsigned long long wait_ns;     // limit of every mbarrier wait (2 s unless the test hook shortened it)
     int withhold;                   // test hook: ring stage whose copies the first CTA never issues (-1: none)
@@ -632,15 +635,17 @@ int persistent_ctas_per_sm();
 int persistent_max_seqs();
 // SMs of the current device (paged_attention.cu).
 int num_sms();
-// One decode pass (bf16 cache, one partition per sequence) writing each
-// (sequence, query head)'s normalised partial into ws_o [B, Hq, D] and its
-// (m, l) into ws_ml [B, Hq, 2] instead of the output: the tails of the
-// shared-prefix cascade (paged_attention.cu). units: room for B unit entries
-// and their count (the longest-first order), or null for grid order.
-pkv_status decode_to_partial(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
-                             const int32_t* context_lens, float scale, int num_seqs, int num_q_heads,
-                             int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
-                             int ctx_cap, float* ws_o, float* ws_ml, uint2* units, cudaStream_t st);
+// The tails of the shared-prefix cascade (paged_attention_mq.cu): one decode
+// pass (bf16 cache, one partition per sequence) over the table rows past the
+// prefix, in the longest-first order that `units` already lists (B entries and
+// their count, from list_units), launched as a programmatic dependent of the
+// call before it on the stream, which has written the prefix's partials; each
+// (sequence, query head) merges them into its result and writes the output.
+pkv_status decode_tails_with_prefix(void* out, pkv_dtype out_dtype, const void* q, const void* k_cache,
+                                    const void* v_cache, const int32_t* block_tables, const uint2* units,
+                                    float scale, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                    int block_size, int max_blocks_per_seq, int num_blocks, int ctx_cap,
+                                    const float* pre_o, const float* pre_ml, int pre_parts, cudaStream_t st);
 
 }  // namespace attn
 }  // namespace pkv

@@ -39,6 +39,7 @@
 #include <type_traits>
 
 #include "attention_common.cuh"
+#include "plan_units.cuh"
 
 namespace pkv {
 namespace attn {
@@ -164,124 +165,23 @@ __global__ void __launch_bounds__(GROUPS * D) merge_partitions_kernel(const Para
 }
 
 // ---------------------------------------------------------------------------
-// Longest-first schedule of the partitioned kernel (one CTA).
-//
-// A grid sized for the longest context leaves most rows without work when
-// lengths are mixed, and CTAs taken in grid order start long partitions late:
-// measured with per-CTA timestamps, a 7B-shaped batch streamed ~7.5 TB/s while
-// all 444 CTA slots were busy, then spent its last 35 of 210 us finishing late
-// long sequences, and the long-context grid had 5528 empty CTAs among 872 with
-// work. This kernel lists the live (sequence, partition) units: every full
-// partition first, then each sequence's last partition by decreasing size (a
-// sequence of length 0 last: its CTA writes the zero output). Row y of the
-// partition grid takes unit y; rows past the list exit at the end of dispatch.
+// Longest-first schedule of the partitioned kernel (one CTA; plan_units.cuh).
 // It flags lengths outside [0, ctx_cap] and lists them clamped.
 // ---------------------------------------------------------------------------
-constexpr int kPlanThreads = 256;
-
-// Exclusive scan of one value per thread over the CTA; *total gets the sum.
-__device__ __forceinline__ int cta_exclusive_scan(int v, int* s_warp, int* total) {
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    int incl = v;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += t;
-    }
-    if (lane == 31) s_warp[wid] = incl;
-    __syncthreads();
-    if (wid == 0) {
-        int w = lane < kPlanThreads / 32 ? s_warp[lane] : 0;
-        int wi = w;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, wi, off);
-            if (lane >= off) wi += t;
-        }
-        if (lane < kPlanThreads / 32) s_warp[lane] = wi - w;
-        if (lane == 31) s_warp[kPlanThreads / 32] = wi;
-    }
-    __syncthreads();
-    const int r = s_warp[wid] + incl - v;
-    *total = s_warp[kPlanThreads / 32];
-    __syncthreads();                                            // s_warp is reused by the next scan
-    return r;
-}
-
 __global__ void __launch_bounds__(kPlanThreads) plan_units_kernel(const Params p) {
     // the partition kernel may start its CTAs now; they wait for the list in-kernel
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    __shared__ int hist[kPlanMaxBins];                          // tails per size (blocks), then their offsets
-    __shared__ int s_warp[kPlanThreads / 32 + 1];
-    __shared__ int s_first[kPlanThreads];                       // a pass's first full unit per sequence
-    __shared__ int s_ctx[kPlanThreads];
-    const int B = p.num_seqs, pb = p.part_blocks, bsz = p.block_size, tid = threadIdx.x;
-    for (int b = tid; b < pb; b += kPlanThreads) hist[b] = 0;
-    __syncthreads();
-    // full partitions, listed sequence-major; the tails counted by size
-    int nfull = 0;
-    int ctx_keep = 0;                                           // this thread's length when B fits one pass
-    for (int s0 = 0; s0 < B; s0 += kPlanThreads) {
-        const int sq = s0 + tid;
-        int full = 0, ctx = 0;
-        if (sq < B) {
-            ctx = p.context_lens[sq];
-            if (ctx < 0 || ctx > p.ctx_cap) {
-                flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
-                ctx = ctx < 0 ? 0 : p.ctx_cap;
+    const int cap = p.ctx_cap;
+    list_units(
+        [&](int sq, bool first) {
+            int ctx = p.context_lens[sq];
+            if (ctx < 0 || ctx > cap) {
+                if (first) flag_error(p.err, PKV_ERR_DEVICE_BOUNDS);
+                ctx = ctx < 0 ? 0 : cap;
             }
-            const int nb = (ctx + bsz - 1) / bsz;
-            full = nb / pb;
-            if (nb % pb != 0 || nb == 0) atomicAdd(&hist[nb % pb], 1);
-        }
-        ctx_keep = ctx;
-        int chunk = 0;
-        const int off = cta_exclusive_scan(full, s_warp, &chunk);
-        s_first[tid] = off;
-        s_ctx[tid] = ctx;
-        __syncthreads();
-        // the pass's full units, spread over the threads: unit u belongs to the
-        // last sequence whose first unit is <= u (binary search)
-        for (int u = tid; u < chunk; u += kPlanThreads) {
-            int lo = 0, hi = kPlanThreads - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (s_first[mid] <= u) lo = mid; else hi = mid - 1;
-            }
-            p.units[nfull + u] = make_uint2(((unsigned)(s0 + lo) << 16) | (unsigned)(u - s_first[lo]),
-                                            (unsigned)s_ctx[lo]);
-        }
-        nfull += chunk;
-        __syncthreads();                                        // s_first / s_ctx are reused by the next pass
-    }
-    // tail offsets in decreasing size: offset(size b) = tails longer than b
-    int ntail = 0;
-    for (int b0 = 0; b0 < pb; b0 += kPlanThreads) {
-        const int b = pb - 1 - (b0 + tid);                        // sizes from the largest down
-        const int h = b >= 0 ? hist[b] : 0;
-        int chunk = 0;
-        const int off = ntail + cta_exclusive_scan(h, s_warp, &chunk);
-        if (b >= 0) hist[b] = nfull + off;
-        ntail += chunk;
-        __syncthreads();
-    }
-    // the tails, each at the next free place of its size
-    for (int s0 = 0; s0 < B; s0 += kPlanThreads) {
-        const int sq = s0 + tid;
-        if (sq < B) {
-            int ctx = ctx_keep;
-            if (B > kPlanThreads) {
-                ctx = p.context_lens[sq];
-                ctx = ctx < 0 ? 0 : (ctx > p.ctx_cap ? p.ctx_cap : ctx);
-            }
-            const int nb = (ctx + bsz - 1) / bsz;
-            if (nb % pb != 0 || nb == 0) {
-                const int at = atomicAdd(&hist[nb % pb], 1);
-                p.units[at] = make_uint2(((unsigned)sq << 16) | (unsigned)(nb / pb), (unsigned)ctx);
-            }
-        }
-    }
-    if (tid == 0) *p.unit_count = nfull + ntail;
+            return ctx;
+        },
+        p.num_seqs, p.part_blocks, p.block_size, p.units, p.unit_count);
 }
 
 // ---------------------------------------------------------------------------
@@ -470,10 +370,11 @@ namespace attn {
 // One decode call. kv_dtype: the cache storage (f32, bf16 or fp8 e4m3); q is
 // kv_dtype for f32 / bf16 caches and bf16 for an fp8 cache, whose K and V
 // scales fold into the logit scale and the output.
-pkv_status decode_to_partial(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
-                             const int32_t* context_lens, float scale, int num_seqs, int num_q_heads,
-                             int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
-                             int ctx_cap, float* ws_o, float* ws_ml, uint2* units, cudaStream_t st) {
+pkv_status decode_tails_with_prefix(void* out, pkv_dtype out_dtype, const void* q, const void* k_cache,
+                                    const void* v_cache, const int32_t* block_tables, const uint2* units,
+                                    float scale, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                    int block_size, int max_blocks_per_seq, int num_blocks, int ctx_cap,
+                                    const float* pre_o, const float* pre_ml, int pre_parts, cudaStream_t st) {
     const int group = num_q_heads / num_kv_heads;
     int* err = device_error_word();
     if (!err) return PKV_ERR_CUDA;
@@ -483,12 +384,14 @@ pkv_status decode_to_partial(const void* q, const void* k_cache, const void* v_c
         !make_cache_map(&mv, v_cache, PKV_BF16, num_blocks, block_size, num_kv_heads, head_dim, use_mma))
         return PKV_ERR_CUDA;
     Params p{};
+    p.out = out;
     p.q = q;
     p.block_tables = block_tables;
-    p.context_lens = context_lens;
+    p.context_lens = nullptr;                                   // each unit carries its (tail) length
     p.err = err;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.out_scale = 1.0f;
+    p.out_f32 = out_dtype == PKV_F32;
     p.num_q_heads = num_q_heads;
     p.num_kv_heads = num_kv_heads;
     p.group = group;
@@ -499,21 +402,14 @@ pkv_status decode_to_partial(const void* q, const void* k_cache, const void* v_c
     p.part_blocks = std::max(1, (ctx_cap + block_size - 1) / block_size);   // one partition per sequence
     p.num_parts = 1;
     p.num_seqs = num_seqs;
-    p.ws_o = ws_o;
-    p.ws_ml = ws_ml;
-    p.partials_only = 1;
+    p.units = const_cast<uint2*>(units);
+    p.unit_count = const_cast<int*>(reinterpret_cast<const int*>(units + num_seqs));
+    p.pre_o = pre_o;
+    p.pre_ml = pre_ml;
+    p.pre_parts = pre_parts;
     p.withhold = -1;
     p.wait_ns = kDefaultWaitNs;
-    dim3 grid(num_kv_heads, 1, num_seqs);
-    if (units && num_seqs >= 2 && p.part_blocks <= kPlanMaxBins) {
-        // longest first: the plan kernel sorts the sequences by length, the
-        // decode grid (a programmatic dependent) takes them in that order
-        p.units = units;
-        p.unit_count = reinterpret_cast<int*>(units + num_seqs);
-        plan_units_kernel<<<1, kPlanThreads, 0, st>>>(p);
-        if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
-        grid = dim3(num_kv_heads, num_seqs, 1);
-    }
+    const dim3 grid(num_kv_heads, num_seqs, 1);                 // row y takes listed unit y
     cudaError_t e;
     switch (block_size) {
         case 8: e = dispatch_partitioned<8>(PKV_BF16, use_mma, head_dim, group, num_kv_heads, mk, mv, p, grid, st); break;

@@ -277,11 +277,33 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 O += red_o[(w * K::MAXG + h) * D + d] * sc;
             }
         }
-        const float val = L > 0.f ? O / L : 0.f;
         const int64_t qh = (int64_t)seq * p.num_q_heads + qh0 + hd * group + h;
-        if (nparts <= 1 && !p.partials_only) {
-            store_out(p, qh * D + d, val);
+        if (nparts <= 1 && p.pre_parts > 0) {
+            // the shared prefix's partials and this tail: out = sum w_i o_i / sum w_i
+            const float* pm = p.pre_ml + qh * p.pre_parts * 2;
+            const float* po = p.pre_o + qh * p.pre_parts * D + d;
+            float Mx = M;
+            for (int i = 0; i < p.pre_parts; ++i) Mx = fmaxf(Mx, pm[2 * i]);
+            float Lx = 0.f, Ox = 0.f;
+            if (Mx != kNegInf) {
+                if (M != kNegInf) {
+                    const float sc = fast_exp2(M - Mx);
+                    Lx = L * sc;
+                    Ox = O * sc;
+                }
+                for (int i = 0; i < p.pre_parts; ++i) {
+                    const float mi = pm[2 * i];
+                    if (mi == kNegInf) continue;
+                    const float w = pm[2 * i + 1] * fast_exp2(mi - Mx);
+                    Lx += w;
+                    Ox += w * po[(int64_t)i * D];
+                }
+            }
+            store_out(p, qh * D + d, Lx > 0.f ? Ox / Lx : 0.f);
+        } else if (nparts <= 1) {
+            store_out(p, qh * D + d, L > 0.f ? O / L : 0.f);
         } else {
+            const float val = L > 0.f ? O / L : 0.f;
             p.ws_o[(qh * C + part) * D + d] = val;
             if (d == 0) {
                 p.ws_ml[(qh * C + part) * 2 + 0] = M;

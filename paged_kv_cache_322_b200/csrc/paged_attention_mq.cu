@@ -27,6 +27,7 @@
 #include <cmath>
 
 #include "attention_common.cuh"
+#include "plan_units.cuh"
 
 namespace pkv {
 namespace attn {
@@ -773,11 +774,11 @@ pkv_status pkv_paged_attention_multi_query(void* out, pkv_dtype out_dtype, const
 // blocks once. The batch's B decode queries attend to the prefix as B query
 // tokens of one sequence with the causal mask off (the tcgen05 kernel: every
 // KV head's prefix tiles are loaded once for all B x G rows; the prefix is cut
-// into partitions so the call fills the GPU), each sequence's query attends to
-// its own tail (the decode kernel, tokens prefix .. ctx - 1 through the table
-// entries past the prefix's blocks); all write normalised partials (o / l, m, l)
-// into slots (the prefix's partitions, then the tail), and an exact log-sum-exp
-// merge of the slots gives softmax over the whole context. Not a step of the
+// into partitions so the call fills the GPU, each writing a normalised partial
+// (o / l, m, l)); then each sequence's query attends to its own tail (the decode
+// kernel, tokens prefix .. ctx - 1 through the table entries past the prefix's
+// blocks, longest tail first), and merges the prefix's partials into its result
+// by the exact log-sum-exp rule before writing the output. Not a step of the
 // pages' method, which reads a shared block once per sequence that maps it.
 // ---------------------------------------------------------------------------
 namespace pkv {
@@ -787,10 +788,8 @@ namespace {
 struct CascadeWs {
     float* pre_o;    // [B, Hq, prefix partitions, D]
     float* pre_ml;   // [B, Hq, prefix partitions, 2]
-    float* tail_o;   // [B, Hq, D]
-    float* tail_ml;  // [B, Hq, 2]
-    uint2* units;    // the tails' longest-first list: B entries and their count
-    int32_t* ints;   // tail lengths [B], prefix length [1], prefix query starts [2]
+    uint2* units;    // the tails' list: B entries and their count
+    int32_t* ints;   // the prefix call's length [1] and query starts [2]
 };
 
 // Prefix partitions: at most one wave of the prefix call's CTAs (KV heads x row
@@ -811,16 +810,15 @@ int cascade_prefix_part_tokens(int prefix, int parts) {
 
 // The workspace's regions in order, each 256-byte aligned.
 size_t cascade_region(int i, int num_seqs, int num_q_heads, int head_dim, int pre_parts) {
-    const size_t rows_t = (size_t)num_seqs * num_q_heads, rows_p = rows_t * pre_parts;
-    const size_t sz[6] = {rows_p * head_dim * 4, rows_p * 2 * 4, rows_t * head_dim * 4, rows_t * 2 * 4,
-                          (size_t)num_seqs * sizeof(uint2) + sizeof(int), ((size_t)num_seqs + 3) * 4};
+    const size_t rows_p = (size_t)num_seqs * num_q_heads * pre_parts;
+    const size_t sz[4] = {rows_p * head_dim * 4, rows_p * 2 * 4, (size_t)num_seqs * sizeof(uint2) + sizeof(int), 3 * 4};
     size_t off = 0;
     for (int k = 0; k < i; ++k) off += (sz[k] + 255) & ~size_t(255);
     return off;
 }
 
 size_t cascade_ws_bytes(int num_seqs, int num_q_heads, int head_dim, int pre_parts) {
-    return cascade_region(6, num_seqs, num_q_heads, head_dim, pre_parts);
+    return cascade_region(4, num_seqs, num_q_heads, head_dim, pre_parts);
 }
 
 CascadeWs cascade_ws(void* workspace, int num_seqs, int num_q_heads, int head_dim, int pre_parts) {
@@ -829,70 +827,42 @@ CascadeWs cascade_ws(void* workspace, int num_seqs, int num_q_heads, int head_di
     CascadeWs w;
     w.pre_o = reinterpret_cast<float*>(at(0));
     w.pre_ml = reinterpret_cast<float*>(at(1));
-    w.tail_o = reinterpret_cast<float*>(at(2));
-    w.tail_ml = reinterpret_cast<float*>(at(3));
-    w.units = reinterpret_cast<uint2*>(at(4));
-    w.ints = reinterpret_cast<int32_t*>(at(5));
+    w.units = reinterpret_cast<uint2*>(at(2));
+    w.ints = reinterpret_cast<int32_t*>(at(3));
     return w;
 }
 
-// The calls' lengths: sequence s's tail is ctx_s - prefix tokens (at least 1:
-// its own new token; a shorter context is flagged and read as prefix + 1, a
-// longer one than the cap as the cap); the prefix call has one sequence of B
-// queries.
-__global__ void cascade_prep_kernel(const int32_t* context_lens, int32_t* ints, int num_seqs, int prefix, int cap,
-                                    int* err) {
-    int32_t* tail_len = ints;
-    int32_t* pre_len = ints + num_seqs;
-    int32_t* pre_qs = pre_len + 1;
-    for (int s = threadIdx.x; s < num_seqs; s += blockDim.x) {
+// The plan of the call (one CTA of kPlanThreads): sequence s's tail is ctx_s -
+// prefix tokens (at least 1: its own new token; a shorter context is flagged
+// and read as prefix + 1, one past the cap as the cap), listed longest first
+// (list_units; in sequence order when a tail of tail_cap tokens spans more
+// blocks than the list's size bins), and the prefix call's descriptors: one
+// sequence of `prefix` tokens with B queries.
+__global__ void __launch_bounds__(kPlanThreads) cascade_plan_kernel(const int32_t* context_lens, CascadeWs ws,
+                                                                     int num_seqs, int prefix, int cap, int block_size,
+                                                                     int* err) {
+    const int tail_cap = cap - prefix;
+    auto tail = [&](int s, bool first) {
         int c = context_lens[s];
         if (c <= prefix || c > cap) {
-            flag_error(err, PKV_ERR_DEVICE_BOUNDS);
+            if (first) flag_error(err, PKV_ERR_DEVICE_BOUNDS);
             c = c <= prefix ? prefix + 1 : cap;
         }
-        tail_len[s] = c - prefix;
+        return c - prefix;
+    };
+    const int pb = (tail_cap + block_size - 1) / block_size;  // the tails' one partition, in blocks
+    if (pb <= kPlanMaxBins) {
+        list_units(tail, num_seqs, pb, block_size, ws.units, reinterpret_cast<int*>(ws.units + num_seqs));
+    } else {
+        for (int s = threadIdx.x; s < num_seqs; s += kPlanThreads)
+            ws.units[s] = make_uint2((unsigned)s << 16, (unsigned)tail(s, true));
+        if (threadIdx.x == 0) *reinterpret_cast<int*>(ws.units + num_seqs) = num_seqs;
     }
     if (threadIdx.x == 0) {
-        pre_len[0] = prefix;
-        pre_qs[0] = 0;
-        pre_qs[1] = num_seqs;
+        ws.ints[0] = prefix;
+        ws.ints[1] = 0;
+        ws.ints[2] = num_seqs;
     }
-}
-
-// out[s, h] from the prefix's partials and the tail's: M = max m_i,
-// w_i = l_i 2^(m_i - M), out = sum w_i o_i / sum w_i. grid (Hq, B), D threads;
-// a programmatic dependent of the tails' decode grid: it waits for that grid
-// (and so for everything before it on the stream) in-kernel.
-template <int D>
-__global__ void __launch_bounds__(D) cascade_merge_kernel(void* out, int out_f32, CascadeWs ws, int num_q_heads,
-                                                          int pre_parts) {
-    const int64_t qh = (int64_t)blockIdx.y * num_q_heads + blockIdx.x;
-    const int d = threadIdx.x;
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    const float* ml = ws.pre_ml + qh * pre_parts * 2;
-    const float* o = ws.pre_o + qh * pre_parts * D + d;
-    const float mt = ws.tail_ml[qh * 2], lt = ws.tail_ml[qh * 2 + 1];
-    float M = mt;
-    for (int i = 0; i < pre_parts; ++i) M = fmaxf(M, ml[2 * i]);
-    float L = 0.f, acc = 0.f;
-    if (M != kNegInf) {
-        for (int i = 0; i < pre_parts; ++i) {
-            const float mi = ml[2 * i];
-            if (mi == kNegInf) continue;
-            const float w = ml[2 * i + 1] * fast_exp2(mi - M);
-            L += w;
-            acc += w * o[(int64_t)i * D];
-        }
-        if (mt != kNegInf) {
-            const float w = lt * fast_exp2(mt - M);
-            L += w;
-            acc += w * ws.tail_o[qh * D + d];
-        }
-    }
-    const float v = L > 0.f ? acc / L : 0.f;
-    if (out_f32) static_cast<float*>(out)[qh * D + d] = v;
-    else static_cast<__nv_bfloat16*>(out)[qh * D + d] = __float2bfloat16_rn(v);
 }
 
 }  // namespace
@@ -946,7 +916,8 @@ pkv_status pkv_paged_attention_decode_shared_prefix(void* out, pkv_dtype out_dty
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const CascadeWs ws = cascade_ws(workspace, num_seqs, num_q_heads, head_dim, npre);
     const int tail_cap = max_context_len - prefix_tokens;
-    cascade_prep_kernel<<<1, 256, 0, st>>>(context_lens, ws.ints, num_seqs, prefix_tokens, max_context_len, err);
+    cascade_plan_kernel<<<1, kPlanThreads, 0, st>>>(context_lens, ws, num_seqs, prefix_tokens, max_context_len,
+                                                     block_size, err);
     if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
 
     MqParams p{};
@@ -975,8 +946,8 @@ pkv_status pkv_paged_attention_decode_shared_prefix(void* out, pkv_dtype out_dty
             return PKV_ERR_CUDA;
         MqParams pp = p;
         pp.block_tables = block_tables;                         // row 0: its first prefix / bs entries
-        pp.context_lens = ws.ints + num_seqs;
-        pp.query_start = ws.ints + num_seqs + 1;
+        pp.context_lens = ws.ints;
+        pp.query_start = ws.ints + 1;
         pp.num_seqs = 1;
         pp.num_tokens = num_seqs;
         pp.max_blocks = max_blocks_per_seq;
@@ -990,30 +961,11 @@ pkv_status pkv_paged_attention_decode_shared_prefix(void* out, pkv_dtype out_dty
         dim3 grid(num_kv_heads, npre, pp.row_tiles);
         if (launch_mq_tc_bs(block_size, mqm, mk, mv, pp, grid, st) != cudaSuccess) return PKV_ERR_CUDA;
     }
-    // 2. each sequence's tail: its query over tokens prefix .. ctx - 1 (the decode kernel, longest tail first)
-    {
-        const pkv_status ts = decode_to_partial(q, k_cache, v_cache, block_tables + prefix_tokens / block_size,
-                                                ws.ints, scale, num_seqs, num_q_heads, num_kv_heads, head_dim,
-                                                block_size, max_blocks_per_seq, num_blocks, tail_cap, ws.tail_o,
-                                                ws.tail_ml, ws.units, st);
-        if (ts != PKV_OK) return ts;
-    }
-    // 3. the exact merge of the partials
-    {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(num_q_heads, num_seqs);
-        cfg.blockDim = dim3(128);
-        cfg.stream = st;
-        cudaLaunchAttribute at[1];
-        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        at[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = at;
-        cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, cascade_merge_kernel<128>, out, (int)(out_dtype == PKV_F32), ws, num_q_heads,
-                               npre) != cudaSuccess)
-            return PKV_ERR_CUDA;
-    }
-    return PKV_OK;
+    // 2. each sequence's tail: its query over tokens prefix .. ctx - 1 (the decode kernel, longest tail
+    //    first), merged with the prefix's partials into the output
+    return decode_tails_with_prefix(out, out_dtype, q, k_cache, v_cache, block_tables + prefix_tokens / block_size,
+                                    ws.units, scale, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                    max_blocks_per_seq, num_blocks, tail_cap, ws.pre_o, ws.pre_ml, npre, st);
 }
 
 }  // extern "C"

@@ -522,10 +522,10 @@ def test_shared_prefix_host_refusals(lib):
     a workspace below its size."""
     fake = ctypes.c_void_p(1 << 20)
     ws_need = lib.pkv_paged_attention_shared_prefix_workspace_bytes(32, 32, 32, 128, 1008)
-    rows = 32 * 32 * 2                             # at least one prefix partial and the tail's per row
-    assert ws_need >= rows * (128 * 4 + 2 * 4) + 32 * 8 + 4 + (32 + 3) * 4
-    # at most one prefix partial per 128-token tile: 1008 tokens -> 8 tiles; six 256-byte aligned regions
-    assert ws_need <= 32 * 32 * 9 * (128 * 4 + 2 * 4) + 32 * 8 + 4 + (32 + 3) * 4 + 6 * 256
+    rows = 32 * 32                                 # (sequence, query head) rows: one prefix partial at least
+    assert ws_need >= rows * (128 * 4 + 2 * 4) + 32 * 8 + 4 + 3 * 4
+    # at most one prefix partial per 128-token tile: 1008 tokens -> 8 tiles; four 256-byte aligned regions
+    assert ws_need <= 8 * rows * (128 * 4 + 2 * 4) + 32 * 8 + 4 + 3 * 4 + 4 * 256
     bad = ctypes.c_size_t(-1).value
     assert lib.pkv_paged_attention_shared_prefix_workspace_bytes(0, 32, 32, 128, 1008) == bad
     assert lib.pkv_paged_attention_shared_prefix_workspace_bytes(32, 32, 5, 128, 1008) == bad
