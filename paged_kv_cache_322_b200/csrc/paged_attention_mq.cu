@@ -519,8 +519,10 @@ namespace attn {
 namespace {
 
 template <int BSZ>
+// pdl: launched as a programmatic dependent of the kernel before it on the
+// stream (its CTAs wait for that grid in-kernel).
 cudaError_t launch_mq_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const MqParams& p,
-                         dim3 grid, cudaStream_t st) {
+                         dim3 grid, cudaStream_t st, bool pdl) {
     auto kern = tc::paged_mq_tc_kernel<BSZ>;
     static std::atomic<uint64_t> done_mask{0};
     int dev = 0;
@@ -531,17 +533,30 @@ cudaError_t launch_mq_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
         if (e != cudaSuccess) return e;
         done_mask.fetch_or(bit);
     }
+    if (pdl) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(tc::THREADS);
+        cfg.dynamicSmemBytes = tc::SMEM;
+        cfg.stream = st;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, p);
+    }
     kern<<<grid, tc::THREADS, tc::SMEM, st>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_mq_tc_bs(int bs, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                            const MqParams& p, dim3 grid, cudaStream_t st) {
+                            const MqParams& p, dim3 grid, cudaStream_t st, bool pdl = false) {
     switch (bs) {
-        case 8: return launch_mq_tc<8>(mq, mk, mv, p, grid, st);
-        case 16: return launch_mq_tc<16>(mq, mk, mv, p, grid, st);
-        case 32: return launch_mq_tc<32>(mq, mk, mv, p, grid, st);
-        default: return launch_mq_tc<64>(mq, mk, mv, p, grid, st);
+        case 8: return launch_mq_tc<8>(mq, mk, mv, p, grid, st, pdl);
+        case 16: return launch_mq_tc<16>(mq, mk, mv, p, grid, st, pdl);
+        case 32: return launch_mq_tc<32>(mq, mk, mv, p, grid, st, pdl);
+        default: return launch_mq_tc<64>(mq, mk, mv, p, grid, st, pdl);
     }
 }
 
@@ -841,6 +856,8 @@ CascadeWs cascade_ws(void* workspace, int num_seqs, int num_q_heads, int head_di
 __global__ void __launch_bounds__(kPlanThreads) cascade_plan_kernel(const int32_t* context_lens, CascadeWs ws,
                                                                      int num_seqs, int prefix, int cap, int block_size,
                                                                      int* err) {
+    // the prefix call may start its CTAs now; they wait for this grid in-kernel
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tail_cap = cap - prefix;
     auto tail = [&](int s, bool first) {
         int c = context_lens[s];
@@ -959,7 +976,7 @@ pkv_status pkv_paged_attention_decode_shared_prefix(void* out, pkv_dtype out_dty
         pp.causal = 0;
         pp.slot = 0;
         dim3 grid(num_kv_heads, npre, pp.row_tiles);
-        if (launch_mq_tc_bs(block_size, mqm, mk, mv, pp, grid, st) != cudaSuccess) return PKV_ERR_CUDA;
+        if (launch_mq_tc_bs(block_size, mqm, mk, mv, pp, grid, st, /*pdl=*/true) != cudaSuccess) return PKV_ERR_CUDA;
     }
     // 2. each sequence's tail: its query over tokens prefix .. ctx - 1 (the decode kernel, longest tail
     //    first), merged with the prefix's partials into the output

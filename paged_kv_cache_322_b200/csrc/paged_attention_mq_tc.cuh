@@ -168,6 +168,9 @@ paged_mq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int seq = blockIdx.z / p.row_tiles, tile = blockIdx.z - seq * p.row_tiles;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.group;
+    // launched as a programmatic dependent (the shared-prefix cascade), the CTAs
+    // wait here for the grid that wrote the call's lengths; a no-op otherwise
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     int q0, n, c;
     mq_sequence(p, seq, q0, n, c);
     const int row_begin = tile * ROWS;
