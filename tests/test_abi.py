@@ -542,3 +542,23 @@ def test_shared_prefix_host_refusals(lib):
     assert call(prefix=1000) == 1                  # PKV_ERR_INVALID_ARG: not whole blocks
     assert call(prefix=1504, maxlen=1500) == 1     # the prefix reaches the longest context
     assert call(ws_n=ws_need - 1) == 1             # workspace too small
+
+
+def test_shared_prefix_workspace_follows_the_prefix_partition_rule(lib):
+    """The shared-prefix workspace holds one normalised partial per (sequence,
+    query head, prefix partition) plus the tails' unit list and the prefix
+    call's descriptors, each region 256-byte aligned. Prefix partitions: at most
+    one wave of the prefix call's CTAs (KV heads x 128-row tiles x partitions,
+    one CTA per SM; without a GPU the library assumes 148 SMs), at most one per
+    128-token tile of the prefix, at least one."""
+    def r256(x):
+        return (x + 255) // 256 * 256
+
+    for B, hq, hkv, prefix in [(32, 32, 32, 1008), (8, 64, 8, 4000), (200, 8, 8, 64), (4, 128, 8, 16),
+                               (64, 32, 4, 8192), (33, 33, 1, 128)]:
+        group = hq // hkv
+        row_tiles = -(-B * group // 128)
+        parts = max(1, min(max(1, 148 // (hkv * row_tiles)), -(-prefix // 128)))
+        rows = B * hq * parts
+        want = r256(rows * 128 * 4) + r256(rows * 2 * 4) + r256(B * 8 + 4) + r256(12)
+        assert lib.pkv_paged_attention_shared_prefix_workspace_bytes(B, hq, hkv, 128, prefix) == want, (B, hq, hkv)
