@@ -338,12 +338,13 @@ pkv_status pkv_paged_attention_multi_query(
  * 提升数倍", Memory Sharing). The result is pkv_paged_attention_decode's
  * (softmax over each sequence's whole context), computed as a cascade that
  * reads the shared blocks once instead of once per sequence: the B queries
- * attend to the prefix as one block of B x group rows per KV head, each query
- * to its own tail, and the partial softmaxes merge exactly. The prefix is cut
- * into partitions of whole 128-token tiles, at most one wave of its call's CTAs
- * (KV heads x 128-row tiles x partitions), each writing its own partial. The
- * cascade is not a step of the pages' method (their kernel walks each sequence's
- * table).
+ * attend to the prefix as one block of B x group rows per KV head (its tokens
+ * cut into partitions of whole 128-token tiles, at most one wave of the prefix
+ * call's CTAs: KV heads x 128-row tiles x partitions, each writing a partial),
+ * then each query to its own tail, longest tail first, merging the prefix's
+ * partials into its result by the exact log-sum-exp rule before it writes the
+ * output. Three kernels on `stream`, no host synchronisation. The cascade is not
+ * a step of the pages' method (their kernel walks each sequence's table).
  *
  *   prefix_tokens  host; the first prefix_tokens / block_size entries of every
  *                  row of block_tables are the same blocks (the caller's
@@ -358,7 +359,11 @@ pkv_status pkv_paged_attention_multi_query(
  *                  (size_t)-1 for arguments it cannot size.
  * Other arguments as pkv_paged_attention_decode. Supported: bf16 caches, head_dim
  * 128, groups 1, 2, 4, 8, 16, block sizes 8-64, num_seqs x group >= 32 (the
- * prefix runs on the tcgen05 multi-query kernel); PKV_ERR_UNSUPPORTED otherwise.
+ * prefix runs on the tcgen05 multi-query kernel), num_seqs <= 65535;
+ * PKV_ERR_UNSUPPORTED otherwise. Host-side argument errors (a prefix that is not
+ * whole blocks or reaches max_context_len, a table too narrow for
+ * max_context_len, a null or misaligned pointer, a small workspace) return
+ * PKV_ERR_INVALID_ARG before any launch.
  */
 size_t pkv_paged_attention_shared_prefix_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads,
                                                         int head_dim, int prefix_tokens);
