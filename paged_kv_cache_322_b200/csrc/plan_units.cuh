@@ -13,6 +13,8 @@
 // partition grid takes unit y; rows past the list exit at the end of dispatch.
 #pragma once
 
+#include "attention_common.cuh"
+
 namespace pkv {
 namespace attn {
 
