@@ -299,6 +299,19 @@ def mq_attention_bytes(lens_after, n: int, hq: int, hkv: int, d: int, bs: int) -
             int(sum(-(-int(c) // bs) for c in lens_after)) * 4)
 
 
+def decode_launches(num_seqs: int, part: int, part_used: int, maxctx: int, block_size: int) -> int:
+    """Kernels one decode attention call launches: the plan kernel when the
+    library lists units longest first (two or more sequences, at most 65535
+    units, partitions of at most 4096 blocks), the partition kernel, and the
+    merge when the longest context spans more than one partition; the
+    persistent schedule (part -1) is one kernel."""
+    if part == -1:
+        return 1
+    parts = max(1, -(-maxctx // part_used))
+    plan = 1 if (num_seqs >= 2 and num_seqs * parts <= 65535 and part_used // block_size <= 4096) else 0
+    return plan + 1 + (1 if parts > 1 else 0)
+
+
 def append_bytes(w: wl.Workload) -> int:
     n = w.num_kv_heads * w.head_dim
     return w.num_seqs * (2 * n * (w.in_bytes + w.elt_bytes) + 8)   # K and V rows read and written, slot ids
@@ -394,7 +407,7 @@ def run_pkv(args, ws, rank, local):
     attn_avg_ms = statistics.mean(attn_ms)
     attn_bytes_avg = statistics.mean(s["bytes_attn"] for s in timed)
     achieved = attn_bytes_avg / (attn_avg_ms * 1e-3) / 1e9
-    launches_per_step = 2 + (1 if (part_used > 0 and maxctx > part_used) else 0)
+    launches_per_step = 1 + decode_launches(w.num_seqs, part, part_used, maxctx, w.block_size)   # + the append
     del steps
 
     # ---- end to end through the C ABI from host buffers: pkv_decode_step ----
@@ -872,7 +885,7 @@ def run_shared_prefix(args, ws, rank, local):
                      "algorithmic_bytes_per_launch": int(au), "bytes_basis": "unique", "traffic": None},
         "e2e": e2e,
         "cascade": cascade,
-        "gpu_launches": (3 + (1 if (part_used > 0 and maxctx > part_used) else 0)) * K,
+        "gpu_launches": (2 + decode_launches(B, part, part_used, maxctx, bs)) * K,   # + copy_blocks, append
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,
     }
