@@ -94,3 +94,24 @@ def test_reference_arm_line(monkeypatch):
     assert r["impl"] == "reference" and r["value"] > 0 and r["ms_per_step"] > 0 and r["config"]["global_batch"] == 2
     assert r["cpu_baseline"]["kind"] == "oracle" and r["cpu_baseline"]["cores"] >= 1
     assert r["e2e"]["h2d_bytes_per_step"] == 0 and r["e2e"]["d2h_bytes_per_step"] == 0
+
+
+@pytest.mark.parametrize("B,maxctx,part,bs", [(64, 2060, 0, 16), (1, 4096, 0, 16), (16, 32768, 512, 16),
+                                              (32, 1552, 0, 16), (4000, 4096, 256, 16), (2, 70000, 0, 16),
+                                              (8, 300, 64, 8)])
+def test_decode_launch_count_matches_the_library_schedule(B, maxctx, part, bs):
+    """gpu_launches counts the plan kernel exactly when the library lists units
+    longest first — which shows in the workspace it asks for: the unit list at
+    its front, before any split-K partials."""
+    from paged_kv_cache_322_b200 import binding
+    hq, hkv, d = 32, 8, 128
+    mb = -(-maxctx // bs)
+    pt = binding.partition_tokens(B, hq, hkv, d, bs, mb, maxctx, part)
+    ws = binding.workspace_bytes(B, hq, hkv, d, bs, mb, maxctx, part)
+    parts = -(-maxctx // pt)
+    partials = 0
+    if parts > 1:
+        rows = B * hq * parts
+        partials = (rows * d * 4 + 255) // 256 * 256 + rows * 2 * 4
+    plan = ws - partials > 0
+    assert bench.decode_launches(B, part, pt, maxctx, bs) == int(plan) + 1 + int(parts > 1)
